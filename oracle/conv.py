@@ -1,0 +1,168 @@
+"""The CGTP convolution, its adjoints and the per-atom forces (fp64).
+
+Test infrastructure only (see ``oracle/__init__``).
+
+Definition ("LunaTP: Enabling Efficient and Scalable Tensor Product for
+Equivariant MLIPs", abstract: CGTP convolutions; selection rules from "Tensor
+Decomposition Networks ...", reply to reviewer S6y1).  For every edge
+e = (j -> i) with edge vector r_e, real harmonics Y_e = Y(r_e/|r_e|) and
+weights W_e[p][u]:
+
+    out[i][l3, m3][u] = sum_{e in row i} sum_{p=(l1,l2,l3)} W_e[p][u]
+                        sum_{m1,m2} C^p[m1,m2,m3] x[j][l1,m1][u] Y_e[l2,m2]
+
+Readings where the pages are silent: no normalisation constants (no
+1/sqrt(degree), no path normalisation); paths that share l3 are summed into
+one output block; feature layout [node][l*l + m + l][u].
+
+This module evaluates the sum literally: every path, every nonzero
+(m1, m2, m3), every edge, vectorised only over channels and edge chunks.  It
+does not factor the per-edge matrix sum_m2 C Y out of the channel loop.
+
+Backward (the bilinear adjoints of the same sum, cf. the closed-form
+gradients of a bilinear tensor product in the reply to reviewer S6y1):
+
+    grad_x[j][l1,m1][u] = sum_{e: src=j} sum_p W_e[p][u] sum_{m2,m3} C Y_e[l2,m2] g[i][l3,m3][u]
+    grad_W[e][p][u]     = sum_{m1,m2,m3} C x[j][l1,m1][u] Y_e[l2,m2] g[i][l3,m3][u]
+    grad_Y[e][l2,m2]    = sum_p sum_{m1,m3} C sum_u W_e[p][u] x[j][l1,m1][u] g[i][l3,m3][u]
+    grad_r[e]           = (dY_e/dr_e)^T grad_Y[e]
+
+Forces: with r_e = pos_j - pos_i, dE/dpos_j += grad_r[e] and
+dE/dpos_i -= grad_r[e]; the force is F = -dE/dpos.
+"""
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+from .cg import paths, real_cg
+from .graph import edge_dst
+from .sh import real_sh, real_sh_jacobian
+
+
+def path_nonzeros(lmax_in, lmax_sh, lmax_out):
+    """[(p, row_in, row_sh, row_out, C)] for every nonzero real CG entry,
+    rows being offsets into the concatenated l = 0..L layouts."""
+    out = []
+    for p, (l1, l2, l3) in enumerate(paths(lmax_in, lmax_sh, lmax_out)):
+        C = real_cg(l1, l2, l3)
+        for a, b, c in zip(*np.nonzero(C)):
+            out.append((p, l1 * l1 + int(a), l2 * l2 + int(b), l3 * l3 + int(c), float(C[a, b, c])))
+    return out
+
+
+def _chunks(n, size):
+    return [(s, min(n, s + size)) for s in range(0, n, size)]
+
+
+def _map_chunks(fn, n, chunk, threads):
+    parts = _chunks(n, chunk)
+    if threads <= 1 or len(parts) <= 1:
+        return [fn(s, e) for s, e in parts]
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        return list(ex.map(lambda se: fn(*se), parts))
+
+
+def edge_messages(src, edge_vec, x, w, lmax_in, lmax_sh, lmax_out):
+    """m[e][l3,m3][u]: the contribution of edge e to its destination row."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    E, u = w.shape[0], x.shape[2]
+    Y = real_sh(edge_vec, lmax_sh)
+    xs = x[src]
+    m = np.zeros((E, (lmax_out + 1) ** 2, u))
+    for p, ri, rs, ro, c in path_nonzeros(lmax_in, lmax_sh, lmax_out):
+        m[:, ro, :] += c * w[:, p, :] * xs[:, ri, :] * Y[:, rs][:, None]
+    return m
+
+
+def conv_forward(row_ptr, col, edge_vec, x, w, lmax_in, lmax_sh, lmax_out,
+                 threads=1, chunk=4096):
+    """out [N][(lmax_out+1)^2][u] in fp64."""
+    row_ptr = np.asarray(row_ptr, dtype=np.int64)
+    col = np.asarray(col, dtype=np.int64)
+    x = np.asarray(x, dtype=np.float64)
+    n, u = row_ptr.size - 1, x.shape[2]
+    dst = edge_dst(row_ptr)
+
+    def part(s, e):
+        o = np.zeros((n, (lmax_out + 1) ** 2, u))
+        m = edge_messages(col[s:e], np.asarray(edge_vec)[s:e], x, np.asarray(w)[s:e],
+                          lmax_in, lmax_sh, lmax_out)
+        np.add.at(o, dst[s:e], m)
+        return o
+
+    out = np.zeros((n, (lmax_out + 1) ** 2, u))
+    for o in _map_chunks(part, col.size, chunk, threads):
+        out += o
+    return out
+
+
+def conv_forward_rows(row_ptr, col, edge_vec, x, w, lmax_in, lmax_sh, lmax_out, rows):
+    """Output rows ``rows`` only (for sampling graphs too large to evaluate)."""
+    row_ptr = np.asarray(row_ptr, dtype=np.int64)
+    res = []
+    for i in rows:
+        s, e = row_ptr[i], row_ptr[i + 1]
+        m = edge_messages(np.asarray(col)[s:e], np.asarray(edge_vec)[s:e], x,
+                          np.asarray(w)[s:e], lmax_in, lmax_sh, lmax_out)
+        res.append(m.sum(axis=0))
+    return np.stack(res) if res else np.zeros((0, (lmax_out + 1) ** 2, np.asarray(x).shape[2]))
+
+
+def edge_backward(src, dst, edge_vec, x, w, g, lmax_in, lmax_sh, lmax_out):
+    """Per-edge adjoints: (msg_x [E][(lmax_in+1)^2][u], grad_w [E][P][u], grad_r [E][3])."""
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    E, P, u = w.shape
+    Y = real_sh(edge_vec, lmax_sh)
+    J = real_sh_jacobian(edge_vec, lmax_sh)
+    xs, gd = x[src], g[dst]
+    mx = np.zeros((E, (lmax_in + 1) ** 2, u))
+    gw = np.zeros((E, P, u))
+    gY = np.zeros((E, (lmax_sh + 1) ** 2))
+    for p, ri, rs, ro, c in path_nonzeros(lmax_in, lmax_sh, lmax_out):
+        mx[:, ri, :] += c * w[:, p, :] * Y[:, rs][:, None] * gd[:, ro, :]
+        gw[:, p, :] += c * xs[:, ri, :] * Y[:, rs][:, None] * gd[:, ro, :]
+        gY[:, rs] += c * np.sum(w[:, p, :] * xs[:, ri, :] * gd[:, ro, :], axis=1)
+    gr = np.einsum("eb,ebk->ek", gY, J)
+    return mx, gw, gr
+
+
+def conv_backward(row_ptr, col, edge_vec, x, w, grad_out, lmax_in, lmax_sh, lmax_out,
+                  threads=1, chunk=4096):
+    """(grad_x [N][(lmax_in+1)^2][u], grad_w [E][P][u], grad_edge_vec [E][3]) in fp64."""
+    row_ptr = np.asarray(row_ptr, dtype=np.int64)
+    col = np.asarray(col, dtype=np.int64)
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w)
+    n, u = row_ptr.size - 1, x.shape[2]
+    E, P = col.size, w.shape[1]
+    dst = edge_dst(row_ptr)
+    grad_w = np.zeros((E, P, u))
+    grad_r = np.zeros((E, 3))
+
+    def part(s, e):
+        gx = np.zeros((n, (lmax_in + 1) ** 2, u))
+        mx, gw, gr = edge_backward(col[s:e], dst[s:e], np.asarray(edge_vec)[s:e], x, w[s:e],
+                                   grad_out, lmax_in, lmax_sh, lmax_out)
+        np.add.at(gx, col[s:e], mx)
+        grad_w[s:e] = gw
+        grad_r[s:e] = gr
+        return gx
+
+    grad_x = np.zeros((n, (lmax_in + 1) ** 2, u))
+    for gx in _map_chunks(part, E, chunk, threads):
+        grad_x += gx
+    return grad_x, grad_w, grad_r
+
+
+def edge_forces(row_ptr, col, grad_edge_vec, n_nodes):
+    """F = -dE/dpos from dE/dr_e, with r_e = pos_src - pos_dst."""
+    col = np.asarray(col, dtype=np.int64)
+    dst = edge_dst(row_ptr).astype(np.int64)
+    gr = np.asarray(grad_edge_vec, dtype=np.float64)
+    dEdpos = np.zeros((n_nodes, 3))
+    np.add.at(dEdpos, col, gr)
+    np.add.at(dEdpos, dst, -gr)
+    return -dEdpos
