@@ -1,0 +1,245 @@
+"""Python binding of libcgtp.so over torch CUDA tensors.
+
+Argument marshalling only: every step runs in the library's kernels; torch
+supplies device memory and the current stream.  Tensors must be CUDA,
+contiguous, fp32 (features, weights, vectors) or int32 (indices), in the
+layouts of include/cgtp.h.
+"""
+import ctypes
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from ._lib import call, lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(t, dtype, name):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def n_paths(lmax_in, lmax_sh, lmax_out):
+    return sum(1 for l1 in range(lmax_in + 1) for l2 in range(lmax_sh + 1)
+               for l3 in range(abs(l1 - l2), min(l1 + l2, lmax_out) + 1))
+
+
+def supported(lmax_in, lmax_sh, lmax_out):
+    return bool(lib().cgtp_supported(lmax_in, lmax_sh, lmax_out))
+
+
+def cg_block(l1, l2, l3):
+    """Dense real CG block of one path from the library's host generator (no GPU)."""
+    import numpy as np
+    out = np.zeros((2 * l1 + 1) * (2 * l2 + 1) * (2 * l3 + 1), dtype=np.float64)
+    call("cgtp_cg_block", l1, l2, l3, out.ctypes.data_as(ctypes.c_void_p))
+    return out.reshape(2 * l1 + 1, 2 * l2 + 1, 2 * l3 + 1)
+
+
+@dataclass
+class Graph:
+    n_nodes: int
+    n_edges: int
+    row_ptr: torch.Tensor   # [N+1] int32
+    col: torch.Tensor       # [E] int32, source of each edge
+    edge_vec: torch.Tensor  # [E][3] fp32, pos_src - pos_dst
+    csc_ptr: torch.Tensor   # [N+1] int32
+    csc_edge: torch.Tensor  # [E] int32
+    csc_dst: torch.Tensor   # [E] int32
+
+
+def build_graph(pos, rc, box=None, graph_ptr=None, max_edges=None, n_edges_out=None):
+    """Neighbour list on the device.  Reads the edge count back once (4 bytes);
+    if it exceeds the capacity, rebuilds with exactly enough room."""
+    _check(pos, torch.float32, "pos")
+    _check(graph_ptr, torch.int32, "graph_ptr")
+    n = pos.shape[0]
+    dev = pos.device
+    if max_edges is None:
+        max_edges = max(64, 64 * n)
+    while True:
+        row_ptr = torch.empty(n + 1, dtype=torch.int32, device=dev)
+        csc_ptr = torch.empty(n + 1, dtype=torch.int32, device=dev)
+        col = torch.empty(max(max_edges, 1), dtype=torch.int32, device=dev)
+        ev = torch.empty((max(max_edges, 1), 3), dtype=torch.float32, device=dev)
+        ce = torch.empty(max(max_edges, 1), dtype=torch.int32, device=dev)
+        cd = torch.empty(max(max_edges, 1), dtype=torch.int32, device=dev)
+        ne = n_edges_out if n_edges_out is not None else torch.empty(1, dtype=torch.int32, device=dev)
+        call("cgtp_graph_build", _ptr(pos), n, ctypes.c_float(0.0 if box is None else float(box)),
+             ctypes.c_float(float(rc)), _ptr(graph_ptr), 0 if graph_ptr is None else graph_ptr.numel() - 1,
+             _ptr(row_ptr), _ptr(col), _ptr(ev), _ptr(csc_ptr), _ptr(ce), _ptr(cd), max_edges, _ptr(ne),
+             _stream())
+        E = int(ne.item())
+        if E <= max_edges:
+            return Graph(n, E, row_ptr, col[:E], ev[:E], csc_ptr, ce[:E], cd[:E])
+        max_edges = E
+
+
+def csr_transpose(n, row_ptr, col):
+    """(csc_ptr, csc_edge, csc_dst) of an arbitrary CSR graph."""
+    _check(row_ptr, torch.int32, "row_ptr")
+    _check(col, torch.int32, "col")
+    E = col.numel()
+    dev = row_ptr.device
+    csc_ptr = torch.empty(n + 1, dtype=torch.int32, device=dev)
+    ce = torch.empty(max(E, 1), dtype=torch.int32, device=dev)
+    cd = torch.empty(max(E, 1), dtype=torch.int32, device=dev)
+    ws = torch.empty(max(n, 1), dtype=torch.int32, device=dev)
+    call("cgtp_csr_transpose", n, E, _ptr(row_ptr), _ptr(col), _ptr(csc_ptr), _ptr(ce), _ptr(cd), _ptr(ws),
+         ws.numel() * 4, _stream())
+    return csc_ptr, ce[:E], cd[:E]
+
+
+def graph_check(n, row_ptr, col, edge_vec):
+    """Device-side validation flags (see cgtp_graph_check)."""
+    flags = torch.empty(1, dtype=torch.int32, device=row_ptr.device)
+    call("cgtp_graph_check", n, col.numel(), _ptr(row_ptr), _ptr(col), _ptr(edge_vec), _ptr(flags), _stream())
+    return int(flags.item())
+
+
+def spherical_harmonics(lmax_sh, edge_vec, with_grad=False):
+    _check(edge_vec, torch.float32, "edge_vec")
+    E = edge_vec.shape[0]
+    NS = (lmax_sh + 1) ** 2
+    Y = torch.empty((E, NS), dtype=torch.float32, device=edge_vec.device)
+    dY = torch.empty((E, NS, 3), dtype=torch.float32, device=edge_vec.device) if with_grad else None
+    call("cgtp_spherical_harmonics", lmax_sh, E, _ptr(edge_vec), _ptr(Y), _ptr(dY), _stream())
+    return (Y, dY) if with_grad else Y
+
+
+def forces(graph, grad_edge_vec, out=None):
+    _check(grad_edge_vec, torch.float32, "grad_edge_vec")
+    if out is None:
+        out = torch.empty((graph.n_nodes, 3), dtype=torch.float32, device=grad_edge_vec.device)
+    call("cgtp_forces", graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr), _ptr(graph.csc_ptr),
+         _ptr(graph.csc_edge), _ptr(grad_edge_vec), _ptr(out), _stream())
+    return out
+
+
+class Plan:
+    """Paths and CG coefficients of one irreps shape (lmax_in, lmax_sh, lmax_out, mult)."""
+
+    def __init__(self, lmax_in, lmax_sh, lmax_out, mult):
+        self.lmax_in, self.lmax_sh, self.lmax_out, self.mult = lmax_in, lmax_sh, lmax_out, mult
+        h = ctypes.c_void_p()
+        call("cgtp_plan_create", lmax_in, lmax_sh, lmax_out, mult, ctypes.byref(h))
+        self._h = h
+        n = ctypes.c_int()
+        nnz = ctypes.c_int()
+        call("cgtp_plan_info", h, ctypes.byref(n), None, ctypes.byref(nnz))
+        buf = (ctypes.c_int * (3 * n.value))()
+        call("cgtp_plan_info", h, ctypes.byref(n), ctypes.cast(buf, ctypes.c_void_p), ctypes.byref(nnz))
+        self.n_paths = n.value
+        self.n_cg_nonzero = nnz.value
+        self.paths = [tuple(buf[3 * k:3 * k + 3]) for k in range(n.value)]
+        self.ni, self.ns, self.no = (lmax_in + 1) ** 2, (lmax_sh + 1) ** 2, (lmax_out + 1) ** 2
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            try:
+                lib().cgtp_plan_destroy(h)
+            except Exception:
+                pass
+            self._h = None
+
+    # ------------------------------------------------------------ convolution
+    def conv_forward(self, graph, x, w, out=None):
+        _check(x, torch.float32, "x")
+        _check(w, torch.float32, "w")
+        if out is None:
+            out = torch.empty((graph.n_nodes, self.no, self.mult), dtype=torch.float32, device=x.device)
+        call("cgtp_conv_forward", self._h, graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr), _ptr(graph.col),
+             _ptr(graph.edge_vec), _ptr(x), _ptr(w), _ptr(out), _stream())
+        return out
+
+    def conv_backward_workspace_bytes(self, n_edges):
+        b = ctypes.c_size_t()
+        call("cgtp_conv_backward_workspace_size", self._h, n_edges, ctypes.byref(b))
+        return b.value
+
+    def conv_backward(self, graph, x, w, grad_out, want_x=True, want_w=True, want_r=True,
+                      grad_x=None, grad_w=None, grad_edge_vec=None, workspace=None):
+        _check(x, torch.float32, "x")
+        _check(w, torch.float32, "w")
+        _check(grad_out, torch.float32, "grad_out")
+        dev = x.device
+        E = graph.n_edges
+        if want_x and grad_x is None:
+            grad_x = torch.empty((graph.n_nodes, self.ni, self.mult), dtype=torch.float32, device=dev)
+        if want_w and grad_w is None:
+            grad_w = torch.empty((E, self.n_paths, self.mult), dtype=torch.float32, device=dev)
+        if want_r and grad_edge_vec is None:
+            grad_edge_vec = torch.empty((E, 3), dtype=torch.float32, device=dev)
+        ws_bytes = 0
+        if want_r:
+            ws_bytes = self.conv_backward_workspace_bytes(E)
+            if workspace is None:
+                workspace = torch.empty(max(ws_bytes // 4, 64), dtype=torch.float32, device=dev)
+        call("cgtp_conv_backward", self._h, graph.n_nodes, E, _ptr(graph.csc_ptr), _ptr(graph.csc_edge),
+             _ptr(graph.csc_dst), _ptr(graph.edge_vec), _ptr(x), _ptr(w), _ptr(grad_out),
+             _ptr(grad_x if want_x else None), _ptr(grad_w if want_w else None),
+             _ptr(grad_edge_vec if want_r else None), _ptr(workspace if want_r else None),
+             workspace.numel() * 4 if (want_r and workspace is not None) else 0, _stream())
+        return (grad_x if want_x else None, grad_w if want_w else None, grad_edge_vec if want_r else None)
+
+    # ------------------------------------------------------------ radial network
+    def radial_forward(self, edge_vec, rc, W1, W2, out=None):
+        _check(edge_vec, torch.float32, "edge_vec")
+        _check(W1, torch.float32, "W1")
+        _check(W2, torch.float32, "W2")
+        E = edge_vec.shape[0]
+        if out is None:
+            out = torch.empty((E, self.n_paths, self.mult), dtype=torch.float32, device=edge_vec.device)
+        call("cgtp_radial_forward", self._h, E, _ptr(edge_vec), ctypes.c_float(float(rc)), _ptr(W1), _ptr(W2),
+             _ptr(out), _stream())
+        return out
+
+    def radial_backward(self, edge_vec, rc, W1, W2, grad_w, grad_edge_vec):
+        """Adds dL/d edge_vec through the weights into grad_edge_vec (in place)."""
+        _check(grad_w, torch.float32, "grad_w")
+        _check(grad_edge_vec, torch.float32, "grad_edge_vec")
+        call("cgtp_radial_backward", self._h, edge_vec.shape[0], _ptr(edge_vec), ctypes.c_float(float(rc)),
+             _ptr(W1), _ptr(W2), _ptr(grad_w), _ptr(grad_edge_vec), _stream())
+        return grad_edge_vec
+
+    # ------------------------------------------------------------ edge-free product
+    def tp_forward(self, x, y, w, out=None):
+        for t, nm in ((x, "x"), (y, "y"), (w, "w")):
+            _check(t, torch.float32, nm)
+        B = x.shape[0]
+        if out is None:
+            out = torch.empty((B, self.no, self.mult), dtype=torch.float32, device=x.device)
+        call("cgtp_tp_forward", self._h, B, _ptr(x), _ptr(y), _ptr(w), _ptr(out), _stream())
+        return out
+
+    def tp_backward(self, x, y, w, grad_z, want_x=True, want_y=True, want_w=True):
+        B = x.shape[0]
+        dev = x.device
+        gx = torch.empty_like(x) if want_x else None
+        gy = torch.empty_like(y) if want_y else None
+        gw = torch.empty_like(w) if want_w else None
+        ws = None
+        nb = 0
+        if want_w:
+            b = ctypes.c_size_t()
+            call("cgtp_tp_backward_workspace_size", self._h, B, ctypes.byref(b))
+            nb = b.value
+            ws = torch.empty(max(nb // 4, 64), dtype=torch.float32, device=dev)
+        call("cgtp_tp_backward", self._h, B, _ptr(x), _ptr(y), _ptr(w), _ptr(grad_z), _ptr(gx), _ptr(gy),
+             _ptr(gw), _ptr(ws), nb, _stream())
+        return gx, gy, gw

@@ -1,0 +1,378 @@
+// C ABI of libcgtp.so: argument checks, plans, coefficient-table upload and
+// dispatch to the per-shape kernels.  Declared in include/cgtp.h.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "cg_table.h"
+#include "configs.h"
+#include "launch.h"
+#include "structure.h"
+#include "../../include/cgtp.h"
+
+namespace cgtp {
+
+// ---------------------------------------------------------------- uploaders
+static std::vector<UploadFn>& uploaders() {
+  static std::vector<UploadFn> v;
+  return v;
+}
+int register_table_uploader(UploadFn fn) {
+  uploaders().push_back(fn);
+  return 1;
+}
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+cgtp_status cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int)e;
+  return CGTP_ERR_CUDA;
+}
+
+struct HostTables {
+  float cg[kTableSize];
+  float shk[kShkSize];
+  int status = -1;
+};
+
+HostTables& host_tables() {
+  static HostTables t;
+  static std::once_flag once;
+  std::call_once(once, [] { t.status = build_constant_tables(t.cg, t.shk); });
+  return t;
+}
+
+std::mutex g_dev_mutex;
+std::vector<int> g_uploaded;  // per device: 1 once the tables are in its constant memory
+std::vector<int> g_num_sms;
+
+cgtp_status ensure_device(int* num_sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if ((int)g_uploaded.size() <= dev) {
+    g_uploaded.resize(dev + 1, 0);
+    g_num_sms.resize(dev + 1, 0);
+  }
+  if (!g_uploaded[dev]) {
+    HostTables& t = host_tables();
+    if (t.status != 0) return CGTP_ERR_TABLE;
+    for (UploadFn fn : uploaders()) {
+      e = fn(t.cg, t.shk);
+      if (e != cudaSuccess) return cuda_fail(e);
+    }
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_num_sms[dev] = sms;
+    g_uploaded[dev] = 1;
+  }
+  *num_sms = g_num_sms[dev];
+  return CGTP_OK;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+#define CGTP_LIST_ENTRY(a, b, c) {a, b, c},
+struct Shape {
+  int li, ls, lo;
+};
+const Shape kShapes[] = {CGTP_CONFIGS(CGTP_LIST_ENTRY)};
+
+}  // namespace
+}  // namespace cgtp
+
+using namespace cgtp;
+
+struct cgtp_plan_s {
+  int li, ls, lo, mult;
+  int n_paths;
+  int nnz;
+  std::vector<int> paths;
+};
+
+extern "C" {
+
+const char* cgtp_status_string(cgtp_status s) {
+  switch (s) {
+    case CGTP_OK: return "CGTP_OK";
+    case CGTP_ERR_INVALID_ARG: return "CGTP_ERR_INVALID_ARG";
+    case CGTP_ERR_UNSUPPORTED: return "CGTP_ERR_UNSUPPORTED";
+    case CGTP_ERR_BAD_GRAPH: return "CGTP_ERR_BAD_GRAPH";
+    case CGTP_ERR_OOM: return "CGTP_ERR_OOM";
+    case CGTP_ERR_CUDA: return "CGTP_ERR_CUDA";
+    case CGTP_ERR_TABLE: return "CGTP_ERR_TABLE";
+    case CGTP_ERR_WORKSPACE: return "CGTP_ERR_WORKSPACE";
+  }
+  return "CGTP_ERR_UNKNOWN";
+}
+
+int cgtp_last_cuda_error(void) { return g_last_cuda_error; }
+
+int cgtp_supported(int li, int ls, int lo) {
+  for (const Shape& s : kShapes)
+    if (s.li == li && s.ls == ls && s.lo == lo) return 1;
+  return 0;
+}
+
+cgtp_status cgtp_cg_block(int l1, int l2, int l3, double* out) {
+  if (out == nullptr || l1 < 0 || l2 < 0 || l3 < 0 || l1 > kLmaxTab || l2 > kLmaxTab || l3 > kLmaxTab)
+    return CGTP_ERR_INVALID_ARG;
+  double disc = 0.0;
+  real_cg_block(l1, l2, l3, out, &disc);
+  return disc > 1e-12 ? CGTP_ERR_TABLE : CGTP_OK;
+}
+
+cgtp_status cgtp_plan_create(int li, int ls, int lo, int mult, cgtp_plan* plan) {
+  if (plan == nullptr) return CGTP_ERR_INVALID_ARG;
+  *plan = nullptr;
+  if (li < 0 || ls < 0 || lo < 0 || mult <= 0 || mult % 4 != 0) return CGTP_ERR_INVALID_ARG;
+  if (!cgtp_supported(li, ls, lo)) return CGTP_ERR_UNSUPPORTED;
+  if (host_tables().status != 0) return CGTP_ERR_TABLE;
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  cgtp_plan_s* p = new (std::nothrow) cgtp_plan_s();
+  if (p == nullptr) return CGTP_ERR_OOM;
+  const PathData d = make_paths(li, ls, lo);
+  p->li = li;
+  p->ls = ls;
+  p->lo = lo;
+  p->mult = mult;
+  p->n_paths = d.np;
+  p->nnz = d.nnz;
+  for (int k = 0; k < d.np; ++k) {
+    p->paths.push_back(d.l1[k]);
+    p->paths.push_back(d.l2[k]);
+    p->paths.push_back(d.l3[k]);
+  }
+  *plan = p;
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_plan_destroy(cgtp_plan plan) {
+  delete plan;
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_plan_info(cgtp_plan plan, int* n_paths, int* paths, int* n_nonzero) {
+  if (plan == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (n_paths) *n_paths = plan->n_paths;
+  if (paths)
+    for (size_t k = 0; k < plan->paths.size(); ++k) paths[k] = plan->paths[k];
+  if (n_nonzero) *n_nonzero = plan->nnz;
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_graph_build(const float* pos, int n, float box_len, float rc, const int* graph_ptr,
+                             int n_graphs, int* row_ptr, int* col, float* edge_vec, int* csc_ptr,
+                             int* csc_edge, int* csc_dst, int max_edges, int* n_edges, void* stream) {
+  if (n < 0 || max_edges < 0 || !(rc > 0.f) || row_ptr == nullptr || csc_ptr == nullptr || n_edges == nullptr)
+    return CGTP_ERR_INVALID_ARG;
+  if (n > 0 && pos == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (max_edges > 0 && (col == nullptr || edge_vec == nullptr || csc_edge == nullptr || csc_dst == nullptr))
+    return CGTP_ERR_INVALID_ARG;
+  if (graph_ptr != nullptr && n_graphs < 1) return CGTP_ERR_INVALID_ARG;
+  if (box_len > 0.f && !((double)rc < 0.5 * (double)box_len)) return CGTP_ERR_INVALID_ARG;
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  cudaError_t e = launch_graph_build(pos, n, box_len, rc, graph_ptr, n_graphs, row_ptr, col, edge_vec, csc_ptr,
+                                     csc_edge, csc_dst, max_edges, n_edges, sms, (cudaStream_t)stream);
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
+cgtp_status cgtp_csr_transpose(int n, int n_edges, const int* row_ptr, const int* col, int* csc_ptr, int* csc_edge,
+                               int* csc_dst, void* workspace, size_t workspace_bytes, void* stream) {
+  if (n < 0 || n_edges < 0 || row_ptr == nullptr || csc_ptr == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (n_edges > 0 && (col == nullptr || csc_edge == nullptr || csc_dst == nullptr)) return CGTP_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < sizeof(int) * (size_t)(n > 0 ? n : 1)) return CGTP_ERR_WORKSPACE;
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  cudaError_t e = launch_csr_transpose(n, n_edges, row_ptr, col, csc_ptr, csc_edge, csc_dst, (int*)workspace, sms,
+                                       (cudaStream_t)stream);
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
+cgtp_status cgtp_graph_check(int n, int n_edges, const int* row_ptr, const int* col, const float* edge_vec,
+                             int* flags, void* stream) {
+  if (n < 0 || n_edges < 0 || row_ptr == nullptr || flags == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (n_edges > 0 && (col == nullptr || edge_vec == nullptr)) return CGTP_ERR_INVALID_ARG;
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  cudaError_t e = launch_graph_check(n, n_edges, row_ptr, col, edge_vec, flags, sms, (cudaStream_t)stream);
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
+cgtp_status cgtp_spherical_harmonics(int lmax_sh, int n_edges, const float* edge_vec, float* Y, float* dY,
+                                     void* stream) {
+  if (lmax_sh < 0 || lmax_sh > kLmaxTab || n_edges < 0) return CGTP_ERR_INVALID_ARG;
+  if (n_edges > 0 && (edge_vec == nullptr || (Y == nullptr && dY == nullptr))) return CGTP_ERR_INVALID_ARG;
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  cudaError_t e = launch_sh(lmax_sh, n_edges, edge_vec, Y, dY, sms, (cudaStream_t)stream);
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
+cgtp_status cgtp_conv_forward(cgtp_plan p, int n_nodes, int n_edges, const int* row_ptr, const int* col,
+                              const float* edge_vec, const float* x, const float* w, float* out, void* stream) {
+  if (p == nullptr || n_nodes < 0 || n_edges < 0 || row_ptr == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (n_nodes > 0 && (x == nullptr || out == nullptr)) return CGTP_ERR_INVALID_ARG;
+  if (n_edges > 0 && (col == nullptr || edge_vec == nullptr || w == nullptr)) return CGTP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(out)) return CGTP_ERR_INVALID_ARG;
+  if (n_nodes == 0) return CGTP_OK;
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  ConvFwdArgs a{n_nodes, row_ptr, col, edge_vec, x, w, out, p->mult};
+  cudaError_t e = cudaErrorNotSupported;
+#define CGTP_FWD_ENTRY(A, B, C) \
+  if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_fwd<A, B, C>(a, sms, (cudaStream_t)stream);
+  CGTP_CONFIGS(CGTP_FWD_ENTRY)
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
+static int bwd_slices(cgtp_plan p) {
+  int s = 0;
+#define CGTP_SLICES_ENTRY(A, B, C) \
+  if (p->li == A && p->ls == B && p->lo == C) s = conv_bwd_slices<A, B, C>(p->mult);
+  CGTP_CONFIGS(CGTP_SLICES_ENTRY)
+  return s;
+}
+
+cgtp_status cgtp_conv_backward_workspace_size(cgtp_plan p, int n_edges, size_t* bytes) {
+  if (p == nullptr || n_edges < 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
+  const size_t ns = (size_t)(p->ls + 1) * (p->ls + 1);
+  const size_t b = sizeof(float) * (size_t)bwd_slices(p) * (size_t)n_edges * ns;
+  *bytes = (b + 255) & ~(size_t)255;
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_conv_backward(cgtp_plan p, int n_nodes, int n_edges, const int* csc_ptr, const int* csc_edge,
+                               const int* csc_dst, const float* edge_vec, const float* x, const float* w,
+                               const float* grad_out, float* grad_x, float* grad_w, float* grad_edge_vec,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  if (p == nullptr || n_nodes < 0 || n_edges < 0 || csc_ptr == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (n_nodes > 0 && (x == nullptr || grad_out == nullptr)) return CGTP_ERR_INVALID_ARG;
+  if (n_edges > 0 && (csc_edge == nullptr || csc_dst == nullptr || edge_vec == nullptr || w == nullptr))
+    return CGTP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(grad_out) || !aligned16(grad_x) || !aligned16(grad_w))
+    return CGTP_ERR_INVALID_ARG;
+  if (grad_edge_vec != nullptr && n_edges > 0) {
+    size_t need = 0;
+    cgtp_conv_backward_workspace_size(p, n_edges, &need);
+    if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
+      return CGTP_ERR_WORKSPACE;
+  }
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (n_nodes == 0) return CGTP_OK;
+  if (n_edges == 0) {  // no edges: every gradient is zero
+    cudaError_t e = cudaSuccess;
+    if (grad_x) e = cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)n_nodes * (p->li + 1) * (p->li + 1) * p->mult, s);
+    return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+  }
+  ConvBwdArgs a{n_nodes, n_edges, csc_ptr, csc_edge, csc_dst, edge_vec, x, w, grad_out,
+                grad_x, grad_w, grad_edge_vec, (float*)workspace, p->mult};
+  cudaError_t e = cudaErrorNotSupported;
+#define CGTP_BWD_ENTRY(A, B, C) \
+  if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_bwd<A, B, C>(a, sms, s);
+  CGTP_CONFIGS(CGTP_BWD_ENTRY)
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
+cgtp_status cgtp_forces(int n_nodes, int n_edges, const int* row_ptr, const int* csc_ptr, const int* csc_edge,
+                        const float* grad_edge_vec, float* forces, void* stream) {
+  if (n_nodes < 0 || n_edges < 0 || row_ptr == nullptr || csc_ptr == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (n_nodes > 0 && forces == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (n_edges > 0 && (csc_edge == nullptr || grad_edge_vec == nullptr)) return CGTP_ERR_INVALID_ARG;
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  cudaError_t e = launch_forces(n_nodes, row_ptr, csc_ptr, csc_edge, grad_edge_vec, forces, sms, (cudaStream_t)stream);
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
+cgtp_status cgtp_radial_forward(cgtp_plan p, int n_edges, const float* edge_vec, float rc, const float* W1,
+                                const float* W2, float* w, void* stream) {
+  if (p == nullptr || n_edges < 0 || !(rc > 0.f)) return CGTP_ERR_INVALID_ARG;
+  if (n_edges > 0 && (edge_vec == nullptr || W1 == nullptr || W2 == nullptr || w == nullptr))
+    return CGTP_ERR_INVALID_ARG;
+  if (!aligned16(W2) || !aligned16(w)) return CGTP_ERR_INVALID_ARG;
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  cudaError_t e = launch_radial_fwd(n_edges, p->n_paths * p->mult, edge_vec, rc, W1, W2, w, (cudaStream_t)stream);
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
+cgtp_status cgtp_radial_backward(cgtp_plan p, int n_edges, const float* edge_vec, float rc, const float* W1,
+                                 const float* W2, const float* grad_w, float* grad_edge_vec, void* stream) {
+  if (p == nullptr || n_edges < 0 || !(rc > 0.f)) return CGTP_ERR_INVALID_ARG;
+  if (n_edges > 0 && (edge_vec == nullptr || W1 == nullptr || W2 == nullptr || grad_w == nullptr ||
+                      grad_edge_vec == nullptr))
+    return CGTP_ERR_INVALID_ARG;
+  if (!aligned16(W2) || !aligned16(grad_w)) return CGTP_ERR_INVALID_ARG;
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  cudaError_t e = launch_radial_bwd(n_edges, p->n_paths * p->mult, edge_vec, rc, W1, W2, grad_w, grad_edge_vec,
+                                    (cudaStream_t)stream);
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
+cgtp_status cgtp_tp_forward(cgtp_plan p, int batch, const float* x, const float* y, const float* w, float* z,
+                            void* stream) {
+  if (p == nullptr || batch < 0) return CGTP_ERR_INVALID_ARG;
+  if (batch > 0 && (x == nullptr || y == nullptr || w == nullptr || z == nullptr)) return CGTP_ERR_INVALID_ARG;
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  TPArgs a{batch, x, y, w, nullptr, z, nullptr, nullptr, nullptr, nullptr, p->mult};
+  cudaError_t e = cudaErrorNotSupported;
+#define CGTP_TPF_ENTRY(A, B, C) \
+  if (p->li == A && p->ls == B && p->lo == C) e = launch_tp_fwd<A, B, C>(a, sms, (cudaStream_t)stream);
+  CGTP_CONFIGS(CGTP_TPF_ENTRY)
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
+cgtp_status cgtp_tp_backward_workspace_size(cgtp_plan p, int batch, size_t* bytes) {
+  if (p == nullptr || batch < 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
+  const size_t b = sizeof(float) * (size_t)tp_chunks(batch) * p->n_paths * p->mult;
+  *bytes = (b + 255) & ~(size_t)255;
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_tp_backward(cgtp_plan p, int batch, const float* x, const float* y, const float* w,
+                             const float* grad_z, float* grad_x, float* grad_y, float* grad_w, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  if (p == nullptr || batch < 0) return CGTP_ERR_INVALID_ARG;
+  if (batch > 0 && (x == nullptr || y == nullptr || w == nullptr || grad_z == nullptr)) return CGTP_ERR_INVALID_ARG;
+  if (grad_w != nullptr) {
+    size_t need = 0;
+    cgtp_tp_backward_workspace_size(p, batch, &need);
+    if (workspace == nullptr || workspace_bytes < need) return CGTP_ERR_WORKSPACE;
+  }
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  TPArgs a{batch, x, y, w, grad_z, nullptr, grad_x, grad_y, grad_w, grad_w ? (float*)workspace : nullptr, p->mult};
+  cudaError_t e = cudaErrorNotSupported;
+#define CGTP_TPB_ENTRY(A, B, C) \
+  if (p->li == A && p->ls == B && p->lo == C) e = launch_tp_bwd<A, B, C>(a, sms, (cudaStream_t)stream);
+  CGTP_CONFIGS(CGTP_TPB_ENTRY)
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,112 @@
+// Device-side helpers shared by the kernels: compile-time loops, the
+// constant-memory coefficient tables, cache-hinted vector loads and the
+// launch-argument structs.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <type_traits>
+#include <utility>
+
+#include "structure.h"
+
+namespace cgtp {
+
+// ---- compile-time loop: f(std::integral_constant<int, I>) for I in [B, E) ----
+template <int B, class F, int... Is>
+__device__ __forceinline__ void static_for_impl(F&& f, std::integer_sequence<int, Is...>) {
+  (f(std::integral_constant<int, B + Is>{}), ...);
+}
+template <int B, int E, class F>
+__device__ __forceinline__ void static_for(F&& f) {
+  if constexpr (E > B) static_for_impl<B>(f, std::make_integer_sequence<int, E - B>{});
+}
+
+// ---- coefficient tables.  Every translation unit that needs them holds its
+// own constant-memory copy and registers an uploader at load time; plan
+// creation runs every registered uploader once per device. ----
+using UploadFn = cudaError_t (*)(const float* cg, const float* shk);
+int register_table_uploader(UploadFn fn);  // host, defined in abi.cu
+
+#define CGTP_DEFINE_CONSTANT_TABLES()                                              \
+  static __constant__ float c_cg[kTableSize];                                      \
+  static __constant__ float c_shk[kShkSize];                                       \
+  static cudaError_t upload_tables_here(const float* cg, const float* shk) {       \
+    cudaError_t e = cudaMemcpyToSymbol(c_cg, cg, sizeof(float) * kTableSize);      \
+    if (e != cudaSuccess) return e;                                                \
+    return cudaMemcpyToSymbol(c_shk, shk, sizeof(float) * kShkSize);               \
+  }                                                                                \
+  static const int tables_registered_here = register_table_uploader(&upload_tables_here);
+
+// ---- loads / stores with cache hints ----
+__device__ __forceinline__ float4 ld_stream(const float* p) {  // read once: evict first
+  return __ldcs(reinterpret_cast<const float4*>(p));
+}
+__device__ __forceinline__ float4 ld_ro(const float* p) {  // read-only, reused: cached
+  return __ldg(reinterpret_cast<const float4*>(p));
+}
+__device__ __forceinline__ void st_stream(float* p, float4 v) {
+  __stcs(reinterpret_cast<float4*>(p), v);
+}
+__device__ __forceinline__ void st_f4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+
+__device__ __forceinline__ void f4_to(float (&a)[4], float4 v) {
+  a[0] = v.x; a[1] = v.y; a[2] = v.z; a[3] = v.w;
+}
+__device__ __forceinline__ float4 to_f4(const float (&a)[4]) { return make_float4(a[0], a[1], a[2], a[3]); }
+
+// ---- launch arguments ----
+struct ConvFwdArgs {
+  int n_nodes;
+  const int* row_ptr;
+  const int* col;
+  const float* edge_vec;
+  const float* x;
+  const float* w;
+  float* out;
+  int mult;
+};
+
+struct ConvBwdArgs {
+  int n_nodes;
+  int n_edges;
+  const int* csc_ptr;
+  const int* csc_edge;
+  const int* csc_dst;
+  const float* edge_vec;
+  const float* x;
+  const float* w;
+  const float* grad_out;
+  float* grad_x;
+  float* grad_w;
+  float* grad_edge_vec;
+  float* grad_sh;   // workspace [slices][n_edges][NS]
+  int mult;
+};
+
+struct TPArgs {
+  int batch;
+  const float* x;
+  const float* y;
+  const float* w;
+  const float* grad_z;  // bwd
+  float* z;             // fwd
+  float* grad_x;
+  float* grad_y;
+  float* grad_w;
+  float* partial;       // workspace [chunks][P][mult]
+  int mult;
+};
+
+// Edge-free tensor product: batch rows per block and the number of batch
+// chunks whose grad_w partials the backward keeps in its workspace.
+constexpr int kTpRows = 8;
+constexpr int kTpChunksMax = 64;
+inline int tp_chunks(int batch) {
+  int ch = (batch + kTpRows - 1) / kTpRows;
+  if (ch > kTpChunksMax) ch = kTpChunksMax;
+  return ch < 1 ? 1 : ch;
+}
+
+}  // namespace cgtp

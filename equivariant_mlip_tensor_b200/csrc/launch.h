@@ -1,0 +1,39 @@
+// Host-side launchers of every kernel family (defined in the .cu files; the
+// per-shape ones are instantiated once per entry of configs.h).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace cgtp {
+
+template <int LI, int LS, int LO>
+cudaError_t launch_conv_fwd(const ConvFwdArgs& a, int num_sms, cudaStream_t stream);
+template <int LI, int LS, int LO>
+cudaError_t launch_conv_bwd(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);
+template <int LI, int LS, int LO>
+int conv_bwd_slices(int mult);
+template <int LI, int LS, int LO>
+cudaError_t launch_tp_fwd(const TPArgs& a, int num_sms, cudaStream_t stream);
+template <int LI, int LS, int LO>
+cudaError_t launch_tp_bwd(const TPArgs& a, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_graph_build(const float* pos, int n, float box_len, float rc, const int* graph_ptr,
+                               int n_graphs, int* row_ptr, int* col, float* edge_vec, int* csc_ptr,
+                               int* csc_edge, int* csc_dst, int max_edges, int* n_edges, int num_sms,
+                               cudaStream_t stream);
+cudaError_t launch_csr_transpose(int n, int n_edges, const int* row_ptr, const int* col, int* csc_ptr,
+                                 int* csc_edge, int* csc_dst, int* ws, int num_sms, cudaStream_t stream);
+cudaError_t launch_graph_check(int n, int n_edges, const int* row_ptr, const int* col, const float* edge_vec,
+                               int* flags, int num_sms, cudaStream_t stream);
+cudaError_t launch_radial_fwd(int n_edges, int N, const float* ev, float rc, const float* W1, const float* W2,
+                              float* w, cudaStream_t stream);
+cudaError_t launch_radial_bwd(int n_edges, int N, const float* ev, float rc, const float* W1, const float* W2,
+                              const float* gw, float* gev, cudaStream_t stream);
+cudaError_t launch_forces(int n, const int* row_ptr, const int* csc_ptr, const int* csc_edge, const float* g,
+                          float* F, int num_sms, cudaStream_t stream);
+cudaError_t launch_sh(int lmax_sh, int n_edges, const float* ev, float* Y, float* dY, int num_sms,
+                      cudaStream_t stream);
+
+}  // namespace cgtp

@@ -1,0 +1,224 @@
+/*
+ * cgtp.h -- C ABI of the B200 (sm_100a) Clebsch-Gordan tensor-product
+ * convolution library (libcgtp.so).
+ *
+ * The operation ("LunaTP: Enabling Efficient and Scalable Tensor Product for
+ * Equivariant MLIPs", abstract: node-centric CGTP convolutions and their
+ * derivatives; selection rules from "Tensor Decomposition Networks for
+ * Accelerating Machine Learning Force Field Computations", reply to reviewer
+ * S6y1).  For every directed edge e = (j -> i) with edge vector
+ * r_e = pos_j - pos_i, real spherical harmonics Y_e = Y(r_e / |r_e|) and
+ * weights W_e[p][u]:
+ *
+ *   out[i][l3,m3][u] = sum_{e in row i} sum_{p=(l1,l2,l3)} W_e[p][u]
+ *                      sum_{m1,m2} C^p[m1,m2,m3] x[j][l1,m1][u] Y_e[l2,m2]
+ *
+ * over every path with l1 <= lmax_in, l2 <= lmax_sh and
+ * |l1-l2| <= l3 <= min(l1+l2, lmax_out).  Paths are numbered in
+ * lexicographic (l1, l2, l3) order.
+ *
+ * Conventions shared by every entry point
+ *  - Layouts: irreps features are [node][l*l + m + l][u] with the channel u
+ *    fastest (fp32); weights are [edge][path][u] (fp32); edge vectors are
+ *    [edge][3] (fp32); the real basis orders the l = 1 block as (y, z, x);
+ *    harmonics use component normalisation (sum_m Y_lm^2 = 2l + 1,
+ *    Y_00 = 1); CG coefficients are the unitary real-basis ones.
+ *  - Graphs: CSR by destination (row_ptr [N+1], col [E] = source of each
+ *    edge, rows ascending, sources ascending within a row).  The CSC view by
+ *    source (csc_ptr [N+1], csc_edge [E] = CSR edge number, csc_dst [E] =
+ *    destination) lists each source's edges in ascending destination order.
+ *    All indices are int32.
+ *  - Pointers: "device" arguments are caller-owned device memory; the
+ *    library never frees or retains them.  Feature, weight and output arrays
+ *    must be 16-byte aligned (they are read and written as float4).
+ *  - Streams: every call is asynchronous on the given cudaStream_t (passed
+ *    as void*, NULL = legacy default stream); nothing synchronises unless
+ *    stated.
+ *  - Errors: every call returns a cgtp_status.  Invalid arguments are found
+ *    on the host before any launch (CGTP_ERR_INVALID_ARG /
+ *    CGTP_ERR_UNSUPPORTED) and nothing is launched.  A launch failure
+ *    returns CGTP_ERR_CUDA; cgtp_last_cuda_error() gives the CUDA code.
+ *    Nothing aborts, throws or exits across this boundary.
+ *  - Zero-length edges (coincident atoms) have no direction: their
+ *    harmonics are Y_00 = 1 and 0 for l > 0, with a zero derivative.
+ */
+#ifndef CGTP_H
+#define CGTP_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CGTP_OK = 0,
+  CGTP_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, negative size, ...  */
+  CGTP_ERR_UNSUPPORTED = 2,  /* (lmax_in, lmax_sh, lmax_out, mult) not built  */
+  CGTP_ERR_BAD_GRAPH = 3,    /* reported by cgtp_graph_check                   */
+  CGTP_ERR_OOM = 4,          /* host allocation failed                          */
+  CGTP_ERR_CUDA = 5,         /* a CUDA runtime call or launch failed            */
+  CGTP_ERR_TABLE = 6,        /* CG table construction failed its own checks    */
+  CGTP_ERR_WORKSPACE = 7     /* workspace missing or smaller than required      */
+} cgtp_status;
+
+typedef struct cgtp_plan_s* cgtp_plan;
+
+/* Human-readable name of a status code (static string). */
+const char* cgtp_status_string(cgtp_status s);
+
+/* CUDA error code (cudaError_t as int) of the last CGTP_ERR_CUDA on this
+ * host thread, 0 if none. */
+int cgtp_last_cuda_error(void);
+
+/* ---------------------------------------------------------------------------
+ * Plan: the path list and the real CG coefficients for one irreps shape.
+ * ("Tensor Decomposition Networks ...", reply to S6y1: only triples obeying
+ * |l1-l2| <= l3 <= l1+l2 and m3 = m1+m2 are nonzero.)
+ * Builds the coefficients on the host (fp64, by the angular-momentum
+ * lowering operator and the complex-to-real change of basis), checks them,
+ * and uploads them once per device to constant memory (synchronous copy on
+ * the current device).  mult must be a positive multiple of 4.
+ * Supported (lmax_in, lmax_sh, lmax_out): see cgtp_supported().
+ * Returns CGTP_ERR_UNSUPPORTED for shapes that are not compiled in.
+ * ------------------------------------------------------------------------- */
+cgtp_status cgtp_plan_create(int lmax_in, int lmax_sh, int lmax_out, int mult, cgtp_plan* plan);
+cgtp_status cgtp_plan_destroy(cgtp_plan plan);
+
+/* 1 if kernels for this (lmax_in, lmax_sh, lmax_out) are compiled in. */
+int cgtp_supported(int lmax_in, int lmax_sh, int lmax_out);
+
+/* Number of paths; if paths_l1l2l3 is not NULL it receives 3*n_paths ints
+ * (l1, l2, l3 per path, lexicographic).  n_cg_nonzero (nullable) receives
+ * the number of nonzero real CG entries over all paths.  Host only. */
+cgtp_status cgtp_plan_info(cgtp_plan plan, int* n_paths, int* paths_l1l2l3, int* n_cg_nonzero);
+
+/* Host-only: the dense real-basis CG block of path (l1, l2, l3), all <= 4,
+ * as (2l1+1)*(2l2+1)*(2l3+1) doubles in [m1][m2][m3] order, computed by the
+ * same generator that feeds the kernels.  Needs no GPU. */
+cgtp_status cgtp_cg_block(int l1, int l2, int l3, double* out);
+
+/* ---------------------------------------------------------------------------
+ * Neighbour list (CSR by destination + CSC by source), brute force over the
+ * candidate pairs of each graph, bit-exact contract:
+ *   d = p_j - p_i per axis in fp64 (positions upcast from fp32);
+ *   periodic box (side box_len > 0): d <- d - L*rint(d/L), each operation
+ *   rounded separately (rint: halves to even); box_len <= 0 means no box;
+ *   edge when ((dx*dx + dy*dy) + dz*dz) < rc*rc in fp64 without fused
+ *   multiply-add, rc*rc formed in fp64 from the fp32 cutoff, i != j;
+ *   edge_vec = (float)d.
+ * pos: device [n][3].  graph_ptr: device [n_graphs+1] start offsets of
+ * contiguous graphs (pairs only within a graph), or NULL for one graph.
+ * Outputs (device): row_ptr [n+1], col [max_edges], edge_vec [max_edges][3],
+ * csc_ptr [n+1], csc_edge [max_edges], csc_dst [max_edges], n_edges [1].
+ * If the true edge count exceeds max_edges, *n_edges holds the true count,
+ * row_ptr is complete, and only the edges below max_edges are written (the
+ * caller must check *n_edges and rebuild with more room).  The CSC arrays
+ * use the symmetry of the predicate (j in N(i) iff i in N(j)).
+ * Requires rc < box_len/2 with a box.  No host synchronisation.
+ * ------------------------------------------------------------------------- */
+cgtp_status cgtp_graph_build(const float* pos, int n, float box_len, float rc,
+                             const int* graph_ptr, int n_graphs,
+                             int* row_ptr, int* col, float* edge_vec,
+                             int* csc_ptr, int* csc_edge, int* csc_dst,
+                             int max_edges, int* n_edges, void* stream);
+
+/* CSC view of an arbitrary CSR graph (no symmetry assumed).
+ * workspace: device, at least n*sizeof(int) bytes (zeroed by the call). */
+cgtp_status cgtp_csr_transpose(int n, int n_edges, const int* row_ptr, const int* col,
+                               int* csc_ptr, int* csc_edge, int* csc_dst,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* Device-side validation of a CSR graph: sets bits of *flags (device int,
+ * cleared by the call): 1 = row_ptr not monotone or row_ptr[0] != 0 or
+ * row_ptr[n] != n_edges, 2 = col out of range, 4 = zero-length edge vector,
+ * 8 = non-finite edge vector. */
+cgtp_status cgtp_graph_check(int n, int n_edges, const int* row_ptr, const int* col,
+                             const float* edge_vec, int* flags, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Real spherical harmonics of edge directions (materialised; the
+ * convolution kernels compute them in registers).  Y: device
+ * [n_edges][(lmax_sh+1)^2]; dY (nullable): device [n_edges][(lmax_sh+1)^2][3]
+ * = dY/d(edge_vec).  lmax_sh <= 4.
+ * ------------------------------------------------------------------------- */
+cgtp_status cgtp_spherical_harmonics(int lmax_sh, int n_edges, const float* edge_vec,
+                                     float* Y, float* dY, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Convolution forward (node-centric: one owner per destination row, no
+ * atomics).  x: [n_nodes][(lmax_in+1)^2][mult]; w: [n_edges][n_paths][mult];
+ * out: [n_nodes][(lmax_out+1)^2][mult] (overwritten).
+ * ------------------------------------------------------------------------- */
+cgtp_status cgtp_conv_forward(cgtp_plan plan, int n_nodes, int n_edges,
+                              const int* row_ptr, const int* col, const float* edge_vec,
+                              const float* x, const float* w, float* out, void* stream);
+
+/* Bytes of device workspace cgtp_conv_backward needs when grad_edge_vec is
+ * requested (0 otherwise is also accepted). */
+cgtp_status cgtp_conv_backward_workspace_size(cgtp_plan plan, int n_edges, size_t* bytes);
+
+/* ---------------------------------------------------------------------------
+ * Convolution backward, node-centric over sources (CSC), one read of W:
+ *   grad_x[j] = sum_{e: src=j} sum_p W_e[p] (T_e^p)^T grad_out[dst(e)]
+ *   grad_w[e][p][u] = sum C x[j] Y_e grad_out[i]
+ *   grad_edge_vec[e] = (dY_e/dr_e)^T sum_u sum_p W x grad_out C
+ * with T_e^p[m1][m3] = sum_m2 C^p[m1,m2,m3] Y_e[l2,m2].
+ * grad_x, grad_w, grad_edge_vec are nullable (not computed when NULL) and
+ * overwritten.  grad_edge_vec needs workspace of the size reported by
+ * cgtp_conv_backward_workspace_size (device, 256-byte aligned).
+ * ------------------------------------------------------------------------- */
+cgtp_status cgtp_conv_backward(cgtp_plan plan, int n_nodes, int n_edges,
+                               const int* csc_ptr, const int* csc_edge, const int* csc_dst,
+                               const float* edge_vec, const float* x, const float* w,
+                               const float* grad_out, float* grad_x, float* grad_w,
+                               float* grad_edge_vec, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Per-atom forces from edge-vector gradients, F = -dE/dpos with
+ * r_e = pos_src - pos_dst:  F[n] = sum_{e: dst=n} g[e] - sum_{e: src=n} g[e].
+ * Segmented sums over the CSR row and the CSC row of each node; no atomics.
+ * forces: device [n_nodes][3], overwritten.
+ * ------------------------------------------------------------------------- */
+cgtp_status cgtp_forces(int n_nodes, int n_edges, const int* row_ptr, const int* csc_ptr,
+                        const int* csc_edge, const float* grad_edge_vec, float* forces,
+                        void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Radial weight network: 8 Gaussians on [0, rc] (centres k*rc/7, width
+ * rc/7) -> a = phi @ W1 [8][64] -> SiLU -> w = h @ W2 [64][n_paths*mult],
+ * no biases.  w: [n_edges][n_paths][mult], overwritten.
+ * ------------------------------------------------------------------------- */
+cgtp_status cgtp_radial_forward(cgtp_plan plan, int n_edges, const float* edge_vec, float rc,
+                                const float* W1, const float* W2, float* w, void* stream);
+
+/* dL/d edge_vec through the radial weights, ADDED to grad_edge_vec:
+ * grad_edge_vec[e] += (sum_k (grad_w W2^T)_k SiLU'(a_k) (W1 dphi/dr)_k) r_e/|r_e|. */
+cgtp_status cgtp_radial_backward(cgtp_plan plan, int n_edges, const float* edge_vec, float rc,
+                                 const float* W1, const float* W2, const float* grad_w,
+                                 float* grad_edge_vec, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Edge-free channelwise tensor product of batched pairs ("Tensor
+ * Decomposition Networks ...", reply to S6y1: the exact CG product, timed at
+ * batch 1000 and multiplicity 128):
+ *   z[b][l3,m3][u] = sum_p w[p][u] sum C^p[m1,m2,m3] x[b][l1,m1][u] y[b][l2,m2][u]
+ * x: [batch][(lmax_in+1)^2][mult], y: [batch][(lmax_sh+1)^2][mult],
+ * w: [n_paths][mult], z: [batch][(lmax_out+1)^2][mult] (overwritten).
+ * ------------------------------------------------------------------------- */
+cgtp_status cgtp_tp_forward(cgtp_plan plan, int batch, const float* x, const float* y,
+                            const float* w, float* z, void* stream);
+
+cgtp_status cgtp_tp_backward_workspace_size(cgtp_plan plan, int batch, size_t* bytes);
+
+/* grad_x, grad_y, grad_w nullable, overwritten; grad_w (the sum over the
+ * batch) needs the workspace reported by cgtp_tp_backward_workspace_size. */
+cgtp_status cgtp_tp_backward(cgtp_plan plan, int batch, const float* x, const float* y,
+                             const float* w, const float* grad_z, float* grad_x, float* grad_y,
+                             float* grad_w, void* workspace, size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CGTP_H */
