@@ -1,0 +1,461 @@
+"""Benchmark: CGTP convolution edges/s (forward + backward) on the molecular
+batch workload (256 graphs x 30 atoms, L_in = L_out = 2, harmonics l <= 4,
+mult 128), one B200 per rank.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {cgtp,reference}]
+
+A timed step is one pass of the convolution over the resident batch:
+harmonics + forward (one kernel), backward over sources (grad_x, grad_W and
+the per-edge harmonic gradient), the harmonic Jacobian (grad_edge_vec) and
+the per-atom forces.  The neighbour list and the radial weight network run
+in a second timed loop ("pipeline": positions -> graph -> weights -> forward
+-> backward -> radial backward -> forces) reported beside the headline.
+Every rank processes its own batch (weak scaling, no collective on the data
+path); timing uses CUDA events on the launching stream, between a barrier
+and a device synchronisation, and the slowest rank's time.
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload on this host's cores (rank 0 only).
+"""
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from equivariant_mlip_tensor_b200 import synthetic  # noqa: E402
+
+METRIC = "CGTP conv edges/s (fwd+bwd) at L=2, mult=128; % of HBM roofline"
+UNIT = "edges/s"
+WORKLOAD = ("molecules: 256 graphs x 30 atoms uniform in an 8 A cube (0.9 A rejection), cutoff 5 A, "
+            "one CSR over the batch; x 128x(l=0..2), harmonics l<=4, outputs l<=2, 19 paths, "
+            "weights from the radial network; energy = sum of l=0 outputs")
+
+
+def _load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs", 6650.0), "measured"
+    return 6650.0, "fallback"
+
+
+def _cores():
+    return len(os.sched_getaffinity(0))
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling (every 200 ms) during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            self.f = os.fdopen(fd, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": float(max(smax)) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- algorithmic bytes
+def conv_bytes(n, E, P, u, ni, ns, no, slices):
+    """Algorithmic bytes of one forward and one backward launch (fp32/int32)."""
+    fwd = 4 * (E * P * u + n * ni * u + n * no * u + 3 * E + E + (n + 1))
+    bwd = 4 * (2 * E * P * u + 2 * n * ni * u + n * no * u + 3 * E + 2 * E + (n + 1)
+               + slices * E * ns)
+    return fwd, bwd
+
+
+def structural_counts(li, ls, lo):
+    """(T entries, CG entries, sum of 2l3+1) over the paths, from the real-basis
+    selection rules (|m3| in {|m1|+|m2|, ||m1|-|m2||}, parity of the negative m's)."""
+    def ok(l1, l2, l3, a, b, c):
+        if abs(c) not in (abs(a) + abs(b), abs(abs(a) - abs(b))):
+            return False
+        return ((a < 0) + (b < 0) + (c < 0)) % 2 == (l1 + l2 + l3) % 2
+    nT = nnz = osum = 0
+    for l1 in range(li + 1):
+        for l2 in range(ls + 1):
+            for l3 in range(abs(l1 - l2), min(l1 + l2, lo) + 1):
+                osum += 2 * l3 + 1
+                for a in range(-l1, l1 + 1):
+                    for c in range(-l3, l3 + 1):
+                        k = sum(ok(l1, l2, l3, a, b, c) for b in range(-l2, l2 + 1))
+                        nnz += k
+                        nT += k > 0
+    return nT, nnz, osum
+
+
+def conv_flops(E, u, nT, nnz, no_sum, P):
+    """Algorithmic FLOPs (FMA = 2) with the per-edge T factorisation:
+    forward sum_p(|T^p| + (2l3+1)) per channel-edge; backward t, grad_W, s,
+    grad_x and the channel dot products (4 |T| + 2 sum(2l3+1)) per
+    channel-edge plus nnz per lane."""
+    fwd = 2 * E * u * (nT + no_sum)
+    bwd = 2 * E * u * (3 * nT + 2 * no_sum) + 2 * E * nnz * (u // 4)
+    return fwd, bwd
+
+
+# ---------------------------------------------------------------- reference arm / CPU baseline
+def oracle_step(w, n_graphs_sample, threads):
+    """The oracle's fwd + bwd + forces over the first n_graphs_sample graphs."""
+    from oracle import conv as oconv
+    from oracle import graph as ograph
+    from oracle import radial as oradial
+    n = n_graphs_sample * w.graph_size
+    pos, gid = w.pos[:n], w.graph_id[:n]
+    L = (w.lmax_in, w.lmax_sh, w.lmax_out)
+    o = ograph.neighbour_list(pos, w.rc, None, gid)
+    Wo = oradial.radial_forward(o["edge_vec"], w.W1, w.W2, w.rc, w.n_paths, w.mult)
+    chunk = max(256, -(-o["col"].size // threads))
+    t0 = time.perf_counter()
+    oconv.conv_forward(o["row_ptr"], o["col"], o["edge_vec"], w.x[:n], Wo, *L, threads=threads, chunk=chunk)
+    _, _, gr = oconv.conv_backward(o["row_ptr"], o["col"], o["edge_vec"], w.x[:n], Wo, w.grad_out[:n], *L,
+                                   threads=threads, chunk=chunk)
+    oconv.edge_forces(o["row_ptr"], o["col"], gr, n)
+    dt = time.perf_counter() - t0
+    return o["col"].size, dt
+
+
+def cpu_baseline(w, budget_s=15.0):
+    threads = _cores()
+    E1, dt1 = oracle_step(w, 2, threads)
+    rate = E1 / dt1
+    n_g = int(max(2, min(w.pos.shape[0] // w.graph_size, budget_s * rate / (E1 / 2))))
+    E, dt = oracle_step(w, n_g, threads)
+    return {"value": E / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"first {n_g} of 256 molecules ({E} edges): fp64 NumPy forward + backward + forces, "
+                      f"{threads} threads over edge chunks, {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = synthetic.molecules()
+    threads = _cores()
+    n_g = 4
+    times, edges = [], 0
+    for _ in range(args.warmup):
+        oracle_step(w, n_g, threads)
+    for _ in range(args.steps):
+        E, dt = oracle_step(w, n_g, threads)
+        times.append(dt)
+        edges = E
+    ms = 1e3 * float(np.mean(times))
+    value = edges / (ms / 1e3)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)", "impl": "reference",
+            "config": {"workload": WORKLOAD, "sample": f"first {n_g} molecules per step ({edges} edges)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"first {n_g} of 256 molecules per step ({edges} edges)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    from equivariant_mlip_tensor_b200 import api
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+
+    w = synthetic.molecules(seed=4 + 1000 * rank)
+    L = (w.lmax_in, w.lmax_sh, w.lmax_out)
+    n, u = w.n_nodes, w.mult
+    ni, ns, no = (L[0] + 1) ** 2, (L[1] + 1) ** 2, (L[2] + 1) ** 2
+    stream = torch.cuda.current_stream()
+
+    # resident inputs
+    pos = torch.from_numpy(w.pos).to(dev)
+    gp = torch.from_numpy(np.arange(0, n + 1, w.graph_size, dtype=np.int32)).to(dev)
+    x = torch.from_numpy(w.x).to(dev)
+    go = torch.from_numpy(w.grad_out).to(dev)
+    W1 = torch.from_numpy(w.W1).to(dev)
+    W2 = torch.from_numpy(w.W2).to(dev)
+    plan = api.Plan(*L, u)
+    g = api.build_graph(pos, w.rc, graph_ptr=gp, max_edges=int(1.25 * 13 * n))
+    E, P = g.n_edges, plan.n_paths
+    W = plan.radial_forward(g.edge_vec, w.rc, W1, W2)
+    out = torch.empty((n, no, u), dtype=torch.float32, device=dev)
+    gx = torch.empty((n, ni, u), dtype=torch.float32, device=dev)
+    gw = torch.empty((E, P, u), dtype=torch.float32, device=dev)
+    gr = torch.empty((E, 3), dtype=torch.float32, device=dev)
+    F = torch.empty((n, 3), dtype=torch.float32, device=dev)
+    ws_bytes = plan.conv_backward_workspace_bytes(E)
+    ws = torch.empty(ws_bytes // 4 + 64, dtype=torch.float32, device=dev)
+
+    def conv_step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        plan.conv_forward(g, x, W, out=out)
+        if ev is not None:
+            ev[1].record(stream)
+        plan.conv_backward(g, x, W, go, grad_x=gx, grad_w=gw, grad_edge_vec=gr, workspace=ws)
+        if ev is not None:
+            ev[2].record(stream)
+        api.forces(g, gr, out=F)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        conv_step()
+    torch.cuda.synchronize()
+
+    # per-kernel breakdown (separate loop, events between launches)
+    nb = min(args.steps, 200)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nb)]
+    barrier()
+    torch.cuda.synchronize()
+    for k in range(nb):
+        conv_step(evs[k])
+    torch.cuda.synchronize()
+    t_fwd = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    t_bwd = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    t_frc = float(np.mean([e[2].elapsed_time(e[3]) for e in evs]))
+
+    # headline timed region: exactly K steps between barrier + synchronize
+    clocks = ClockSampler(local)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    e0.record(stream)
+    for _ in range(args.steps):
+        conv_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    t_local = e0.elapsed_time(e1) / 1e3
+    t = max_over_ranks(t_local)
+    edges_all = sum_over_ranks(float(E))
+    value = edges_all * args.steps / t
+    ms_step = 1e3 * t / args.steps
+
+    # pipeline: positions -> graph -> radial weights -> conv -> radial backward -> forces
+    ne_dev = torch.empty(1, dtype=torch.int32, device=dev)
+    cap = g.col.numel() if g.col.numel() >= E else E
+    bufs = dict(row_ptr=torch.empty(n + 1, dtype=torch.int32, device=dev),
+                col=torch.empty(cap, dtype=torch.int32, device=dev),
+                ev=torch.empty((cap, 3), dtype=torch.float32, device=dev),
+                csc_ptr=torch.empty(n + 1, dtype=torch.int32, device=dev),
+                ce=torch.empty(cap, dtype=torch.int32, device=dev),
+                cd=torch.empty(cap, dtype=torch.int32, device=dev))
+    from equivariant_mlip_tensor_b200._lib import call
+    import ctypes
+
+    def P_(t):
+        return ctypes.c_void_p(t.data_ptr())
+
+    gpipe = api.Graph(n, E, bufs["row_ptr"], bufs["col"][:E], bufs["ev"][:E], bufs["csc_ptr"],
+                      bufs["ce"][:E], bufs["cd"][:E])
+    Wp = torch.empty_like(W)
+
+    def pipeline_step(evp=None, pos_t=pos):
+        if evp is not None:
+            evp[0].record(stream)
+        call("cgtp_graph_build", P_(pos_t), n, ctypes.c_float(0.0), ctypes.c_float(w.rc), P_(gp), gp.numel() - 1,
+             P_(bufs["row_ptr"]), P_(bufs["col"]), P_(bufs["ev"]), P_(bufs["csc_ptr"]), P_(bufs["ce"]),
+             P_(bufs["cd"]), cap, P_(ne_dev), ctypes.c_void_p(stream.cuda_stream))
+        if evp is not None:
+            evp[1].record(stream)
+        plan.radial_forward(gpipe.edge_vec, w.rc, W1, W2, out=Wp)
+        if evp is not None:
+            evp[2].record(stream)
+        plan.conv_forward(gpipe, x, Wp, out=out)
+        plan.conv_backward(gpipe, x, Wp, go, grad_x=gx, grad_w=gw, grad_edge_vec=gr, workspace=ws)
+        if evp is not None:
+            evp[3].record(stream)
+        plan.radial_backward(gpipe.edge_vec, w.rc, W1, W2, gw, gr)
+        if evp is not None:
+            evp[4].record(stream)
+        api.forces(gpipe, gr, out=F)
+        if evp is not None:
+            evp[5].record(stream)
+
+    for _ in range(3):
+        pipeline_step()
+    torch.cuda.synchronize()
+    assert int(ne_dev.item()) == E
+    npipe = max(20, min(args.steps // 4, 500))
+    evp = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(npipe)]
+    barrier()
+    torch.cuda.synchronize()
+    for k in range(npipe):
+        pipeline_step(evp[k])
+    torch.cuda.synchronize()
+    seg = np.mean([[e[i].elapsed_time(e[i + 1]) for i in range(5)] for e in evp], axis=0)
+    t_pipe = max_over_ranks(float(np.mean([e[0].elapsed_time(e[5]) for e in evp])) / 1e3)
+    pipe_value = edges_all / t_pipe
+
+    # e2e through the public API with host buffers: pinned positions, features and
+    # output gradient in; forces out, every step
+    pos_h = torch.from_numpy(w.pos).pin_memory()
+    x_h = torch.from_numpy(w.x).pin_memory()
+    go_h = torch.from_numpy(w.grad_out).pin_memory()
+    F_h = torch.empty((n, 3), dtype=torch.float32).pin_memory()
+    pos_d = torch.empty_like(pos)
+
+    def e2e_step():
+        pos_d.copy_(pos_h, non_blocking=True)
+        x.copy_(x_h, non_blocking=True)
+        go.copy_(go_h, non_blocking=True)
+        pipeline_step(pos_t=pos_d)
+        F_h.copy_(F, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    ne2e = max(10, min(args.steps // 10, 200))
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    a0.record(stream)
+    for _ in range(ne2e):
+        e2e_step()
+    a1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = max_over_ranks(a0.elapsed_time(a1) / 1e3 / ne2e)
+    h2d = pos_h.numel() * 4 + x_h.numel() * 4 + go_h.numel() * 4
+    d2h = F_h.numel() * 4
+
+    # roofline of the dominant kernel (the backward)
+    hbm, peak_kind = _load_peaks()
+    slices = max(1, int(ws_bytes // (4 * E * ns))) if E else 1
+    b_fwd, b_bwd = conv_bytes(n, E, P, u, ni, ns, no, slices)
+    dominant = "conv_bwd" if t_bwd >= t_fwd else "conv_fwd"
+    b_dom, t_dom = (b_bwd, t_bwd) if dominant == "conv_bwd" else (b_fwd, t_fwd)
+    achieved = b_dom / (t_dom / 1e3) / 1e9
+    nT, nnz, no_sum = structural_counts(*L)
+    f_fwd, f_bwd = conv_flops(E, u, nT, nnz, no_sum, P)
+    step_bytes = b_fwd + b_bwd + 4 * (E * 3 * 2 + n * 3 + 2 * (n + 1) + 2 * E)
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded); weights from the radial network",
+        "config": {"workload": WORKLOAD, "n_nodes": n, "n_edges": E, "paths": P, "mult": u,
+                   "l2": "inputs larger than L2 (W is %.0f MB per rank, read twice per step)" % (E * P * u * 4 / 1e6),
+                   "parallelism": f"independent batch per rank (dp{world})"},
+        "gpu_launches": 4 * args.steps,
+        "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None, "peak_kind": peak_kind,
+                     "alg_bytes_per_launch": b_dom},
+        "kernels_ms": {"conv_fwd": t_fwd, "conv_bwd_incl_sh_jacobian": t_bwd, "forces": t_frc},
+        "step_hbm_frac": (step_bytes / (ms_step / 1e3) / 1e9) / hbm,
+        "fp32_tflops": {"conv_fwd": f_fwd / (t_fwd / 1e3) / 1e12, "conv_bwd": f_bwd / (t_bwd / 1e3) / 1e12},
+        "pipeline": {"value": pipe_value, "unit": UNIT, "ms_per_step": t_pipe * 1e3,
+                     "stages_ms": {"graph": float(seg[0]), "radial_fwd": float(seg[1]),
+                                   "conv_fwd_bwd": float(seg[2]), "radial_bwd": float(seg[3]),
+                                   "forces": float(seg[4])}},
+        "e2e": {"value": edges_all / t_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "what": "pinned host positions, features, output gradient -> graph, radial weights, conv fwd+bwd, "
+                        "radial bwd, forces -> host forces"},
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["cgtp", "reference"], default="cgtp")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

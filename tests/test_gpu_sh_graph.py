@@ -39,8 +39,8 @@ def test_harmonics_and_jacobian(api, lmax):
     for k in range(v.shape[0]):
         s = np.max(np.abs(Jo[k]))
         assert np.max(np.abs(J[k] - Jo[k])) <= GRAD_TOL * max(s, 1e-30) + 1e-30
-    Y2 = api.spherical_harmonics(lmax, cuda(v))
-    assert np.array_equal(host(Y2), host(Y))
+    Y2 = api.spherical_harmonics(lmax, cuda(v))  # value-only path (rsqrt) vs the dual-number path
+    assert rel_err(host(Y2), Yo) < FWD_TOL
 
 
 def _compare_graph(g, o):
