@@ -236,7 +236,7 @@ def run_gpu(args):
         dist.all_reduce(t, op=dist.ReduceOp.SUM)
         return float(t.item())
 
-    w = synthetic.molecules(seed=4 + 1000 * rank)
+    w = synthetic.molecules(seed=4 + 1000 * rank, n_graphs=args.graphs)
     L = (w.lmax_in, w.lmax_sh, w.lmax_out)
     n, u = w.n_nodes, w.mult
     ni, ns, no = (L[0] + 1) ** 2, (L[1] + 1) ** 2, (L[2] + 1) ** 2
@@ -309,6 +309,16 @@ def run_gpu(args):
     edges_all = sum_over_ranks(float(E))
     value = edges_all * args.steps / t
     ms_step = 1e3 * t / args.steps
+
+    if args.conv_only:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                              "ms_per_step": ms_step, "n_edges": E,
+                              "kernels_ms": {"conv_fwd": t_fwd, "conv_bwd_incl_sh_jacobian": t_bwd,
+                                             "forces": t_frc}}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
 
     # pipeline: positions -> graph -> radial weights -> conv -> radial backward -> forces
     ne_dev = torch.empty(1, dtype=torch.int32, device=dev)
@@ -449,6 +459,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["cgtp", "reference"], default="cgtp")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graphs", type=int, default=256, help="molecules per rank (profiling uses fewer)")
+    ap.add_argument("--conv-only", action="store_true",
+                    help="time only the convolution step (no pipeline / e2e / CPU baseline); for profiling")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

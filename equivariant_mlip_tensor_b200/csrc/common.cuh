@@ -22,6 +22,14 @@ template <int B, int E, class F>
 __device__ __forceinline__ void static_for(F&& f) {
   if constexpr (E > B) static_for_impl<B>(f, std::make_integer_sequence<int, E - B>{});
 }
+template <int B, class F, int... Is>
+void static_for_host_impl(F&& f, std::integer_sequence<int, Is...>) {
+  (f(std::integral_constant<int, B + Is>{}), ...);
+}
+template <int B, int E, class F>
+void static_for_host(F&& f) {
+  if constexpr (E > B) static_for_host_impl<B>(f, std::make_integer_sequence<int, E - B>{});
+}
 
 // ---- coefficient tables.  Every translation unit that needs them holds its
 // own constant-memory copy and registers an uploader at load time; plan
@@ -50,6 +58,12 @@ __device__ __forceinline__ void st_stream(float* p, float4 v) {
   __stcs(reinterpret_cast<float4*>(p), v);
 }
 __device__ __forceinline__ void st_f4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+
+// Bulk prefetch of [p, p + bytes) into L2 (one TMA instruction; p and bytes
+// multiples of 16).
+__device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 
 __device__ __forceinline__ void f4_to(float (&a)[4], float4 v) {
   a[0] = v.x; a[1] = v.y; a[2] = v.z; a[3] = v.w;

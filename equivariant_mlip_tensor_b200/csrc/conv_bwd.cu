@@ -1,11 +1,10 @@
 // CGTP convolution backward, node-centric over sources (CSC), for sm_100a.
 //
 // For edge e = (j -> i) with T_e^p[m1][m3] = sum_m2 C^p[m1,m2,m3] Y_e[l2,m2]:
-//   t_p[m3][u]      = sum_m1 T_e^p[m1][m3] x[j][l1,m1][u]
-//   grad_W[e][p][u] = sum_m3 g[i][l3,m3][u] t_p[m3][u]
-//   s_p[m3][u]      = W_e[p][u] g[i][l3,m3][u]
-//   grad_x[j][l1,m1][u] += sum_m3 T_e^p[m1][m3] s_p[m3][u]
-//   grad_Y[e][l2,m2] = sum_p sum_{m1,m3} C^p[m1,m2,m3] sum_u x[j][l1,m1][u] s_p[m3][u]
+//   h_p[m1][u]      = sum_m3 T_e^p[m1][m3] g[i][l3,m3][u]
+//   grad_x[j][l1,m1][u] += W_e[p][u] h_p[m1][u]
+//   grad_W[e][p][u] = sum_m1 x[j][l1,m1][u] h_p[m1][u]
+//   grad_Y[e][l2,m2] = sum_p sum_{m1,m3} C^p[m1,m2,m3] sum_u W_e[p][u] x[j][l1,m1][u] g[i][l3,m3][u]
 // (the adjoints of the bilinear convolution; cf. the closed-form gradients
 // of a bilinear tensor product in "Tensor Decomposition Networks ...",
 // reply to reviewer S6y1, and the derivative computation of "LunaTP ...",
@@ -23,6 +22,7 @@ namespace cgtp {
 CGTP_DEFINE_CONSTANT_TABLES()
 }  // namespace cgtp
 
+#include "conv_common.cuh"
 #include "sh.cuh"
 
 namespace cgtp {
@@ -31,91 +31,54 @@ namespace {
 
 constexpr int kBwdThreads = 128;
 
-template <int VEC>
-struct VecIO;
-template <>
-struct VecIO<4> {
-  static __device__ __forceinline__ void ld(float (&a)[4], const float* p) { f4_to(a, __ldg(reinterpret_cast<const float4*>(p))); }
-  static __device__ __forceinline__ void ld_stream(float (&a)[4], const float* p) { f4_to(a, __ldcs(reinterpret_cast<const float4*>(p))); }
-  static __device__ __forceinline__ void st(float* p, const float (&a)[4]) { *reinterpret_cast<float4*>(p) = to_f4(a); }
-  static __device__ __forceinline__ void st_stream(float* p, const float (&a)[4]) { __stcs(reinterpret_cast<float4*>(p), to_f4(a)); }
-};
-template <>
-struct VecIO<2> {
-  static __device__ __forceinline__ void ld(float (&a)[2], const float* p) {
-    const float2 v = __ldg(reinterpret_cast<const float2*>(p));
-    a[0] = v.x; a[1] = v.y;
-  }
-  static __device__ __forceinline__ void ld_stream(float (&a)[2], const float* p) {
-    const float2 v = __ldcs(reinterpret_cast<const float2*>(p));
-    a[0] = v.x; a[1] = v.y;
-  }
-  static __device__ __forceinline__ void st(float* p, const float (&a)[2]) { *reinterpret_cast<float2*>(p) = make_float2(a[0], a[1]); }
-  static __device__ __forceinline__ void st_stream(float* p, const float (&a)[2]) { __stcs(reinterpret_cast<float2*>(p), make_float2(a[0], a[1])); }
-};
-
-template <class PS>
-__device__ __forceinline__ void compute_T_bwd(const float (&Y)[PS::NS], float* __restrict__ T) {
-  static_for<0, PS::NP>([&](auto Pc) {
-    constexpr int P = decltype(Pc)::value;
-    constexpr int l1 = PS::D.l1[P], l2 = PS::D.l2[P], l3 = PS::D.l3[P];
-    static_for<0, 2 * l3 + 1>([&](auto M3c) {
-      constexpr int m3 = decltype(M3c)::value - l3;
-      static_for<0, 2 * l1 + 1>([&](auto M1c) {
-        constexpr int m1 = decltype(M1c)::value - l1;
-        constexpr int ti = PS::t_index(P, m1, m3);
-        if constexpr (ti >= 0) {
-          float v = 0.f;
-          static_for<0, 2 * l2 + 1>([&](auto M2c) {
-            constexpr int m2 = decltype(M2c)::value - l2;
-            if constexpr (cg_allowed(l1, l2, l3, m1, m2, m3)) {
-              v = fmaf(c_cg[table_index(l1, l2, l3, m1, m2, m3)], Y[l2 * l2 + l2 + m2], v);
-            }
-          });
-          T[ti] = v;
-        }
-      });
-    });
-    static_for<PS::D.tbase[P] + PS::D.tcount[P], PS::D.tbase[P + 1]>([&](auto Kc) {
-      T[decltype(Kc)::value] = 0.f;
-    });
-  });
+template <class PS, class GR>
+constexpr bool grp_has_l2(int l2) {
+  for (int k = 0; k < GR::D.n; ++k)
+    if (PS::D.l2[GR::D.path[k]] == l2) return true;
+  return false;
 }
 
-template <class PS>
-constexpr bool first_of_l2(int k) {
-  return k == 0 || PS::D.l2[PS::D.by_l2[k - 1]] != PS::D.l2[PS::D.by_l2[k]];
-}
-
-// One edge of the CSC row.  Paths are visited in (l2, l1, l3) order so that
-// only one l2 block of the grad_Y partial is live at a time; each finished
-// block goes to this lane's row of the shared reduction buffer (gyrow).  Each
-// T entry is loaded once (four at a time) and used for t, grad_x and grad_Y.
-template <class PS, int VEC, bool NEED_GY>
-__device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const float (&xr)[PS::NI][VEC],
-                                         const float (&gr)[PS::NO][VEC], const float* __restrict__ wrow,
-                                         float* __restrict__ gwrow, int mult, float (&gx)[PS::NI][VEC],
-                                         float* __restrict__ gyrow) {
+// One edge of the CSC row, the paths of one group (l1 = GR's value).  Per
+// path, with h[m1] = sum_m3 T[m1][m3] g[m3] (one pass over the structural
+// nonzeros of T):
+//   grad_x[m1] += W h[m1],   grad_W = sum_m1 x[m1] h[m1],
+// and, for grad_Y, the channel sums sum_u W x[m1] g[m3] of every T entry
+// contracted with the CG coefficients.  Paths are visited in (l2, ...) order
+// so that only one l2 block of the grad_Y partial is live at a time; each
+// finished block goes to this lane's row of the shared reduction buffer
+// (gyrow).  The edge's weight rows and its destination's output-gradient
+// rows come from this lane's pipeline stage.
+template <class PS, class GR, int VEC, bool NEED_GY>
+__device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const float* __restrict__ stage, int rowf,
+                                         const float (&xr)[GR::NOWN][VEC], float* __restrict__ gwrow, int mult,
+                                         float (&gx)[GR::NOWN][VEC], float* __restrict__ gyrow) {
   float gy[PS::NS];
-  static_for<0, PS::NP>([&](auto Kc) {
+  static_for<0, GR::NP>([&](auto Kc) {
     constexpr int K = decltype(Kc)::value;
-    constexpr int P = PS::D.by_l2[K];
+    constexpr int P = GR::D.path[K];
     constexpr int l1 = PS::D.l1[P], l2 = PS::D.l2[P], l3 = PS::D.l3[P];
-    constexpr int tb = PS::D.tbase[P], tc = PS::D.tcount[P];
-    if constexpr (NEED_GY && first_of_l2<PS>(K)) {
+    constexpr int tb = GR::D.lt[K], tc = PS::D.tcount[P];
+    constexpr int g0 = GR::NP + l3 * l3 - GR::D.rlo;  // staged row of grad_out[l3, m3 = -l3]
+    if constexpr (NEED_GY && GR::D.first_l2[K]) {
 #pragma unroll
       for (int m2 = 0; m2 < 2 * l2 + 1; ++m2) gy[l2 * l2 + m2] = 0.f;
     }
     float wv[VEC];
-    VecIO<VEC>::ld_stream(wv, wrow + P * mult);
-    float s[2 * l3 + 1][VEC], t[2 * l3 + 1][VEC];
+    VecIO<VEC>::lds(wv, stage + K * rowf);
+    float gv[2 * l3 + 1][VEC], h[2 * l1 + 1][VEC];
 #pragma unroll
-    for (int m3 = 0; m3 < 2 * l3 + 1; ++m3)
+    for (int m3 = 0; m3 < 2 * l3 + 1; ++m3) VecIO<VEC>::lds(gv[m3], stage + (g0 + m3) * rowf);
 #pragma unroll
-      for (int c = 0; c < VEC; ++c) {
-        s[m3][c] = wv[c] * gr[l3 * l3 + m3][c];
-        t[m3][c] = 0.f;
-      }
+    for (int m1 = 0; m1 < 2 * l1 + 1; ++m1)
+#pragma unroll
+      for (int c = 0; c < VEC; ++c) h[m1][c] = 0.f;
+    float xw[2 * l1 + 1][VEC];  // W x, for the grad_Y channel sums
+    if constexpr (NEED_GY) {
+#pragma unroll
+      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1)
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) xw[m1][c] = wv[c] * xr[m1][c];
+    }
     static_for<0, (tc + 3) / 4>([&](auto Qc) {
       constexpr int q = decltype(Qc)::value;
       const float4 v4 = *reinterpret_cast<const float4*>(T + tb + 4 * q);
@@ -124,17 +87,13 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
         constexpr int k = 4 * q + decltype(Rc)::value;
         if constexpr (k < tc) {
           constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
-          constexpr int r1 = l1 * l1 + l1 + m1;
           const float tv = tv4[decltype(Rc)::value];
 #pragma unroll
-          for (int c = 0; c < VEC; ++c) {
-            t[m3 + l3][c] = fmaf(tv, xr[r1][c], t[m3 + l3][c]);
-            gx[r1][c] = fmaf(tv, s[m3 + l3][c], gx[r1][c]);
-          }
+          for (int c = 0; c < VEC; ++c) h[m1 + l1][c] = fmaf(tv, gv[m3 + l3][c], h[m1 + l1][c]);
           if constexpr (NEED_GY) {
             float av = 0.f;
 #pragma unroll
-            for (int c = 0; c < VEC; ++c) av = fmaf(xr[r1][c], s[m3 + l3][c], av);
+            for (int c = 0; c < VEC; ++c) av = fmaf(xw[m1 + l1][c], gv[m3 + l3][c], av);
             static_for<0, 2 * l2 + 1>([&](auto M2c) {
               constexpr int m2 = decltype(M2c)::value - l2;
               if constexpr (cg_allowed(l1, l2, l3, m1, m2, m3)) {
@@ -145,36 +104,44 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
         }
       });
     });
-    if (gwrow != nullptr) {
-      float gw[VEC];
+    float gw[VEC];
+#pragma unroll
+    for (int c = 0; c < VEC; ++c) gw[c] = 0.f;
+#pragma unroll
+    for (int m1 = 0; m1 < 2 * l1 + 1; ++m1)
 #pragma unroll
       for (int c = 0; c < VEC; ++c) {
-        gw[c] = 0.f;
-#pragma unroll
-        for (int m3 = 0; m3 < 2 * l3 + 1; ++m3) gw[c] = fmaf(gr[l3 * l3 + m3][c], t[m3][c], gw[c]);
+        gx[m1][c] = fmaf(wv[c], h[m1][c], gx[m1][c]);
+        gw[c] = fmaf(xr[m1][c], h[m1][c], gw[c]);
       }
-      VecIO<VEC>::st_stream(gwrow + P * mult, gw);
-    }
-    if constexpr (NEED_GY && PS::D.last_of_l2[K]) {
+    if (gwrow != nullptr) VecIO<VEC>::st_stream(gwrow + P * mult, gw);
+    if constexpr (NEED_GY && GR::D.last_l2[K]) {
 #pragma unroll
       for (int m2 = 0; m2 < 2 * l2 + 1; ++m2) gyrow[l2 * l2 + m2] = gy[l2 * l2 + m2];
     }
   });
 }
 
-template <class PS, int VEC, bool NEED_GY>
+// One launch per path group (the paths with l1 = L1): grad_x rows of that
+// block, grad_W of those paths and a partial grad_Y over those paths.
+template <class PS, int VEC, bool NEED_GY, int L1>
 __global__ void __launch_bounds__(kBwdThreads)
-conv_bwd_kernel(ConvBwdArgs a, int lg_G, int S, int BT, int tstride) {
-  constexpr int NI = PS::NI, NO = PS::NO, NS = PS::NS;
+conv_bwd_kernel(ConvBwdArgs a, int lg_G, int S, int BT, int slice_base) {
+  using GR = Grp<PS, kByL1, L1>;
+  constexpr int NI = PS::NI, NO = PS::NO, NS = PS::NS, NR = GR::NOWN, NT = GR::NT;
+  constexpr int NROWS = GR::NP + GR::NROW;
   constexpr int NSP = NS | 1;  // odd row stride: conflict-free transposed reduction
   extern __shared__ float4 smem_f4[];
   float* smem = reinterpret_cast<float*>(smem_f4);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int G = 1 << lg_G, gpw = 32 >> lg_G;
   const int grp = lane >> lg_G, gl = lane & (G - 1);
-  const int group_floats = BT * tstride + 2 * ((BT + 3) & ~3);
+  const int rowf = G * VEC;
+  const int stage_floats = NROWS * rowf;
+  const int group_floats = BT * NT + 2 * stage_floats + 2 * ((BT + 3) & ~3);
   float* Tg = smem + (warp * gpw + grp) * group_floats;
-  int* Eg = reinterpret_cast<int*>(Tg + BT * tstride);
+  float* St = Tg + BT * NT;
+  int* Eg = reinterpret_cast<int*>(St + 2 * stage_floats);
   int* Ig = Eg + ((BT + 3) & ~3);
   // per warp: 32 x NSP floats for the grad_Y reduction
   float* red = smem + (kBwdThreads / 32) * gpw * group_floats + warp * 32 * NSP;
@@ -194,10 +161,10 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G, int S, int BT, int tstride) {
       k1 = __ldg(a.csc_ptr + node + 1);
     }
     const int maxdeg = __reduce_max_sync(0xffffffffu, k1 - k0);
-    float xr[NI][VEC], gx[NI][VEC];
+    float xr[NR][VEC], gx[NR][VEC];
 #pragma unroll
-    for (int r = 0; r < NI; ++r) {
-      if (active) VecIO<VEC>::ld(xr[r], a.x + (node * NI + r) * a.mult + c0);
+    for (int r = 0; r < NR; ++r) {
+      if (active) VecIO<VEC>::ld(xr[r], a.x + (node * NI + L1 * L1 + r) * a.mult + c0);
       else {
 #pragma unroll
         for (int c = 0; c < VEC; ++c) xr[r][c] = 0.f;
@@ -205,6 +172,22 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G, int S, int BT, int tstride) {
 #pragma unroll
       for (int c = 0; c < VEC; ++c) gx[r][c] = 0.f;
     }
+
+    // copies of edge slot k of the current batch into stage s (this lane's channels only)
+    auto issue = [&](int b0, int k, int s) {
+      if (!(active && k0 + b0 + k < k1)) return;
+      float* dst = St + s * stage_floats + gl * VEC;
+      const float* wrow = a.w + (long long)Eg[k] * PS::NP * a.mult + c0;
+      static_for<0, GR::NP>([&](auto Kc) {
+        constexpr int K = decltype(Kc)::value;
+        constexpr int P = GR::D.path[K];
+        VecIO<VEC>::cp_async(dst + K * rowf, wrow + P * a.mult);
+      });
+      constexpr int rlo = GR::D.rlo;
+      const float* grow = a.grad_out + ((long long)Ig[k] * NO + rlo) * a.mult + c0;
+#pragma unroll
+      for (int r = 0; r < GR::NROW; ++r) VecIO<VEC>::cp_async(dst + (GR::NP + r) * rowf, grow + r * a.mult);
+    };
 
     for (int b0 = 0; b0 < maxdeg; b0 += BT) {
       for (int k = gl; k < BT; k += G) {
@@ -214,39 +197,52 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G, int S, int BT, int tstride) {
           float Y[NS];
           sh_of_vec<PS::LS>(__ldg(a.edge_vec + 3 * (long long)e), __ldg(a.edge_vec + 3 * (long long)e + 1),
                             __ldg(a.edge_vec + 3 * (long long)e + 2), Y);
-          compute_T_bwd<PS>(Y, Tg + k * tstride);
+          compute_T_grp<PS, GR>(Y, Tg + k * NT);
           Eg[k] = e;
           Ig[k] = __ldg(a.csc_dst + kk);
         }
       }
       __syncwarp();
       const int nb = min(BT, maxdeg - b0);
+      issue(b0, 0, 0);
+      cp_async_commit();
       for (int k = 0; k < nb; ++k) {
+        if (k + 1 < nb) issue(b0, k + 1, (k + 1) & 1);
+        cp_async_commit();
+        cp_async_wait<1>();  // this lane's copies of edge k have landed
         const bool valid = active && (k0 + b0 + k) < k1;
         float* rg = red + (grp * G) * NSP;  // this group's rows of the reduction buffer
-        if constexpr (NEED_GY) {
+        if constexpr (NEED_GY) {  // zero the l2 blocks no path of the group touches
+          static_for<0, PS::LS + 1>([&](auto Bc) {
+            constexpr int l2 = decltype(Bc)::value;
+            if constexpr (!grp_has_l2<PS, GR>(l2)) {
 #pragma unroll
-          for (int b = 0; b < NS; ++b) rg[gl * NSP + b] = 0.f;  // l2 blocks no path touches
+              for (int m2 = 0; m2 < 2 * l2 + 1; ++m2) rg[gl * NSP + l2 * l2 + m2] = 0.f;
+            }
+          });
         }
         int e = 0;
         if (valid) {
           e = Eg[k];
-          const long long i = Ig[k];
-          float gr[NO][VEC];
-#pragma unroll
-          for (int r = 0; r < NO; ++r) VecIO<VEC>::ld(gr[r], a.grad_out + (i * NO + r) * a.mult + c0);
-          const long long woff = (long long)e * PS::NP * a.mult + c0;
-          bwd_edge<PS, VEC, NEED_GY>(Tg + k * tstride, xr, gr, a.w + woff,
-                                     a.grad_w ? a.grad_w + woff : nullptr, a.mult, gx, rg + gl * NSP);
+          bwd_edge<PS, GR, VEC, NEED_GY>(Tg + k * NT, St + (k & 1) * stage_floats + gl * VEC, rowf, xr,
+                                         a.grad_w ? a.grad_w + (long long)e * PS::NP * a.mult + c0 : nullptr,
+                                         a.mult, gx, rg + gl * NSP);
         }
         if constexpr (NEED_GY) {
           __syncwarp();
           if (valid) {
-            float* dst = a.grad_sh + ((long long)slice * a.n_edges + e) * NS;
-            for (int b = gl; b < NS; b += G) {
-              float v = 0.f;
-              for (int r = 0; r < G; ++r) v += rg[r * NSP + b];
-              dst[b] = v;
+            float* dst = a.grad_sh + ((long long)(slice_base + slice) * a.n_edges + e) * NS;
+            for (int b = gl; b < NS; b += G) {  // four independent partial sums
+              float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
+              int r = 0;
+              for (; r + 4 <= G; r += 4) {
+                v0 += rg[r * NSP + b];
+                v1 += rg[(r + 1) * NSP + b];
+                v2 += rg[(r + 2) * NSP + b];
+                v3 += rg[(r + 3) * NSP + b];
+              }
+              for (; r < G; ++r) v0 += rg[r * NSP + b];
+              dst[b] = (v0 + v1) + (v2 + v3);
             }
           }
           __syncwarp();
@@ -256,7 +252,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G, int S, int BT, int tstride) {
     }
     if (active && a.grad_x != nullptr) {
 #pragma unroll
-      for (int r = 0; r < NI; ++r) VecIO<VEC>::st(a.grad_x + (node * NI + r) * a.mult + c0, gx[r]);
+      for (int r = 0; r < NR; ++r) VecIO<VEC>::st(a.grad_x + (node * NI + L1 * L1 + r) * a.mult + c0, gx[r]);
     }
   }
 }
@@ -293,65 +289,89 @@ __global__ void sh_backward_kernel(int n_edges, int S, const float* __restrict__
 
 }  // namespace
 
+// Channels per lane: 4 (float4) up to l = 2; 2 for l = 3, whose path groups
+// would otherwise exceed the register file.
 template <class PS>
 constexpr int bwd_vec() {
-  return (PS::NI + PS::NO > 20) ? 2 : 4;
+  return PS::LI >= 3 || PS::LO >= 3 ? 2 : 4;
+}
+
+// channel lanes per group (G) and channel slices (S) of the backward
+template <class PS>
+void bwd_geometry(int mult, int& G, int& lg_G, int& S) {
+  lane_geometry(mult, bwd_vec<PS>(), G, lg_G, S);
 }
 
 template <int LI, int LS, int LO>
 int conv_bwd_slices(int mult) {
   using PS = PathSet<LI, LS, LO>;
+  int G, lg_G, S;
+  bwd_geometry<PS>(mult, G, lg_G, S);
+  return S * (LI + 1);  // one partial grad_Y per (path group, channel slice)
+}
+
+template <class PS, int L1>
+cudaError_t launch_bwd_group(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
+  using GR = Grp<PS, kByL1, L1>;
   constexpr int VEC = bwd_vec<PS>();
-  const int lanes = mult / VEC;
-  int G = 1;
-  while (G < 32 && lanes % (2 * G) == 0) G *= 2;
-  return lanes / G;
+  constexpr int NSP = PS::NS | 1;
+  int G, lg_G, S;
+  bwd_geometry<PS>(a.mult, G, lg_G, S);
+  const bool need_gy = a.grad_edge_vec != nullptr;
+  if constexpr (GR::NP == 0) {  // no path starts from this l1 block: its gradient is zero
+    if (a.grad_x != nullptr) {
+      cudaError_t e = cudaMemset2DAsync(a.grad_x + (size_t)L1 * L1 * a.mult, sizeof(float) * PS::NI * a.mult, 0,
+                                        sizeof(float) * GR::NOWN * a.mult, a.n_nodes, stream);
+      if (e != cudaSuccess) return e;
+    }
+    if (need_gy)
+      for (int s = 0; s < S; ++s) {
+        cudaError_t e = cudaMemsetAsync(a.grad_sh + (size_t)(L1 * S + s) * a.n_edges * PS::NS, 0,
+                                        sizeof(float) * (size_t)a.n_edges * PS::NS, stream);
+        if (e != cudaSuccess) return e;
+      }
+    return cudaSuccess;
+  } else {
+    const int gpw = 32 / G;
+    const int stage_floats = (GR::NP + GR::NROW) * G * VEC;
+    const int BT = pick_batch(gpw, GR::NT, stage_floats);
+    const int group_floats = BT * GR::NT + 2 * stage_floats + 2 * ((BT + 3) & ~3);
+    const size_t smem = sizeof(float) * ((size_t)group_floats * gpw * (kBwdThreads / 32) +
+                                         (need_gy ? (size_t)(kBwdThreads / 32) * 32 * NSP : 0));
+    const long long items = (long long)a.n_nodes * S;
+    const long long groups_per_block = (long long)gpw * (kBwdThreads / 32);
+    const long long blocks = (items + groups_per_block - 1) / groups_per_block;
+    auto run = [&](auto kern) -> cudaError_t {
+      cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e2 != cudaSuccess) return e2;
+      int per_sm = 0;
+      e2 = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBwdThreads, smem);
+      if (e2 != cudaSuccess) return e2;
+      if (per_sm < 1) per_sm = 1;
+      const long long cap = (long long)num_sms * per_sm;
+      long long nb = blocks > cap ? cap : blocks;
+      if (nb < 1) nb = 1;
+      kern<<<(unsigned)nb, kBwdThreads, smem, stream>>>(a, lg_G, S, BT, L1 * S);
+      return cudaGetLastError();
+    };
+    if (need_gy) return run(conv_bwd_kernel<PS, VEC, true, L1>);
+    return run(conv_bwd_kernel<PS, VEC, false, L1>);
+  }
 }
 
 template <int LI, int LS, int LO>
 cudaError_t launch_conv_bwd(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
   using PS = PathSet<LI, LS, LO>;
-  constexpr int VEC = bwd_vec<PS>();
-  constexpr int NSP = PS::NS | 1;
-  const int lanes = a.mult / VEC;
-  int G = 1;
-  while (G < 32 && lanes % (2 * G) == 0) G *= 2;
-  int lg_G = 0;
-  while ((1 << lg_G) < G) ++lg_G;
-  const int S = lanes / G;
-  const int gpw = 32 / G;
-  const int tstride = PS::NT > 0 ? PS::NT : 4;
-  int BT = 4096 / (gpw * tstride);
-  BT = BT < 1 ? 1 : (BT > 32 ? 32 : BT);
-  const int group_floats = BT * tstride + 2 * ((BT + 3) & ~3);
-  const bool need_gy = a.grad_edge_vec != nullptr;
-  const size_t smem = sizeof(float) * ((size_t)group_floats * gpw * (kBwdThreads / 32) +
-                                       (need_gy ? (size_t)(kBwdThreads / 32) * 32 * NSP : 0));
-  const long long items = (long long)a.n_nodes * S;
-  const long long groups_per_block = (long long)gpw * (kBwdThreads / 32);
-  long long blocks = (items + groups_per_block - 1) / groups_per_block;
-  cudaError_t err;
-  auto run = [&](auto kern) -> cudaError_t {
-    cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e2 != cudaSuccess) return e2;
-    int per_sm = 0;
-    e2 = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBwdThreads, smem);
-    if (e2 != cudaSuccess) return e2;
-    if (per_sm < 1) per_sm = 1;
-    const long long cap = (long long)num_sms * per_sm;
-    long long nb = blocks > cap ? cap : blocks;
-    if (nb < 1) nb = 1;
-    kern<<<(unsigned)nb, kBwdThreads, smem, stream>>>(a, lg_G, S, BT, tstride);
-    return cudaGetLastError();
-  };
-  if (need_gy) err = run(conv_bwd_kernel<PS, VEC, true>);
-  else err = run(conv_bwd_kernel<PS, VEC, false>);
-  if (err != cudaSuccess || !need_gy || a.n_edges == 0) return err;
+  cudaError_t err = cudaSuccess;
+  static_for_host<0, LI + 1>([&](auto Lc) {
+    if (err == cudaSuccess) err = launch_bwd_group<PS, decltype(Lc)::value>(a, num_sms, stream);
+  });
+  if (err != cudaSuccess || a.grad_edge_vec == nullptr || a.n_edges == 0) return err;
   const int threads = 256;
   long long nbk = (a.n_edges + threads - 1) / threads;
   if (nbk > (long long)num_sms * 16) nbk = (long long)num_sms * 16;
-  sh_backward_kernel<LS><<<(unsigned)nbk, threads, 0, stream>>>(a.n_edges, S, a.edge_vec, a.grad_sh,
-                                                                 a.grad_edge_vec);
+  sh_backward_kernel<LS><<<(unsigned)nbk, threads, 0, stream>>>(a.n_edges, conv_bwd_slices<LI, LS, LO>(a.mult),
+                                                                 a.edge_vec, a.grad_sh, a.grad_edge_vec);
   return cudaGetLastError();
 }
 

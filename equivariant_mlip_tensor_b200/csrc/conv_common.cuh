@@ -1,0 +1,140 @@
+// Shared pieces of the node-centric convolution kernels: path groups, the
+// per-edge T matrices of a group, vector loads/stores and per-lane
+// asynchronous copies into shared memory.
+//
+// Include after CGTP_DEFINE_CONSTANT_TABLES (uses c_cg).
+#pragma once
+
+namespace cgtp {
+
+// ---- vector I/O of VEC consecutive channels ----
+template <int VEC>
+struct VecIO;
+template <>
+struct VecIO<4> {
+  static __device__ __forceinline__ void ld(float (&a)[4], const float* p) { f4_to(a, __ldg(reinterpret_cast<const float4*>(p))); }
+  static __device__ __forceinline__ void lds(float (&a)[4], const float* p) { f4_to(a, *reinterpret_cast<const float4*>(p)); }
+  static __device__ __forceinline__ void st(float* p, const float (&a)[4]) { *reinterpret_cast<float4*>(p) = to_f4(a); }
+  static __device__ __forceinline__ void st_stream(float* p, const float (&a)[4]) { __stcs(reinterpret_cast<float4*>(p), to_f4(a)); }
+  // asynchronous global -> shared copy of this lane's 16 bytes (L2 only)
+  static __device__ __forceinline__ void cp_async(float* s, const float* g) {
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(s);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(g) : "memory");
+  }
+};
+template <>
+struct VecIO<2> {
+  static __device__ __forceinline__ void ld(float (&a)[2], const float* p) {
+    const float2 v = __ldg(reinterpret_cast<const float2*>(p));
+    a[0] = v.x; a[1] = v.y;
+  }
+  static __device__ __forceinline__ void lds(float (&a)[2], const float* p) {
+    const float2 v = *reinterpret_cast<const float2*>(p);
+    a[0] = v.x; a[1] = v.y;
+  }
+  static __device__ __forceinline__ void st(float* p, const float (&a)[2]) { *reinterpret_cast<float2*>(p) = make_float2(a[0], a[1]); }
+  static __device__ __forceinline__ void st_stream(float* p, const float (&a)[2]) { __stcs(reinterpret_cast<float2*>(p), make_float2(a[0], a[1])); }
+  static __device__ __forceinline__ void cp_async(float* s, const float* g) {
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(s);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sa), "l"(g) : "memory");
+  }
+};
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// ---- path groups ----
+// The convolution kernels split the paths into groups that share one l
+// value: the backward groups by l1 (each group owns a block of grad_x rows),
+// the forward by l3 (each group owns a block of output rows).  One launch
+// per group keeps the per-thread state and the unrolled code small.
+enum GroupKind { kByL1 = 0, kByL3 = 1, kAll = 2 };
+
+template <class PS, int KIND, int V>
+struct Grp {
+  struct Data {
+    int n;                       // paths in the group
+    int path[kMaxPaths];         // path numbers, sorted by (l2, lexicographic)
+    int lt[kMaxPaths + 1];       // group-local padded T offset of the k-th path
+    bool first_l2[kMaxPaths];    // k-th path is the group's first with its l2
+    bool last_l2[kMaxPaths];     // k-th path is the group's last with its l2
+    int rlo, rhi;                // rows [rlo, rhi) of the gathered node tensor
+  };
+  static constexpr Data make() {
+    Data d{};
+    int lo = 99, hi = -1;
+    for (int b = 0; b <= PS::LS; ++b)
+      for (int p = 0; p < PS::D.np; ++p) {
+        if (PS::D.l2[p] != b) continue;
+        if (KIND != kAll && (KIND == kByL1 ? PS::D.l1[p] : PS::D.l3[p]) != V) continue;
+        d.path[d.n++] = p;
+        const int lo_other = KIND == kByL1 ? PS::D.l3[p] : PS::D.l1[p];
+        lo = lo_other < lo ? lo_other : lo;
+        hi = lo_other > hi ? lo_other : hi;
+      }
+    d.lt[0] = 0;
+    for (int k = 0; k < d.n; ++k) {
+      d.lt[k + 1] = d.lt[k] + (PS::D.tcount[d.path[k]] + 3) / 4 * 4;
+      d.first_l2[k] = k == 0 || PS::D.l2[d.path[k - 1]] != PS::D.l2[d.path[k]];
+      d.last_l2[k] = k + 1 == d.n || PS::D.l2[d.path[k + 1]] != PS::D.l2[d.path[k]];
+    }
+    d.rlo = d.n ? lo * lo : 0;
+    d.rhi = d.n ? (hi + 1) * (hi + 1) : 0;
+    return d;
+  }
+  static constexpr Data D = make();
+  static constexpr int NP = D.n;
+  static constexpr int NT = D.lt[D.n] > 0 ? D.lt[D.n] : 4;  // T floats per edge
+  static constexpr int NROW = D.rhi - D.rlo;              // gathered node rows
+  // rows of the group's own block (all output rows for kAll)
+  static constexpr int NOWN = KIND == kAll ? PS::NO : 2 * V + 1;
+  static constexpr int OWN0 = KIND == kAll ? 0 : V * V;    // first own row
+};
+
+// T^p[m1][m3] = sum_m2 C^p[m1,m2,m3] Y[l2,m2] for the group's paths, packed
+// per path in (m3, m1) order, each path padded to a multiple of 4 floats.
+template <class PS, class GR>
+__device__ __forceinline__ void compute_T_grp(const float (&Y)[PS::NS], float* __restrict__ T) {
+  static_for<0, GR::NP>([&](auto Kc) {
+    constexpr int K = decltype(Kc)::value;
+    constexpr int P = GR::D.path[K];
+    constexpr int l1 = PS::D.l1[P], l2 = PS::D.l2[P], l3 = PS::D.l3[P];
+    constexpr int tc = PS::D.tcount[P], base = GR::D.lt[K];
+    static_for<0, tc>([&](auto Ec) {
+      constexpr int k = decltype(Ec)::value;
+      constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
+      float v = 0.f;
+      static_for<0, 2 * l2 + 1>([&](auto M2c) {
+        constexpr int m2 = decltype(M2c)::value - l2;
+        if constexpr (cg_allowed(l1, l2, l3, m1, m2, m3)) {
+          v = fmaf(c_cg[table_index(l1, l2, l3, m1, m2, m3)], Y[l2 * l2 + l2 + m2], v);
+        }
+      });
+      T[base + k] = v;
+    });
+    static_for<base + tc, GR::D.lt[K + 1]>([&](auto Zc) { T[decltype(Zc)::value] = 0.f; });
+  });
+}
+
+// Edges per batch: T matrices of BT edges per group of lanes, sized so that a
+// group's shared memory stays near 24 KB.
+inline int pick_batch(int gpw, int t_floats, int stage_floats, int budget_floats = 6144) {
+  const int budget = budget_floats / gpw - 2 * stage_floats;
+  int bt = budget / (t_floats + 3);
+  if (bt > 16) bt = 16;
+  return bt < 1 ? 1 : bt;
+}
+
+// Channel lanes per group (G, a power of two <= 32) and channel slices S for
+// mult channels at VEC channels per lane.
+inline void lane_geometry(int mult, int vec, int& G, int& lg_G, int& S) {
+  const int lanes = mult / vec;
+  G = 1;
+  while (G < 32 && lanes % (2 * G) == 0) G *= 2;
+  lg_G = 0;
+  while ((1 << lg_G) < G) ++lg_G;
+  S = lanes / G;
+}
+
+}  // namespace cgtp

@@ -5,115 +5,132 @@
 //
 // ("LunaTP: Enabling Efficient and Scalable Tensor Product for Equivariant
 // MLIPs", abstract: node-centric execution, path-group parallelism and reuse;
-// this kernel is our own design for the B200.)
+// the kernel below is our own design for the B200.)
 //
-// Mapping.  A group of G lanes (G a power of two <= 32) owns one (row, channel
-// slice) work item; each lane owns 4 consecutive channels (float4).  The
-// group walks its row's edges in batches of BT: first every lane computes the
-// harmonics and the packed T matrices of one edge of the batch (channel
-// independent, coefficients from constant memory, so a batch costs one pass
-// of this code whatever its size) into shared memory; then all lanes sweep
-// the batch, streaming W_e (the dominant HBM stream, read once with an
-// evict-first hint), gathering x_j (L2 resident), and accumulating the
-// output row in registers.  Each output element is written once; there are
-// no atomics.  The loops over paths, m3 and m1 are unrolled at compile time
-// over the structural nonzero pattern of the real CG coefficients, so every
-// register index is static.
+// Mapping.  A group of G lanes (G a power of two <= 32) owns one
+// (row, channel slice) work item; each lane owns 4 consecutive channels.
+// (Optionally one launch per output block l3, each over that block's paths.)
+// The lanes walk the row's edges in batches of BT: first every lane
+// computes the harmonics and the group's packed T matrices of one edge of
+// the batch (channel independent; coefficients are constant-memory operands)
+// into shared memory; then the lanes sweep the batch with a two-stage
+// pipeline: while edge k is computed, each lane's cp.async copies of edge
+// k+1's weight rows (the HBM stream, read once) and of its source's feature
+// rows (L2 resident) land in shared memory.  The output rows accumulate in
+// registers and are written once; there are no atomics.  Loops over paths
+// and over the structural nonzeros of T are unrolled at compile time, so
+// every register index is static.
 #include "common.cuh"
 
 namespace cgtp {
 CGTP_DEFINE_CONSTANT_TABLES()
 }  // namespace cgtp
 
+#include "conv_common.cuh"
 #include "sh.cuh"
 
 namespace cgtp {
-
 namespace {
 
 constexpr int kFwdThreads = 128;
+constexpr int kFwdVec = 4;
 
-// T matrices of one edge from its harmonics (packed layout of PathSet).
-template <class PS>
-__device__ __forceinline__ void compute_T(const float (&Y)[PS::NS], float* __restrict__ T) {
-  static_for<0, PS::NP>([&](auto Pc) {
-    constexpr int P = decltype(Pc)::value;
-    constexpr int l1 = PS::D.l1[P], l2 = PS::D.l2[P], l3 = PS::D.l3[P];
-    static_for<0, 2 * l3 + 1>([&](auto M3c) {
-      constexpr int m3 = decltype(M3c)::value - l3;
-      static_for<0, 2 * l1 + 1>([&](auto M1c) {
-        constexpr int m1 = decltype(M1c)::value - l1;
-        constexpr int ti = PS::t_index(P, m1, m3);
-        if constexpr (ti >= 0) {
-          float v = 0.f;
-          static_for<0, 2 * l2 + 1>([&](auto M2c) {
-            constexpr int m2 = decltype(M2c)::value - l2;
-            if constexpr (cg_allowed(l1, l2, l3, m1, m2, m3)) {
-              constexpr int ci = table_index(l1, l2, l3, m1, m2, m3);
-              v = fmaf(c_cg[ci], Y[l2 * l2 + l2 + m2], v);
-            }
-          });
-          T[ti] = v;
-        }
-      });
-    });
-    // zero the padding so that float4 reads of the block see finite values
-    static_for<PS::D.tbase[P] + PS::D.tcount[P], PS::D.tbase[P + 1]>([&](auto Kc) {
-      T[decltype(Kc)::value] = 0.f;
-    });
-  });
-}
+// Stage x rows through the cp.async pipeline (1) or gather them with cached
+// loads after an L2 prefetch (0); path groups by l3 (1) or one group (0).
+#ifndef CGTP_FWD_STAGE_X
+#define CGTP_FWD_STAGE_X 1
+#endif
+#ifndef CGTP_FWD_GROUPED
+#define CGTP_FWD_GROUPED 0
+#endif
+constexpr bool kStageX = CGTP_FWD_STAGE_X != 0;
 
-// One edge: acc[l3,m3][c] += sum_p W[p][c] sum_m1 T[p][m1][m3] x[l1,m1][c].
-template <class PS>
-__device__ __forceinline__ void fwd_edge(const float* __restrict__ T, const float (&xr)[PS::NI][4],
-                                         const float* __restrict__ wrow, int mult,
-                                         float (&acc)[PS::NO][4]) {
-  static_for<0, PS::NP>([&](auto Pc) {
-    constexpr int P = decltype(Pc)::value;
+// One edge: acc[m3][c] += sum_p W[p][c] sum_m1 T[p][m1][m3] x[l1,m1][c] for the group's paths.
+template <class PS, class GR>
+__device__ __forceinline__ void fwd_edge(const float* __restrict__ T, const float* __restrict__ stage, int rowf,
+                                         const float* __restrict__ xg, int mult,
+                                         float (&acc)[GR::NOWN][kFwdVec]) {
+  float xr[GR::NROW][kFwdVec];
+#pragma unroll
+  for (int r = 0; r < GR::NROW; ++r) {
+    if constexpr (kStageX) VecIO<kFwdVec>::lds(xr[r], stage + (GR::NP + r) * rowf);
+    else VecIO<kFwdVec>::ld(xr[r], xg + r * mult);
+  }
+  static_for<0, GR::NP>([&](auto Kc) {
+    constexpr int K = decltype(Kc)::value;
+    constexpr int P = GR::D.path[K];
     constexpr int l1 = PS::D.l1[P], l3 = PS::D.l3[P];
-    constexpr int tb = PS::D.tbase[P], tn = PS::D.tbase[P + 1] - PS::D.tbase[P];
-    float wv[4];
-    f4_to(wv, ld_stream(wrow + P * mult));
-    float tl[tn > 0 ? tn : 4];
-    static_for<0, tn / 4>([&](auto Qc) {
-      constexpr int q = decltype(Qc)::value;
-      const float4 v = *reinterpret_cast<const float4*>(T + tb + 4 * q);
-      tl[4 * q + 0] = v.x;
-      tl[4 * q + 1] = v.y;
-      tl[4 * q + 2] = v.z;
-      tl[4 * q + 3] = v.w;
-    });
-    static_for<0, 2 * l3 + 1>([&](auto M3c) {
-      constexpr int m3 = decltype(M3c)::value - l3;
-      float t[4] = {0.f, 0.f, 0.f, 0.f};
-      static_for<0, 2 * l1 + 1>([&](auto M1c) {
-        constexpr int m1 = decltype(M1c)::value - l1;
-        constexpr int ti = PS::t_index(P, m1, m3);
-        if constexpr (ti >= 0) {
+    constexpr int tc = PS::D.tcount[P], tb = GR::D.lt[K];
+    float wv[kFwdVec];
+    VecIO<kFwdVec>::lds(wv, stage + K * rowf);
+    constexpr int o3 = l3 * l3 - GR::OWN0;  // first own row of this path's output block
+    if constexpr (2 * l3 + 1 <= 2 * l1 + 1) {
+      // t[m3] = sum_m1 T x[m1], then out[m3] += W t[m3]
+      float t[2 * l3 + 1][kFwdVec];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) t[c] = fmaf(tl[ti - tb], xr[l1 * l1 + l1 + m1][c], t[c]);
-        }
+      for (int m3 = 0; m3 < 2 * l3 + 1; ++m3)
+#pragma unroll
+        for (int c = 0; c < kFwdVec; ++c) t[m3][c] = 0.f;
+      static_for<0, (tc + 3) / 4>([&](auto Qc) {
+        constexpr int q = decltype(Qc)::value;
+        const float4 v4 = *reinterpret_cast<const float4*>(T + tb + 4 * q);
+        const float tv4[4] = {v4.x, v4.y, v4.z, v4.w};
+        static_for<0, 4>([&](auto Rc) {
+          constexpr int k = 4 * q + decltype(Rc)::value;
+          if constexpr (k < tc) {
+            constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
+            constexpr int rx = l1 * l1 + l1 + m1 - GR::D.rlo;
+#pragma unroll
+            for (int c = 0; c < kFwdVec; ++c) t[m3 + l3][c] = fmaf(tv4[decltype(Rc)::value], xr[rx][c], t[m3 + l3][c]);
+          }
+        });
       });
 #pragma unroll
-      for (int c = 0; c < 4; ++c) acc[l3 * l3 + l3 + m3][c] = fmaf(wv[c], t[c], acc[l3 * l3 + l3 + m3][c]);
-    });
+      for (int m3 = 0; m3 < 2 * l3 + 1; ++m3)
+#pragma unroll
+        for (int c = 0; c < kFwdVec; ++c) acc[o3 + m3][c] = fmaf(wv[c], t[m3][c], acc[o3 + m3][c]);
+    } else {
+      // xw[m1] = W x[m1], then out[m3] += sum_m1 T xw[m1]
+      float xw[2 * l1 + 1][kFwdVec];
+#pragma unroll
+      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1)
+#pragma unroll
+        for (int c = 0; c < kFwdVec; ++c) xw[m1][c] = wv[c] * xr[l1 * l1 + m1 - GR::D.rlo][c];
+      static_for<0, (tc + 3) / 4>([&](auto Qc) {
+        constexpr int q = decltype(Qc)::value;
+        const float4 v4 = *reinterpret_cast<const float4*>(T + tb + 4 * q);
+        const float tv4[4] = {v4.x, v4.y, v4.z, v4.w};
+        static_for<0, 4>([&](auto Rc) {
+          constexpr int k = 4 * q + decltype(Rc)::value;
+          if constexpr (k < tc) {
+            constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
+#pragma unroll
+            for (int c = 0; c < kFwdVec; ++c)
+              acc[o3 + m3 + l3][c] = fmaf(tv4[decltype(Rc)::value], xw[m1 + l1][c], acc[o3 + m3 + l3][c]);
+          }
+        });
+      });
+    }
   });
 }
 
-template <class PS>
+template <class PS, int KIND, int L3>
 __global__ void __launch_bounds__(kFwdThreads)
-conv_fwd_kernel(ConvFwdArgs a, int lg_G, int S, int BT, int tstride) {
-  constexpr int NI = PS::NI, NO = PS::NO, NS = PS::NS;
+conv_fwd_kernel(ConvFwdArgs a, int lg_G, int S, int BT) {
+  using GR = Grp<PS, KIND, L3>;
+  constexpr int NI = PS::NI, NO = PS::NO, NS = PS::NS, NT = GR::NT;
+  constexpr int NROWS = GR::NP + (kStageX ? GR::NROW : 0);
   extern __shared__ float4 smem_f4[];
   float* smem = reinterpret_cast<float*>(smem_f4);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int G = 1 << lg_G, gpw = 32 >> lg_G;
   const int grp = lane >> lg_G, gl = lane & (G - 1);
-  // per group: BT rows of T (stride tstride floats, 16-byte aligned) + BT source ids
-  const int group_floats = BT * tstride + ((BT + 3) & ~3);
+  const int rowf = G * kFwdVec;                    // floats per staged row
+  const int stage_floats = NROWS * rowf;
+  const int group_floats = BT * NT + 2 * stage_floats + ((BT + 3) & ~3);
   float* Tg = smem + (warp * gpw + grp) * group_floats;
-  int* Jg = reinterpret_cast<int*>(Tg + BT * tstride);
+  float* St = Tg + BT * NT;                        // two pipeline stages
+  int* Jg = reinterpret_cast<int*>(St + 2 * stage_floats);
 
   const long long n_items = (long long)a.n_nodes * S;
   const long long warps_total = (long long)gridDim.x * (kFwdThreads / 32);
@@ -123,16 +140,37 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G, int S, int BT, int tstride) {
     const bool active = item < n_items;
     const int node = active ? int(item / S) : 0;
     const int slice = active ? int(item % S) : 0;
-    const int c0 = (slice * G + gl) * 4;
+    const int c0 = (slice * G + gl) * kFwdVec;
     int e0 = 0, e1 = 0;
     if (active) {
       e0 = __ldg(a.row_ptr + node);
       e1 = __ldg(a.row_ptr + node + 1);
     }
     const int maxdeg = __reduce_max_sync(0xffffffffu, e1 - e0);
-    float acc[NO][4];
+    float acc[GR::NOWN][kFwdVec];
 #pragma unroll
-    for (int k = 0; k < NO; ++k) acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.f;
+    for (int r = 0; r < GR::NOWN; ++r)
+#pragma unroll
+      for (int c = 0; c < kFwdVec; ++c) acc[r][c] = 0.f;
+
+    // copies of edge slot k of the current batch into stage s (this lane's channels only)
+    auto issue = [&](int b0, int k, int s) {
+      const int e = e0 + b0 + k;
+      if (!(active && e < e1)) return;
+      float* dst = St + s * stage_floats + gl * kFwdVec;
+      const float* wrow = a.w + (long long)e * PS::NP * a.mult + c0;
+      static_for<0, GR::NP>([&](auto Kc) {
+        constexpr int K = decltype(Kc)::value;
+        constexpr int P = GR::D.path[K];
+        VecIO<kFwdVec>::cp_async(dst + K * rowf, wrow + P * a.mult);
+      });
+      if constexpr (kStageX) {
+        constexpr int rlo = GR::D.rlo;
+        const float* xrow = a.x + ((long long)Jg[k] * NI + rlo) * a.mult + c0;
+#pragma unroll
+        for (int r = 0; r < GR::NROW; ++r) VecIO<kFwdVec>::cp_async(dst + (GR::NP + r) * rowf, xrow + r * a.mult);
+      }
+    };
 
     for (int b0 = 0; b0 < maxdeg; b0 += BT) {
       for (int k = gl; k < BT; k += G) {
@@ -141,28 +179,68 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G, int S, int BT, int tstride) {
           float Y[NS];
           sh_of_vec<PS::LS>(__ldg(a.edge_vec + 3 * (long long)e), __ldg(a.edge_vec + 3 * (long long)e + 1),
                             __ldg(a.edge_vec + 3 * (long long)e + 2), Y);
-          compute_T<PS>(Y, Tg + k * tstride);
-          Jg[k] = __ldg(a.col + e);
+          compute_T_grp<PS, GR>(Y, Tg + k * NT);
+          const int j = __ldg(a.col + e);
+          if constexpr (!kStageX) {
+            constexpr int rlo = GR::D.rlo;
+            prefetch_l2(a.x + ((long long)j * NI + rlo) * a.mult, (unsigned)(GR::NROW * a.mult * 4));
+          }
+          Jg[k] = j;
         }
       }
       __syncwarp();
       const int nb = min(BT, maxdeg - b0);
+      issue(b0, 0, 0);
+      cp_async_commit();
       for (int k = 0; k < nb; ++k) {
-        const int e = e0 + b0 + k;
-        if (active && e < e1) {
-          const long long j = Jg[k];
-          float xr[NI][4];
-#pragma unroll
-          for (int r = 0; r < NI; ++r) f4_to(xr[r], ld_ro(a.x + (j * NI + r) * a.mult + c0));
-          fwd_edge<PS>(Tg + k * tstride, xr, a.w + (long long)e * PS::NP * a.mult + c0, a.mult, acc);
+        if (k + 1 < nb) issue(b0, k + 1, (k + 1) & 1);
+        cp_async_commit();
+        cp_async_wait<1>();  // this lane's copies of edge k have landed
+        if (active && e0 + b0 + k < e1) {
+          constexpr int rlo = GR::D.rlo;
+          fwd_edge<PS, GR>(Tg + k * NT, St + (k & 1) * stage_floats + gl * kFwdVec, rowf,
+                           a.x + ((long long)Jg[k] * NI + rlo) * a.mult + c0, a.mult, acc);
         }
       }
       __syncwarp();
     }
     if (active) {
 #pragma unroll
-      for (int r = 0; r < NO; ++r) st_f4(a.out + ((long long)node * NO + r) * a.mult + c0, to_f4(acc[r]));
+      for (int r = 0; r < GR::NOWN; ++r)
+        VecIO<kFwdVec>::st(a.out + ((long long)node * NO + GR::OWN0 + r) * a.mult + c0, acc[r]);
     }
+  }
+}
+
+template <class PS, int KIND, int L3>
+cudaError_t launch_fwd_group(const ConvFwdArgs& a, int num_sms, cudaStream_t stream) {
+  using GR = Grp<PS, KIND, L3>;
+  if constexpr (GR::NP == 0) {  // no path reaches this output block: it is zero
+    return cudaMemset2DAsync(a.out + (size_t)GR::OWN0 * a.mult, sizeof(float) * PS::NO * a.mult, 0,
+                             sizeof(float) * GR::NOWN * a.mult, a.n_nodes, stream);
+  } else {
+    int G, lg_G, S;
+    lane_geometry(a.mult, kFwdVec, G, lg_G, S);
+    const int gpw = 32 / G;
+    const int stage_floats = (GR::NP + (kStageX ? GR::NROW : 0)) * G * kFwdVec;
+    const int BT = pick_batch(gpw, GR::NT, stage_floats, KIND == kAll ? 12288 : 6144);
+    const int group_floats = BT * GR::NT + 2 * stage_floats + ((BT + 3) & ~3);
+    const size_t smem = sizeof(float) * (size_t)group_floats * gpw * (kFwdThreads / 32);
+    auto kern = conv_fwd_kernel<PS, KIND, L3>;
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFwdThreads, smem);
+    if (err != cudaSuccess) return err;
+    if (per_sm < 1) per_sm = 1;
+    const long long items = (long long)a.n_nodes * S;
+    const long long groups_per_block = (long long)gpw * (kFwdThreads / 32);
+    long long blocks = (items + groups_per_block - 1) / groups_per_block;
+    const long long cap = (long long)num_sms * per_sm;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    kern<<<(unsigned)blocks, kFwdThreads, smem, stream>>>(a, lg_G, S, BT);
+    return cudaGetLastError();
   }
 }
 
@@ -171,34 +249,15 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G, int S, int BT, int tstride) {
 template <int LI, int LS, int LO>
 cudaError_t launch_conv_fwd(const ConvFwdArgs& a, int num_sms, cudaStream_t stream) {
   using PS = PathSet<LI, LS, LO>;
-  const int lanes = a.mult / 4;
-  int G = 1;
-  while (G < 32 && lanes % (2 * G) == 0) G *= 2;
-  int lg_G = 0;
-  while ((1 << lg_G) < G) ++lg_G;
-  const int S = lanes / G;
-  const int gpw = 32 / G;
-  const int tstride = PS::NT > 0 ? PS::NT : 4;
-  // batch size: about 16 KB of T per warp, at least one edge per lane when possible
-  int BT = 4096 / (gpw * tstride);
-  BT = BT < 1 ? 1 : (BT > 32 ? 32 : BT);
-  const int group_floats = BT * tstride + ((BT + 3) & ~3);
-  const size_t smem = sizeof(float) * (size_t)group_floats * gpw * (kFwdThreads / 32);
-  auto kern = conv_fwd_kernel<PS>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (err != cudaSuccess) return err;
-  int per_sm = 0;
-  err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFwdThreads, smem);
-  if (err != cudaSuccess) return err;
-  if (per_sm < 1) per_sm = 1;
-  const long long items = (long long)a.n_nodes * S;
-  const long long groups_per_block = (long long)gpw * (kFwdThreads / 32);
-  long long blocks = (items + groups_per_block - 1) / groups_per_block;
-  const long long cap = (long long)num_sms * per_sm;
-  if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
-  kern<<<(unsigned)blocks, kFwdThreads, smem, stream>>>(a, lg_G, S, BT, tstride);
-  return cudaGetLastError();
+  if constexpr (CGTP_FWD_GROUPED == 0) {
+    return launch_fwd_group<PS, kAll, 0>(a, num_sms, stream);
+  } else {
+    cudaError_t err = cudaSuccess;
+    static_for_host<0, LO + 1>([&](auto Lc) {
+      if (err == cudaSuccess) err = launch_fwd_group<PS, kByL3, decltype(Lc)::value>(a, num_sms, stream);
+    });
+    return err;
+  }
 }
 
 // One translation unit per shape (the build passes CGTP_CFG_LI/LS/LO).
