@@ -122,12 +122,20 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
   });
 }
 
-// One launch per path group (the paths with l1 = L1): grad_x rows of that
-// block, grad_W of those paths and a partial grad_Y over those paths.
-template <class PS, int VEC, bool NEED_GY, int L1>
+// Unrolled instructions per edge and lane allowed in one backward launch.
+constexpr int kBwdBudget = 1100;
+
+template <class PS, int VEC, bool NEED_GY>
+using BwdPlan = Plan<PS, kByL1, VEC, NEED_GY, kBwdBudget>;
+
+// One launch per chunk (paths of one l1 block): grad_x rows of that block
+// (written by the block's first chunk, accumulated by the others), grad_W
+// of the chunk's paths and a partial grad_Y over them.
+template <class PS, int VEC, bool NEED_GY, int CH>
 __global__ void __launch_bounds__(kBwdThreads)
 conv_bwd_kernel(ConvBwdArgs a, int lg_G, int S, int BT, int slice_base) {
-  using GR = Grp<PS, kByL1, L1>;
+  using GR = ChunkGrp<PS, BwdPlan<PS, VEC, NEED_GY>, CH, kByL1>;
+  constexpr int L1 = GR::KEY;
   constexpr int NI = PS::NI, NO = PS::NO, NS = PS::NS, NR = GR::NOWN, NT = GR::NT;
   constexpr int NROWS = GR::NP + GR::NROW;
   constexpr int NSP = NS | 1;  // odd row stride: conflict-free transposed reduction
@@ -169,8 +177,12 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G, int S, int BT, int slice_base) {
 #pragma unroll
         for (int c = 0; c < VEC; ++c) xr[r][c] = 0.f;
       }
+      if (!GR::FIRST && active && a.grad_x != nullptr) {
+        VecIO<VEC>::ld(gx[r], a.grad_x + (node * NI + L1 * L1 + r) * a.mult + c0);
+      } else {
 #pragma unroll
-      for (int c = 0; c < VEC; ++c) gx[r][c] = 0.f;
+        for (int c = 0; c < VEC; ++c) gx[r][c] = 0.f;
+      }
     }
 
     // copies of edge slot k of the current batch into stage s (this lane's channels only)
@@ -307,65 +319,73 @@ int conv_bwd_slices(int mult) {
   using PS = PathSet<LI, LS, LO>;
   int G, lg_G, S;
   bwd_geometry<PS>(mult, G, lg_G, S);
-  return S * (LI + 1);  // one partial grad_Y per (path group, channel slice)
+  return S * BwdPlan<PS, bwd_vec<PS>(), true>::N;  // one partial grad_Y per (chunk, channel slice)
 }
 
-template <class PS, int L1>
-cudaError_t launch_bwd_group(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
-  using GR = Grp<PS, kByL1, L1>;
+template <class PS, bool NEED_GY, int CH>
+cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
   constexpr int VEC = bwd_vec<PS>();
+  using GR = ChunkGrp<PS, BwdPlan<PS, VEC, NEED_GY>, CH, kByL1>;
   constexpr int NSP = PS::NS | 1;
   int G, lg_G, S;
   bwd_geometry<PS>(a.mult, G, lg_G, S);
-  const bool need_gy = a.grad_edge_vec != nullptr;
-  if constexpr (GR::NP == 0) {  // no path starts from this l1 block: its gradient is zero
-    if (a.grad_x != nullptr) {
-      cudaError_t e = cudaMemset2DAsync(a.grad_x + (size_t)L1 * L1 * a.mult, sizeof(float) * PS::NI * a.mult, 0,
-                                        sizeof(float) * GR::NOWN * a.mult, a.n_nodes, stream);
-      if (e != cudaSuccess) return e;
-    }
-    if (need_gy)
-      for (int s = 0; s < S; ++s) {
-        cudaError_t e = cudaMemsetAsync(a.grad_sh + (size_t)(L1 * S + s) * a.n_edges * PS::NS, 0,
-                                        sizeof(float) * (size_t)a.n_edges * PS::NS, stream);
-        if (e != cudaSuccess) return e;
-      }
-    return cudaSuccess;
-  } else {
-    const int gpw = 32 / G;
-    const int stage_floats = (GR::NP + GR::NROW) * G * VEC;
-    const int BT = pick_batch(gpw, GR::NT, stage_floats);
-    const int group_floats = BT * GR::NT + 2 * stage_floats + 2 * ((BT + 3) & ~3);
-    const size_t smem = sizeof(float) * ((size_t)group_floats * gpw * (kBwdThreads / 32) +
-                                         (need_gy ? (size_t)(kBwdThreads / 32) * 32 * NSP : 0));
-    const long long items = (long long)a.n_nodes * S;
-    const long long groups_per_block = (long long)gpw * (kBwdThreads / 32);
-    const long long blocks = (items + groups_per_block - 1) / groups_per_block;
-    auto run = [&](auto kern) -> cudaError_t {
-      cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e2 != cudaSuccess) return e2;
-      int per_sm = 0;
-      e2 = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBwdThreads, smem);
-      if (e2 != cudaSuccess) return e2;
-      if (per_sm < 1) per_sm = 1;
-      const long long cap = (long long)num_sms * per_sm;
-      long long nb = blocks > cap ? cap : blocks;
-      if (nb < 1) nb = 1;
-      kern<<<(unsigned)nb, kBwdThreads, smem, stream>>>(a, lg_G, S, BT, L1 * S);
-      return cudaGetLastError();
-    };
-    if (need_gy) return run(conv_bwd_kernel<PS, VEC, true, L1>);
-    return run(conv_bwd_kernel<PS, VEC, false, L1>);
-  }
+  const int gpw = 32 / G;
+  const int stage_floats = (GR::NP + GR::NROW) * G * VEC;
+  const int BT = pick_batch(gpw, GR::NT, stage_floats);
+  const int group_floats = BT * GR::NT + 2 * stage_floats + 2 * ((BT + 3) & ~3);
+  const size_t smem = sizeof(float) * ((size_t)group_floats * gpw * (kBwdThreads / 32) +
+                                       (NEED_GY ? (size_t)(kBwdThreads / 32) * 32 * NSP : 0));
+  const long long items = (long long)a.n_nodes * S;
+  const long long groups_per_block = (long long)gpw * (kBwdThreads / 32);
+  const long long blocks = (items + groups_per_block - 1) / groups_per_block;
+  auto kern = conv_bwd_kernel<PS, VEC, NEED_GY, CH>;
+  cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e2 != cudaSuccess) return e2;
+  int per_sm = 0;
+  e2 = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBwdThreads, smem);
+  if (e2 != cudaSuccess) return e2;
+  if (per_sm < 1) per_sm = 1;
+  const long long cap = (long long)num_sms * per_sm;
+  long long nb = blocks > cap ? cap : blocks;
+  if (nb < 1) nb = 1;
+  kern<<<(unsigned)nb, kBwdThreads, smem, stream>>>(a, lg_G, S, BT, CH * S);
+  return cudaGetLastError();
+}
+
+// grad_x blocks that no path reaches (l1 with no path) are zero.
+template <class PS>
+cudaError_t zero_unreached_grad_x(const ConvBwdArgs& a, cudaStream_t stream) {
+  if (a.grad_x == nullptr) return cudaSuccess;
+  cudaError_t err = cudaSuccess;
+  static_for_host<0, PS::LI + 1>([&](auto Lc) {
+    constexpr int l1 = decltype(Lc)::value;
+    constexpr bool reached = [] {
+      for (int p = 0; p < PS::D.np; ++p)
+        if (PS::D.l1[p] == l1) return true;
+      return false;
+    }();
+    if (!reached && err == cudaSuccess)
+      err = cudaMemset2DAsync(a.grad_x + (size_t)l1 * l1 * a.mult, sizeof(float) * PS::NI * a.mult, 0,
+                              sizeof(float) * (2 * l1 + 1) * a.mult, a.n_nodes, stream);
+  });
+  return err;
+}
+
+template <class PS, bool NEED_GY>
+cudaError_t launch_bwd_chunks(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
+  constexpr int NCH = BwdPlan<PS, bwd_vec<PS>(), NEED_GY>::N;
+  cudaError_t err = zero_unreached_grad_x<PS>(a, stream);
+  static_for_host<0, NCH>([&](auto Cc) {
+    if (err == cudaSuccess) err = launch_bwd_chunk<PS, NEED_GY, decltype(Cc)::value>(a, num_sms, stream);
+  });
+  return err;
 }
 
 template <int LI, int LS, int LO>
 cudaError_t launch_conv_bwd(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
   using PS = PathSet<LI, LS, LO>;
-  cudaError_t err = cudaSuccess;
-  static_for_host<0, LI + 1>([&](auto Lc) {
-    if (err == cudaSuccess) err = launch_bwd_group<PS, decltype(Lc)::value>(a, num_sms, stream);
-  });
+  const cudaError_t err = a.grad_edge_vec != nullptr ? launch_bwd_chunks<PS, true>(a, num_sms, stream)
+                                                     : launch_bwd_chunks<PS, false>(a, num_sms, stream);
   if (err != cudaSuccess || a.grad_edge_vec == nullptr || a.n_edges == 0) return err;
   const int threads = 256;
   long long nbk = (a.n_edges + threads - 1) / threads;

@@ -117,6 +117,104 @@ __device__ __forceinline__ void compute_T_grp(const float (&Y)[PS::NS], float* _
   });
 }
 
+// ---- chunks: the launches of a kernel family ----
+// Paths sorted by (key, l2, lexicographic), key = l1 (backward) or l3
+// (forward), are cut into runs with one key value whose unrolled code per
+// edge stays below a budget: a loop body much larger than about 20 KB of
+// instructions stops fitting the instruction cache and the warps stall on
+// instruction fetch.  Every run is one launch; the first run of a key
+// initialises that key's block of rows, later runs add to it.
+struct ChunkPlan {
+  int n;                        // chunks
+  int key[kMaxPaths];           // key value (l1 or l3) of chunk c
+  int first[kMaxPaths];         // chunk c is order[first[c] .. first[c] + count[c])
+  int count[kMaxPaths];
+  bool first_of_key[kMaxPaths];
+  int order[kMaxPaths];         // paths sorted by (key, l2, lexicographic)
+};
+
+// Estimated unrolled instructions per edge and lane for one path.
+template <class PS>
+constexpr int path_cost(int p, int kind, int vec, bool gy) {
+  const int tc = PS::D.tcount[p], n1 = 2 * PS::D.l1[p] + 1, n3 = 2 * PS::D.l3[p] + 1;
+  if (kind == kByL3) return tc * vec + (tc + 3) / 4 + 1 + (n1 < n3 ? n1 : n3) * vec + 4;
+  return tc * vec + (gy ? tc * vec + path_entries(PS::D.l1[p], PS::D.l2[p], PS::D.l3[p]) + n1 * vec : 0) +
+         (tc + 3) / 4 + n3 + 2 * n1 * vec + 6;
+}
+
+template <class PS>
+constexpr ChunkPlan make_chunk_plan(int kind, int vec, bool gy, int budget) {
+  ChunkPlan c{};
+  int k = 0;
+  const int kmax = kind == kByL1 ? PS::LI : PS::LO;
+  for (int key = 0; key <= kmax; ++key)
+    for (int b = 0; b <= PS::LS; ++b)
+      for (int p = 0; p < PS::D.np; ++p)
+        if (PS::D.l2[p] == b && (kind == kByL1 ? PS::D.l1[p] : PS::D.l3[p]) == key) c.order[k++] = p;
+  int start = 0;
+  while (start < k) {
+    const int key = kind == kByL1 ? PS::D.l1[c.order[start]] : PS::D.l3[c.order[start]];
+    int end = start, cost = 0;
+    while (end < k && (kind == kByL1 ? PS::D.l1[c.order[end]] : PS::D.l3[c.order[end]]) == key) {
+      const int pc = path_cost<PS>(c.order[end], kind, vec, gy);
+      if (end > start && cost + pc > budget) break;
+      cost += pc;
+      ++end;
+    }
+    c.key[c.n] = key;
+    c.first[c.n] = start;
+    c.count[c.n] = end - start;
+    c.first_of_key[c.n] = c.n == 0 || c.key[c.n - 1] != key;
+    ++c.n;
+    start = end;
+  }
+  return c;
+}
+
+template <class PS, int KIND, int VEC, bool GY, int BUDGET>
+struct Plan {
+  static constexpr ChunkPlan P = make_chunk_plan<PS>(KIND, VEC, GY, BUDGET);
+  static constexpr int N = P.n;
+};
+
+// The paths of chunk CH of plan PL, with the same interface as Grp.
+template <class PS, class PL, int CH>
+struct Chunk {
+  using Data = typename Grp<PS, kAll, 0>::Data;
+  static constexpr int KEY = PL::P.key[CH];
+  static constexpr bool FIRST = PL::P.first_of_key[CH];
+  static constexpr Data make(bool by_l1) {
+    Data d{};
+    int lo = 99, hi = -1;
+    for (int k = 0; k < PL::P.count[CH]; ++k) {
+      const int p = PL::P.order[PL::P.first[CH] + k];
+      d.path[d.n++] = p;
+      const int other = by_l1 ? PS::D.l3[p] : PS::D.l1[p];
+      lo = other < lo ? other : lo;
+      hi = other > hi ? other : hi;
+    }
+    d.lt[0] = 0;
+    for (int k = 0; k < d.n; ++k) {
+      d.lt[k + 1] = d.lt[k] + (PS::D.tcount[d.path[k]] + 3) / 4 * 4;
+      d.first_l2[k] = k == 0 || PS::D.l2[d.path[k - 1]] != PS::D.l2[d.path[k]];
+      d.last_l2[k] = k + 1 == d.n || PS::D.l2[d.path[k + 1]] != PS::D.l2[d.path[k]];
+    }
+    d.rlo = d.n ? lo * lo : 0;
+    d.rhi = d.n ? (hi + 1) * (hi + 1) : 0;
+    return d;
+  }
+};
+template <class PS, class PL, int CH, int KIND>
+struct ChunkGrp : Chunk<PS, PL, CH> {
+  using Base = Chunk<PS, PL, CH>;
+  static constexpr typename Base::Data D = Base::make(KIND == kByL1);
+  static constexpr int NP = D.n;
+  static constexpr int NT = D.lt[D.n] > 0 ? D.lt[D.n] : 4;
+  static constexpr int NROW = D.rhi - D.rlo;
+  static constexpr int NOWN = 2 * Base::KEY + 1;
+  static constexpr int OWN0 = Base::KEY * Base::KEY;
+};
+
 // Edges per batch: T matrices of BT edges per group of lanes, sized so that a
 // group's shared memory stays near 24 KB.
 inline int pick_batch(int gpw, int t_floats, int stage_floats, int budget_floats = 6144) {
