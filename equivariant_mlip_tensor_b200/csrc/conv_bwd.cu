@@ -32,10 +32,13 @@ namespace {
 constexpr int kBwdThreads = 128;
 
 template <class PS, class GR>
-constexpr bool grp_has_l2(int l2) {
-  for (int k = 0; k < GR::D.n; ++k)
-    if (PS::D.l2[GR::D.path[k]] == l2) return true;
-  return false;
+constexpr unsigned touched_sh_mask() {
+  unsigned m = 0;
+  for (int k = 0; k < GR::D.n; ++k) {
+    const int l2 = PS::D.l2[GR::D.path[k]];
+    for (int b = l2 * l2; b < (l2 + 1) * (l2 + 1); ++b) m |= 1u << b;
+  }
+  return m;
 }
 
 // One edge of the CSC row, the paths of one group (l1 = GR's value).  Per
@@ -45,13 +48,13 @@ constexpr bool grp_has_l2(int l2) {
 // and, for grad_Y, the channel sums sum_u W x[m1] g[m3] of every T entry
 // contracted with the CG coefficients.  Paths are visited in (l2, ...) order
 // so that only one l2 block of the grad_Y partial is live at a time; each
-// finished block goes to this lane's row of the shared reduction buffer
-// (gyrow).  The edge's weight rows and its destination's output-gradient
+// finished block goes to this lane's column of the shared reduction buffer
+// (gyrow, row stride rs).  The edge's weight rows and its destination's output-gradient
 // rows come from this lane's pipeline stage.
 template <class PS, class GR, int VEC, bool NEED_GY>
 __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const float* __restrict__ stage, int rowf,
                                          const float (&xr)[GR::NOWN][VEC], float* __restrict__ gwrow, int mult,
-                                         float (&gx)[GR::NOWN][VEC], float* __restrict__ gyrow) {
+                                         float (&gx)[GR::NOWN][VEC], float* __restrict__ gyrow, int rs) {
   float gy[PS::NS];
   static_for<0, GR::NP>([&](auto Kc) {
     constexpr int K = decltype(Kc)::value;
@@ -117,7 +120,7 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
     if (gwrow != nullptr) VecIO<VEC>::st_stream(gwrow + P * mult, gw);
     if constexpr (NEED_GY && GR::D.last_l2[K]) {
 #pragma unroll
-      for (int m2 = 0; m2 < 2 * l2 + 1; ++m2) gyrow[l2 * l2 + m2] = gy[l2 * l2 + m2];
+      for (int m2 = 0; m2 < 2 * l2 + 1; ++m2) gyrow[(l2 * l2 + m2) * rs] = gy[l2 * l2 + m2];
     }
   });
 }
@@ -131,14 +134,20 @@ using BwdPlan = Plan<PS, kByL1, VEC, NEED_GY, kBwdBudget>;
 // One launch per chunk (paths of one l1 block): grad_x rows of that block
 // (written by the block's first chunk, accumulated by the others), grad_W
 // of the chunk's paths and a partial grad_Y over them.
-template <class PS, int VEC, bool NEED_GY, int CH>
+template <class PS, int VEC, bool NEED_GY, int CH, int KMULT>
 __global__ void __launch_bounds__(kBwdThreads)
-conv_bwd_kernel(ConvBwdArgs a, int lg_G, int S, int BT, int slice_base) {
+conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt) {
+  // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x VEC
+  // channels, so every row offset below folds into an immediate.
+  const int mult = KMULT ? KMULT : a.mult;
+  const int lg_G = KMULT ? 5 : lg_G_rt;
+  const int S = KMULT ? KMULT / (32 * VEC) : S_rt;
+  const int slice_base = KMULT ? CH * S : slice_base_rt;
   using GR = ChunkGrp<PS, BwdPlan<PS, VEC, NEED_GY>, CH, kByL1>;
   constexpr int L1 = GR::KEY;
   constexpr int NI = PS::NI, NO = PS::NO, NS = PS::NS, NR = GR::NOWN, NT = GR::NT;
   constexpr int NROWS = GR::NP + GR::NROW;
-  constexpr int NSP = NS | 1;  // odd row stride: conflict-free transposed reduction
+  constexpr unsigned GY_MASK = touched_sh_mask<PS, GR>();  // harmonics this chunk's paths reach
   extern __shared__ float4 smem_f4[];
   float* smem = reinterpret_cast<float*>(smem_f4);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -151,8 +160,11 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G, int S, int BT, int slice_base) {
   float* St = Tg + BT * NT;
   int* Eg = reinterpret_cast<int*>(St + 2 * stage_floats);
   int* Ig = Eg + ((BT + 3) & ~3);
-  // per warp: 32 x NSP floats for the grad_Y reduction
-  float* red = smem + (kBwdThreads / 32) * gpw * group_floats + warp * 32 * NSP;
+  // grad_Y reduction buffer, per group of lanes: NS rows (one per harmonic)
+  // of G lane partials, row stride rs = G + 4 (float4 aligned, and rows read
+  // by the 8 lanes of one 128-bit access phase fall in distinct banks)
+  const int rs = G + 4;
+  float* red = smem + (kBwdThreads / 32) * gpw * group_floats + (warp * gpw + grp) * NS * rs;
 
   const long long n_items = (long long)a.n_nodes * S;
   const long long warps_total = (long long)gridDim.x * (kBwdThreads / 32);
@@ -172,13 +184,13 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G, int S, int BT, int slice_base) {
     float xr[NR][VEC], gx[NR][VEC];
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
-      if (active) VecIO<VEC>::ld(xr[r], a.x + (node * NI + L1 * L1 + r) * a.mult + c0);
+      if (active) VecIO<VEC>::ld(xr[r], a.x + (node * NI + L1 * L1 + r) * mult + c0);
       else {
 #pragma unroll
         for (int c = 0; c < VEC; ++c) xr[r][c] = 0.f;
       }
       if (!GR::FIRST && active && a.grad_x != nullptr) {
-        VecIO<VEC>::ld(gx[r], a.grad_x + (node * NI + L1 * L1 + r) * a.mult + c0);
+        VecIO<VEC>::ld(gx[r], a.grad_x + (node * NI + L1 * L1 + r) * mult + c0);
       } else {
 #pragma unroll
         for (int c = 0; c < VEC; ++c) gx[r][c] = 0.f;
@@ -189,16 +201,16 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G, int S, int BT, int slice_base) {
     auto issue = [&](int b0, int k, int s) {
       if (!(active && k0 + b0 + k < k1)) return;
       float* dst = St + s * stage_floats + gl * VEC;
-      const float* wrow = a.w + (long long)Eg[k] * PS::NP * a.mult + c0;
+      const float* wrow = a.w + (long long)Eg[k] * PS::NP * mult + c0;
       static_for<0, GR::NP>([&](auto Kc) {
         constexpr int K = decltype(Kc)::value;
         constexpr int P = GR::D.path[K];
-        VecIO<VEC>::cp_async(dst + K * rowf, wrow + P * a.mult);
+        VecIO<VEC>::cp_async(dst + K * rowf, wrow + P * mult);
       });
       constexpr int rlo = GR::D.rlo;
-      const float* grow = a.grad_out + ((long long)Ig[k] * NO + rlo) * a.mult + c0;
+      const float* grow = a.grad_out + ((long long)Ig[k] * NO + rlo) * mult + c0;
 #pragma unroll
-      for (int r = 0; r < GR::NROW; ++r) VecIO<VEC>::cp_async(dst + (GR::NP + r) * rowf, grow + r * a.mult);
+      for (int r = 0; r < GR::NROW; ++r) VecIO<VEC>::cp_async(dst + (GR::NP + r) * rowf, grow + r * mult);
     };
 
     for (int b0 = 0; b0 < maxdeg; b0 += BT) {
@@ -223,38 +235,36 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G, int S, int BT, int slice_base) {
         cp_async_commit();
         cp_async_wait<1>();  // this lane's copies of edge k have landed
         const bool valid = active && (k0 + b0 + k) < k1;
-        float* rg = red + (grp * G) * NSP;  // this group's rows of the reduction buffer
-        if constexpr (NEED_GY) {  // zero the l2 blocks no path of the group touches
-          static_for<0, PS::LS + 1>([&](auto Bc) {
-            constexpr int l2 = decltype(Bc)::value;
-            if constexpr (!grp_has_l2<PS, GR>(l2)) {
-#pragma unroll
-              for (int m2 = 0; m2 < 2 * l2 + 1; ++m2) rg[gl * NSP + l2 * l2 + m2] = 0.f;
-            }
-          });
-        }
         int e = 0;
         if (valid) {
           e = Eg[k];
           bwd_edge<PS, GR, VEC, NEED_GY>(Tg + k * NT, St + (k & 1) * stage_floats + gl * VEC, rowf, xr,
-                                         a.grad_w ? a.grad_w + (long long)e * PS::NP * a.mult + c0 : nullptr,
-                                         a.mult, gx, rg + gl * NSP);
+                                         a.grad_w ? a.grad_w + (long long)e * PS::NP * mult + c0 : nullptr,
+                                         mult, gx, red + gl, rs);
         }
         if constexpr (NEED_GY) {
           __syncwarp();
           if (valid) {
             float* dst = a.grad_sh + ((long long)(slice_base + slice) * a.n_edges + e) * NS;
-            for (int b = gl; b < NS; b += G) {  // four independent partial sums
-              float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
-              int r = 0;
-              for (; r + 4 <= G; r += 4) {
-                v0 += rg[r * NSP + b];
-                v1 += rg[(r + 1) * NSP + b];
-                v2 += rg[(r + 2) * NSP + b];
-                v3 += rg[(r + 3) * NSP + b];
+            for (int b = gl; b < NS; b += G) {  // column sums; harmonics the chunk never reaches get 0
+              float v = 0.f;
+              if ((GY_MASK >> b) & 1u) {
+                const float* row = red + b * rs;
+                if (G % 4 == 0) {
+                  float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                  for (int r = 0; r < G; r += 4) {
+                    const float4 q4 = *reinterpret_cast<const float4*>(row + r);
+                    s4.x += q4.x;
+                    s4.y += q4.y;
+                    s4.z += q4.z;
+                    s4.w += q4.w;
+                  }
+                  v = (s4.x + s4.y) + (s4.z + s4.w);
+                } else {
+                  for (int r = 0; r < G; ++r) v += row[r];
+                }
               }
-              for (; r < G; ++r) v0 += rg[r * NSP + b];
-              dst[b] = (v0 + v1) + (v2 + v3);
+              dst[b] = v;
             }
           }
           __syncwarp();
@@ -264,7 +274,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G, int S, int BT, int slice_base) {
     }
     if (active && a.grad_x != nullptr) {
 #pragma unroll
-      for (int r = 0; r < NR; ++r) VecIO<VEC>::st(a.grad_x + (node * NI + L1 * L1 + r) * a.mult + c0, gx[r]);
+      for (int r = 0; r < NR; ++r) VecIO<VEC>::st(a.grad_x + (node * NI + L1 * L1 + r) * mult + c0, gx[r]);
     }
   }
 }
@@ -326,7 +336,6 @@ template <class PS, bool NEED_GY, int CH>
 cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
   constexpr int VEC = bwd_vec<PS>();
   using GR = ChunkGrp<PS, BwdPlan<PS, VEC, NEED_GY>, CH, kByL1>;
-  constexpr int NSP = PS::NS | 1;
   int G, lg_G, S;
   bwd_geometry<PS>(a.mult, G, lg_G, S);
   const int gpw = 32 / G;
@@ -334,11 +343,11 @@ cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t str
   const int BT = pick_batch(gpw, GR::NT, stage_floats);
   const int group_floats = BT * GR::NT + 2 * stage_floats + 2 * ((BT + 3) & ~3);
   const size_t smem = sizeof(float) * ((size_t)group_floats * gpw * (kBwdThreads / 32) +
-                                       (NEED_GY ? (size_t)(kBwdThreads / 32) * 32 * NSP : 0));
+                                       (NEED_GY ? (size_t)(kBwdThreads / 32) * gpw * PS::NS * (G + 4) : 0));
   const long long items = (long long)a.n_nodes * S;
   const long long groups_per_block = (long long)gpw * (kBwdThreads / 32);
   const long long blocks = (items + groups_per_block - 1) / groups_per_block;
-  auto kern = conv_bwd_kernel<PS, VEC, NEED_GY, CH>;
+  auto kern = a.mult == 128 ? conv_bwd_kernel<PS, VEC, NEED_GY, CH, 128> : conv_bwd_kernel<PS, VEC, NEED_GY, CH, 0>;
   cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e2 != cudaSuccess) return e2;
   int per_sm = 0;

@@ -114,9 +114,14 @@ __device__ __forceinline__ void fwd_edge(const float* __restrict__ T, const floa
   });
 }
 
-template <class PS, int KIND, int L3>
+template <class PS, int KIND, int L3, int KMULT>
 __global__ void __launch_bounds__(kFwdThreads)
-conv_fwd_kernel(ConvFwdArgs a, int lg_G, int S, int BT) {
+conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
+  // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x 4
+  // channels, so every row offset below folds into an immediate.
+  const int mult = KMULT ? KMULT : a.mult;
+  const int lg_G = KMULT ? 5 : lg_G_rt;
+  const int S = KMULT ? KMULT / (32 * kFwdVec) : S_rt;
   using GR = Grp<PS, KIND, L3>;
   constexpr int NI = PS::NI, NO = PS::NO, NS = PS::NS, NT = GR::NT;
   constexpr int NROWS = GR::NP + (kStageX ? GR::NROW : 0);
@@ -158,17 +163,17 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G, int S, int BT) {
       const int e = e0 + b0 + k;
       if (!(active && e < e1)) return;
       float* dst = St + s * stage_floats + gl * kFwdVec;
-      const float* wrow = a.w + (long long)e * PS::NP * a.mult + c0;
+      const float* wrow = a.w + (long long)e * PS::NP * mult + c0;
       static_for<0, GR::NP>([&](auto Kc) {
         constexpr int K = decltype(Kc)::value;
         constexpr int P = GR::D.path[K];
-        VecIO<kFwdVec>::cp_async(dst + K * rowf, wrow + P * a.mult);
+        VecIO<kFwdVec>::cp_async(dst + K * rowf, wrow + P * mult);
       });
       if constexpr (kStageX) {
         constexpr int rlo = GR::D.rlo;
-        const float* xrow = a.x + ((long long)Jg[k] * NI + rlo) * a.mult + c0;
+        const float* xrow = a.x + ((long long)Jg[k] * NI + rlo) * mult + c0;
 #pragma unroll
-        for (int r = 0; r < GR::NROW; ++r) VecIO<kFwdVec>::cp_async(dst + (GR::NP + r) * rowf, xrow + r * a.mult);
+        for (int r = 0; r < GR::NROW; ++r) VecIO<kFwdVec>::cp_async(dst + (GR::NP + r) * rowf, xrow + r * mult);
       }
     };
 
@@ -183,7 +188,7 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G, int S, int BT) {
           const int j = __ldg(a.col + e);
           if constexpr (!kStageX) {
             constexpr int rlo = GR::D.rlo;
-            prefetch_l2(a.x + ((long long)j * NI + rlo) * a.mult, (unsigned)(GR::NROW * a.mult * 4));
+            prefetch_l2(a.x + ((long long)j * NI + rlo) * mult, (unsigned)(GR::NROW * mult * 4));
           }
           Jg[k] = j;
         }
@@ -199,7 +204,7 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G, int S, int BT) {
         if (active && e0 + b0 + k < e1) {
           constexpr int rlo = GR::D.rlo;
           fwd_edge<PS, GR>(Tg + k * NT, St + (k & 1) * stage_floats + gl * kFwdVec, rowf,
-                           a.x + ((long long)Jg[k] * NI + rlo) * a.mult + c0, a.mult, acc);
+                           a.x + ((long long)Jg[k] * NI + rlo) * mult + c0, mult, acc);
         }
       }
       __syncwarp();
@@ -207,7 +212,7 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G, int S, int BT) {
     if (active) {
 #pragma unroll
       for (int r = 0; r < GR::NOWN; ++r)
-        VecIO<kFwdVec>::st(a.out + ((long long)node * NO + GR::OWN0 + r) * a.mult + c0, acc[r]);
+        VecIO<kFwdVec>::st(a.out + ((long long)node * NO + GR::OWN0 + r) * mult + c0, acc[r]);
     }
   }
 }
@@ -226,7 +231,7 @@ cudaError_t launch_fwd_group(const ConvFwdArgs& a, int num_sms, cudaStream_t str
     const int BT = pick_batch(gpw, GR::NT, stage_floats, KIND == kAll ? 12288 : 6144);
     const int group_floats = BT * GR::NT + 2 * stage_floats + ((BT + 3) & ~3);
     const size_t smem = sizeof(float) * (size_t)group_floats * gpw * (kFwdThreads / 32);
-    auto kern = conv_fwd_kernel<PS, KIND, L3>;
+    auto kern = a.mult == 128 ? conv_fwd_kernel<PS, KIND, L3, 128> : conv_fwd_kernel<PS, KIND, L3, 0>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
     int per_sm = 0;
