@@ -178,13 +178,11 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
     };
 
     for (int b0 = 0; b0 < maxdeg; b0 += BT) {
+      // sources of every slot, then the first slot's copies, so that they fly
+      // while the T matrices of the batch are computed
       for (int k = gl; k < BT; k += G) {
         const int e = e0 + b0 + k;
         if (active && e < e1) {
-          float Y[NS];
-          sh_of_vec<PS::LS>(__ldg(a.edge_vec + 3 * (long long)e), __ldg(a.edge_vec + 3 * (long long)e + 1),
-                            __ldg(a.edge_vec + 3 * (long long)e + 2), Y);
-          compute_T_grp<PS, GR>(Y, Tg + k * NT);
           const int j = __ldg(a.col + e);
           if constexpr (!kStageX) {
             constexpr int rlo = GR::D.rlo;
@@ -197,6 +195,16 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
       const int nb = min(BT, maxdeg - b0);
       issue(b0, 0, 0);
       cp_async_commit();
+      for (int k = gl; k < BT; k += G) {
+        const int e = e0 + b0 + k;
+        if (active && e < e1) {
+          float Y[NS];
+          sh_of_vec<PS::LS>(__ldg(a.edge_vec + 3 * (long long)e), __ldg(a.edge_vec + 3 * (long long)e + 1),
+                            __ldg(a.edge_vec + 3 * (long long)e + 2), Y);
+          compute_T_grp<PS, GR>(Y, Tg + k * NT);
+        }
+      }
+      __syncwarp();
       for (int k = 0; k < nb; ++k) {
         if (k + 1 < nb) issue(b0, k + 1, (k + 1) & 1);
         cp_async_commit();
