@@ -376,3 +376,71 @@ cgtp_status cgtp_tp_backward(cgtp_plan p, int batch, const float* x, const float
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the edge-free tensor-product backward.
+//
+// Some callers cannot allocate device memory when they call this library:
+// a host framework that owns all device memory through its own allocator and
+// forbids direct cudaMalloc, or a time-stepping loop (molecular dynamics)
+// that must not allocate after set-up because an allocation can stall the
+// device or fail part-way through a run.  cgtp_tp_backward needs a caller
+// workspace for its per-chunk grad_w partial sums; this variant keeps them
+// instead in the fixed array below, which every GPU that loads the library
+// holds until the process exits.
+namespace cgtp {
+namespace {
+
+// 2 MiB: tp_chunks(batch) * n_paths * mult floats must fit (at most 64
+// chunks, so n_paths * mult <= 8192, e.g. 34 paths x 128 channels at l = 3).
+constexpr size_t kTpNoAllocFloats = size_t(1) << 19;
+static __device__ __align__(256) float g_tp_noalloc_scratch[kTpNoAllocFloats];
+
+std::mutex g_noalloc_mutex;
+std::vector<float*> g_noalloc_ptr;  // device address of the array, per device (nullptr until looked up)
+
+// The array's name in host code is only a host-side stand-in; the device
+// address is looked up once per device, with that device current.
+cgtp_status noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if ((int)g_noalloc_ptr.size() <= dev) g_noalloc_ptr.resize(dev + 1, nullptr);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_tp_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return CGTP_OK;
+}
+
+}  // namespace
+}  // namespace cgtp
+
+extern "C" cgtp_status cgtp_tp_backward_noalloc(cgtp_plan p, int batch, const float* x, const float* y,
+                                                const float* w, const float* grad_z, float* grad_x,
+                                                float* grad_y, float* grad_w, void* stream) {
+  if (p == nullptr || batch < 0) return CGTP_ERR_INVALID_ARG;
+  if (batch > 0 && (x == nullptr || y == nullptr || w == nullptr || grad_z == nullptr)) return CGTP_ERR_INVALID_ARG;
+  float* scratch = nullptr;
+  if (grad_w != nullptr) {
+    const size_t need = (size_t)tp_chunks(batch) * p->n_paths * p->mult;
+    if (need > kTpNoAllocFloats) return CGTP_ERR_WORKSPACE;  // beyond the built-in scratch
+  }
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  if (grad_w != nullptr) {
+    st = noalloc_scratch(&scratch);
+    if (st != CGTP_OK) return st;
+  }
+  TPArgs a{batch, x, y, w, grad_z, nullptr, grad_x, grad_y, grad_w, scratch, p->mult};
+  cudaError_t e = cudaErrorNotSupported;
+#define CGTP_TPB_NOALLOC_ENTRY(A, B, C) \
+  if (p->li == A && p->ls == B && p->lo == C) e = launch_tp_bwd<A, B, C>(a, sms, (cudaStream_t)stream);
+  CGTP_CONFIGS(CGTP_TPB_NOALLOC_ENTRY)
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}

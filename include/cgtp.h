@@ -218,6 +218,30 @@ cgtp_status cgtp_tp_backward(cgtp_plan plan, int batch, const float* x, const fl
                              const float* w, const float* grad_z, float* grad_x, float* grad_y,
                              float* grad_w, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Allocation-free cgtp_tp_backward (an addition of this library; the paper
+ * has no counterpart).  For callers that cannot allocate device memory when
+ * they call in: a host framework that owns all device memory through its own
+ * allocator and forbids direct cudaMalloc, or a time-stepping loop that must
+ * not allocate after set-up.  Same arguments and results as
+ * cgtp_tp_backward, without the workspace: the grad_w partial sums live in a
+ * fixed 2 MiB array inside the library (held on every device that loads it
+ * until the process exits).  Allocates nothing.
+ *  - Limit: tp_chunks(batch) * n_paths * mult <= 524288 floats, where the
+ *    number of batch chunks is min(ceil(batch / 8), 64); so n_paths * mult
+ *    <= 8192 always fits.  Larger requests return CGTP_ERR_WORKSPACE and
+ *    launch nothing.
+ *  - The first call on a device (with grad_w requested) looks up the array's
+ *    device address (cudaGetSymbolAddress) with that device current; make
+ *    that first call before any stream capture.
+ *  - Every call shares the array; it keeps the last call's partial sums,
+ *    which each call overwrites completely before reading.  Calls that
+ *    overlap on the GPU (different streams, no ordering) race on it.
+ * ------------------------------------------------------------------------- */
+cgtp_status cgtp_tp_backward_noalloc(cgtp_plan plan, int batch, const float* x, const float* y,
+                                     const float* w, const float* grad_z, float* grad_x, float* grad_y,
+                                     float* grad_w, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
