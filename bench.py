@@ -428,7 +428,7 @@ def run_gpu(args):
         "config": {"workload": WORKLOAD, "n_nodes": n, "n_edges": E, "paths": P, "mult": u,
                    "l2": "inputs larger than L2 (W is %.0f MB per rank, read twice per step)" % (E * P * u * 4 / 1e6),
                    "parallelism": f"independent batch per rank (dp{world})"},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": (3 + slices) * args.steps,  # forward, backward chunks, harmonic Jacobian, forces
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": None, "peak_kind": peak_kind,
                      "alg_bytes_per_launch": b_dom},
