@@ -205,38 +205,19 @@ def run_reference(args):
 # ---------------------------------------------------------------- GPU arm
 def run_gpu(args):
     import torch
-    import torch.distributed as dist
 
     from equivariant_mlip_tensor_b200 import api
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from equivariant_mlip_tensor_b200.ranks import Group, Ranks, shard_seed, throughput
+
+    ranks = Ranks.from_env()
+    world, rank, local = ranks.world, ranks.rank, ranks.local
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    group = Group(ranks, "nccl", dev)
+    barrier, max_over_ranks = group.barrier, group.max
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    def sum_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.SUM)
-        return float(t.item())
-
-    w = synthetic.molecules(seed=4 + 1000 * rank, n_graphs=args.graphs)
+    w = synthetic.molecules(seed=shard_seed(4, rank), n_graphs=args.graphs)
     L = (w.lmax_in, w.lmax_sh, w.lmax_out)
     n, u = w.n_nodes, w.mult
     ni, ns, no = (L[0] + 1) ** 2, (L[1] + 1) ** 2, (L[2] + 1) ** 2
@@ -304,11 +285,8 @@ def run_gpu(args):
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
-    t_local = e0.elapsed_time(e1) / 1e3
-    t = max_over_ranks(t_local)
-    edges_all = sum_over_ranks(float(E))
-    value = edges_all * args.steps / t
-    ms_step = 1e3 * t / args.steps
+    value, ms_step = throughput(group, float(E), e0.elapsed_time(e1) / 1e3, args.steps)
+    edges_all = group.sum(float(E))
 
     if args.conv_only:
         if rank == 0:
@@ -316,8 +294,7 @@ def run_gpu(args):
                               "ms_per_step": ms_step, "n_edges": E,
                               "kernels_ms": {"conv_fwd": t_fwd, "conv_bwd_incl_sh_jacobian": t_bwd,
                                              "forces": t_frc}}), flush=True)
-        if world > 1:
-            dist.destroy_process_group()
+        group.close()
         return 0
 
     # pipeline: positions -> graph -> radial weights -> conv -> radial backward -> forces
@@ -418,8 +395,7 @@ def run_gpu(args):
     f_fwd, f_bwd = conv_flops(E, u, nT, nnz, no_sum, P)
     step_bytes = b_fwd + b_bwd + 4 * (E * 3 * 2 + n * 3 + 2 * (n + 1) + 2 * E)
     if rank != 0:
-        if world > 1:
-            dist.destroy_process_group()
+        group.close()
         return 0
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -447,8 +423,7 @@ def run_gpu(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    group.close()
     return 0
 
 
