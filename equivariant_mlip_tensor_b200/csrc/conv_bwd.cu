@@ -29,7 +29,30 @@ namespace cgtp {
 
 namespace {
 
-constexpr int kBwdThreads = 128;
+// Warps per block, persistent grid or one group of lanes per item, and the
+// shared-memory budget per warp (floats) that sizes the edge batch (as in
+// the forward: one-warp blocks let the block scheduler balance the rows).
+#ifndef CGTP_BWD_WARPS
+#define CGTP_BWD_WARPS 1
+#endif
+#ifndef CGTP_BWD_PERSISTENT
+#define CGTP_BWD_PERSISTENT 0
+#endif
+#ifndef CGTP_BWD_BATCH_FLOATS
+#define CGTP_BWD_BATCH_FLOATS 6144
+#endif
+#ifndef CGTP_BWD_MAX_BATCH
+#define CGTP_BWD_MAX_BATCH 16
+#endif
+#ifndef CGTP_BWD_MINB
+#define CGTP_BWD_MINB 0
+#endif
+constexpr int kBwdThreads = 32 * CGTP_BWD_WARPS;
+#if CGTP_BWD_MINB > 0
+#define CGTP_BWD_BOUNDS __launch_bounds__(kBwdThreads, CGTP_BWD_MINB)
+#else
+#define CGTP_BWD_BOUNDS __launch_bounds__(kBwdThreads)
+#endif
 
 template <class PS, class GR>
 constexpr unsigned touched_sh_mask() {
@@ -135,7 +158,7 @@ using BwdPlan = Plan<PS, kByL1, VEC, NEED_GY, kBwdBudget>;
 // (written by the block's first chunk, accumulated by the others), grad_W
 // of the chunk's paths and a partial grad_Y over them.
 template <class PS, int VEC, bool NEED_GY, int CH, int KMULT>
-__global__ void __launch_bounds__(kBwdThreads)
+__global__ void CGTP_BWD_BOUNDS
 conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt) {
   // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x VEC
   // channels, so every row offset below folds into an immediate.
@@ -340,7 +363,7 @@ cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t str
   bwd_geometry<PS>(a.mult, G, lg_G, S);
   const int gpw = 32 / G;
   const int stage_floats = (GR::NP + GR::NROW) * G * VEC;
-  const int BT = pick_batch(gpw, GR::NT, stage_floats);
+  const int BT = pick_batch(gpw, GR::NT, stage_floats, CGTP_BWD_BATCH_FLOATS, CGTP_BWD_MAX_BATCH);
   const int group_floats = BT * GR::NT + 2 * stage_floats + 2 * ((BT + 3) & ~3);
   const size_t smem = sizeof(float) * ((size_t)group_floats * gpw * (kBwdThreads / 32) +
                                        (NEED_GY ? (size_t)(kBwdThreads / 32) * gpw * PS::NS * (G + 4) : 0));
@@ -350,11 +373,13 @@ cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t str
   auto kern = a.mult == 128 ? conv_bwd_kernel<PS, VEC, NEED_GY, CH, 128> : conv_bwd_kernel<PS, VEC, NEED_GY, CH, 0>;
   cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e2 != cudaSuccess) return e2;
-  int per_sm = 0;
-  e2 = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBwdThreads, smem);
-  if (e2 != cudaSuccess) return e2;
-  if (per_sm < 1) per_sm = 1;
-  const long long cap = (long long)num_sms * per_sm;
+  long long cap = 0x7fffffffLL;  // the kernel loops over items beyond the grid
+  if (CGTP_BWD_PERSISTENT) {
+    int per_sm = 0;
+    e2 = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBwdThreads, smem);
+    if (e2 != cudaSuccess) return e2;
+    cap = (long long)num_sms * (per_sm < 1 ? 1 : per_sm);
+  }
   long long nb = blocks > cap ? cap : blocks;
   if (nb < 1) nb = 1;
   kern<<<(unsigned)nb, kBwdThreads, smem, stream>>>(a, lg_G, S, BT, CH * S);

@@ -217,10 +217,10 @@ struct ChunkGrp : Chunk<PS, PL, CH> {
 
 // Edges per batch: T matrices of BT edges per group of lanes, sized so that a
 // group's shared memory stays near 24 KB.
-inline int pick_batch(int gpw, int t_floats, int stage_floats, int budget_floats = 6144) {
+inline int pick_batch(int gpw, int t_floats, int stage_floats, int budget_floats = 6144, int max_bt = 16) {
   const int budget = budget_floats / gpw - 2 * stage_floats;
   int bt = budget / (t_floats + 3);
-  if (bt > 16) bt = 16;
+  if (bt > max_bt) bt = max_bt;
   return bt < 1 ? 1 : bt;
 }
 

@@ -32,7 +32,32 @@ CGTP_DEFINE_CONSTANT_TABLES()
 namespace cgtp {
 namespace {
 
-constexpr int kFwdThreads = 128;
+// Warps per block, whether the grid is persistent (one wave that loops over
+// the work items) or one group of lanes per item, and the shared-memory
+// budget per warp (floats) that sizes the edge batch.  One-warp blocks over
+// one item each let the block scheduler balance rows of unequal degree: an
+// SM takes a new row as soon as any of its warps finishes one.
+#ifndef CGTP_FWD_WARPS
+#define CGTP_FWD_WARPS 1
+#endif
+#ifndef CGTP_FWD_PERSISTENT
+#define CGTP_FWD_PERSISTENT 0
+#endif
+#ifndef CGTP_FWD_BATCH_FLOATS
+#define CGTP_FWD_BATCH_FLOATS 12288
+#endif
+#ifndef CGTP_FWD_MAX_BATCH
+#define CGTP_FWD_MAX_BATCH 16
+#endif
+#ifndef CGTP_FWD_MINB
+#define CGTP_FWD_MINB 0
+#endif
+constexpr int kFwdThreads = 32 * CGTP_FWD_WARPS;
+#if CGTP_FWD_MINB > 0
+#define CGTP_FWD_BOUNDS __launch_bounds__(kFwdThreads, CGTP_FWD_MINB)
+#else
+#define CGTP_FWD_BOUNDS __launch_bounds__(kFwdThreads)
+#endif
 constexpr int kFwdVec = 4;
 
 // Stage x rows through the cp.async pipeline (1) or gather them with cached
@@ -115,7 +140,7 @@ __device__ __forceinline__ void fwd_edge(const float* __restrict__ T, const floa
 }
 
 template <class PS, int KIND, int L3, int KMULT>
-__global__ void __launch_bounds__(kFwdThreads)
+__global__ void CGTP_FWD_BOUNDS
 conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
   // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x 4
   // channels, so every row offset below folds into an immediate.
@@ -236,20 +261,23 @@ cudaError_t launch_fwd_group(const ConvFwdArgs& a, int num_sms, cudaStream_t str
     lane_geometry(a.mult, kFwdVec, G, lg_G, S);
     const int gpw = 32 / G;
     const int stage_floats = (GR::NP + (kStageX ? GR::NROW : 0)) * G * kFwdVec;
-    const int BT = pick_batch(gpw, GR::NT, stage_floats, KIND == kAll ? 12288 : 6144);
+    const int BT = pick_batch(gpw, GR::NT, stage_floats, KIND == kAll ? CGTP_FWD_BATCH_FLOATS : 6144,
+                               CGTP_FWD_MAX_BATCH);
     const int group_floats = BT * GR::NT + 2 * stage_floats + ((BT + 3) & ~3);
     const size_t smem = sizeof(float) * (size_t)group_floats * gpw * (kFwdThreads / 32);
     auto kern = a.mult == 128 ? conv_fwd_kernel<PS, KIND, L3, 128> : conv_fwd_kernel<PS, KIND, L3, 0>;
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFwdThreads, smem);
-    if (err != cudaSuccess) return err;
-    if (per_sm < 1) per_sm = 1;
     const long long items = (long long)a.n_nodes * S;
     const long long groups_per_block = (long long)gpw * (kFwdThreads / 32);
     long long blocks = (items + groups_per_block - 1) / groups_per_block;
-    const long long cap = (long long)num_sms * per_sm;
+    long long cap = 0x7fffffffLL;  // the kernel loops over items beyond the grid
+    if (CGTP_FWD_PERSISTENT) {
+      int per_sm = 0;
+      err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFwdThreads, smem);
+      if (err != cudaSuccess) return err;
+      cap = (long long)num_sms * (per_sm < 1 ? 1 : per_sm);
+    }
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     kern<<<(unsigned)blocks, kFwdThreads, smem, stream>>>(a, lg_G, S, BT);
