@@ -47,6 +47,35 @@ int register_table_uploader(UploadFn fn);  // host, defined in abi.cu
   }                                                                                \
   static const int tables_registered_here = register_table_uploader(&upload_tables_here);
 
+// ---- programmatic dependent launch (sm_90 and later) ----
+// A grid launched with programmatic stream serialization may start once every
+// block of the grid before it has called grid_dependents_launch() (or
+// exited); grid_dependency_wait() then blocks until that preceding grid has
+// completed and its writes are visible.  Both are no-ops for a grid launched
+// in plain stream order.
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Host: launch kern<<<grid, block, smem, stream>>>(args...), with programmatic
+// stream serialization when pdl is set.
+template <class... P, class... A>
+cudaError_t launch_kernel(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool pdl,
+                          A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
+
 // ---- loads / stores with cache hints ----
 __device__ __forceinline__ float4 ld_stream(const float* p) {  // read once: evict first
   return __ldcs(reinterpret_cast<const float4*>(p));

@@ -149,7 +149,10 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
 }
 
 // Unrolled instructions per edge and lane allowed in one backward launch.
-constexpr int kBwdBudget = 1100;
+#ifndef CGTP_BWD_BUDGET
+#define CGTP_BWD_BUDGET 1100
+#endif
+constexpr int kBwdBudget = CGTP_BWD_BUDGET;
 
 template <class PS, int VEC, bool NEED_GY>
 using BwdPlan = Plan<PS, kByL1, VEC, NEED_GY, kBwdBudget>;
@@ -189,6 +192,10 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
   const int rs = G + 4;
   float* red = smem + (kBwdThreads / 32) * gpw * group_floats + (warp * gpw + grp) * NS * rs;
 
+  // The next chunk of this call may start on SMs this grid leaves idle: no
+  // chunk reads what another writes, except a chunk that adds onto an
+  // earlier chunk's grad_x rows, and that one waits for it below.
+  grid_dependents_launch();
   const long long n_items = (long long)a.n_nodes * S;
   const long long warps_total = (long long)gridDim.x * (kBwdThreads / 32);
   for (long long base = ((long long)blockIdx.x * (kBwdThreads / 32) + warp) * gpw; base < n_items;
@@ -212,12 +219,8 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
 #pragma unroll
         for (int c = 0; c < VEC; ++c) xr[r][c] = 0.f;
       }
-      if (!GR::FIRST && active && a.grad_x != nullptr) {
-        VecIO<VEC>::ld(gx[r], a.grad_x + (node * NI + L1 * L1 + r) * mult + c0);
-      } else {
 #pragma unroll
-        for (int c = 0; c < VEC; ++c) gx[r][c] = 0.f;
-      }
+      for (int c = 0; c < VEC; ++c) gx[r][c] = 0.f;
     }
 
     // copies of edge slot k of the current batch into stage s (this lane's channels only)
@@ -296,6 +299,18 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
       __syncwarp();
     }
     if (active && a.grad_x != nullptr) {
+      if constexpr (!GR::FIRST) {
+        // rows of an l1 block that an earlier chunk of this call wrote: wait
+        // for that grid (the preceding launch) and add onto its values
+        grid_dependency_wait();
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          float prev[VEC];
+          VecIO<VEC>::ld(prev, a.grad_x + (node * NI + L1 * L1 + r) * mult + c0);
+#pragma unroll
+          for (int c = 0; c < VEC; ++c) gx[r][c] += prev[c];
+        }
+      }
 #pragma unroll
       for (int r = 0; r < NR; ++r) VecIO<VEC>::st(a.grad_x + (node * NI + L1 * L1 + r) * mult + c0, gx[r]);
     }
@@ -336,9 +351,18 @@ __global__ void sh_backward_kernel(int n_edges, int S, const float* __restrict__
 
 // Channels per lane: 4 (float4) up to l = 2; 2 for l = 3, whose path groups
 // would otherwise exceed the register file.
+// Programmatic dependent launch between the chunks of one backward call
+// (1) or plain stream order (0).
+#ifndef CGTP_BWD_PDL
+#define CGTP_BWD_PDL 1
+#endif
+
+#ifndef CGTP_BWD_VEC
+#define CGTP_BWD_VEC 0  // 0: by shape as above
+#endif
 template <class PS>
 constexpr int bwd_vec() {
-  return PS::LI >= 3 || PS::LO >= 3 ? 2 : 4;
+  return CGTP_BWD_VEC ? CGTP_BWD_VEC : (PS::LI >= 3 || PS::LO >= 3 ? 2 : 4);
 }
 
 // channel lanes per group (G) and channel slices (S) of the backward
@@ -382,8 +406,9 @@ cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t str
   }
   long long nb = blocks > cap ? cap : blocks;
   if (nb < 1) nb = 1;
-  kern<<<(unsigned)nb, kBwdThreads, smem, stream>>>(a, lg_G, S, BT, CH * S);
-  return cudaGetLastError();
+  // Every chunk but the call's first may overlap the one before it.
+  return launch_kernel(kern, dim3((unsigned)nb), dim3(kBwdThreads), smem, stream, CGTP_BWD_PDL && CH > 0, a, lg_G,
+                       S, BT, CH * S);
 }
 
 // grad_x blocks that no path reaches (l1 with no path) are zero.

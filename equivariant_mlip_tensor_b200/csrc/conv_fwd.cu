@@ -50,7 +50,7 @@ namespace {
 #define CGTP_FWD_MAX_BATCH 16
 #endif
 #ifndef CGTP_FWD_MINB
-#define CGTP_FWD_MINB 0
+#define CGTP_FWD_MINB 1
 #endif
 constexpr int kFwdThreads = 32 * CGTP_FWD_WARPS;
 #if CGTP_FWD_MINB > 0
@@ -58,7 +58,10 @@ constexpr int kFwdThreads = 32 * CGTP_FWD_WARPS;
 #else
 #define CGTP_FWD_BOUNDS __launch_bounds__(kFwdThreads)
 #endif
-constexpr int kFwdVec = 4;
+#ifndef CGTP_FWD_VEC
+#define CGTP_FWD_VEC 4
+#endif
+constexpr int kFwdVec = CGTP_FWD_VEC;  // channels per lane
 
 // Stage x rows through the cp.async pipeline (1) or gather them with cached
 // loads after an L2 prefetch (0); path groups by l3 (1) or one group (0).
