@@ -104,6 +104,36 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ---------------------------------------------------------------- measured DRAM traffic
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch of each kernel
+# family at the molecules workload (97 480 edges), from an ncu capture
+# (profiles/conv_molecules_traffic.md), with a hash of the kernel sources it
+# was taken on: traffic is reported only while the sources are unchanged.
+KERNEL_HEADERS = ("common.cuh", "conv_common.cuh", "sh.cuh", "structure.h")
+MEASURED_TRAFFIC = {
+    "conv_fwd": {"bytes": 1025952000, "n_edges": 97480, "sources": ("conv_fwd.cu",) + KERNEL_HEADERS,
+                 "sha256_16": "88771e3801183127"},
+    "conv_bwd": {"bytes": 2062707456, "n_edges": 97480, "sources": ("conv_bwd.cu",) + KERNEL_HEADERS,
+                 "sha256_16": "efbbeca031725577"},
+}
+
+
+def measured_traffic(kernel, n_edges):
+    """Measured DRAM bytes of one launch scaled to n_edges, or None when the
+    kernel's sources changed since the capture."""
+    import hashlib
+    rec = MEASURED_TRAFFIC.get(kernel)
+    if rec is None:
+        return None
+    m = hashlib.sha256()
+    for name in rec["sources"]:
+        with open(os.path.join(ROOT, "equivariant_mlip_tensor_b200", "csrc", name), "rb") as f:
+            m.update(f.read())
+    if m.hexdigest()[:16] != rec["sha256_16"]:
+        return None
+    return rec["bytes"] * n_edges / rec["n_edges"]
+
+
 # ---------------------------------------------------------------- algorithmic bytes
 def conv_bytes(n, E, P, u, ni, ns, no, slices):
     """Algorithmic bytes of one forward and one backward launch (fp32/int32)."""
@@ -200,6 +230,82 @@ def run_reference(args):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ---------------------------------------------------------------- every workload size
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12  # SMs x FP32 lanes x FMA x max clock
+
+
+def _time_ms(torch, fn, reps):
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def config_table(torch, api, dev, hbm, reps=20):
+    """Forward and backward of every workload (sizes of the pages' configurations),
+    each against the HBM and FP32 rooflines, plus the edge-free tensor product."""
+    rows = []
+    for name in ("tiny", "bulk", "bulk_large", "molecules"):
+        w = synthetic.WORKLOADS[name]()
+        L = (w.lmax_in, w.lmax_sh, w.lmax_out)
+        n, u = w.n_nodes, w.mult
+        ni, ns, no = (L[0] + 1) ** 2, (L[1] + 1) ** 2, (L[2] + 1) ** 2
+        gp = None
+        if w.graph_id is not None:
+            gp = torch.from_numpy(np.arange(0, n + 1, w.graph_size, dtype=np.int32)).to(dev)
+        g = api.build_graph(torch.from_numpy(w.pos).to(dev), w.rc, box=w.box, graph_ptr=gp)
+        plan = api.Plan(*L, u)
+        E, P = g.n_edges, plan.n_paths
+        W = plan.radial_forward(g.edge_vec, w.rc, torch.from_numpy(w.W1).to(dev), torch.from_numpy(w.W2).to(dev))
+        x = torch.from_numpy(w.x).to(dev)
+        go = torch.from_numpy(w.grad_out).to(dev)
+        out = torch.empty((n, no, u), dtype=torch.float32, device=dev)
+        gx = torch.empty((n, ni, u), dtype=torch.float32, device=dev)
+        gw = torch.empty_like(W)
+        gr = torch.empty((E, 3), dtype=torch.float32, device=dev)
+        F = torch.empty((n, 3), dtype=torch.float32, device=dev)
+        ws_bytes = plan.conv_backward_workspace_bytes(E)
+        ws = torch.empty(ws_bytes // 4 + 64, dtype=torch.float32, device=dev)
+        k = max(3, reps if E < 500_000 else reps // 4)
+        t_f = _time_ms(torch, lambda: plan.conv_forward(g, x, W, out=out), k)
+        t_b = _time_ms(torch, lambda: plan.conv_backward(g, x, W, go, grad_x=gx, grad_w=gw, grad_edge_vec=gr,
+                                                          workspace=ws), k)
+        t_frc = _time_ms(torch, lambda: api.forces(g, gr, out=F), k)
+        slices = max(1, int(ws_bytes // (4 * E * ns))) if E else 1
+        b_f, b_b = conv_bytes(n, E, P, u, ni, ns, no, slices)
+        nT, nnz, no_sum = structural_counts(*L)
+        f_f, f_b = conv_flops(E, u, nT, nnz, no_sum, P)
+        rows.append({"workload": name, "L": list(L), "mult": u, "n_nodes": n, "n_edges": E, "paths": P,
+                     "fwd_ms": t_f, "bwd_ms": t_b, "forces_ms": t_frc,
+                     "edges_per_s_fwd_bwd": E / ((t_f + t_b) / 1e3),
+                     "hbm_frac": {"fwd": b_f / (t_f / 1e3) / 1e9 / hbm, "bwd": b_b / (t_b / 1e3) / 1e9 / hbm},
+                     "fp32_frac": {"fwd": f_f / (t_f / 1e3) / 1e12 / FP32_PEAK_TFLOPS,
+                                   "bwd": f_b / (t_b / 1e3) / 1e12 / FP32_PEAK_TFLOPS}})
+        del W, gw, out, gx, gr, F, ws, x, go, g
+        torch.cuda.empty_cache()
+    t = synthetic.tp_batch()
+    L = (t.lmax_in, t.lmax_sh, t.lmax_out)
+    plan = api.Plan(*L, t.mult)
+    xs, ys, ws_, gz = (torch.from_numpy(a).to(dev) for a in (t.x, t.y, t.w, t.grad_z))
+    z = torch.empty_like(gz)
+    t_f = _time_ms(torch, lambda: plan.tp_forward(xs, ys, ws_, out=z), reps)
+    t_b = _time_ms(torch, lambda: plan.tp_backward(xs, ys, ws_, gz), reps)
+    B, u = t.x.shape[0], t.mult
+    ni, ns, no = (L[0] + 1) ** 2, (L[1] + 1) ** 2, (L[2] + 1) ** 2
+    b_f = 4 * (B * u * (ni + ns + no) + t.w.size)
+    b_b = 4 * (B * u * (2 * ni + 2 * ns + no) + 2 * t.w.size)
+    rows.append({"workload": "tp_batch (edge-free tensor product)", "L": list(L), "mult": u, "batch": B,
+                 "fwd_ms": t_f, "bwd_ms": t_b, "pairs_per_s_fwd_bwd": B / ((t_f + t_b) / 1e3),
+                 "hbm_frac": {"fwd": b_f / (t_f / 1e3) / 1e9 / hbm, "bwd": b_b / (t_b / 1e3) / 1e9 / hbm}})
+    return rows
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -391,6 +497,7 @@ def run_gpu(args):
     dominant = "conv_bwd" if t_bwd >= t_fwd else "conv_fwd"
     b_dom, t_dom = (b_bwd, t_bwd) if dominant == "conv_bwd" else (b_fwd, t_fwd)
     achieved = b_dom / (t_dom / 1e3) / 1e9
+    traffic = measured_traffic(dominant, E)
     nT, nnz, no_sum = structural_counts(*L)
     f_fwd, f_bwd = conv_flops(E, u, nT, nnz, no_sum, P)
     step_bytes = b_fwd + b_bwd + 4 * (E * 3 * 2 + n * 3 + 2 * (n + 1) + 2 * E)
@@ -406,8 +513,9 @@ def run_gpu(args):
                    "parallelism": f"independent batch per rank (dp{world})"},
         "gpu_launches": (3 + slices) * args.steps,  # forward, backward chunks, harmonic Jacobian, forces
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None, "peak_kind": peak_kind,
-                     "alg_bytes_per_launch": b_dom},
+                     "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
+                     "alg_bytes_per_launch": b_dom,
+                     "traffic_over_alg": traffic / b_dom if traffic else None},
         "kernels_ms": {"conv_fwd": t_fwd, "conv_bwd_incl_sh_jacobian": t_bwd, "forces": t_frc},
         "step_hbm_frac": (step_bytes / (ms_step / 1e3) / 1e9) / hbm,
         "fp32_tflops": {"conv_fwd": f_fwd / (t_fwd / 1e3) / 1e12, "conv_bwd": f_bwd / (t_bwd / 1e3) / 1e12},
@@ -420,6 +528,8 @@ def run_gpu(args):
                         "radial bwd, forces -> host forces"},
         "clocks": clk,
     }
+    if rank == 0 and not args.no_configs:
+        line["configs"] = config_table(torch, api, dev, hbm)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
@@ -434,6 +544,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["cgtp", "reference"], default="cgtp")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-workload table")
     ap.add_argument("--graphs", type=int, default=256, help="molecules per rank (profiling uses fewer)")
     ap.add_argument("--conv-only", action="store_true",
                     help="time only the convolution step (no pipeline / e2e / CPU baseline); for profiling")
