@@ -90,6 +90,7 @@ struct Grp {
   // rows of the group's own block (all output rows for kAll)
   static constexpr int NOWN = KIND == kAll ? PS::NO : 2 * V + 1;
   static constexpr int OWN0 = KIND == kAll ? 0 : V * V;    // first own row
+  static constexpr bool FIRST = true;                      // initialises its rows
 };
 
 // T^p[m1][m3] = sum_m2 C^p[m1,m2,m3] Y[l2,m2] for the group's paths, packed

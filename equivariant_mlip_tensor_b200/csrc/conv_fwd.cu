@@ -64,14 +64,21 @@ constexpr int kFwdThreads = 32 * CGTP_FWD_WARPS;
 constexpr int kFwdVec = CGTP_FWD_VEC;  // channels per lane
 
 // Stage x rows through the cp.async pipeline (1) or gather them with cached
-// loads after an L2 prefetch (0); path groups by l3 (1) or one group (0).
+// loads after an L2 prefetch (0).
 #ifndef CGTP_FWD_STAGE_X
 #define CGTP_FWD_STAGE_X 1
 #endif
-#ifndef CGTP_FWD_GROUPED
-#define CGTP_FWD_GROUPED 0
-#endif
 constexpr bool kStageX = CGTP_FWD_STAGE_X != 0;
+
+// One launch over all paths while their unrolled code per edge and lane stays
+// within CGTP_FWD_SINGLE_MAX instructions; otherwise one launch per chunk of
+// paths with one l3, each within CGTP_FWD_BUDGET (the instruction cache).
+#ifndef CGTP_FWD_SINGLE_MAX
+#define CGTP_FWD_SINGLE_MAX 1600
+#endif
+#ifndef CGTP_FWD_BUDGET
+#define CGTP_FWD_BUDGET 1100
+#endif
 
 // One edge: acc[m3][c] += sum_p W[p][c] sum_m1 T[p][m1][m3] x[l1,m1][c] for the group's paths.
 template <class PS, class GR>
@@ -142,7 +149,10 @@ __device__ __forceinline__ void fwd_edge(const float* __restrict__ T, const floa
   });
 }
 
-template <class PS, int KIND, int L3, int KMULT>
+// GR: the launch's paths (all of them, or one chunk of one l3 block).  A
+// chunk that continues an l3 block another chunk of the call started adds
+// onto that chunk's rows (GR::FIRST false).
+template <class PS, class GR, int KMULT>
 __global__ void CGTP_FWD_BOUNDS
 conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
   // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x 4
@@ -150,7 +160,6 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
   const int mult = KMULT ? KMULT : a.mult;
   const int lg_G = KMULT ? 5 : lg_G_rt;
   const int S = KMULT ? KMULT / (32 * kFwdVec) : S_rt;
-  using GR = Grp<PS, KIND, L3>;
   constexpr int NI = PS::NI, NO = PS::NO, NS = PS::NS, NT = GR::NT;
   constexpr int NROWS = GR::NP + (kStageX ? GR::NROW : 0);
   extern __shared__ float4 smem_f4[];
@@ -165,6 +174,9 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
   float* St = Tg + BT * NT;                        // two pipeline stages
   int* Jg = reinterpret_cast<int*>(St + 2 * stage_floats);
 
+  // The next chunk of this call may start on SMs this grid leaves idle (see
+  // the launcher: chunks write disjoint rows unless one continues another).
+  grid_dependents_launch();
   const long long n_items = (long long)a.n_nodes * S;
   const long long warps_total = (long long)gridDim.x * (kFwdThreads / 32);
   for (long long base = ((long long)blockIdx.x * (kFwdThreads / 32) + warp) * gpw; base < n_items;
@@ -246,6 +258,17 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
       __syncwarp();
     }
     if (active) {
+      if constexpr (!GR::FIRST) {
+        // rows of an l3 block that the preceding launch wrote: wait for it, add
+        grid_dependency_wait();
+#pragma unroll
+        for (int r = 0; r < GR::NOWN; ++r) {
+          float prev[kFwdVec];
+          VecIO<kFwdVec>::ld(prev, a.out + ((long long)node * NO + GR::OWN0 + r) * mult + c0);
+#pragma unroll
+          for (int c = 0; c < kFwdVec; ++c) acc[r][c] += prev[c];
+        }
+      }
 #pragma unroll
       for (int r = 0; r < GR::NOWN; ++r)
         VecIO<kFwdVec>::st(a.out + ((long long)node * NO + GR::OWN0 + r) * mult + c0, acc[r]);
@@ -253,39 +276,60 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
   }
 }
 
-template <class PS, int KIND, int L3>
-cudaError_t launch_fwd_group(const ConvFwdArgs& a, int num_sms, cudaStream_t stream) {
-  using GR = Grp<PS, KIND, L3>;
-  if constexpr (GR::NP == 0) {  // no path reaches this output block: it is zero
-    return cudaMemset2DAsync(a.out + (size_t)GR::OWN0 * a.mult, sizeof(float) * PS::NO * a.mult, 0,
-                             sizeof(float) * GR::NOWN * a.mult, a.n_nodes, stream);
-  } else {
-    int G, lg_G, S;
-    lane_geometry(a.mult, kFwdVec, G, lg_G, S);
-    const int gpw = 32 / G;
-    const int stage_floats = (GR::NP + (kStageX ? GR::NROW : 0)) * G * kFwdVec;
-    const int BT = pick_batch(gpw, GR::NT, stage_floats, KIND == kAll ? CGTP_FWD_BATCH_FLOATS : 6144,
-                               CGTP_FWD_MAX_BATCH);
-    const int group_floats = BT * GR::NT + 2 * stage_floats + ((BT + 3) & ~3);
-    const size_t smem = sizeof(float) * (size_t)group_floats * gpw * (kFwdThreads / 32);
-    auto kern = a.mult == 128 ? conv_fwd_kernel<PS, KIND, L3, 128> : conv_fwd_kernel<PS, KIND, L3, 0>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+template <class PS, class GR>
+cudaError_t launch_fwd_group(const ConvFwdArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
+  int G, lg_G, S;
+  lane_geometry(a.mult, kFwdVec, G, lg_G, S);
+  const int gpw = 32 / G;
+  const int stage_floats = (GR::NP + (kStageX ? GR::NROW : 0)) * G * kFwdVec;
+  const int BT = pick_batch(gpw, GR::NT, stage_floats, CGTP_FWD_BATCH_FLOATS, CGTP_FWD_MAX_BATCH);
+  const int group_floats = BT * GR::NT + 2 * stage_floats + ((BT + 3) & ~3);
+  const size_t smem = sizeof(float) * (size_t)group_floats * gpw * (kFwdThreads / 32);
+  auto kern = a.mult == 128 ? conv_fwd_kernel<PS, GR, 128> : conv_fwd_kernel<PS, GR, 0>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  const long long items = (long long)a.n_nodes * S;
+  const long long groups_per_block = (long long)gpw * (kFwdThreads / 32);
+  long long blocks = (items + groups_per_block - 1) / groups_per_block;
+  long long cap = 0x7fffffffLL;  // the kernel loops over items beyond the grid
+  if (CGTP_FWD_PERSISTENT) {
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFwdThreads, smem);
     if (err != cudaSuccess) return err;
-    const long long items = (long long)a.n_nodes * S;
-    const long long groups_per_block = (long long)gpw * (kFwdThreads / 32);
-    long long blocks = (items + groups_per_block - 1) / groups_per_block;
-    long long cap = 0x7fffffffLL;  // the kernel loops over items beyond the grid
-    if (CGTP_FWD_PERSISTENT) {
-      int per_sm = 0;
-      err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFwdThreads, smem);
-      if (err != cudaSuccess) return err;
-      cap = (long long)num_sms * (per_sm < 1 ? 1 : per_sm);
-    }
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
-    kern<<<(unsigned)blocks, kFwdThreads, smem, stream>>>(a, lg_G, S, BT);
-    return cudaGetLastError();
+    cap = (long long)num_sms * (per_sm < 1 ? 1 : per_sm);
   }
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return launch_kernel(kern, dim3((unsigned)blocks), dim3(kFwdThreads), smem, stream, pdl, a, lg_G, S, BT);
+}
+
+// Unrolled instructions per edge and lane of all paths in one launch.
+template <class PS>
+constexpr int fwd_all_cost() {
+  int c = 0;
+  for (int p = 0; p < PS::D.np; ++p) c += path_cost<PS>(p, kByL3, kFwdVec, false);
+  return c;
+}
+
+template <class PS>
+using FwdPlan = Plan<PS, kByL3, kFwdVec, false, CGTP_FWD_BUDGET>;
+
+// Output blocks l3 that no path reaches are zero.
+template <class PS>
+cudaError_t zero_unreached_out(const ConvFwdArgs& a, cudaStream_t stream) {
+  cudaError_t err = cudaSuccess;
+  static_for_host<0, PS::LO + 1>([&](auto Lc) {
+    constexpr int l3 = decltype(Lc)::value;
+    constexpr bool reached = [] {
+      for (int p = 0; p < PS::D.np; ++p)
+        if (PS::D.l3[p] == l3) return true;
+      return false;
+    }();
+    if (!reached && err == cudaSuccess)
+      err = cudaMemset2DAsync(a.out + (size_t)l3 * l3 * a.mult, sizeof(float) * PS::NO * a.mult, 0,
+                              sizeof(float) * (2 * l3 + 1) * a.mult, a.n_nodes, stream);
+  });
+  return err;
 }
 
 }  // namespace
@@ -293,12 +337,16 @@ cudaError_t launch_fwd_group(const ConvFwdArgs& a, int num_sms, cudaStream_t str
 template <int LI, int LS, int LO>
 cudaError_t launch_conv_fwd(const ConvFwdArgs& a, int num_sms, cudaStream_t stream) {
   using PS = PathSet<LI, LS, LO>;
-  if constexpr (CGTP_FWD_GROUPED == 0) {
-    return launch_fwd_group<PS, kAll, 0>(a, num_sms, stream);
+  if constexpr (fwd_all_cost<PS>() <= CGTP_FWD_SINGLE_MAX) {
+    // all paths in one launch (it writes every output row, reached or not)
+    return launch_fwd_group<PS, Grp<PS, kAll, 0>>(a, num_sms, false, stream);
   } else {
-    cudaError_t err = cudaSuccess;
-    static_for_host<0, LO + 1>([&](auto Lc) {
-      if (err == cudaSuccess) err = launch_fwd_group<PS, kByL3, decltype(Lc)::value>(a, num_sms, stream);
+    cudaError_t err = zero_unreached_out<PS>(a, stream);
+    static_for_host<0, FwdPlan<PS>::N>([&](auto Cc) {
+      constexpr int CH = decltype(Cc)::value;
+      // every chunk but the call's first may overlap the one before it
+      if (err == cudaSuccess)
+        err = launch_fwd_group<PS, ChunkGrp<PS, FwdPlan<PS>, CH, kByL3>>(a, num_sms, CH > 0, stream);
     });
     return err;
   }
