@@ -152,10 +152,16 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
 #ifndef CGTP_BWD_BUDGET
 #define CGTP_BWD_BUDGET 1100
 #endif
-constexpr int kBwdBudget = CGTP_BWD_BUDGET;
+#ifndef CGTP_BWD_BUDGET_L3
+#define CGTP_BWD_BUDGET_L3 800  // l = 3 chunks carry more registers per path
+#endif
+template <class PS>
+constexpr int bwd_budget() {
+  return PS::LI >= 3 || PS::LO >= 3 ? CGTP_BWD_BUDGET_L3 : CGTP_BWD_BUDGET;
+}
 
 template <class PS, int VEC, bool NEED_GY>
-using BwdPlan = Plan<PS, kByL1, VEC, NEED_GY, kBwdBudget>;
+using BwdPlan = Plan<PS, kByL1, VEC, NEED_GY, bwd_budget<PS>()>;
 
 // One launch per chunk (paths of one l1 block): grad_x rows of that block
 // (written by the block's first chunk, accumulated by the others), grad_W
@@ -349,20 +355,20 @@ __global__ void sh_backward_kernel(int n_edges, int S, const float* __restrict__
 
 }  // namespace
 
-// Channels per lane: 4 (float4) up to l = 2; 2 for l = 3, whose path groups
-// would otherwise exceed the register file.
 // Programmatic dependent launch between the chunks of one backward call
 // (1) or plain stream order (0).
 #ifndef CGTP_BWD_PDL
 #define CGTP_BWD_PDL 1
 #endif
 
+// Channels per lane (float4: measured faster than 2 at every shape with
+// one-warp blocks and budgeted chunks).
 #ifndef CGTP_BWD_VEC
-#define CGTP_BWD_VEC 0  // 0: by shape as above
+#define CGTP_BWD_VEC 4
 #endif
 template <class PS>
 constexpr int bwd_vec() {
-  return CGTP_BWD_VEC ? CGTP_BWD_VEC : (PS::LI >= 3 || PS::LO >= 3 ? 2 : 4);
+  return CGTP_BWD_VEC;
 }
 
 // channel lanes per group (G) and channel slices (S) of the backward
