@@ -36,7 +36,7 @@ import numpy as np
 
 from .cg import paths, real_cg
 from .graph import edge_dst
-from .sh import real_sh, real_sh_jacobian
+from .sh import real_sh, real_sh_hessian, real_sh_jacobian
 
 
 def path_nonzeros(lmax_in, lmax_sh, lmax_out):
@@ -166,3 +166,71 @@ def edge_forces(row_ptr, col, grad_edge_vec, n_nodes):
     np.add.at(dEdpos, col, gr)
     np.add.at(dEdpos, dst, -gr)
     return -dEdpos
+
+
+def conv_double_backward(row_ptr, col, edge_vec, x, w, grad_out, gg_x, gg_w, gg_r,
+                         lmax_in, lmax_sh, lmax_out):
+    """Adjoint of the backward: the gradients of
+
+        L = <gg_x, grad_x> + <gg_w, grad_w> + <gg_r, grad_r>
+
+    (grad_x, grad_w, grad_r = conv_backward(x, w, grad_out, edge_vec)) with
+    respect to x, w, grad_out and the edge vectors, for cotangents gg_x
+    [N][(lmax_in+1)^2][u], gg_w [E][P][u] and gg_r [E][3] (any may be None).
+    This is the second derivative that force training needs ("LunaTP ...",
+    abstract: higher-order derivative computation).
+
+    Written out per nonzero (p, m1, m2, m3) of each edge e = (j -> i), with
+    uY[e] = (dY_e/dr_e) gg_r[e] (the directional derivative of the harmonics)
+    and gY[e] the harmonic gradient of the backward, L is
+
+        sum_e sum_nz C sum_u g[i,m3,u] (gg_x[j,m1,u] W[e,p,u] Y[e,m2]
+                                        + gg_w[e,p,u] x[j,m1,u] Y[e,m2]
+                                        + uY[e,m2] W[e,p,u] x[j,m1,u])
+
+    so that, term by term,
+        dL/dg[i,m3,u] = sum_e sum_nz C (gg_x W Y + gg_w x Y + uY W x)
+        dL/dx[j,m1,u] = sum_e sum_nz C g (gg_w Y + uY W)
+        dL/dW[e,p,u]  = sum_nz(p) C g (gg_x Y + uY x)
+        dL/dr_e       = (dY/dr)^T [sum_nz C sum_u g (gg_x W + gg_w x)]
+                        + sum_m2 gY[e,m2] (d2Y[e,m2]/dr2) gg_r[e].
+    Returns (d_x, d_w, d_grad_out, d_edge_vec) in fp64.
+    """
+    row_ptr = np.asarray(row_ptr, dtype=np.int64)
+    src = np.asarray(col, dtype=np.int64)
+    dst = edge_dst(row_ptr).astype(np.int64)
+    ev = np.asarray(edge_vec, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    g = np.asarray(grad_out, dtype=np.float64)
+    n, u = row_ptr.size - 1, x.shape[2]
+    E, P = src.size, w.shape[1]
+    ns = (lmax_sh + 1) ** 2
+    ggx = np.zeros_like(x) if gg_x is None else np.asarray(gg_x, dtype=np.float64)
+    ggw = np.zeros_like(w) if gg_w is None else np.asarray(gg_w, dtype=np.float64)
+    ggr = np.zeros((E, 3)) if gg_r is None else np.asarray(gg_r, dtype=np.float64)
+    Y = real_sh(ev, lmax_sh)
+    J = real_sh_jacobian(ev, lmax_sh)
+    H = real_sh_hessian(ev, lmax_sh)
+    uY = np.einsum("ebk,ek->eb", J, ggr)
+    xs, gd, ggxs = x[src], g[dst], ggx[src]
+    d_g_edge = np.zeros((E, g.shape[1], u))
+    d_x_edge = np.zeros((E, x.shape[1], u))
+    d_w = np.zeros((E, P, u))
+    dY_expl = np.zeros((E, ns))
+    gY = np.zeros((E, ns))
+    for p, ri, rs, ro, c in path_nonzeros(lmax_in, lmax_sh, lmax_out):
+        Yc, uc = Y[:, rs][:, None], uY[:, rs][:, None]
+        Wp, ggwp = w[:, p, :], ggw[:, p, :]
+        d_g_edge[:, ro, :] += c * (ggxs[:, ri, :] * Wp * Yc + ggwp * xs[:, ri, :] * Yc + uc * Wp * xs[:, ri, :])
+        d_x_edge[:, ri, :] += c * gd[:, ro, :] * (ggwp * Yc + uc * Wp)
+        d_w[:, p, :] += c * gd[:, ro, :] * (ggxs[:, ri, :] * Yc + uc * xs[:, ri, :])
+        dY_expl[:, rs] += c * np.sum(gd[:, ro, :] * (ggxs[:, ri, :] * Wp + ggwp * xs[:, ri, :]), axis=1)
+        gY[:, rs] += c * np.sum(Wp * xs[:, ri, :] * gd[:, ro, :], axis=1)
+    d_g = np.zeros_like(g)
+    np.add.at(d_g, dst, d_g_edge)
+    d_x = np.zeros_like(x)
+    np.add.at(d_x, src, d_x_edge)
+    d_r = np.einsum("eb,ebk->ek", dY_expl, J) + np.einsum("eb,ebjk,ek->ej", gY, H, ggr)
+    return d_x, d_w, d_g, d_r
+

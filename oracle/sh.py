@@ -40,8 +40,8 @@ def _legendre_deriv_coeffs(l, m):
 
 def _re_im_power(x, y, m):
     """Re and Im of (x + i y)^m as real polynomials in x and y (binomial sum)."""
-    re = np.zeros_like(x)
-    im = np.zeros_like(x)
+    re = 0 * x
+    im = 0 * x
     for p in range(m + 1):
         term = math.comb(m, p) * x ** (m - p) * y ** p
         # i^p cycles 1, i, -1, -i
@@ -57,8 +57,10 @@ def _re_im_power(x, y, m):
     return re, im
 
 
-def _sh_unit(x, y, z, lmax):
-    """Real harmonics of a unit vector given by arrays x, y, z (real or complex)."""
+def _sh_blocks(x, y, z, lmax):
+    """The (lmax+1)^2 real harmonics of a unit vector given by x, y, z, as a
+    list in lm order; x, y, z may be real or complex arrays or any number type
+    with +, -, * and integer powers."""
     out = []
     for l in range(lmax + 1):
         block = [None] * (2 * l + 1)
@@ -72,7 +74,12 @@ def _sh_unit(x, y, z, lmax):
                 block[l + m] = norm * dP * re
                 block[l - m] = norm * dP * im
         out.extend(block)
-    return np.stack(out, axis=-1)
+    return out
+
+
+def _sh_unit(x, y, z, lmax):
+    """Real harmonics of a unit vector given by arrays x, y, z (real or complex)."""
+    return np.stack(_sh_blocks(x, y, z, lmax), axis=-1)
 
 
 def real_sh(vec, lmax):
@@ -138,3 +145,20 @@ def real_sh_legendre(vec, lmax):
             block[l - m] = norm * P[(l, m)] * np.sin(m * phi)
         out.extend(block)
     return np.stack(out, axis=-1)
+
+
+def real_sh_hessian(vec, lmax):
+    """d2Y_lm(vec/|vec|)/dvec2, shape [..., (lmax+1)^2, 3, 3], by second-order
+    forward-mode differentiation (``oracle.jet``) of the same polynomial
+    harmonics of the normalised vector.  Zero vectors get a zero Hessian."""
+    from .jet import Jet
+    v = np.asarray(vec, dtype=np.float64)
+    r2 = np.sum(v * v, axis=-1)
+    safe = np.where(r2 > 0, 1.0, 0.0)[..., None] * v + np.where(r2 > 0, 0.0, 1.0)[..., None] * np.array([0.0, 0.0, 1.0])
+    x, y, z = Jet.variables(safe)
+    inv = (x * x + y * y + z * z).sqrt().reciprocal()
+    blocks = _sh_blocks(x * inv, y * inv, z * inv, lmax)
+    H = np.stack([b.h for b in blocks], axis=-3)
+    H[r2 == 0] = 0.0
+    return H
+
