@@ -197,6 +197,38 @@ class Plan:
              workspace.numel() * 4 if (want_r and workspace is not None) else 0, _stream())
         return (grad_x if want_x else None, grad_w if want_w else None, grad_edge_vec if want_r else None)
 
+    def conv_double_backward_workspace_bytes(self, n_edges):
+        b = ctypes.c_size_t()
+        call("cgtp_conv_double_backward_workspace_size", self._h, n_edges, ctypes.byref(b))
+        return b.value
+
+    def conv_double_backward(self, graph, x, w, grad_out, gg_x=None, gg_w=None, gg_edge_vec=None,
+                             want_x=True, want_w=True, want_grad_out=True, want_r=True, workspace=None):
+        """Adjoint of conv_backward: gradients of <gg_x, grad_x> + <gg_w, grad_w>
+        + <gg_edge_vec, grad_edge_vec> with respect to (x, w, grad_out, edge_vec)."""
+        for t, nm in ((x, "x"), (w, "w"), (grad_out, "grad_out")):
+            _check(t, torch.float32, nm)
+        for t, nm in ((gg_x, "gg_x"), (gg_w, "gg_w"), (gg_edge_vec, "gg_edge_vec")):
+            if t is not None:
+                _check(t, torch.float32, nm)
+        dev = x.device
+        E = graph.n_edges
+        d_x = torch.empty_like(x) if want_x else None
+        d_w = torch.empty((E, self.n_paths, self.mult), dtype=torch.float32, device=dev) if want_w else None
+        d_g = torch.empty_like(grad_out) if want_grad_out else None
+        d_r = torch.empty((E, 3), dtype=torch.float32, device=dev) if want_r else None
+        nb = 0
+        if want_r or gg_edge_vec is not None:
+            nb = self.conv_double_backward_workspace_bytes(E)
+            if workspace is None:
+                workspace = torch.empty(max(nb // 4, 64), dtype=torch.float32, device=dev)
+        call("cgtp_conv_double_backward", self._h, graph.n_nodes, E, _ptr(graph.row_ptr), _ptr(graph.col),
+             _ptr(graph.csc_ptr), _ptr(graph.csc_edge), _ptr(graph.csc_dst), _ptr(graph.edge_vec), _ptr(x),
+             _ptr(w), _ptr(grad_out), _ptr(gg_x), _ptr(gg_w), _ptr(gg_edge_vec), _ptr(d_x), _ptr(d_w), _ptr(d_g),
+             _ptr(d_r), _ptr(workspace if nb else None), workspace.numel() * 4 if (nb and workspace is not None) else 0,
+             _stream())
+        return d_x, d_w, d_g, d_r
+
     # ------------------------------------------------------------ radial network
     def radial_forward(self, edge_vec, rc, W1, W2, out=None):
         _check(edge_vec, torch.float32, "edge_vec")

@@ -292,6 +292,144 @@ cgtp_status cgtp_conv_backward(cgtp_plan p, int n_nodes, int n_edges, const int*
   return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
 }
 
+// ---- double backward: the adjoint of cgtp_conv_backward ----
+static cudaError_t dispatch_fwd(cgtp_plan p, const ConvFwdArgs& a, int sms, cudaStream_t s) {
+  cudaError_t e = cudaErrorNotSupported;
+#define CGTP_DFWD_ENTRY(A, B, C) \
+  if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_fwd<A, B, C>(a, sms, s);
+  CGTP_CONFIGS(CGTP_DFWD_ENTRY)
+  return e;
+}
+static cudaError_t dispatch_bwd(cgtp_plan p, const ConvBwdArgs& a, int sms, cudaStream_t s) {
+  cudaError_t e = cudaErrorNotSupported;
+#define CGTP_DBWD_ENTRY(A, B, C) \
+  if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_bwd<A, B, C>(a, sms, s);
+  CGTP_CONFIGS(CGTP_DBWD_ENTRY)
+  return e;
+}
+
+cgtp_status cgtp_conv_double_backward_workspace_size(cgtp_plan p, int n_edges, size_t* bytes) {
+  if (p == nullptr || n_edges < 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
+  const size_t ns = (size_t)(p->ls + 1) * (p->ls + 1);
+  const size_t u = (sizeof(float) * (size_t)n_edges * ns + 255) & ~(size_t)255;
+  size_t bw = 0;
+  cgtp_conv_backward_workspace_size(p, n_edges, &bw);
+  *bytes = u + bw;
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_conv_double_backward(cgtp_plan p, int n_nodes, int n_edges, const int* row_ptr, const int* col,
+                                      const int* csc_ptr, const int* csc_edge, const int* csc_dst,
+                                      const float* edge_vec, const float* x, const float* w, const float* grad_out,
+                                      const float* gg_x, const float* gg_w, const float* gg_edge_vec, float* d_x,
+                                      float* d_w, float* d_grad_out, float* d_edge_vec, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (p == nullptr || n_nodes < 0 || n_edges < 0 || row_ptr == nullptr || csc_ptr == nullptr)
+    return CGTP_ERR_INVALID_ARG;
+  if (n_nodes > 0 && (x == nullptr || grad_out == nullptr)) return CGTP_ERR_INVALID_ARG;
+  if (n_edges > 0 && (col == nullptr || csc_edge == nullptr || csc_dst == nullptr || edge_vec == nullptr ||
+                      w == nullptr))
+    return CGTP_ERR_INVALID_ARG;
+  for (const void* q : {(const void*)x, (const void*)w, (const void*)grad_out, (const void*)gg_x, (const void*)gg_w,
+                        (const void*)d_x, (const void*)d_w, (const void*)d_grad_out})
+    if (!aligned16(q)) return CGTP_ERR_INVALID_ARG;
+  const size_t ns = (size_t)(p->ls + 1) * (p->ls + 1);
+  const size_t u_bytes = (sizeof(float) * (size_t)n_edges * ns + 255) & ~(size_t)255;
+  const bool need_ws = n_edges > 0 && (gg_edge_vec != nullptr || d_edge_vec != nullptr);
+  if (need_ws) {
+    size_t need = 0;
+    cgtp_conv_double_backward_workspace_size(p, n_edges, &need);
+    if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
+      return CGTP_ERR_WORKSPACE;
+  }
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (n_nodes == 0) return CGTP_OK;
+  const size_t nx = (size_t)n_nodes * (p->li + 1) * (p->li + 1) * p->mult;
+  const size_t ng = (size_t)n_nodes * (p->lo + 1) * (p->lo + 1) * p->mult;
+  const size_t nw = (size_t)n_edges * p->n_paths * p->mult;
+  cudaError_t e = cudaSuccess;
+  auto zero = [&](float* q, size_t n) {
+    if (q != nullptr && n > 0 && e == cudaSuccess) e = cudaMemsetAsync(q, 0, sizeof(float) * n, s);
+  };
+  if (n_edges == 0) {  // nothing depends on anything: every gradient is zero
+    zero(d_x, nx);
+    zero(d_grad_out, ng);
+    return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+  }
+  float* uY = need_ws ? (float*)workspace : nullptr;                      // [E][NS] = (dY/dr) gg_edge_vec
+  float* gsh = need_ws ? (float*)((char*)workspace + u_bytes) : nullptr;  // harmonic-gradient partials
+  const bool gr = gg_edge_vec != nullptr;
+  if (gr) e = launch_sh_dir(p->ls, n_edges, edge_vec, gg_edge_vec, uY, sms, s);
+
+  // d grad_out: forward convolutions with one argument replaced at a time
+  //   (Y -> uY), (x -> gg_x), (W -> gg_w), summed
+  if (d_grad_out != nullptr) {
+    bool init = false;
+    auto fwd = [&](const float* xx, const float* ww, const float* sh) {
+      if (e != cudaSuccess) return;
+      ConvFwdArgs a{n_nodes, row_ptr, col, edge_vec, xx, ww, d_grad_out, p->mult};
+      a.sh = sh;
+      a.accumulate = init ? 1 : 0;
+      e = dispatch_fwd(p, a, sms, s);
+      init = true;
+    };
+    if (gr) fwd(x, w, uY);
+    if (gg_x) fwd(gg_x, w, nullptr);
+    if (gg_w) fwd(x, gg_w, nullptr);
+    if (!init) zero(d_grad_out, ng);
+  }
+
+  // d x and d W: backward convolutions, (Y -> uY) for both, then
+  //   d x += grad_x with W -> gg_w and d W += grad_w with x -> gg_x (one launch)
+  if (d_x != nullptr || d_w != nullptr) {
+    bool init_x = false, init_w = false;
+    if (gr && e == cudaSuccess) {
+      ConvBwdArgs a{n_nodes, n_edges, csc_ptr, csc_edge, csc_dst, edge_vec, x, w, grad_out,
+                    d_x, d_w, nullptr, nullptr, p->mult};
+      a.sh = uY;
+      e = dispatch_bwd(p, a, sms, s);
+      init_x = d_x != nullptr;
+      init_w = d_w != nullptr;
+    }
+    float* ox = gg_w ? d_x : nullptr;
+    float* ow = gg_x ? d_w : nullptr;
+    if ((ox != nullptr || ow != nullptr) && e == cudaSuccess) {
+      // the two outputs accumulate together: both were written above or neither
+      ConvBwdArgs a{n_nodes, n_edges, csc_ptr, csc_edge, csc_dst, edge_vec, gg_x ? gg_x : x, gg_w ? gg_w : w,
+                    grad_out, ox, ow, nullptr, nullptr, p->mult};
+      a.accumulate = gr ? 1 : 0;
+      e = dispatch_bwd(p, a, sms, s);
+      init_x = init_x || ox != nullptr;
+      init_w = init_w || ow != nullptr;
+    }
+    if (!init_x) zero(d_x, nx);
+    if (!init_w) zero(d_w, nw);
+  }
+
+  // d edge_vec: (dY/dr)^T of the harmonic gradients with x -> gg_x and with
+  //   W -> gg_w, plus sum_b G_b (d2Y_b/dr2) gg_edge_vec with G the backward's own
+  if (d_edge_vec != nullptr) {
+    bool init = false;
+    auto gy = [&](const float* xx, const float* ww, int mode_set, int mode_add) {
+      if (e != cudaSuccess) return;
+      ConvBwdArgs a{n_nodes, n_edges, csc_ptr, csc_edge, csc_dst, edge_vec, xx, ww, grad_out,
+                    nullptr, nullptr, d_edge_vec, gsh, p->mult};
+      a.gr_mode = init ? mode_add : mode_set;
+      a.gr_dir = gg_edge_vec;
+      e = dispatch_bwd(p, a, sms, s);
+      init = true;
+    };
+    if (gg_x) gy(gg_x, w, 0, 1);
+    if (gg_w) gy(x, gg_w, 0, 1);
+    if (gr) gy(x, w, 3, 2);
+    if (!init) zero(d_edge_vec, (size_t)n_edges * 3);
+  }
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
 cgtp_status cgtp_forces(int n_nodes, int n_edges, const int* row_ptr, const int* csc_ptr, const int* csc_edge,
                         const float* grad_edge_vec, float* forces, void* stream) {
   if (n_nodes < 0 || n_edges < 0 || row_ptr == nullptr || csc_ptr == nullptr) return CGTP_ERR_INVALID_ARG;

@@ -109,6 +109,10 @@ struct ConvFwdArgs {
   const float* w;
   float* out;
   int mult;
+  // optional: per-edge harmonics [n_edges][(L_sh+1)^2] used instead of
+  // Y(edge_vec) (the double backward substitutes directional derivatives)
+  const float* sh = nullptr;
+  int accumulate = 0;  // add onto out instead of overwriting it
 };
 
 struct ConvBwdArgs {
@@ -126,6 +130,13 @@ struct ConvBwdArgs {
   float* grad_edge_vec;
   float* grad_sh;   // workspace [slices][n_edges][NS]
   int mult;
+  const float* sh = nullptr;  // optional per-edge harmonics replacing Y(edge_vec)
+  int accumulate = 0;         // add onto grad_x and grad_w instead of overwriting them
+  // grad_edge_vec from the harmonic gradient G (summed over the slices):
+  // 0: = (dY/dr)^T G, 1: += (dY/dr)^T G, 2: += sum_b G_b (d2Y_b/dr2) gr_dir,
+  // 3: = sum_b G_b (d2Y_b/dr2) gr_dir
+  int gr_mode = 0;
+  const float* gr_dir = nullptr;  // [n_edges][3], for gr_mode 2 and 3
 };
 
 struct TPArgs {

@@ -76,7 +76,7 @@ constexpr unsigned touched_sh_mask() {
 // rows come from this lane's pipeline stage.
 template <class PS, class GR, int VEC, bool NEED_GY>
 __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const float* __restrict__ stage, int rowf,
-                                         const float (&xr)[GR::NOWN][VEC], float* __restrict__ gwrow, int mult,
+                                         const float (&xr)[GR::NOWN][VEC], float* __restrict__ gwrow, bool acc, int mult,
                                          float (&gx)[GR::NOWN][VEC], float* __restrict__ gyrow, int rs) {
   float gy[PS::NS];
   static_for<0, GR::NP>([&](auto Kc) {
@@ -140,7 +140,15 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
         gx[m1][c] = fmaf(wv[c], h[m1][c], gx[m1][c]);
         gw[c] = fmaf(xr[m1][c], h[m1][c], gw[c]);
       }
-    if (gwrow != nullptr) VecIO<VEC>::st_stream(gwrow + P * mult, gw);
+    if (gwrow != nullptr) {
+      if (acc) {
+        float prev[VEC];
+        VecIO<VEC>::ld(prev, gwrow + P * mult);
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) gw[c] += prev[c];
+      }
+      VecIO<VEC>::st_stream(gwrow + P * mult, gw);
+    }
     if constexpr (NEED_GY && GR::D.last_l2[K]) {
 #pragma unroll
       for (int m2 = 0; m2 < 2 * l2 + 1; ++m2) gyrow[(l2 * l2 + m2) * rs] = gy[l2 * l2 + m2];
@@ -251,8 +259,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
         if (active && kk < k1) {
           const int e = __ldg(a.csc_edge + kk);
           float Y[NS];
-          sh_of_vec<PS::LS>(__ldg(a.edge_vec + 3 * (long long)e), __ldg(a.edge_vec + 3 * (long long)e + 1),
-                            __ldg(a.edge_vec + 3 * (long long)e + 2), Y);
+          edge_sh<PS::LS>(a.sh, a.edge_vec, e, Y);
           compute_T_grp<PS, GR>(Y, Tg + k * NT);
           Eg[k] = e;
           Ig[k] = __ldg(a.csc_dst + kk);
@@ -272,7 +279,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
           e = Eg[k];
           bwd_edge<PS, GR, VEC, NEED_GY>(Tg + k * NT, St + (k & 1) * stage_floats + gl * VEC, rowf, xr,
                                          a.grad_w ? a.grad_w + (long long)e * PS::NP * mult + c0 : nullptr,
-                                         mult, gx, red + gl, rs);
+                                         a.accumulate != 0, mult, gx, red + gl, rs);
         }
         if constexpr (NEED_GY) {
           __syncwarp();
@@ -305,10 +312,10 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
       __syncwarp();
     }
     if (active && a.grad_x != nullptr) {
-      if constexpr (!GR::FIRST) {
-        // rows of an l1 block that an earlier chunk of this call wrote: wait
-        // for that grid (the preceding launch) and add onto its values
-        grid_dependency_wait();
+      if (!GR::FIRST || a.accumulate) {
+        // rows of an l1 block that an earlier chunk of this call wrote (wait
+        // for that grid, the preceding launch), or the caller's values
+        if constexpr (!GR::FIRST) grid_dependency_wait();
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
           float prev[VEC];
@@ -323,10 +330,10 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
   }
 }
 
-// grad_edge_vec[e] = (dY_e/dr_e)^T sum_s grad_sh[s][e]
+// grad_edge_vec[e] (= or +=) (dY_e/dr_e)^T sum_s grad_sh[s][e]
 template <int LS>
 __global__ void sh_backward_kernel(int n_edges, int S, const float* __restrict__ edge_vec,
-                                   const float* __restrict__ grad_sh, float* __restrict__ grad_edge_vec) {
+                                   const float* __restrict__ grad_sh, float* __restrict__ grad_edge_vec, int add) {
   constexpr int NS = (LS + 1) * (LS + 1);
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n_edges;
        e += (long long)gridDim.x * blockDim.x) {
@@ -346,6 +353,49 @@ __global__ void sh_backward_kernel(int n_edges, int S, const float* __restrict__
       d0 = fmaf(g[b], Y[b].d0, d0);
       d1 = fmaf(g[b], Y[b].d1, d1);
       d2 = fmaf(g[b], Y[b].d2, d2);
+    }
+    if (add) {
+      d0 += grad_edge_vec[3 * e];
+      d1 += grad_edge_vec[3 * e + 1];
+      d2 += grad_edge_vec[3 * e + 2];
+    }
+    grad_edge_vec[3 * e] = d0;
+    grad_edge_vec[3 * e + 1] = d1;
+    grad_edge_vec[3 * e + 2] = d2;
+  }
+}
+
+// grad_edge_vec[e] (= or +=) sum_b G_b (d2Y_b/dr2) q_e with G = sum_s grad_sh[s][e]:
+// the second-order term of the double backward (q = the cotangent of grad_edge_vec).
+template <int LS>
+__global__ void sh_backward_hess_kernel(int n_edges, int S, const float* __restrict__ edge_vec,
+                                        const float* __restrict__ grad_sh, const float* __restrict__ q,
+                                        float* __restrict__ grad_edge_vec, int add) {
+  constexpr int NS = (LS + 1) * (LS + 1);
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n_edges;
+       e += (long long)gridDim.x * blockDim.x) {
+    float g[NS];
+#pragma unroll
+    for (int b = 0; b < NS; ++b) g[b] = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float* src = grad_sh + ((long long)s * n_edges + e) * NS;
+#pragma unroll
+      for (int b = 0; b < NS; ++b) g[b] += src[b];
+    }
+    HDual Y[NS];
+    sh_hess_of_vec<LS>(edge_vec[3 * e], edge_vec[3 * e + 1], edge_vec[3 * e + 2], q[3 * e], q[3 * e + 1],
+                       q[3 * e + 2], Y);
+    float d0 = 0.f, d1 = 0.f, d2 = 0.f;
+#pragma unroll
+    for (int b = 0; b < NS; ++b) {
+      d0 = fmaf(g[b], Y[b].d0.e, d0);
+      d1 = fmaf(g[b], Y[b].d1.e, d1);
+      d2 = fmaf(g[b], Y[b].d2.e, d2);
+    }
+    if (add) {
+      d0 += grad_edge_vec[3 * e];
+      d1 += grad_edge_vec[3 * e + 1];
+      d2 += grad_edge_vec[3 * e + 2];
     }
     grad_edge_vec[3 * e] = d0;
     grad_edge_vec[3 * e + 1] = d1;
@@ -439,7 +489,7 @@ cudaError_t zero_unreached_grad_x(const ConvBwdArgs& a, cudaStream_t stream) {
 template <class PS, bool NEED_GY>
 cudaError_t launch_bwd_chunks(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
   constexpr int NCH = BwdPlan<PS, bwd_vec<PS>(), NEED_GY>::N;
-  cudaError_t err = zero_unreached_grad_x<PS>(a, stream);
+  cudaError_t err = a.accumulate ? cudaSuccess : zero_unreached_grad_x<PS>(a, stream);
   static_for_host<0, NCH>([&](auto Cc) {
     if (err == cudaSuccess) err = launch_bwd_chunk<PS, NEED_GY, decltype(Cc)::value>(a, num_sms, stream);
   });
@@ -455,8 +505,15 @@ cudaError_t launch_conv_bwd(const ConvBwdArgs& a, int num_sms, cudaStream_t stre
   const int threads = 256;
   long long nbk = (a.n_edges + threads - 1) / threads;
   if (nbk > (long long)num_sms * 16) nbk = (long long)num_sms * 16;
-  sh_backward_kernel<LS><<<(unsigned)nbk, threads, 0, stream>>>(a.n_edges, conv_bwd_slices<LI, LS, LO>(a.mult),
-                                                                 a.edge_vec, a.grad_sh, a.grad_edge_vec);
+  const int S = conv_bwd_slices<LI, LS, LO>(a.mult);
+  if (a.gr_mode >= 2) {
+    if (a.gr_dir == nullptr) return cudaErrorInvalidValue;
+    sh_backward_hess_kernel<LS><<<(unsigned)nbk, threads, 0, stream>>>(a.n_edges, S, a.edge_vec, a.grad_sh, a.gr_dir,
+                                                                      a.grad_edge_vec, a.gr_mode == 2);
+  } else {
+    sh_backward_kernel<LS><<<(unsigned)nbk, threads, 0, stream>>>(a.n_edges, S, a.edge_vec, a.grad_sh,
+                                                                 a.grad_edge_vec, a.gr_mode == 1);
+  }
   return cudaGetLastError();
 }
 

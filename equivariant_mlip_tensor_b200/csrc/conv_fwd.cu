@@ -239,8 +239,7 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
         const int e = e0 + b0 + k;
         if (active && e < e1) {
           float Y[NS];
-          sh_of_vec<PS::LS>(__ldg(a.edge_vec + 3 * (long long)e), __ldg(a.edge_vec + 3 * (long long)e + 1),
-                            __ldg(a.edge_vec + 3 * (long long)e + 2), Y);
+          edge_sh<PS::LS>(a.sh, a.edge_vec, e, Y);
           compute_T_grp<PS, GR>(Y, Tg + k * NT);
         }
       }
@@ -258,9 +257,10 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
       __syncwarp();
     }
     if (active) {
-      if constexpr (!GR::FIRST) {
-        // rows of an l3 block that the preceding launch wrote: wait for it, add
-        grid_dependency_wait();
+      if (!GR::FIRST || a.accumulate) {
+        // rows of an l3 block that the preceding launch wrote (wait for it),
+        // or the caller's values to add onto
+        if constexpr (!GR::FIRST) grid_dependency_wait();
 #pragma unroll
         for (int r = 0; r < GR::NOWN; ++r) {
           float prev[kFwdVec];
@@ -341,7 +341,7 @@ cudaError_t launch_conv_fwd(const ConvFwdArgs& a, int num_sms, cudaStream_t stre
     // all paths in one launch (it writes every output row, reached or not)
     return launch_fwd_group<PS, Grp<PS, kAll, 0>>(a, num_sms, false, stream);
   } else {
-    cudaError_t err = zero_unreached_out<PS>(a, stream);
+    cudaError_t err = a.accumulate ? cudaSuccess : zero_unreached_out<PS>(a, stream);
     static_for_host<0, FwdPlan<PS>::N>([&](auto Cc) {
       constexpr int CH = decltype(Cc)::value;
       // every chunk but the call's first may overlap the one before it

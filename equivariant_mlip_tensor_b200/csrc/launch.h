@@ -35,5 +35,7 @@ cudaError_t launch_forces(int n, const int* row_ptr, const int* csc_ptr, const i
                           float* F, int num_sms, cudaStream_t stream);
 cudaError_t launch_sh(int lmax_sh, int n_edges, const float* ev, float* Y, float* dY, int num_sms,
                       cudaStream_t stream);
+cudaError_t launch_sh_dir(int lmax_sh, int n_edges, const float* ev, const float* q, float* u, int num_sms,
+                          cudaStream_t stream);
 
 }  // namespace cgtp

@@ -64,7 +64,37 @@ __global__ void sh_kernel(int n_edges, const float* __restrict__ ev, float* __re
   }
 }
 
+// u[e] = (dY_e/dr_e) q[e]: the harmonics' derivative along a per-edge direction.
+template <int LS>
+__global__ void sh_dir_kernel(int n_edges, const float* __restrict__ ev, const float* __restrict__ q,
+                              float* __restrict__ u) {
+  constexpr int NS = (LS + 1) * (LS + 1);
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n_edges;
+       e += (long long)gridDim.x * blockDim.x) {
+    Dual1 y[NS];
+    sh_dir_of_vec<LS>(ev[3 * e], ev[3 * e + 1], ev[3 * e + 2], q[3 * e], q[3 * e + 1], q[3 * e + 2], y);
+#pragma unroll
+    for (int b = 0; b < NS; ++b) u[e * NS + b] = y[b].e;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_sh_dir(int lmax_sh, int n_edges, const float* ev, const float* q, float* u, int num_sms,
+                          cudaStream_t stream) {
+  if (n_edges == 0) return cudaSuccess;
+  long long b = ((long long)n_edges + 127) / 128;
+  if (b > num_sms * 16LL) b = num_sms * 16LL;
+  switch (lmax_sh) {
+    case 0: sh_dir_kernel<0><<<(int)b, 128, 0, stream>>>(n_edges, ev, q, u); break;
+    case 1: sh_dir_kernel<1><<<(int)b, 128, 0, stream>>>(n_edges, ev, q, u); break;
+    case 2: sh_dir_kernel<2><<<(int)b, 128, 0, stream>>>(n_edges, ev, q, u); break;
+    case 3: sh_dir_kernel<3><<<(int)b, 128, 0, stream>>>(n_edges, ev, q, u); break;
+    case 4: sh_dir_kernel<4><<<(int)b, 128, 0, stream>>>(n_edges, ev, q, u); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
 
 cudaError_t launch_forces(int n, const int* row_ptr, const int* csc_ptr, const int* csc_edge, const float* g,
                           float* F, int num_sms, cudaStream_t stream) {

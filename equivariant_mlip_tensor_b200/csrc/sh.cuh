@@ -37,6 +37,41 @@ __device__ __forceinline__ Dual3 operator*(float s, const Dual3& a) {
   return Dual3(s * a.v, s * a.d0, s * a.d1, s * a.d2);
 }
 
+// Value plus derivative along one direction q: f + t q.grad f (first order).
+struct Dual1 {
+  float v, e;
+  __device__ __forceinline__ Dual1() : v(0.f), e(0.f) {}
+  __device__ __forceinline__ explicit Dual1(float c) : v(c), e(0.f) {}
+  __device__ __forceinline__ Dual1(float a, float b) : v(a), e(b) {}
+};
+__device__ __forceinline__ Dual1 operator+(const Dual1& a, const Dual1& b) { return Dual1(a.v + b.v, a.e + b.e); }
+__device__ __forceinline__ Dual1 operator-(const Dual1& a, const Dual1& b) { return Dual1(a.v - b.v, a.e - b.e); }
+__device__ __forceinline__ Dual1 operator*(const Dual1& a, const Dual1& b) {
+  return Dual1(a.v * b.v, fmaf(a.v, b.e, a.e * b.v));
+}
+__device__ __forceinline__ Dual1 operator*(float s, const Dual1& a) { return Dual1(s * a.v, s * a.e); }
+
+// Gradient with respect to the edge vector of a Dual1-valued function: the
+// t-part of component k is (d2f/dr2 q)_k, a Hessian-vector product.
+struct HDual {
+  Dual1 v, d0, d1, d2;
+  __device__ __forceinline__ HDual() {}
+  __device__ __forceinline__ explicit HDual(float c) : v(c) {}
+  __device__ __forceinline__ HDual(Dual1 a, Dual1 b, Dual1 c, Dual1 d) : v(a), d0(b), d1(c), d2(d) {}
+};
+__device__ __forceinline__ HDual operator+(const HDual& a, const HDual& b) {
+  return HDual(a.v + b.v, a.d0 + b.d0, a.d1 + b.d1, a.d2 + b.d2);
+}
+__device__ __forceinline__ HDual operator-(const HDual& a, const HDual& b) {
+  return HDual(a.v - b.v, a.d0 - b.d0, a.d1 - b.d1, a.d2 - b.d2);
+}
+__device__ __forceinline__ HDual operator*(const HDual& a, const HDual& b) {
+  return HDual(a.v * b.v, a.v * b.d0 + a.d0 * b.v, a.v * b.d1 + a.d1 * b.v, a.v * b.d2 + a.d2 * b.v);
+}
+__device__ __forceinline__ HDual operator*(float s, const HDual& a) {
+  return HDual(s * a.v, s * a.d0, s * a.d1, s * a.d2);
+}
+
 __device__ __forceinline__ float scal(float c) { return c; }
 
 template <class S>
@@ -111,6 +146,62 @@ static __device__ __forceinline__ void sh_grad_of_vec(float vx, float vy, float 
 #pragma unroll
     for (int k = 0; k < (LS + 1) * (LS + 1); ++k) Y[k] = Dual3(0.f);
     Y[0] = Dual3(1.f);
+  }
+}
+
+// Directional derivative (dY/dr) q of the harmonics: Y[b].e for every b.
+template <int LS>
+static __device__ __forceinline__ void sh_dir_of_vec(float vx, float vy, float vz, float qx, float qy, float qz,
+                                                     Dual1 (&Y)[(LS + 1) * (LS + 1)]) {
+  const float r2 = fmaf(vx, vx, fmaf(vy, vy, vz * vz));
+  if (r2 > 0.f) {
+    const float inv = rsqrtf(r2);
+    // d(r2^-1/2) = -r2^-3/2 (v . q) along q
+    const float vq = fmaf(vx, qx, fmaf(vy, qy, vz * qz));
+    const Dual1 invd(inv, -inv * inv * inv * vq);
+    sh_unit<LS, Dual1>(Dual1(vx, qx) * invd, Dual1(vy, qy) * invd, Dual1(vz, qz) * invd, Y);
+  } else {
+#pragma unroll
+    for (int k = 0; k < (LS + 1) * (LS + 1); ++k) Y[k] = Dual1(0.f);
+    Y[0] = Dual1(1.f);
+  }
+}
+
+// Harmonics with their gradient and the Hessian-vector product along q:
+// Y[b].dk.v = dY_b/dr_k and Y[b].dk.e = (d2Y_b/dr2 q)_k.
+template <int LS>
+static __device__ __forceinline__ void sh_hess_of_vec(float vx, float vy, float vz, float qx, float qy, float qz,
+                                                      HDual (&Y)[(LS + 1) * (LS + 1)]) {
+  const float r2 = fmaf(vx, vx, fmaf(vy, vy, vz * vz));
+  if (r2 > 0.f) {
+    const Dual1 one(1.f), zero(0.f);
+    const HDual X(Dual1(vx, qx), one, zero, zero), Yv(Dual1(vy, qy), zero, one, zero),
+        Z(Dual1(vz, qz), zero, zero, one);
+    // s = r2 as an HDual, then s^-1/2 by the chain rule at both orders:
+    // f = s^-1/2, f' = -s^-3/2 / 2, f'' = 3 s^-5/2 / 4, each carried along q.
+    const HDual s = X * X + Yv * Yv + Z * Z;
+    const float inv = rsqrtf(s.v.v);
+    const float f0 = inv, f1 = -0.5f * inv * inv * inv, f2 = 0.75f * inv * inv * inv * inv * inv;
+    const Dual1 fs(f0, f1 * s.v.e), dfs(f1, f2 * s.v.e);
+    const HDual invd(fs, dfs * s.d0, dfs * s.d1, dfs * s.d2);
+    sh_unit<LS, HDual>(X * invd, Yv * invd, Z * invd, Y);
+  } else {
+#pragma unroll
+    for (int k = 0; k < (LS + 1) * (LS + 1); ++k) Y[k] = HDual(0.f);
+    Y[0] = HDual(1.f);
+  }
+}
+
+// Harmonics of edge e: the caller's per-edge values when given, else Y(edge_vec[e]).
+template <int LS>
+static __device__ __forceinline__ void edge_sh(const float* __restrict__ sh, const float* __restrict__ edge_vec,
+                                               long long e, float (&Y)[(LS + 1) * (LS + 1)]) {
+  constexpr int NS = (LS + 1) * (LS + 1);
+  if (sh != nullptr) {
+#pragma unroll
+    for (int b = 0; b < NS; ++b) Y[b] = __ldg(sh + e * NS + b);
+  } else {
+    sh_of_vec<LS>(__ldg(edge_vec + 3 * e), __ldg(edge_vec + 3 * e + 1), __ldg(edge_vec + 3 * e + 2), Y);
   }
 }
 

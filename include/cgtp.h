@@ -175,6 +175,39 @@ cgtp_status cgtp_conv_backward(cgtp_plan plan, int n_nodes, int n_edges,
                                float* grad_edge_vec, void* workspace, size_t workspace_bytes,
                                void* stream);
 
+/* Bytes of device workspace cgtp_conv_double_backward needs when
+ * gg_edge_vec or d_edge_vec is given. */
+cgtp_status cgtp_conv_double_backward_workspace_size(cgtp_plan plan, int n_edges, size_t* bytes);
+
+/* ---------------------------------------------------------------------------
+ * Double backward: the adjoint of cgtp_conv_backward, the higher-order
+ * derivative that force training needs ("LunaTP ...", abstract: derivative
+ * computation).  With (grad_x, grad_w, grad_edge_vec) the outputs of
+ * cgtp_conv_backward for (x, w, grad_out, edge_vec) and cotangents gg_x
+ * [n_nodes][(lmax_in+1)^2][mult], gg_w [n_edges][n_paths][mult] and
+ * gg_edge_vec [n_edges][3] (each nullable = zero), the call returns the
+ * gradients of
+ *   L = <gg_x, grad_x> + <gg_w, grad_w> + <gg_edge_vec, grad_edge_vec>
+ * with respect to x (d_x), w (d_w), grad_out (d_grad_out) and the edge
+ * vectors (d_edge_vec), each nullable (not computed) and overwritten.
+ * Every term is one of the first-order convolutions with one argument
+ * replaced (Y by (dY/dr) gg_edge_vec, x by gg_x, W by gg_w), plus
+ * sum_b G_b (d2Y_b/dr2) gg_edge_vec with G the backward's harmonic gradient;
+ * all run in this library's kernels.  Needs both graph views (CSR for the
+ * d_grad_out sums, CSC for d_x).  When gg_edge_vec or d_edge_vec is given,
+ * workspace (device, 256-byte aligned) of the size reported by
+ * cgtp_conv_double_backward_workspace_size is required
+ * (CGTP_ERR_WORKSPACE otherwise).
+ * ------------------------------------------------------------------------- */
+cgtp_status cgtp_conv_double_backward(cgtp_plan plan, int n_nodes, int n_edges,
+                                      const int* row_ptr, const int* col,
+                                      const int* csc_ptr, const int* csc_edge, const int* csc_dst,
+                                      const float* edge_vec, const float* x, const float* w,
+                                      const float* grad_out, const float* gg_x, const float* gg_w,
+                                      const float* gg_edge_vec, float* d_x, float* d_w,
+                                      float* d_grad_out, float* d_edge_vec, void* workspace,
+                                      size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Per-atom forces from edge-vector gradients, F = -dE/dpos with
  * r_e = pos_src - pos_dst:  F[n] = sum_{e: dst=n} g[e] - sum_{e: src=n} g[e].
