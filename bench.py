@@ -111,10 +111,10 @@ class ClockSampler:
 # was taken on: traffic is reported only while the sources are unchanged.
 KERNEL_HEADERS = ("common.cuh", "conv_common.cuh", "sh.cuh", "structure.h")
 MEASURED_TRAFFIC = {
-    "conv_fwd": {"bytes": 1025952000, "n_edges": 97480, "sources": ("conv_fwd.cu",) + KERNEL_HEADERS,
-                 "sha256_16": "88771e3801183127"},
-    "conv_bwd": {"bytes": 2062707456, "n_edges": 97480, "sources": ("conv_bwd.cu",) + KERNEL_HEADERS,
-                 "sha256_16": "efbbeca031725577"},
+    "conv_fwd": {"bytes": 1022236160, "n_edges": 97480, "sources": ("conv_fwd.cu",) + KERNEL_HEADERS,
+                 "sha256_16": "e371af1a1d48edcc"},
+    "conv_bwd": {"bytes": 2062439424, "n_edges": 97480, "sources": ("conv_bwd.cu",) + KERNEL_HEADERS,
+                 "sha256_16": "64f00dd54890ea3c"},
 }
 
 
@@ -289,6 +289,21 @@ def config_table(torch, api, dev, hbm, reps=20):
                      "hbm_frac": {"fwd": b_f / (t_f / 1e3) / 1e9 / hbm, "bwd": b_b / (t_b / 1e3) / 1e9 / hbm},
                      "fp32_frac": {"fwd": f_f / (t_f / 1e3) / 1e12 / FP32_PEAK_TFLOPS,
                                    "bwd": f_b / (t_b / 1e3) / 1e12 / FP32_PEAK_TFLOPS}})
+        if name == "molecules":
+            # double backward (adjoint of the backward) with all three cotangents
+            ggx, ggw, ggr = torch.randn_like(x), torch.randn_like(W), torch.randn((E, 3), device=dev)
+            dws = torch.empty(plan.conv_double_backward_workspace_bytes(E) // 4 + 64, dtype=torch.float32,
+                              device=dev)
+            t_d = _time_ms(torch, lambda: plan.conv_double_backward(g, x, W, go, gg_x=ggx, gg_w=ggw,
+                                                                    gg_edge_vec=ggr, workspace=dws), k)
+            # algorithmic bytes: read x, gg_x, W, gg_w, grad_out, gg_r, edge vectors; write d_x, d_W,
+            # d_grad_out, d_edge_vec
+            b_d = 4 * (3 * E * P * u + 3 * n * ni * u + 2 * n * no * u + 9 * E + 2 * (n + 1) + 2 * E)
+            rows.append({"workload": "molecules double backward (adjoint of the backward, all cotangents)",
+                         "L": list(L), "mult": u, "n_edges": E, "ms": t_d, "edges_per_s": E / (t_d / 1e3),
+                         "hbm_frac": b_d / (t_d / 1e3) / 1e9 / hbm,
+                         "launches": "3 forward + 2 backward + 3 harmonic-gradient passes + 1 directional harmonics"})
+            del ggx, ggw, ggr, dws
         del W, gw, out, gx, gr, F, ws, x, go, g
         torch.cuda.empty_cache()
     t = synthetic.tp_batch()

@@ -174,7 +174,9 @@ using BwdPlan = Plan<PS, kByL1, VEC, NEED_GY, bwd_budget<PS>()>;
 // One launch per chunk (paths of one l1 block): grad_x rows of that block
 // (written by the block's first chunk, accumulated by the others), grad_W
 // of the chunk's paths and a partial grad_Y over them.
-template <class PS, int VEC, bool NEED_GY, int CH, int KMULT>
+// EXT: the double backward's variant (per-edge harmonics given by the caller,
+// results added onto the outputs); the plain variant compiles without either.
+template <class PS, int VEC, bool NEED_GY, int CH, int KMULT, bool EXT>
 __global__ void CGTP_BWD_BOUNDS
 conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt) {
   // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x VEC
@@ -259,7 +261,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
         if (active && kk < k1) {
           const int e = __ldg(a.csc_edge + kk);
           float Y[NS];
-          edge_sh<PS::LS>(a.sh, a.edge_vec, e, Y);
+          edge_sh<PS::LS>(EXT ? a.sh : nullptr, a.edge_vec, e, Y);
           compute_T_grp<PS, GR>(Y, Tg + k * NT);
           Eg[k] = e;
           Ig[k] = __ldg(a.csc_dst + kk);
@@ -279,7 +281,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
           e = Eg[k];
           bwd_edge<PS, GR, VEC, NEED_GY>(Tg + k * NT, St + (k & 1) * stage_floats + gl * VEC, rowf, xr,
                                          a.grad_w ? a.grad_w + (long long)e * PS::NP * mult + c0 : nullptr,
-                                         a.accumulate != 0, mult, gx, red + gl, rs);
+                                         EXT && a.accumulate != 0, mult, gx, red + gl, rs);
         }
         if constexpr (NEED_GY) {
           __syncwarp();
@@ -312,7 +314,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
       __syncwarp();
     }
     if (active && a.grad_x != nullptr) {
-      if (!GR::FIRST || a.accumulate) {
+      if (!GR::FIRST || (EXT && a.accumulate)) {
         // rows of an l1 block that an earlier chunk of this call wrote (wait
         // for that grid, the preceding launch), or the caller's values
         if constexpr (!GR::FIRST) grid_dependency_wait();
@@ -450,7 +452,9 @@ cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t str
   const long long items = (long long)a.n_nodes * S;
   const long long groups_per_block = (long long)gpw * (kBwdThreads / 32);
   const long long blocks = (items + groups_per_block - 1) / groups_per_block;
-  auto kern = a.mult == 128 ? conv_bwd_kernel<PS, VEC, NEED_GY, CH, 128> : conv_bwd_kernel<PS, VEC, NEED_GY, CH, 0>;
+  auto kern = (a.sh != nullptr || a.accumulate) ? conv_bwd_kernel<PS, VEC, NEED_GY, CH, 0, true>
+               : a.mult == 128                 ? conv_bwd_kernel<PS, VEC, NEED_GY, CH, 128, false>
+                                               : conv_bwd_kernel<PS, VEC, NEED_GY, CH, 0, false>;
   cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e2 != cudaSuccess) return e2;
   long long cap = 0x7fffffffLL;  // the kernel loops over items beyond the grid
