@@ -234,3 +234,38 @@ def conv_double_backward(row_ptr, col, edge_vec, x, w, grad_out, gg_x, gg_w, gg_
     d_r = np.einsum("eb,ebk->ek", dY_expl, J) + np.einsum("eb,ebjk,ek->ej", gY, H, ggr)
     return d_x, d_w, d_g, d_r
 
+
+def conv_uvw_forward(row_ptr, col, edge_vec, x, w, mix, lmax_in, lmax_sh, lmax_out):
+    """Fully connected ("uvw") convolution: the per-path messages of the
+    channelwise convolution, summed over each row but kept per path, then
+    mixed across channels by a dense matrix per path ("Tensor Decomposition
+    Networks ...", reply to reviewer cmnz: the fully connected CG tensor
+    product of Equiformer):
+
+        t[i][p][m3][u]   = sum_{e in row i} W_e[p][u] sum_{m1,m2} C^p x[j][l1,m1][u] Y_e[l2,m2]
+        out[i][l3,m3][v] = sum_{p: l3(p) = l3} sum_u t[i][p][m3][u] mix[p][u][v]
+
+    mix is [P][u][v]; out is [N][(lmax_out+1)^2][v] in fp64.  With every
+    mix[p] the identity this is conv_forward.
+    """
+    row_ptr = np.asarray(row_ptr, dtype=np.int64)
+    src = np.asarray(col, dtype=np.int64)
+    dst = edge_dst(row_ptr).astype(np.int64)
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    mix = np.asarray(mix, dtype=np.float64)
+    n, u = row_ptr.size - 1, x.shape[2]
+    P, v = mix.shape[0], mix.shape[2]
+    Y = real_sh(edge_vec, lmax_sh)
+    xs = x[src]
+    pl = paths(lmax_in, lmax_sh, lmax_out)
+    t = np.zeros((n, P, (lmax_out + 1) ** 2, u))  # rows of l3(p) used only
+    for p, ri, rs, ro, c in path_nonzeros(lmax_in, lmax_sh, lmax_out):
+        msg = c * w[:, p, :] * xs[:, ri, :] * Y[:, rs][:, None]
+        np.add.at(t[:, p, ro, :], dst, msg)
+    out = np.zeros((n, (lmax_out + 1) ** 2, v))
+    for p, (l1, l2, l3) in enumerate(pl):
+        rows = slice(l3 * l3, (l3 + 1) * (l3 + 1))
+        out[:, rows, :] += np.einsum("imu,uv->imv", t[:, p, rows, :], mix[p])
+    return out
+
