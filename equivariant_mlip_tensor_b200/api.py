@@ -229,6 +229,26 @@ class Plan:
              _stream())
         return d_x, d_w, d_g, d_r
 
+    def uvw_forward_workspace_bytes(self, n_nodes, mult_out):
+        b = ctypes.c_size_t()
+        call("cgtp_uvw_forward_workspace_size", self._h, n_nodes, mult_out, ctypes.byref(b))
+        return b.value
+
+    def uvw_forward(self, graph, x, w, mix, out=None, workspace=None):
+        """Fully connected convolution: per-path messages mixed by mix [P][mult][mult_out]."""
+        for t, nm in ((x, "x"), (w, "w"), (mix, "mix")):
+            _check(t, torch.float32, nm)
+        mult_out = mix.shape[2]
+        if out is None:
+            out = torch.empty((graph.n_nodes, self.no, mult_out), dtype=torch.float32, device=x.device)
+        nb = self.uvw_forward_workspace_bytes(graph.n_nodes, mult_out)
+        if workspace is None:
+            workspace = torch.empty(max(nb // 4, 64), dtype=torch.float32, device=x.device)
+        call("cgtp_uvw_forward", self._h, graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr), _ptr(graph.col),
+             _ptr(graph.edge_vec), _ptr(x), _ptr(w), _ptr(mix), mult_out, _ptr(out), _ptr(workspace),
+             workspace.numel() * 4, _stream())
+        return out
+
     # ------------------------------------------------------------ radial network
     def radial_forward(self, edge_vec, rc, W1, W2, out=None):
         _check(edge_vec, torch.float32, "edge_vec")

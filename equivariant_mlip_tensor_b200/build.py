@@ -24,7 +24,26 @@ ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
                      "-Xcompiler", "-fPIC", "-I", CSRC, "-I", INCLUDE]
 PER_SHAPE = ["conv_fwd.cu", "conv_bwd.cu", "tp.cu"]
-SHAPE_FREE = ["graph.cu", "radial.cu", "misc.cu", "abi.cu", "cg_table.cpp"]
+SHAPE_FREE = ["graph.cu", "radial.cu", "misc.cu", "abi.cu", "cg_table.cpp", "uvw.cu"]
+
+
+def cutlass_include():
+    """Include directories of a CUTLASS (>= 4) header tree for the tensor-core
+    GEMM of the fully connected convolution: $CUTLASS_HOME, else the trees
+    vendored in this Python environment's packages.  None if there is none
+    (uvw.cu then builds without it and its entry point reports unsupported)."""
+    import site
+    cands = []
+    if os.environ.get("CUTLASS_HOME"):
+        cands.append(os.environ["CUTLASS_HOME"])
+    for sp in site.getsitepackages():
+        cands += [os.path.join(sp, "flashinfer", "data", "cutlass"), os.path.join(sp, "tilelang", "3rdparty", "cutlass")]
+    for c in cands:
+        inc = os.path.join(c, "include")
+        if os.path.exists(os.path.join(inc, "cutlass", "gemm", "collective", "builders", "sm100_9xBF16_umma_builder.inl")):
+            util = os.path.join(c, "tools", "util", "include")
+            return [inc] + ([util] if os.path.isdir(util) else [])
+    return None
 
 
 def nvcc():
@@ -58,7 +77,11 @@ def _jobs():
             jobs.append((os.path.join(CSRC, src), obj, defs))
     for src in SHAPE_FREE:
         obj = os.path.join(BUILD, src.rsplit(".", 1)[0] + ".o")
-        jobs.append((os.path.join(CSRC, src), obj, []))
+        defs = []
+        if src == "uvw.cu":
+            inc = cutlass_include()
+            defs = (sum((["-I", d] for d in inc), []) + ["-diag-suppress", "20012,177"]) if inc else ["-DCGTP_NO_CUTLASS"]
+        jobs.append((os.path.join(CSRC, src), obj, defs))
     return jobs
 
 

@@ -430,6 +430,83 @@ cgtp_status cgtp_conv_double_backward(cgtp_plan p, int n_nodes, int n_edges, con
   return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
 }
 
+// ---- fully connected (uvw) convolution ----
+struct UvwLayout {
+  int order[kMaxPaths];
+  int count_l3[kLmaxTab + 1];
+  size_t t_floats, packed_floats;
+};
+static bool uvw_layout(cgtp_plan p, int n_nodes, int mult_out, UvwLayout* L) {
+  bool found = false;
+#define CGTP_UVW_ORDER_ENTRY(A, B, C) \
+  if (p->li == A && p->ls == B && p->lo == C) { conv_path_order<A, B, C>(L->order, L->count_l3); found = true; }
+  CGTP_CONFIGS(CGTP_UVW_ORDER_ENTRY)
+  if (!found) return false;
+  L->t_floats = L->packed_floats = 0;
+  for (int l3 = 0; l3 <= p->lo; ++l3) {
+    L->t_floats += (size_t)n_nodes * (2 * l3 + 1) * L->count_l3[l3] * p->mult;
+    L->packed_floats += (size_t)(2 * l3 + 1) * L->count_l3[l3] * p->mult * mult_out;
+  }
+  return true;
+}
+static size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+cgtp_status cgtp_uvw_forward_workspace_size(cgtp_plan p, int n_nodes, int mult_out, size_t* bytes) {
+  if (p == nullptr || n_nodes < 0 || mult_out <= 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
+  UvwLayout L;
+  if (!uvw_layout(p, n_nodes, mult_out, &L)) return CGTP_ERR_UNSUPPORTED;
+  *bytes = round256(sizeof(float) * L.t_floats) + round256(sizeof(float) * L.packed_floats) +
+           uvw_gemm_workspace(n_nodes, p->lo, L.count_l3, p->mult, mult_out);
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_uvw_forward(cgtp_plan p, int n_nodes, int n_edges, const int* row_ptr, const int* col,
+                             const float* edge_vec, const float* x, const float* w, const float* mix, int mult_out,
+                             float* out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (p == nullptr || n_nodes < 0 || n_edges < 0 || row_ptr == nullptr || mult_out <= 0 || mix == nullptr)
+    return CGTP_ERR_INVALID_ARG;
+  if (n_nodes > 0 && (x == nullptr || out == nullptr)) return CGTP_ERR_INVALID_ARG;
+  if (n_edges > 0 && (col == nullptr || edge_vec == nullptr || w == nullptr)) return CGTP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(out)) return CGTP_ERR_INVALID_ARG;
+  if (p->mult % 4 != 0 || mult_out % 4 != 0) return CGTP_ERR_UNSUPPORTED;  // 16-byte GEMM rows
+  if (n_nodes == 0) return CGTP_OK;
+  size_t need = 0;
+  cgtp_status st = cgtp_uvw_forward_workspace_size(p, n_nodes, mult_out, &need);
+  if (st != CGTP_OK) return st;
+  if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
+    return CGTP_ERR_WORKSPACE;
+  int sms = 0;
+  st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  UvwLayout L;
+  uvw_layout(p, n_nodes, mult_out, &L);
+  float* t = (float*)workspace;
+  float* packed = (float*)((char*)workspace + round256(sizeof(float) * L.t_floats));
+  void* gws = (char*)packed + round256(sizeof(float) * L.packed_floats);
+  const size_t gws_bytes = workspace_bytes - round256(sizeof(float) * L.t_floats) -
+                           round256(sizeof(float) * L.packed_floats);
+  // stage 1: per-path messages t (channelwise convolution, paths kept apart)
+  ConvFwdArgs a{n_nodes, row_ptr, col, edge_vec, x, w, t, p->mult};
+  cudaError_t e = cudaErrorNotSupported;
+#define CGTP_UVW_PATHS_ENTRY(A, B, C) \
+  if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_paths<A, B, C>(a, sms, s);
+  CGTP_CONFIGS(CGTP_UVW_PATHS_ENTRY)
+  if (e != cudaSuccess) return cuda_fail(e);
+  // stage 2: per-l3 mixing GEMMs; output blocks no path reaches are zero
+  e = launch_uvw_pack(p->n_paths, p->mult, mult_out, p->lo, L.order, L.count_l3, mix, packed, s);
+  for (int l3 = 0; l3 <= p->lo && e == cudaSuccess; ++l3)
+    if (L.count_l3[l3] == 0) {
+      const int no = (p->lo + 1) * (p->lo + 1);
+      e = cudaMemset2DAsync(out + (size_t)l3 * l3 * mult_out, sizeof(float) * no * mult_out, 0,
+                            sizeof(float) * (2 * l3 + 1) * mult_out, n_nodes, s);
+    }
+  if (e == cudaSuccess) e = launch_uvw_gemm(n_nodes, p->lo, L.count_l3, p->mult, mult_out, t, packed, out, gws,
+                                            gws_bytes, s);
+  if (e == cudaErrorNotSupported) return CGTP_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
 cgtp_status cgtp_forces(int n_nodes, int n_edges, const int* row_ptr, const int* csc_ptr, const int* csc_edge,
                         const float* grad_edge_vec, float* forces, void* stream) {
   if (n_nodes < 0 || n_edges < 0 || row_ptr == nullptr || csc_ptr == nullptr) return CGTP_ERR_INVALID_ARG;

@@ -91,6 +91,7 @@ struct Grp {
   static constexpr int NOWN = KIND == kAll ? PS::NO : 2 * V + 1;
   static constexpr int OWN0 = KIND == kAll ? 0 : V * V;    // first own row
   static constexpr bool FIRST = true;                      // initialises its rows
+  static constexpr bool PERPATH = false;                   // one row block per l3, paths summed
 };
 
 // T^p[m1][m3] = sum_m2 C^p[m1,m2,m3] Y[l2,m2] for the group's paths, packed
@@ -143,8 +144,11 @@ constexpr int path_cost(int p, int kind, int vec, bool gy) {
          (tc + 3) / 4 + n3 + 2 * n1 * vec + 6;
 }
 
+// max_rows (forward by l3 only): at most this many output rows (sum of
+// 2 l3 + 1 over the chunk's paths), for kernels that keep one block of rows
+// per path.
 template <class PS>
-constexpr ChunkPlan make_chunk_plan(int kind, int vec, bool gy, int budget) {
+constexpr ChunkPlan make_chunk_plan(int kind, int vec, bool gy, int budget, int max_rows = 1 << 30) {
   ChunkPlan c{};
   int k = 0;
   const int kmax = kind == kByL1 ? PS::LI : PS::LO;
@@ -155,11 +159,13 @@ constexpr ChunkPlan make_chunk_plan(int kind, int vec, bool gy, int budget) {
   int start = 0;
   while (start < k) {
     const int key = kind == kByL1 ? PS::D.l1[c.order[start]] : PS::D.l3[c.order[start]];
-    int end = start, cost = 0;
+    int end = start, cost = 0, rows = 0;
     while (end < k && (kind == kByL1 ? PS::D.l1[c.order[end]] : PS::D.l3[c.order[end]]) == key) {
       const int pc = path_cost<PS>(c.order[end], kind, vec, gy);
-      if (end > start && cost + pc > budget) break;
+      const int pr = 2 * PS::D.l3[c.order[end]] + 1;
+      if (end > start && (cost + pc > budget || rows + pr > max_rows)) break;
       cost += pc;
+      rows += pr;
       ++end;
     }
     c.key[c.n] = key;
@@ -172,9 +178,9 @@ constexpr ChunkPlan make_chunk_plan(int kind, int vec, bool gy, int budget) {
   return c;
 }
 
-template <class PS, int KIND, int VEC, bool GY, int BUDGET>
+template <class PS, int KIND, int VEC, bool GY, int BUDGET, int MAX_ROWS = (1 << 30)>
 struct Plan {
-  static constexpr ChunkPlan P = make_chunk_plan<PS>(KIND, VEC, GY, BUDGET);
+  static constexpr ChunkPlan P = make_chunk_plan<PS>(KIND, VEC, GY, BUDGET, MAX_ROWS);
   static constexpr int N = P.n;
 };
 
@@ -207,6 +213,7 @@ struct Chunk {
 };
 template <class PS, class PL, int CH, int KIND>
 struct ChunkGrp : Chunk<PS, PL, CH> {
+  static constexpr bool PERPATH = false;
   using Base = Chunk<PS, PL, CH>;
   static constexpr typename Base::Data D = Base::make(KIND == kByL1);
   static constexpr int NP = D.n;

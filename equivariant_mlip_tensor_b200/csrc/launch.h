@@ -11,6 +11,10 @@ namespace cgtp {
 template <int LI, int LS, int LO>
 cudaError_t launch_conv_fwd(const ConvFwdArgs& a, int num_sms, cudaStream_t stream);
 template <int LI, int LS, int LO>
+cudaError_t launch_conv_paths(const ConvFwdArgs& a, int num_sms, cudaStream_t stream);
+template <int LI, int LS, int LO>
+void conv_path_order(int* order, int* count_l3);
+template <int LI, int LS, int LO>
 cudaError_t launch_conv_bwd(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);
 template <int LI, int LS, int LO>
 int conv_bwd_slices(int mult);
@@ -35,6 +39,14 @@ cudaError_t launch_forces(int n, const int* row_ptr, const int* csc_ptr, const i
                           float* F, int num_sms, cudaStream_t stream);
 cudaError_t launch_sh(int lmax_sh, int n_edges, const float* ev, float* Y, float* dY, int num_sms,
                       cudaStream_t stream);
+// Fully connected convolution, second stage: pack the per-path mixing
+// matrices by l3 and multiply (tensor cores, fp32-accurate).
+cudaError_t launch_uvw_pack(int n_paths, int mult, int mult_out, int lmax_out, const int* order_dev,
+                            const int* count_l3, const float* mix, float* packed, cudaStream_t stream);
+size_t uvw_gemm_workspace(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out);
+cudaError_t launch_uvw_gemm(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out,
+                            const float* t, const float* packed, float* out, void* ws, size_t ws_bytes,
+                            cudaStream_t stream);
 cudaError_t launch_sh_dir(int lmax_sh, int n_edges, const float* ev, const float* q, float* u, int num_sms,
                           cudaStream_t stream);
 

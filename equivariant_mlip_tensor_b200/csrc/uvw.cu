@@ -1,0 +1,154 @@
+// Fully connected ("uvw") convolution, second stage: per l3 block,
+//   out[i][l3, m3][v] = sum_{p: l3(p) = l3} sum_u t[i][p][m3][u] mix[p][u][v]
+// is one dense GEMM with the block's paths concatenated along K
+// (K = paths x mult), batched over m3 ("Tensor Decomposition Networks ...",
+// reply to reviewer cmnz: the fully connected CG tensor product).  The GEMM
+// runs on the 5th-generation tensor cores through CUTLASS's sm100 collective
+// (TMA-staged operands, tcgen05 MMA into tensor memory) in its fp32-accurate
+// mode: each fp32 operand is split into three bf16 terms and the nine
+// products are accumulated in fp32, which keeps the result within fp32
+// rounding of the exact product.  Cluster shape 1x1x1: no multicast loads.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "launch.h"
+
+#if !defined(CGTP_NO_CUTLASS)
+#include "cutlass/cutlass.h"
+#include "cute/tensor.hpp"
+#include "cutlass/epilogue/collective/collective_builder.hpp"
+#include "cutlass/gemm/collective/collective_builder.hpp"
+#include "cutlass/gemm/device/gemm_universal_adapter.h"
+#include "cutlass/gemm/dispatch_policy.hpp"
+#include "cutlass/gemm/kernel/gemm_universal.hpp"
+#include "cutlass/util/packed_stride.hpp"
+#endif
+
+namespace cgtp {
+
+namespace {
+
+struct PathOrder {
+  int order[kMaxPaths];  // path of each rank, ranks grouped by l3
+};
+
+// packed block of l3: [2 l3 + 1 copies][paths of l3 x mult][mult_out]
+__global__ void uvw_pack_kernel(PathOrder po, int mult, int mult_out, int rank0, int npk, int n3,
+                                const float* __restrict__ mix, float* __restrict__ packed) {
+  const long long per_copy = (long long)npk * mult * mult_out;
+  const long long total = per_copy * n3;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i % per_copy;
+    const int v = int(r % mult_out);
+    const long long ku = r / mult_out;
+    const int uu = int(ku % mult), rank = int(ku / mult);
+    packed[i] = mix[((long long)po.order[rank0 + rank] * mult + uu) * mult_out + v];
+  }
+}
+
+#if !defined(CGTP_NO_CUTLASS)
+using namespace cute;
+using TileShape = Shape<_128, _128, _32>;
+using ClusterShape = Shape<_1, _1, _1>;
+constexpr int kAlign = 4;  // floats: 16-byte rows and strides
+using Layout = cutlass::layout::RowMajor;
+using Epilogue = typename cutlass::epilogue::collective::CollectiveBuilder<
+    cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, TileShape, ClusterShape,
+    cutlass::epilogue::collective::EpilogueTileAuto, float, float, float, Layout, kAlign, float, Layout, kAlign,
+    cutlass::epilogue::collective::EpilogueScheduleAuto>::CollectiveOp;
+using Mainloop = typename cutlass::gemm::collective::CollectiveBuilder<
+    cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, float, Layout, kAlign, float, Layout, kAlign, float,
+    TileShape, ClusterShape,
+    cutlass::gemm::collective::StageCountAutoCarveout<static_cast<int>(sizeof(typename Epilogue::SharedStorage))>,
+    cutlass::gemm::KernelTmaWarpSpecialized1SmFastFP32Sm100>::CollectiveOp;
+using Kernel = cutlass::gemm::kernel::GemmUniversal<Shape<int, int, int, int>, Mainloop, Epilogue>;
+using Gemm = cutlass::gemm::device::GemmUniversalAdapter<Kernel>;
+
+// Arguments of the GEMM of one l3 block: A = t block [n_nodes][n3][K] read
+// as n3 batches of [n_nodes][K] (row stride n3 K, batch stride K); B = the
+// packed copies [n3][K][mult_out]; D = out rows (l3, m3) of every node (row
+// stride NO mult_out, batch stride mult_out).
+Gemm::Arguments block_args(int n_nodes, int l3, int lmax_out, int K, int mult_out, const float* t,
+                           const float* packed, float* out) {
+  const int n3 = 2 * l3 + 1, no = (lmax_out + 1) * (lmax_out + 1);
+  using SA = typename Kernel::StrideA;
+  using SB = typename Kernel::StrideB;
+  using SC = typename Kernel::StrideC;
+  using SD = typename Kernel::StrideD;
+  SA sa = cutlass::make_cute_packed_stride(SA{}, make_shape(n_nodes, K, n3));
+  get<0>(sa) = (int64_t)n3 * K;
+  get<2>(sa) = K;
+  SB sb = cutlass::make_cute_packed_stride(SB{}, make_shape(mult_out, K, n3));
+  SD sd = cutlass::make_cute_packed_stride(SD{}, make_shape(n_nodes, mult_out, n3));
+  get<0>(sd) = (int64_t)no * mult_out;
+  get<2>(sd) = mult_out;
+  SC sc = sd;
+  float* D = out + (size_t)l3 * l3 * mult_out;
+  return Gemm::Arguments{cutlass::gemm::GemmUniversalMode::kGemm,
+                         {n_nodes, mult_out, K, n3},
+                         {t, sa, packed, sb},
+                         {{1.f, 0.f}, D, sc, D, sd}};
+}
+#endif
+
+}  // namespace
+
+cudaError_t launch_uvw_pack(int n_paths, int mult, int mult_out, int lmax_out, const int* order, const int* count_l3,
+                            const float* mix, float* packed, cudaStream_t stream) {
+  PathOrder po{};
+  for (int k = 0; k < n_paths && k < kMaxPaths; ++k) po.order[k] = order[k];
+  int rank0 = 0;
+  size_t off = 0;
+  for (int l3 = 0; l3 <= lmax_out; ++l3) {
+    const int npk = count_l3[l3], n3 = 2 * l3 + 1;
+    if (npk > 0) {
+      uvw_pack_kernel<<<256, 256, 0, stream>>>(po, mult, mult_out, rank0, npk, n3, mix, packed + off);
+      const cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    off += (size_t)n3 * npk * mult * mult_out;
+    rank0 += npk;
+  }
+  return cudaSuccess;
+}
+
+size_t uvw_gemm_workspace(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out) {
+#if defined(CGTP_NO_CUTLASS)
+  return 0;
+#else
+  size_t w = 0;
+  for (int l3 = 0; l3 <= lmax_out; ++l3) {
+    if (count_l3[l3] == 0) continue;
+    const size_t b = Gemm::get_workspace_size(
+        block_args(n_nodes, l3, lmax_out, count_l3[l3] * mult, mult_out, nullptr, nullptr, nullptr));
+    w = b > w ? b : w;
+  }
+  return (w + 255) & ~(size_t)255;
+#endif
+}
+
+cudaError_t launch_uvw_gemm(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out, const float* t,
+                            const float* packed, float* out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+#if defined(CGTP_NO_CUTLASS)
+  return cudaErrorNotSupported;
+#else
+  size_t t_off = 0, p_off = 0;
+  for (int l3 = 0; l3 <= lmax_out; ++l3) {
+    const int npk = count_l3[l3], n3 = 2 * l3 + 1, K = npk * mult;
+    if (npk > 0) {
+      Gemm g;
+      auto args = block_args(n_nodes, l3, lmax_out, K, mult_out, t + t_off, packed + p_off, out);
+      if (g.can_implement(args) != cutlass::Status::kSuccess) return cudaErrorNotSupported;
+      if (Gemm::get_workspace_size(args) > ws_bytes) return cudaErrorInvalidValue;
+      if (g.initialize(args, ws, stream) != cutlass::Status::kSuccess) return cudaErrorLaunchFailure;
+      if (g.run(stream) != cutlass::Status::kSuccess) return cudaErrorLaunchFailure;
+    }
+    t_off += (size_t)n_nodes * n3 * K;
+    p_off += (size_t)n3 * K * mult_out;
+  }
+  return cudaGetLastError();
+#endif
+}
+
+}  // namespace cgtp

@@ -208,6 +208,33 @@ cgtp_status cgtp_conv_double_backward(cgtp_plan plan, int n_nodes, int n_edges,
                                       float* d_grad_out, float* d_edge_vec, void* workspace,
                                       size_t workspace_bytes, void* stream);
 
+/* Bytes of device workspace cgtp_uvw_forward needs for n_nodes nodes and
+ * mult_out output channels (per-path messages, packed mixing matrices and
+ * the GEMM's own scratch). */
+cgtp_status cgtp_uvw_forward_workspace_size(cgtp_plan plan, int n_nodes, int mult_out, size_t* bytes);
+
+/* ---------------------------------------------------------------------------
+ * Fully connected ("uvw") convolution forward, the fully connected CG tensor
+ * product of Equiformer ("Tensor Decomposition Networks ...", reply to
+ * reviewer cmnz): the channelwise convolution's per-path messages, summed
+ * over each row but kept per path, then mixed across channels by a dense
+ * matrix per path and summed into l3 blocks:
+ *   t[i][p][m3][u]   = sum_{e in row i} W_e[p][u] sum C^p x[j][l1,m1][u] Y_e[l2,m2]
+ *   out[i][l3,m3][v] = sum_{p: l3(p) = l3} sum_u t[i][p][m3][u] mix[p][u][v]
+ * mix: device [n_paths][mult][mult_out] (paths in the plan's order);
+ * out: device [n_nodes][(lmax_out+1)^2][mult_out] (overwritten).  The
+ * mixing runs on the tensor cores (one GEMM per l3 block, the block's paths
+ * concatenated along K) in an fp32-accurate split-bf16 mode.  mult and
+ * mult_out must be multiples of 4 (CGTP_ERR_UNSUPPORTED otherwise, and when
+ * the library was built without the CUTLASS headers).  workspace: device,
+ * 256-byte aligned, of the size cgtp_uvw_forward_workspace_size reports
+ * (CGTP_ERR_WORKSPACE otherwise).
+ * ------------------------------------------------------------------------- */
+cgtp_status cgtp_uvw_forward(cgtp_plan plan, int n_nodes, int n_edges, const int* row_ptr,
+                             const int* col, const float* edge_vec, const float* x, const float* w,
+                             const float* mix, int mult_out, float* out, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Per-atom forces from edge-vector gradients, F = -dE/dpos with
  * r_e = pos_src - pos_dst:  F[n] = sum_{e: dst=n} g[e] - sum_{e: src=n} g[e].
