@@ -304,6 +304,22 @@ def config_table(torch, api, dev, hbm, reps=20):
                          "hbm_frac": b_d / (t_d / 1e3) / 1e9 / hbm,
                          "launches": "3 forward + 2 backward + 3 harmonic-gradient passes + 1 directional harmonics"})
             del ggx, ggw, ggr, dws
+            # fully connected (uvw) forward, 128 output channels: per-path messages, then one
+            # tensor-core GEMM per l3 block
+            v = 128
+            mix = torch.randn((P, u, v), device=dev) / u ** 0.5
+            uws = torch.empty(plan.uvw_forward_workspace_bytes(n, v) // 4 + 64, dtype=torch.float32, device=dev)
+            uout = torch.empty((n, no, v), dtype=torch.float32, device=dev)
+            t_u = _time_ms(torch, lambda: plan.uvw_forward(g, x, W, mix, out=uout, workspace=uws), k)
+            rows_p = no_sum  # sum over paths of 2 l3 + 1
+            f_gemm = 2.0 * n * rows_p * u * v
+            b_u = 4 * (E * P * u + n * ni * u + n * no * v + P * u * v + 4 * E + (n + 1))
+            rows.append({"workload": "molecules fully connected (uvw) forward, 128 -> 128 channels per path",
+                         "L": list(L), "mult": u, "mult_out": v, "n_edges": E, "ms": t_u,
+                         "edges_per_s": E / (t_u / 1e3), "hbm_frac": b_u / (t_u / 1e3) / 1e9 / hbm,
+                         "mixing_gemm_flops": f_gemm,
+                         "mixing_tflops_if_whole_call": f_gemm / (t_u / 1e3) / 1e12})
+            del mix, uws, uout
         del W, gw, out, gx, gr, F, ws, x, go, g
         torch.cuda.empty_cache()
     t = synthetic.tp_batch()
@@ -321,6 +337,34 @@ def config_table(torch, api, dev, hbm, reps=20):
                  "fwd_ms": t_f, "bwd_ms": t_b, "pairs_per_s_fwd_bwd": B / ((t_f + t_b) / 1e3),
                  "hbm_frac": {"fwd": b_f / (t_f / 1e3) / 1e9 / hbm, "bwd": b_b / (t_b / 1e3) / 1e9 / hbm}})
     return rows
+
+
+def run_op(args):
+    """A short loop of one operation at the molecules workload, for profiling
+    (ncu launch lists): 'uvw' (fully connected forward) or 'double' (double
+    backward)."""
+    import torch
+
+    from equivariant_mlip_tensor_b200 import api
+    dev = torch.device("cuda", 0)
+    w = synthetic.molecules(n_graphs=args.graphs)
+    L = (w.lmax_in, w.lmax_sh, w.lmax_out)
+    n, u = w.n_nodes, w.mult
+    gp = torch.from_numpy(np.arange(0, n + 1, w.graph_size, dtype=np.int32)).to(dev)
+    g = api.build_graph(torch.from_numpy(w.pos).to(dev), w.rc, graph_ptr=gp)
+    plan = api.Plan(*L, u)
+    W = plan.radial_forward(g.edge_vec, w.rc, torch.from_numpy(w.W1).to(dev), torch.from_numpy(w.W2).to(dev))
+    x = torch.from_numpy(w.x).to(dev)
+    go = torch.from_numpy(w.grad_out).to(dev)
+    if args.op == "uvw":
+        mix = torch.randn((plan.n_paths, u, 128), device=dev) / u ** 0.5
+        fn = lambda: plan.uvw_forward(g, x, W, mix)
+    else:
+        ggx, ggw, ggr = torch.randn_like(x), torch.randn_like(W), torch.randn((g.n_edges, 3), device=dev)
+        fn = lambda: plan.conv_double_backward(g, x, W, go, gg_x=ggx, gg_w=ggw, gg_edge_vec=ggr)
+    ms = _time_ms(torch, fn, args.steps)
+    print(json.dumps({"op": args.op, "n_edges": g.n_edges, "ms": ms}), flush=True)
+    return 0
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -560,6 +604,8 @@ def main():
     ap.add_argument("--impl", choices=["cgtp", "reference"], default="cgtp")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-workload table")
+    ap.add_argument("--op", choices=["uvw", "double"], default=None,
+                    help="time one other operation alone (for profiling) instead of the benchmark")
     ap.add_argument("--graphs", type=int, default=256, help="molecules per rank (profiling uses fewer)")
     ap.add_argument("--conv-only", action="store_true",
                     help="time only the convolution step (no pipeline / e2e / CPU baseline); for profiling")
@@ -568,6 +614,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.op is not None:
+        return run_op(args)
     return run_gpu(args)
 
 
