@@ -269,3 +269,52 @@ def conv_uvw_forward(row_ptr, col, edge_vec, x, w, mix, lmax_in, lmax_sh, lmax_o
         out[:, rows, :] += np.einsum("imu,uv->imv", t[:, p, rows, :], mix[p])
     return out
 
+
+def conv_uvw_backward(row_ptr, col, edge_vec, x, w, mix, grad_out, lmax_in, lmax_sh, lmax_out):
+    """Adjoint of conv_uvw_forward for the output gradient g = grad_out
+    [N][(lmax_out+1)^2][v]: (grad_x, grad_w, grad_mix, grad_edge_vec) in fp64.
+
+        gt[i][p][m3][u]  = sum_v g[i][l3,m3][v] mix[p][u][v]
+        grad_mix[p][u][v] = sum_i sum_m3 t[i][p][m3][u] g[i][l3,m3][v]
+    and the channelwise backward with one output gradient per path:
+        grad_x[j][l1,m1][u] = sum_{e: src=j} sum_p W_e[p][u] sum C Y_e gt[i][p][m3][u]
+        grad_W[e][p][u]     = sum C x[j][l1,m1][u] Y_e gt[i][p][m3][u]
+        grad_Y[e][l2,m2]    = sum_p sum C sum_u W_e[p][u] x[j][l1,m1][u] gt[i][p][m3][u]
+        grad_r[e]           = (dY_e/dr_e)^T grad_Y[e]
+    """
+    row_ptr = np.asarray(row_ptr, dtype=np.int64)
+    src = np.asarray(col, dtype=np.int64)
+    dst = edge_dst(row_ptr).astype(np.int64)
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    mix = np.asarray(mix, dtype=np.float64)
+    g = np.asarray(grad_out, dtype=np.float64)
+    n, u = row_ptr.size - 1, x.shape[2]
+    E, P = src.size, w.shape[1]
+    Y = real_sh(edge_vec, lmax_sh)
+    J = real_sh_jacobian(edge_vec, lmax_sh)
+    xs = x[src]
+    pl = paths(lmax_in, lmax_sh, lmax_out)
+    no = (lmax_out + 1) ** 2
+    t = np.zeros((n, P, no, u))
+    for p, ri, rs, ro, c in path_nonzeros(lmax_in, lmax_sh, lmax_out):
+        np.add.at(t[:, p, ro, :], dst, c * w[:, p, :] * xs[:, ri, :] * Y[:, rs][:, None])
+    gt = np.zeros((n, P, no, u))
+    grad_mix = np.zeros_like(mix)
+    for p, (l1, l2, l3) in enumerate(pl):
+        rows = slice(l3 * l3, (l3 + 1) * (l3 + 1))
+        gt[:, p, rows, :] = np.einsum("imv,uv->imu", g[:, rows, :], mix[p])
+        grad_mix[p] = np.einsum("imu,imv->uv", t[:, p, rows, :], g[:, rows, :])
+    gd = gt[dst]  # [E][P][no][u]
+    mx = np.zeros((E, x.shape[1], u))
+    grad_w = np.zeros((E, P, u))
+    gY = np.zeros((E, Y.shape[1]))
+    for p, ri, rs, ro, c in path_nonzeros(lmax_in, lmax_sh, lmax_out):
+        mx[:, ri, :] += c * w[:, p, :] * Y[:, rs][:, None] * gd[:, p, ro, :]
+        grad_w[:, p, :] += c * xs[:, ri, :] * Y[:, rs][:, None] * gd[:, p, ro, :]
+        gY[:, rs] += c * np.sum(w[:, p, :] * xs[:, ri, :] * gd[:, p, ro, :], axis=1)
+    grad_x = np.zeros_like(x)
+    np.add.at(grad_x, src, mx)
+    grad_r = np.einsum("eb,ebk->ek", gY, J)
+    return grad_x, grad_w, grad_mix, grad_r
+

@@ -2,7 +2,8 @@
 mixing reduces it to the channelwise convolution, a pure-Python brute force
 over edges, nonzeros and channels (real CG from the Racah formula, harmonics
 from scipy through the real basis), equivariance under rotations, and
-linearity in the mixing matrices."""
+linearity in the mixing matrices; the backward against the channelwise
+backward (identity mixing) and against central differences of the forward."""
 import numpy as np
 import pytest
 
@@ -76,3 +77,36 @@ def test_linear_in_the_mixing():
     mix2 = np.random.default_rng(5).standard_normal(mix.shape)
     f = lambda m: conv.conv_uvw_forward(nl["row_ptr"], nl["col"], nl["edge_vec"], x, w, m, *L)
     assert np.abs(f(mix + 2.0 * mix2) - f(mix) - 2.0 * f(mix2)).max() <= 1e-12 * np.abs(f(mix)).max()
+
+
+def test_backward_with_identity_mixing_is_channelwise_backward():
+    L = (2, 2, 2)
+    nl, x, w, _ = _problem(6, L, u=3)
+    P = w.shape[1]
+    g = np.random.default_rng(7).standard_normal((x.shape[0], 9, 3))
+    eye = np.stack([np.eye(3)] * P)
+    gx, gw, gm, gr = conv.conv_uvw_backward(nl["row_ptr"], nl["col"], nl["edge_vec"], x, w, eye, g, *L)
+    rx, rw, rr = conv.conv_backward(nl["row_ptr"], nl["col"], nl["edge_vec"], x, w, g, *L)
+    for a, b in ((gx, rx), (gw, rw), (gr, rr)):
+        assert np.abs(a - b).max() <= 1e-12 * np.abs(b).max()
+
+
+@pytest.mark.parametrize("L", [(1, 1, 1), (2, 4, 2)])
+def test_backward_matches_differences_of_forward(L):
+    nl, x, w, mix = _problem(8, L)
+    g = np.random.default_rng(9).standard_normal((x.shape[0], (L[2] + 1) ** 2, mix.shape[2]))
+    rp, col = nl["row_ptr"], nl["col"]
+    ev = nl["edge_vec"].astype(np.float64)
+    grads = conv.conv_uvw_backward(rp, col, ev, x, w, mix, g, *L)
+    f = lambda x_, w_, m_, e_: float(np.sum(g * conv.conv_uvw_forward(rp, col, e_, x_, w_, m_, *L)))
+    rng = np.random.default_rng(10)
+    h = 1e-6
+    base = dict(x_=x, w_=w, m_=mix, e_=ev)
+    for key, grad in zip(("x_", "w_", "m_", "e_"), grads):
+        d = rng.standard_normal(base[key].shape)
+        plus, minus = dict(base), dict(base)
+        plus[key] = base[key] + h * d
+        minus[key] = base[key] - h * d
+        fd = (f(**plus) - f(**minus)) / (2 * h)
+        an = float(np.sum(grad * d))
+        assert abs(fd - an) <= 1e-7 * np.linalg.norm(grad) * np.linalg.norm(d), (key, fd, an)
