@@ -319,7 +319,16 @@ def config_table(torch, api, dev, hbm, reps=20):
                          "edges_per_s": E / (t_u / 1e3), "hbm_frac": b_u / (t_u / 1e3) / 1e9 / hbm,
                          "mixing_gemm_flops": f_gemm,
                          "mixing_tflops_if_whole_call": f_gemm / (t_u / 1e3) / 1e12})
-            del mix, uws, uout
+            ugo = torch.randn((n, no, v), device=dev)
+            bws = torch.empty(plan.uvw_backward_workspace_bytes(n, E, v) // 4 + 64, dtype=torch.float32, device=dev)
+            t_ub = _time_ms(torch, lambda: plan.uvw_backward(g, x, W, mix, ugo, workspace=bws), k)
+            rows.append({"workload": "molecules fully connected (uvw) backward (grad_x, grad_W, grad_mix, grad_r)",
+                         "L": list(L), "mult": u, "mult_out": v, "n_edges": E, "ms": t_ub,
+                         "edges_per_s": E / (t_ub / 1e3),
+                         "tensor_gemm_flops": 2 * f_gemm,
+                         "launches": "2 tensor-core GEMM sets (per-path output gradients, mixing gradient), "
+                                     "per-path backward chunks, per-path forward recompute, harmonic Jacobian"})
+            del mix, uws, uout, ugo, bws
         del W, gw, out, gx, gr, F, ws, x, go, g
         torch.cuda.empty_cache()
     t = synthetic.tp_batch()

@@ -36,6 +36,9 @@ SIGNATURES = {
                                        _p, _p, _p, _p, _p, _sz, _p]),
     "cgtp_uvw_forward_workspace_size": (_i, [_p, _i, _i, ctypes.POINTER(_sz)]),
     "cgtp_uvw_forward": (_i, [_p, _i, _i, _p, _p, _p, _p, _p, _p, _i, _p, _p, _sz, _p]),
+    "cgtp_uvw_backward_workspace_size": (_i, [_p, _i, _i, _i, ctypes.POINTER(_sz)]),
+    "cgtp_uvw_backward": (_i, [_p, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _p, _p, _p, _p, _p, _p,
+                               _sz, _p]),
     "cgtp_forces": (_i, [_i, _i, _p, _p, _p, _p, _p, _p]),
     "cgtp_radial_forward": (_i, [_p, _i, _p, _f, _p, _p, _p, _p]),
     "cgtp_radial_backward": (_i, [_p, _i, _p, _f, _p, _p, _p, _p, _p]),

@@ -249,6 +249,31 @@ class Plan:
              workspace.numel() * 4, _stream())
         return out
 
+    def uvw_backward_workspace_bytes(self, n_nodes, n_edges, mult_out):
+        b = ctypes.c_size_t()
+        call("cgtp_uvw_backward_workspace_size", self._h, n_nodes, n_edges, mult_out, ctypes.byref(b))
+        return b.value
+
+    def uvw_backward(self, graph, x, w, mix, grad_out, want_x=True, want_w=True, want_mix=True, want_r=True,
+                     workspace=None):
+        """Adjoint of uvw_forward: (grad_x, grad_w, grad_mix, grad_edge_vec)."""
+        for t, nm in ((x, "x"), (w, "w"), (mix, "mix"), (grad_out, "grad_out")):
+            _check(t, torch.float32, nm)
+        dev = x.device
+        E, mult_out = graph.n_edges, mix.shape[2]
+        gx = torch.empty_like(x) if want_x else None
+        gw = torch.empty((E, self.n_paths, self.mult), dtype=torch.float32, device=dev) if want_w else None
+        gm = torch.empty_like(mix) if want_mix else None
+        gr = torch.empty((E, 3), dtype=torch.float32, device=dev) if want_r else None
+        nb = self.uvw_backward_workspace_bytes(graph.n_nodes, E, mult_out)
+        if workspace is None:
+            workspace = torch.empty(max(nb // 4, 64), dtype=torch.float32, device=dev)
+        call("cgtp_uvw_backward", self._h, graph.n_nodes, E, _ptr(graph.row_ptr), _ptr(graph.col),
+             _ptr(graph.csc_ptr), _ptr(graph.csc_edge), _ptr(graph.csc_dst), _ptr(graph.edge_vec), _ptr(x), _ptr(w),
+             _ptr(mix), mult_out, _ptr(grad_out), _ptr(gx), _ptr(gw), _ptr(gm), _ptr(gr), _ptr(workspace),
+             workspace.numel() * 4, _stream())
+        return gx, gw, gm, gr
+
     # ------------------------------------------------------------ radial network
     def radial_forward(self, edge_vec, rc, W1, W2, out=None):
         _check(edge_vec, torch.float32, "edge_vec")

@@ -507,6 +507,99 @@ cgtp_status cgtp_uvw_forward(cgtp_plan p, int n_nodes, int n_edges, const int* r
   return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
 }
 
+struct UvwBwdParts {
+  size_t gt, t, packed, part, gemm, bwd;  // bytes of each workspace part
+};
+static bool uvw_bwd_parts(cgtp_plan p, int n_nodes, int n_edges, int mult_out, bool want_mix, bool want_r,
+                          UvwLayout* L, UvwBwdParts* W) {
+  if (!uvw_layout(p, n_nodes, mult_out, L)) return false;
+  size_t part = 0;
+  for (int l3 = 0; l3 <= p->lo; ++l3) part += (size_t)(2 * l3 + 1) * L->count_l3[l3] * p->mult * mult_out;
+  W->gt = round256(sizeof(float) * L->t_floats);
+  W->t = want_mix ? W->gt : 0;
+  W->packed = round256(sizeof(float) * L->packed_floats);
+  W->part = want_mix ? round256(sizeof(float) * part) : 0;
+  W->gemm = uvw_bwd_gemm_workspace(n_nodes, p->lo, L->count_l3, p->mult, mult_out);
+  size_t bw = 0;
+  if (want_r) cgtp_conv_backward_workspace_size(p, n_edges, &bw);
+  W->bwd = bw;
+  return true;
+}
+
+cgtp_status cgtp_uvw_backward_workspace_size(cgtp_plan p, int n_nodes, int n_edges, int mult_out, size_t* bytes) {
+  if (p == nullptr || n_nodes < 0 || n_edges < 0 || mult_out <= 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
+  UvwLayout L;
+  UvwBwdParts W;
+  if (!uvw_bwd_parts(p, n_nodes, n_edges, mult_out, true, true, &L, &W)) return CGTP_ERR_UNSUPPORTED;
+  *bytes = W.gt + W.t + W.packed + W.part + W.gemm + W.bwd;
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_uvw_backward(cgtp_plan p, int n_nodes, int n_edges, const int* row_ptr, const int* col,
+                              const int* csc_ptr, const int* csc_edge, const int* csc_dst, const float* edge_vec,
+                              const float* x, const float* w, const float* mix, int mult_out, const float* grad_out,
+                              float* grad_x, float* grad_w, float* grad_mix, float* grad_edge_vec, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  if (p == nullptr || n_nodes < 0 || n_edges < 0 || row_ptr == nullptr || csc_ptr == nullptr || mult_out <= 0 ||
+      mix == nullptr)
+    return CGTP_ERR_INVALID_ARG;
+  if (n_nodes > 0 && (x == nullptr || grad_out == nullptr)) return CGTP_ERR_INVALID_ARG;
+  if (n_edges > 0 && (col == nullptr || csc_edge == nullptr || csc_dst == nullptr || edge_vec == nullptr ||
+                      w == nullptr))
+    return CGTP_ERR_INVALID_ARG;
+  for (const void* q : {(const void*)x, (const void*)w, (const void*)mix, (const void*)grad_out, (const void*)grad_x,
+                        (const void*)grad_w, (const void*)grad_mix})
+    if (!aligned16(q)) return CGTP_ERR_INVALID_ARG;
+  if (p->mult % 4 != 0 || mult_out % 4 != 0) return CGTP_ERR_UNSUPPORTED;
+  if (n_nodes == 0) return CGTP_OK;
+  UvwLayout L;
+  UvwBwdParts W;
+  if (!uvw_bwd_parts(p, n_nodes, n_edges, mult_out, grad_mix != nullptr, grad_edge_vec != nullptr, &L, &W))
+    return CGTP_ERR_UNSUPPORTED;
+  const size_t need = W.gt + W.t + W.packed + W.part + W.gemm + W.bwd;
+  if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
+    return CGTP_ERR_WORKSPACE;
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  char* ws = (char*)workspace;
+  float* gt = (float*)ws;
+  float* t = (float*)(ws + W.gt);
+  float* packed_t = (float*)(ws + W.gt + W.t);
+  float* part = (float*)(ws + W.gt + W.t + W.packed);
+  void* gws = ws + W.gt + W.t + W.packed + W.part;
+  float* bws = (float*)(ws + W.gt + W.t + W.packed + W.part + W.gemm);
+  // per-path output gradients gt (tensor cores)
+  cudaError_t e = launch_uvw_pack_t(p->n_paths, p->mult, mult_out, p->lo, L.order, L.count_l3, mix, packed_t, s);
+  if (e == cudaSuccess)
+    e = launch_uvw_gt(n_nodes, p->lo, L.count_l3, p->mult, mult_out, grad_out, packed_t, gt, gws, W.gemm, s);
+  // channelwise backward with one output gradient per path
+  if (e == cudaSuccess && (grad_x != nullptr || grad_w != nullptr || grad_edge_vec != nullptr)) {
+    if (n_edges == 0) {
+      if (grad_x) e = cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)n_nodes * (p->li + 1) * (p->li + 1) * p->mult, s);
+    } else {
+      ConvBwdArgs a{n_nodes, n_edges, csc_ptr, csc_edge, csc_dst, edge_vec, x, w, gt,
+                    grad_x, grad_w, grad_edge_vec, bws, p->mult};
+      a.per_path = 1;
+      e = dispatch_bwd(p, a, sms, s);
+    }
+  }
+  // grad_mix from the recomputed per-path messages t (tensor cores)
+  if (e == cudaSuccess && grad_mix != nullptr) {
+    ConvFwdArgs a{n_nodes, row_ptr, col, edge_vec, x, w, t, p->mult};
+    e = cudaErrorNotSupported;
+#define CGTP_UVWB_PATHS_ENTRY(A, B, C) \
+    if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_paths<A, B, C>(a, sms, s);
+    CGTP_CONFIGS(CGTP_UVWB_PATHS_ENTRY)
+    if (e == cudaSuccess)
+      e = launch_uvw_grad_mix(n_nodes, p->n_paths, p->lo, L.order, L.count_l3, p->mult, mult_out, t, grad_out, part,
+                              grad_mix, gws, W.gemm, s);
+  }
+  if (e == cudaErrorNotSupported) return CGTP_ERR_UNSUPPORTED;
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
 cgtp_status cgtp_forces(int n_nodes, int n_edges, const int* row_ptr, const int* csc_ptr, const int* csc_edge,
                         const float* grad_edge_vec, float* forces, void* stream) {
   if (n_nodes < 0 || n_edges < 0 || row_ptr == nullptr || csc_ptr == nullptr) return CGTP_ERR_INVALID_ARG;

@@ -119,6 +119,32 @@ __device__ __forceinline__ void compute_T_grp(const float (&Y)[PS::NS], float* _
   });
 }
 
+// ---- per-path messages (the fully connected convolution) ----
+// The messages of each path are kept apart in blocks by l3: block l3 holds
+// [node][m3][rank][u] for the paths of that l3 in (l2, path number) order
+// (the order in which the chunk planner below visits them), and the blocks
+// follow one another in increasing l3.
+template <class PS>
+constexpr int l3_rank(int p) {
+  int r = 0;
+  for (int q = 0; q < PS::D.np; ++q)
+    if (PS::D.l3[q] == PS::D.l3[p] && (PS::D.l2[q] < PS::D.l2[p] || (PS::D.l2[q] == PS::D.l2[p] && q < p))) ++r;
+  return r;
+}
+template <class PS>
+constexpr int l3_count(int l3) {
+  int n = 0;
+  for (int q = 0; q < PS::D.np; ++q) n += PS::D.l3[q] == l3;
+  return n;
+}
+// rows per node (paths x (2 l3 + 1)) of the blocks before block l3
+template <class PS>
+constexpr int l3_prefix_rows(int l3) {
+  int r = 0;
+  for (int l = 0; l < l3; ++l) r += l3_count<PS>(l) * (2 * l + 1);
+  return r;
+}
+
 // ---- chunks: the launches of a kernel family ----
 // Paths sorted by (key, l2, lexicographic), key = l1 (backward) or l3
 // (forward), are cut into runs with one key value whose unrolled code per

@@ -47,6 +47,14 @@ size_t uvw_gemm_workspace(int n_nodes, int lmax_out, const int* count_l3, int mu
 cudaError_t launch_uvw_gemm(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out,
                             const float* t, const float* packed, float* out, void* ws, size_t ws_bytes,
                             cudaStream_t stream);
+cudaError_t launch_uvw_pack_t(int n_paths, int mult, int mult_out, int lmax_out, const int* order,
+                              const int* count_l3, const float* mix, float* packed_t, cudaStream_t stream);
+size_t uvw_bwd_gemm_workspace(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out);
+cudaError_t launch_uvw_gt(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out, const float* g,
+                          const float* packed_t, float* gt, void* ws, size_t ws_bytes, cudaStream_t stream);
+cudaError_t launch_uvw_grad_mix(int n_nodes, int n_paths, int lmax_out, const int* order, const int* count_l3,
+                                int mult, int mult_out, const float* t, const float* g, float* part,
+                                float* grad_mix, void* ws, size_t ws_bytes, cudaStream_t stream);
 cudaError_t launch_sh_dir(int lmax_sh, int n_edges, const float* ev, const float* q, float* u, int num_sms,
                           cudaStream_t stream);
 

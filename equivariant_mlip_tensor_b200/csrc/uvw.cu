@@ -47,6 +47,38 @@ __global__ void uvw_pack_kernel(PathOrder po, int mult, int mult_out, int rank0,
   }
 }
 
+// packed transposed block of l3: [2 l3 + 1 copies][mult_out][paths of l3 x mult]
+__global__ void uvw_pack_t_kernel(PathOrder po, int mult, int mult_out, int rank0, int npk, int n3,
+                                  const float* __restrict__ mix, float* __restrict__ packed) {
+  const long long K = (long long)npk * mult;
+  const long long per_copy = K * mult_out;
+  const long long total = per_copy * n3;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i % per_copy;
+    const long long ku = r % K;
+    const int v = int(r / K);
+    const int uu = int(ku % mult), rank = int(ku / mult);
+    packed[i] = mix[((long long)po.order[rank0 + rank] * mult + uu) * mult_out + v];
+  }
+}
+
+// grad_mix[p][u][v] = sum_m3 part[m3][rank(p) * mult + u][v] for the paths of one l3 block
+__global__ void uvw_unpack_kernel(PathOrder po, int mult, int mult_out, int rank0, int npk, int n3,
+                                  const float* __restrict__ part, float* __restrict__ grad_mix) {
+  const long long K = (long long)npk * mult;
+  const long long total = K * mult_out;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    float s = 0.f;
+    for (int m3 = 0; m3 < n3; ++m3) s += part[m3 * total + i];
+    const int v = int(i % mult_out);
+    const long long ku = i / mult_out;
+    const int uu = int(ku % mult), rank = int(ku / mult);
+    grad_mix[((long long)po.order[rank0 + rank] * mult + uu) * mult_out + v] = s;
+  }
+}
+
 #if !defined(CGTP_NO_CUTLASS)
 using namespace cute;
 using TileShape = Shape<_128, _128, _32>;
@@ -69,6 +101,67 @@ using Gemm = cutlass::gemm::device::GemmUniversalAdapter<Kernel>;
 // as n3 batches of [n_nodes][K] (row stride n3 K, batch stride K); B = the
 // packed copies [n3][K][mult_out]; D = out rows (l3, m3) of every node (row
 // stride NO mult_out, batch stride mult_out).
+// D = A^T B with A stored K-major (column-major A): the mixing-matrix gradient.
+using LayoutCol = cutlass::layout::ColumnMajor;
+using EpilogueT = Epilogue;
+using MainloopT = typename cutlass::gemm::collective::CollectiveBuilder<
+    cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, float, LayoutCol, kAlign, float, Layout, kAlign, float,
+    TileShape, ClusterShape,
+    cutlass::gemm::collective::StageCountAutoCarveout<static_cast<int>(sizeof(typename EpilogueT::SharedStorage))>,
+    cutlass::gemm::KernelTmaWarpSpecialized1SmFastFP32Sm100>::CollectiveOp;
+using KernelT = cutlass::gemm::kernel::GemmUniversal<Shape<int, int, int, int>, MainloopT, EpilogueT>;
+using GemmT = cutlass::gemm::device::GemmUniversalAdapter<KernelT>;
+
+// gt block l3 = grad_out rows (l3, m3) x packed^T: A = grad_out [n_nodes][v] per
+// m3 batch (row stride NO v, batch stride v), B = [n3][v][K], D = gt block
+// [n_nodes][n3][K] (row stride n3 K, batch stride K).
+Gemm::Arguments block_args_gt(int n_nodes, int l3, int lmax_out, int K, int mult_out, const float* g,
+                              const float* packed_t, float* gt) {
+  const int n3 = 2 * l3 + 1, no = (lmax_out + 1) * (lmax_out + 1);
+  using SA = typename Kernel::StrideA;
+  using SB = typename Kernel::StrideB;
+  using SC = typename Kernel::StrideC;
+  using SD = typename Kernel::StrideD;
+  SA sa = cutlass::make_cute_packed_stride(SA{}, make_shape(n_nodes, mult_out, n3));
+  get<0>(sa) = (int64_t)no * mult_out;
+  get<2>(sa) = mult_out;
+  SB sb = cutlass::make_cute_packed_stride(SB{}, make_shape(K, mult_out, n3));
+  SD sd = cutlass::make_cute_packed_stride(SD{}, make_shape(n_nodes, K, n3));
+  get<0>(sd) = (int64_t)n3 * K;
+  get<2>(sd) = K;
+  SC sc = sd;
+  const float* A = g == nullptr ? nullptr : g + (size_t)l3 * l3 * mult_out;
+  return Gemm::Arguments{cutlass::gemm::GemmUniversalMode::kGemm,
+                         {n_nodes, K, mult_out, n3},
+                         {A, sa, packed_t, sb},
+                         {{1.f, 0.f}, gt, sc, gt, sd}};
+}
+
+// part[m3] = t block (m3)^T x grad_out rows (l3, m3): A = t viewed K-major
+// (column-major [K][n_nodes], column stride n3 K, batch stride K), B =
+// grad_out [n_nodes][v] (row stride NO v, batch stride v), D = [n3][K][v].
+GemmT::Arguments block_args_mix(int n_nodes, int l3, int lmax_out, int K, int mult_out, const float* t,
+                                const float* g, float* part) {
+  const int n3 = 2 * l3 + 1, no = (lmax_out + 1) * (lmax_out + 1);
+  using SA = typename KernelT::StrideA;
+  using SB = typename KernelT::StrideB;
+  using SC = typename KernelT::StrideC;
+  using SD = typename KernelT::StrideD;
+  SA sa = cutlass::make_cute_packed_stride(SA{}, make_shape(K, n_nodes, n3));
+  get<1>(sa) = (int64_t)n3 * K;
+  get<2>(sa) = K;
+  SB sb = cutlass::make_cute_packed_stride(SB{}, make_shape(mult_out, n_nodes, n3));
+  get<1>(sb) = (int64_t)no * mult_out;
+  get<2>(sb) = mult_out;
+  SD sd = cutlass::make_cute_packed_stride(SD{}, make_shape(K, mult_out, n3));
+  SC sc = sd;
+  const float* B = g == nullptr ? nullptr : g + (size_t)l3 * l3 * mult_out;
+  return GemmT::Arguments{cutlass::gemm::GemmUniversalMode::kGemm,
+                          {K, mult_out, n_nodes, n3},
+                          {t, sa, B, sb},
+                          {{1.f, 0.f}, part, sc, part, sd}};
+}
+
 Gemm::Arguments block_args(int n_nodes, int l3, int lmax_out, int K, int mult_out, const float* t,
                            const float* packed, float* out) {
   const int n3 = 2 * l3 + 1, no = (lmax_out + 1) * (lmax_out + 1);
@@ -146,6 +239,101 @@ cudaError_t launch_uvw_gemm(int n_nodes, int lmax_out, const int* count_l3, int 
     }
     t_off += (size_t)n_nodes * n3 * K;
     p_off += (size_t)n3 * K * mult_out;
+  }
+  return cudaGetLastError();
+#endif
+}
+
+cudaError_t launch_uvw_pack_t(int n_paths, int mult, int mult_out, int lmax_out, const int* order,
+                              const int* count_l3, const float* mix, float* packed_t, cudaStream_t stream) {
+  PathOrder po{};
+  for (int k = 0; k < n_paths && k < kMaxPaths; ++k) po.order[k] = order[k];
+  int rank0 = 0;
+  size_t off = 0;
+  for (int l3 = 0; l3 <= lmax_out; ++l3) {
+    const int npk = count_l3[l3], n3 = 2 * l3 + 1;
+    if (npk > 0) {
+      uvw_pack_t_kernel<<<256, 256, 0, stream>>>(po, mult, mult_out, rank0, npk, n3, mix, packed_t + off);
+      const cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    off += (size_t)n3 * npk * mult * mult_out;
+    rank0 += npk;
+  }
+  return cudaSuccess;
+}
+
+size_t uvw_bwd_gemm_workspace(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out) {
+#if defined(CGTP_NO_CUTLASS)
+  return 0;
+#else
+  size_t w = 0;
+  for (int l3 = 0; l3 <= lmax_out; ++l3) {
+    if (count_l3[l3] == 0) continue;
+    const int K = count_l3[l3] * mult;
+    const size_t a = Gemm::get_workspace_size(block_args_gt(n_nodes, l3, lmax_out, K, mult_out, nullptr, nullptr,
+                                                            nullptr));
+    const size_t b = GemmT::get_workspace_size(block_args_mix(n_nodes, l3, lmax_out, K, mult_out, nullptr, nullptr,
+                                                              nullptr));
+    w = a > w ? a : w;
+    w = b > w ? b : w;
+  }
+  return (w + 255) & ~(size_t)255;
+#endif
+}
+
+// gt = per-path output gradients (per l3 block: grad_out rows x packed^T)
+cudaError_t launch_uvw_gt(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out, const float* g,
+                          const float* packed_t, float* gt, void* ws, size_t ws_bytes, cudaStream_t stream) {
+#if defined(CGTP_NO_CUTLASS)
+  return cudaErrorNotSupported;
+#else
+  size_t t_off = 0, p_off = 0;
+  for (int l3 = 0; l3 <= lmax_out; ++l3) {
+    const int npk = count_l3[l3], n3 = 2 * l3 + 1, K = npk * mult;
+    if (npk > 0) {
+      Gemm gm;
+      auto args = block_args_gt(n_nodes, l3, lmax_out, K, mult_out, g, packed_t + p_off, gt + t_off);
+      if (gm.can_implement(args) != cutlass::Status::kSuccess) return cudaErrorNotSupported;
+      if (Gemm::get_workspace_size(args) > ws_bytes) return cudaErrorInvalidValue;
+      if (gm.initialize(args, ws, stream) != cutlass::Status::kSuccess) return cudaErrorLaunchFailure;
+      if (gm.run(stream) != cutlass::Status::kSuccess) return cudaErrorLaunchFailure;
+    }
+    t_off += (size_t)n_nodes * n3 * K;
+    p_off += (size_t)n3 * K * mult_out;
+  }
+  return cudaGetLastError();
+#endif
+}
+
+// grad_mix from the per-path messages t and grad_out (per l3 block, one
+// partial per m3 summed by the unpacking kernel); part: [sum_l3 n3 K v] floats
+cudaError_t launch_uvw_grad_mix(int n_nodes, int n_paths, int lmax_out, const int* order, const int* count_l3,
+                                int mult, int mult_out, const float* t, const float* g, float* part,
+                                float* grad_mix, void* ws, size_t ws_bytes, cudaStream_t stream) {
+#if defined(CGTP_NO_CUTLASS)
+  return cudaErrorNotSupported;
+#else
+  PathOrder po{};
+  for (int k = 0; k < n_paths && k < kMaxPaths; ++k) po.order[k] = order[k];
+  size_t t_off = 0, p_off = 0;
+  int rank0 = 0;
+  for (int l3 = 0; l3 <= lmax_out; ++l3) {
+    const int npk = count_l3[l3], n3 = 2 * l3 + 1, K = npk * mult;
+    if (npk > 0) {
+      GemmT gm;
+      auto args = block_args_mix(n_nodes, l3, lmax_out, K, mult_out, t + t_off, g, part + p_off);
+      if (gm.can_implement(args) != cutlass::Status::kSuccess) return cudaErrorNotSupported;
+      if (GemmT::get_workspace_size(args) > ws_bytes) return cudaErrorInvalidValue;
+      if (gm.initialize(args, ws, stream) != cutlass::Status::kSuccess) return cudaErrorLaunchFailure;
+      if (gm.run(stream) != cutlass::Status::kSuccess) return cudaErrorLaunchFailure;
+      uvw_unpack_kernel<<<256, 256, 0, stream>>>(po, mult, mult_out, rank0, npk, n3, part + p_off, grad_mix);
+      const cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    t_off += (size_t)n_nodes * n3 * K;
+    p_off += (size_t)n3 * K * mult_out;
+    rank0 += npk;
   }
   return cudaGetLastError();
 #endif

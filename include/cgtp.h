@@ -235,6 +235,30 @@ cgtp_status cgtp_uvw_forward(cgtp_plan plan, int n_nodes, int n_edges, const int
                              const float* mix, int mult_out, float* out, void* workspace,
                              size_t workspace_bytes, void* stream);
 
+/* Bytes of device workspace cgtp_uvw_backward needs (with every output). */
+cgtp_status cgtp_uvw_backward_workspace_size(cgtp_plan plan, int n_nodes, int n_edges, int mult_out,
+                                             size_t* bytes);
+
+/* ---------------------------------------------------------------------------
+ * Fully connected convolution backward, the adjoint of cgtp_uvw_forward for
+ * grad_out [n_nodes][(lmax_out+1)^2][mult_out]:
+ *   gt[i][p][m3][u]    = sum_v grad_out[i][l3,m3][v] mix[p][u][v]      (tensor cores)
+ *   grad_mix[p][u][v]  = sum_i sum_m3 t[i][p][m3][u] grad_out[i][l3,m3][v]  (tensor cores,
+ *                        t recomputed)
+ * and the channelwise backward with one output gradient per path (gt):
+ * grad_x [n_nodes][(lmax_in+1)^2][mult], grad_w [n_edges][n_paths][mult],
+ * grad_edge_vec [n_edges][3].  Every output is nullable (not computed) and
+ * overwritten.  Needs both graph views; workspace as reported by
+ * cgtp_uvw_backward_workspace_size (device, 256-byte aligned).
+ * ------------------------------------------------------------------------- */
+cgtp_status cgtp_uvw_backward(cgtp_plan plan, int n_nodes, int n_edges, const int* row_ptr,
+                              const int* col, const int* csc_ptr, const int* csc_edge,
+                              const int* csc_dst, const float* edge_vec, const float* x,
+                              const float* w, const float* mix, int mult_out,
+                              const float* grad_out, float* grad_x, float* grad_w,
+                              float* grad_mix, float* grad_edge_vec, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Per-atom forces from edge-vector gradients, F = -dE/dpos with
  * r_e = pos_src - pos_dst:  F[n] = sum_{e: dst=n} g[e] - sum_{e: src=n} g[e].

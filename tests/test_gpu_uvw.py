@@ -1,7 +1,8 @@
 """GPU parity of the fully connected ("uvw") convolution against the oracle:
-several shapes and output multiplicities, identity mixing against the
-channelwise convolution, sampled rows at the molecules workload, an
-edge-free graph and the host-side errors."""
+forward at several shapes and output multiplicities, identity mixing against
+the channelwise convolution, sampled rows at the molecules workload, an
+edge-free graph and the host-side errors; backward (grad_x, grad_w, grad_mix,
+grad_edge_vec) at four shapes and with each output alone."""
 import ctypes
 
 import numpy as np
@@ -111,3 +112,69 @@ def test_host_errors(api):
     assert f(*args, 8, p(out), p(ws), nb - 256, None) == 7          # workspace too small
     assert f(*args, 8, p(out), None, 0, None) == 7                  # no workspace
     assert f(*args, 8, p(out), p(ws), nb, None) == 0
+
+
+@pytest.mark.parametrize("L,mult,mult_out", [((1, 1, 1), 8, 12), ((2, 2, 2), 32, 16), ((2, 4, 2), 128, 128),
+                                             ((3, 3, 3), 64, 32)])
+def test_backward_matches_oracle(api, L, mult, mult_out):
+    from tests.gpu_common import GRAD_TOL
+    o, g, x, W, mix = _case(api, L, mult, mult_out, 95 + mult)
+    rng = np.random.default_rng(96)
+    go = rng.standard_normal((x.shape[0], (L[2] + 1) ** 2, mult_out)).astype(np.float32)
+    plan = api.Plan(*L, mult)
+    got = plan.uvw_backward(g, cuda(x), cuda(W), cuda(mix), cuda(go))
+    ref = oconv.conv_uvw_backward(o["row_ptr"], o["col"], o["edge_vec"], x, W, mix, go, *L)
+    for name, a, b in zip(("grad_x", "grad_w", "grad_mix", "grad_edge_vec"), got, ref):
+        assert rel_err(host(a), b) <= GRAD_TOL, (name, rel_err(host(a), b))
+
+
+def test_backward_nullable_outputs(api):
+    L, mult, mult_out = (2, 2, 2), 16, 8
+    o, g, x, W, mix = _case(api, L, mult, mult_out, 97)
+    go = np.random.default_rng(98).standard_normal((x.shape[0], 9, mult_out)).astype(np.float32)
+    plan = api.Plan(*L, mult)
+    args = (g, cuda(x), cuda(W), cuda(mix), cuda(go))
+    full = plan.uvw_backward(*args)
+    flags = ("want_x", "want_w", "want_mix", "want_r")
+    for k in range(4):
+        only = plan.uvw_backward(*args, **{f: (f == flags[k]) for f in flags})
+        assert all(only[m] is None for m in range(4) if m != k)
+        # the chunk plan (and so the summation order of grad_x) depends on
+        # whether grad_edge_vec is requested: equal to rounding, not bitwise
+        assert rel_err(host(only[k]), host(full[k]).astype(np.float64)) <= 1e-6
+
+
+def test_backward_molecules_sampled(api):
+    """Full-size backward: per-edge gradients of sampled edges and grad_x rows
+    of sampled sources against the oracle on the sub-graphs that determine them."""
+    from tests.gpu_common import GRAD_TOL
+    w = synthetic.molecules()
+    L = (w.lmax_in, w.lmax_sh, w.lmax_out)
+    n = w.n_nodes
+    g = api.build_graph(cuda(w.pos), w.rc, graph_ptr=cuda(np.arange(0, n + 1, w.graph_size, dtype=np.int32)))
+    o = ograph.neighbour_list(w.pos, w.rc, None, w.graph_id)
+    plan = api.Plan(*L, w.mult)
+    rng = np.random.default_rng(99)
+    E = o["col"].size
+    W = rng.standard_normal((E, plan.n_paths, w.mult)).astype(np.float32)
+    mix = (rng.standard_normal((plan.n_paths, w.mult, 64)) / np.sqrt(w.mult)).astype(np.float32)
+    go = rng.standard_normal((n, 9, 64)).astype(np.float32)
+    gx, gw, gm, gr = plan.uvw_backward(g, cuda(w.x), cuda(W), cuda(mix), cuda(go))
+    rp = o["row_ptr"]
+    dst_all = ograph.edge_dst(rp)
+
+    def sub(edges):
+        edges = np.sort(edges)
+        sp = np.zeros(n + 1, dtype=np.int64)
+        np.add.at(sp, dst_all[edges] + 1, 1)
+        return np.cumsum(sp), o["col"][edges], o["edge_vec"][edges], edges
+
+    edges = rng.choice(E, size=48, replace=False)
+    srp, scol, sev, es = sub(edges)
+    _, rw, _, rr = oconv.conv_uvw_backward(srp, scol, sev, w.x, W[es], mix, go, *L)
+    assert rel_err(host(gw[es.tolist()]), rw) <= GRAD_TOL
+    assert rel_err(host(gr[es.tolist()]), rr) <= GRAD_TOL
+    nodes = np.sort(rng.choice(n, size=8, replace=False))
+    srp, scol, sev, es = sub(np.nonzero(np.isin(o["col"], nodes))[0])
+    rx, _, _, _ = oconv.conv_uvw_backward(srp, scol, sev, w.x, W[es], mix, go, *L)
+    assert rel_err(host(gx[nodes.tolist()]), rx[nodes]) <= GRAD_TOL

@@ -1,7 +1,7 @@
 """Pins of the oracle's fully connected ("uvw") convolution: the identity
 mixing reduces it to the channelwise convolution, a pure-Python brute force
 over edges, nonzeros and channels (real CG from the Racah formula, harmonics
-from scipy through the real basis), equivariance under rotations, and
+from the independent Legendre-recurrence route), equivariance under rotations, and
 linearity in the mixing matrices; the backward against the channelwise
 backward (identity mixing) and against central differences of the forward."""
 import numpy as np
