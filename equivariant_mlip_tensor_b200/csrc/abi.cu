@@ -581,8 +581,10 @@ cgtp_status cgtp_uvw_backward(cgtp_plan p, int n_nodes, int n_edges, const int* 
     } else {
       ConvBwdArgs a{n_nodes, n_edges, csc_ptr, csc_edge, csc_dst, edge_vec, x, w, gt,
                     grad_x, grad_w, grad_edge_vec, bws, p->mult};
-      a.per_path = 1;
-      e = dispatch_bwd(p, a, sms, s);
+      e = cudaErrorNotSupported;
+#define CGTP_UVWB_BWD_ENTRY(A, B, C) \
+      if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_bwd_paths<A, B, C>(a, sms, s);
+      CGTP_CONFIGS(CGTP_UVWB_BWD_ENTRY)
     }
   }
   // grad_mix from the recomputed per-path messages t (tensor cores)

@@ -137,9 +137,6 @@ struct ConvBwdArgs {
   // 3: = sum_b G_b (d2Y_b/dr2) gr_dir
   int gr_mode = 0;
   const float* gr_dir = nullptr;  // [n_edges][3], for gr_mode 2 and 3
-  // grad_out holds one gradient per path (the per-path message layout of the
-  // fully connected convolution) instead of one per output block
-  int per_path = 0;
 };
 
 struct TPArgs {

@@ -64,15 +64,6 @@ constexpr unsigned touched_sh_mask() {
   return m;
 }
 
-// Per-path output gradients: staged rows of path K of the group start at
-// pp_rowoff(K) (each path has its own 2 l3 + 1 rows).
-template <class PS, class GR>
-constexpr int pp_rowoff(int K) {
-  int r = 0;
-  for (int k = 0; k < K; ++k) r += 2 * PS::D.l3[GR::D.path[k]] + 1;
-  return r;
-}
-
 // One edge of the CSC row, the paths of one group (l1 = GR's value).  Per
 // path, with h[m1] = sum_m3 T[m1][m3] g[m3] (one pass over the structural
 // nonzeros of T):
@@ -83,7 +74,7 @@ constexpr int pp_rowoff(int K) {
 // finished block goes to this lane's column of the shared reduction buffer
 // (gyrow, row stride rs).  The edge's weight rows and its destination's output-gradient
 // rows come from this lane's pipeline stage.
-template <class PS, class GR, int VEC, bool NEED_GY, bool PP>
+template <class PS, class GR, int VEC, bool NEED_GY>
 __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const float* __restrict__ stage, int rowf,
                                          const float (&xr)[GR::NOWN][VEC], float* __restrict__ gwrow, bool acc, int mult,
                                          float (&gx)[GR::NOWN][VEC], float* __restrict__ gyrow, int rs) {
@@ -93,8 +84,7 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
     constexpr int P = GR::D.path[K];
     constexpr int l1 = PS::D.l1[P], l2 = PS::D.l2[P], l3 = PS::D.l3[P];
     constexpr int tb = GR::D.lt[K], tc = PS::D.tcount[P];
-    // staged row of grad_out[l3, m3 = -l3] (of this path's own rows when PP)
-    constexpr int g0 = PP ? GR::NP + pp_rowoff<PS, GR>(K) : GR::NP + l3 * l3 - GR::D.rlo;
+    constexpr int g0 = GR::NP + l3 * l3 - GR::D.rlo;  // staged row of grad_out[l3, m3 = -l3]
     if constexpr (NEED_GY && GR::D.first_l2[K]) {
 #pragma unroll
       for (int m2 = 0; m2 < 2 * l2 + 1; ++m2) gy[l2 * l2 + m2] = 0.f;
@@ -186,9 +176,7 @@ using BwdPlan = Plan<PS, kByL1, VEC, NEED_GY, bwd_budget<PS>()>;
 // of the chunk's paths and a partial grad_Y over them.
 // EXT: the double backward's variant (per-edge harmonics given by the caller,
 // results added onto the outputs); the plain variant compiles without either.
-// PP: grad_out is the per-path message layout of the fully connected
-// convolution (each path reads its own rows).
-template <class PS, int VEC, bool NEED_GY, int CH, int KMULT, bool EXT, bool PP>
+template <class PS, int VEC, bool NEED_GY, int CH, int KMULT, bool EXT>
 __global__ void CGTP_BWD_BOUNDS
 conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt) {
   // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x VEC
@@ -200,8 +188,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
   using GR = ChunkGrp<PS, BwdPlan<PS, VEC, NEED_GY>, CH, kByL1>;
   constexpr int L1 = GR::KEY;
   constexpr int NI = PS::NI, NO = PS::NO, NS = PS::NS, NR = GR::NOWN, NT = GR::NT;
-  constexpr int NG = PP ? pp_rowoff<PS, GR>(GR::NP) : GR::NROW;  // staged gradient rows
-  constexpr int NROWS = GR::NP + NG;
+  constexpr int NROWS = GR::NP + GR::NROW;
   constexpr unsigned GY_MASK = touched_sh_mask<PS, GR>();  // harmonics this chunk's paths reach
   extern __shared__ float4 smem_f4[];
   float* smem = reinterpret_cast<float*>(smem_f4);
@@ -262,26 +249,10 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
         constexpr int P = GR::D.path[K];
         VecIO<VEC>::cp_async(dst + K * rowf, wrow + P * mult);
       });
-      if constexpr (PP) {
-        // block l3 of the per-path layout: [node][m3][rank][u]
-        static_for<0, GR::NP>([&](auto Kc) {
-          constexpr int K = decltype(Kc)::value;
-          constexpr int P = GR::D.path[K];
-          constexpr int l3 = PS::D.l3[P], n3 = 2 * l3 + 1;
-          constexpr int npk = l3_count<PS>(l3), rank = l3_rank<PS>(P), pre = l3_prefix_rows<PS>(l3);
-          constexpr int ro = pp_rowoff<PS, GR>(K);
-          const float* base = a.grad_out + (long long)a.n_nodes * mult * pre +
-                              ((long long)Ig[k] * n3 * npk + rank) * mult + c0;
+      constexpr int rlo = GR::D.rlo;
+      const float* grow = a.grad_out + ((long long)Ig[k] * NO + rlo) * mult + c0;
 #pragma unroll
-          for (int m3 = 0; m3 < n3; ++m3)
-            VecIO<VEC>::cp_async(dst + (GR::NP + ro + m3) * rowf, base + (long long)m3 * npk * mult);
-        });
-      } else {
-        constexpr int rlo = GR::D.rlo;
-        const float* grow = a.grad_out + ((long long)Ig[k] * NO + rlo) * mult + c0;
-#pragma unroll
-        for (int r = 0; r < GR::NROW; ++r) VecIO<VEC>::cp_async(dst + (GR::NP + r) * rowf, grow + r * mult);
-      }
+      for (int r = 0; r < GR::NROW; ++r) VecIO<VEC>::cp_async(dst + (GR::NP + r) * rowf, grow + r * mult);
     };
 
     for (int b0 = 0; b0 < maxdeg; b0 += BT) {
@@ -308,7 +279,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
         int e = 0;
         if (valid) {
           e = Eg[k];
-          bwd_edge<PS, GR, VEC, NEED_GY, PP>(Tg + k * NT, St + (k & 1) * stage_floats + gl * VEC, rowf, xr,
+          bwd_edge<PS, GR, VEC, NEED_GY>(Tg + k * NT, St + (k & 1) * stage_floats + gl * VEC, rowf, xr,
                                          a.grad_w ? a.grad_w + (long long)e * PS::NP * mult + c0 : nullptr,
                                          EXT && a.accumulate != 0, mult, gx, red + gl, rs);
         }
@@ -473,8 +444,7 @@ cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t str
   int G, lg_G, S;
   bwd_geometry<PS>(a.mult, G, lg_G, S);
   const int gpw = 32 / G;
-  const int ng = a.per_path ? pp_rowoff<PS, GR>(GR::NP) : GR::NROW;
-  const int stage_floats = (GR::NP + ng) * G * VEC;
+  const int stage_floats = (GR::NP + GR::NROW) * G * VEC;
   const int BT = pick_batch(gpw, GR::NT, stage_floats, CGTP_BWD_BATCH_FLOATS, CGTP_BWD_MAX_BATCH);
   const int group_floats = BT * GR::NT + 2 * stage_floats + 2 * ((BT + 3) & ~3);
   const size_t smem = sizeof(float) * ((size_t)group_floats * gpw * (kBwdThreads / 32) +
@@ -482,11 +452,9 @@ cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t str
   const long long items = (long long)a.n_nodes * S;
   const long long groups_per_block = (long long)gpw * (kBwdThreads / 32);
   const long long blocks = (items + groups_per_block - 1) / groups_per_block;
-  if (a.per_path && (a.sh != nullptr || a.accumulate)) return cudaErrorInvalidValue;
-  auto kern = a.per_path                       ? conv_bwd_kernel<PS, VEC, NEED_GY, CH, 0, false, true>
-              : (a.sh != nullptr || a.accumulate) ? conv_bwd_kernel<PS, VEC, NEED_GY, CH, 0, true, false>
-              : a.mult == 128                   ? conv_bwd_kernel<PS, VEC, NEED_GY, CH, 128, false, false>
-                                                : conv_bwd_kernel<PS, VEC, NEED_GY, CH, 0, false, false>;
+  auto kern = (a.sh != nullptr || a.accumulate) ? conv_bwd_kernel<PS, VEC, NEED_GY, CH, 0, true>
+               : a.mult == 128                 ? conv_bwd_kernel<PS, VEC, NEED_GY, CH, 128, false>
+                                               : conv_bwd_kernel<PS, VEC, NEED_GY, CH, 0, false>;
   cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e2 != cudaSuccess) return e2;
   long long cap = 0x7fffffffLL;  // the kernel loops over items beyond the grid

@@ -98,9 +98,7 @@ __device__ __forceinline__ void fwd_edge(const float* __restrict__ T, const floa
     constexpr int tc = PS::D.tcount[P], tb = GR::D.lt[K];
     float wv[kFwdVec];
     VecIO<kFwdVec>::lds(wv, stage + K * rowf);
-    // first own row of this path's output: its l3 block, or its own block of
-    // 2 l3 + 1 rows when the launch keeps the paths apart
-    constexpr int o3 = GR::PERPATH ? K * (2 * l3 + 1) : l3 * l3 - GR::OWN0;
+    constexpr int o3 = l3 * l3 - GR::OWN0;  // first own row of this path's output block
     if constexpr (2 * l3 + 1 <= 2 * l1 + 1) {
       // t[m3] = sum_m1 T x[m1], then out[m3] += W t[m3]
       float t[2 * l3 + 1][kFwdVec];
@@ -258,20 +256,7 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
       }
       __syncwarp();
     }
-    if constexpr (GR::PERPATH) {
-      // t[node][m3][rank][u] of this l3 block, rank = the path's place among
-      // the block's paths
-      if (active) {
-        constexpr int n3 = 2 * GR::KEY + 1;
-        static_for<0, GR::NP>([&](auto Kc) {
-          constexpr int K = decltype(Kc)::value;
-#pragma unroll
-          for (int m3 = 0; m3 < n3; ++m3)
-            VecIO<kFwdVec>::st(a.out + (((long long)node * n3 + m3) * GR::NPK + GR::PL0 + K) * mult + c0,
-                               acc[K * n3 + m3]);
-        });
-      }
-    } else if (active) {
+    if (active) {
       if (!GR::FIRST || a.accumulate) {
         // rows of an l3 block that the preceding launch wrote (wait for it),
         // or the caller's values to add onto
@@ -329,33 +314,6 @@ constexpr int fwd_all_cost() {
 template <class PS>
 using FwdPlan = Plan<PS, kByL3, kFwdVec, false, CGTP_FWD_BUDGET>;
 
-// Per-path rows (the fully connected convolution's first stage): chunks of
-// same-l3 paths that keep one block of 2 l3 + 1 output rows per path, at most
-// kPathRowsMax rows per chunk (the accumulators stay in registers).
-constexpr int kPathRowsMax = 16;
-template <class PS>
-using PathPlan = Plan<PS, kByL3, kFwdVec, false, CGTP_FWD_BUDGET, kPathRowsMax>;
-
-template <class PS, class PL, int CH>
-struct PathRowsGrp : ChunkGrp<PS, PL, CH, kByL3> {
-  using Base = ChunkGrp<PS, PL, CH, kByL3>;
-  static constexpr bool PERPATH = true;
-  static constexpr int NOWN = Base::NP * (2 * Base::KEY + 1);
-  static constexpr int key_first() {  // first place of this l3 in the plan's order
-    for (int c = 0; c < PL::P.n; ++c)
-      if (PL::P.key[c] == Base::KEY) return PL::P.first[c];
-    return 0;
-  }
-  static constexpr int key_count() {
-    int n = 0;
-    for (int c = 0; c < PL::P.n; ++c)
-      if (PL::P.key[c] == Base::KEY) n += PL::P.count[c];
-    return n;
-  }
-  static constexpr int NPK = key_count();                     // paths with this l3
-  static constexpr int PL0 = PL::P.first[CH] - key_first();   // rank of the chunk's first path
-};
-
 // Output blocks l3 that no path reaches are zero.
 template <class PS>
 cudaError_t zero_unreached_out(const ConvFwdArgs& a, cudaStream_t stream) {
@@ -394,48 +352,8 @@ cudaError_t launch_conv_fwd(const ConvFwdArgs& a, int num_sms, cudaStream_t stre
   }
 }
 
-// Paths in the order of the per-path rows (by l3, then l2, then
-// lexicographic) and the number of paths of each l3.
-template <int LI, int LS, int LO>
-void conv_path_order(int* order, int* count_l3) {
-  using PL = PathPlan<PathSet<LI, LS, LO>>;
-  for (int l = 0; l <= LO; ++l) count_l3[l] = 0;
-  int k = 0;
-  for (int c = 0; c < PL::P.n; ++c)
-    for (int q = 0; q < PL::P.count[c]; ++q) {
-      order[k++] = PL::P.order[PL::P.first[c] + q];
-      ++count_l3[PL::P.key[c]];
-    }
-}
-
-// Per-path messages t (the fully connected convolution's first stage): a.out
-// is t, whose block for l3 holds [n_nodes][2 l3 + 1][paths of l3][mult] and
-// follows the blocks of smaller l3.
-template <int LI, int LS, int LO>
-cudaError_t launch_conv_paths(const ConvFwdArgs& a, int num_sms, cudaStream_t stream) {
-  using PS = PathSet<LI, LS, LO>;
-  using PL = PathPlan<PS>;
-  cudaError_t err = cudaSuccess;
-  static_for_host<0, PL::N>([&](auto Cc) {
-    constexpr int CH = decltype(Cc)::value;
-    using GR = PathRowsGrp<PS, PL, CH>;
-    size_t off = 0;  // floats before the l3 = KEY block
-    for (int c = 0; c < PL::P.n; ++c)
-      if (PL::P.key[c] < GR::KEY) off += (size_t)PL::P.count[c] * (2 * PL::P.key[c] + 1);
-    ConvFwdArgs b = a;
-    b.out = a.out + off * (size_t)a.n_nodes * a.mult;
-    b.accumulate = 0;
-    // chunks write disjoint rows: all but the first may overlap the one before
-    if (err == cudaSuccess) err = launch_fwd_group<PS, GR>(b, num_sms, CH > 0, stream);
-  });
-  return err;
-}
-
 // One translation unit per shape (the build passes CGTP_CFG_LI/LS/LO).
 template cudaError_t launch_conv_fwd<CGTP_CFG_LI, CGTP_CFG_LS, CGTP_CFG_LO>(const ConvFwdArgs&, int,
                                                                          cudaStream_t);
-template cudaError_t launch_conv_paths<CGTP_CFG_LI, CGTP_CFG_LS, CGTP_CFG_LO>(const ConvFwdArgs&, int,
-                                                                           cudaStream_t);
-template void conv_path_order<CGTP_CFG_LI, CGTP_CFG_LS, CGTP_CFG_LO>(int*, int*);
 
 }  // namespace cgtp
