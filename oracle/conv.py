@@ -318,3 +318,24 @@ def conv_uvw_backward(row_ptr, col, edge_vec, x, w, mix, grad_out, lmax_in, lmax
     grad_r = np.einsum("eb,ebk->ek", gY, J)
     return grad_x, grad_w, grad_mix, grad_r
 
+
+def conv_forward_shared(row_ptr, col, edge_vec, x, w_shared, lmax_in, lmax_sh, lmax_out):
+    """Convolution whose weights are shared by every path (path stride 0:
+    W_e[p][u] = w_shared[e][u]; "Tensor Decomposition Networks ...", reply to
+    reviewer oXft: path-weight sharing): conv_forward with the one row repeated
+    for every path."""
+    w_shared = np.asarray(w_shared, dtype=np.float64)
+    P = len(paths(lmax_in, lmax_sh, lmax_out))
+    return conv_forward(row_ptr, col, edge_vec, x, np.repeat(w_shared[:, None, :], P, axis=1),
+                        lmax_in, lmax_sh, lmax_out)
+
+
+def conv_backward_shared(row_ptr, col, edge_vec, x, w_shared, grad_out, lmax_in, lmax_sh, lmax_out):
+    """Adjoint of conv_forward_shared: (grad_x, grad_w_shared [E][u], grad_edge_vec);
+    the shared row's gradient is the sum over paths of the per-path ones."""
+    w_shared = np.asarray(w_shared, dtype=np.float64)
+    P = len(paths(lmax_in, lmax_sh, lmax_out))
+    gx, gw, gr = conv_backward(row_ptr, col, edge_vec, x, np.repeat(w_shared[:, None, :], P, axis=1), grad_out,
+                               lmax_in, lmax_sh, lmax_out)
+    return gx, gw.sum(axis=1), gr
+
