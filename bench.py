@@ -290,6 +290,20 @@ def config_table(torch, api, dev, hbm, reps=20):
                      "fp32_frac": {"fwd": f_f / (t_f / 1e3) / 1e12 / FP32_PEAK_TFLOPS,
                                    "bwd": f_b / (t_b / 1e3) / 1e12 / FP32_PEAK_TFLOPS}})
         if name == "molecules":
+            # weights shared by every path (path stride 0): one weight row per edge
+            wsh = torch.randn((E, u), device=dev)
+            gws = torch.empty_like(wsh)
+            t_sf = _time_ms(torch, lambda: plan.conv_forward_shared(g, x, wsh, out=out), k)
+            t_sb = _time_ms(torch, lambda: plan.conv_backward_shared(g, x, wsh, go, workspace=ws), k)
+            b_sf = 4 * (E * u + n * ni * u + n * no * u + 4 * E + (n + 1))
+            b_sb = 4 * (2 * E * u + 2 * n * ni * u + n * no * u + 5 * E + (n + 1) + slices * E * ns)
+            rows.append({"workload": "molecules, weights shared by every path (path stride 0)",
+                         "L": list(L), "mult": u, "n_edges": E, "fwd_ms": t_sf, "bwd_ms": t_sb,
+                         "edges_per_s_fwd_bwd": E / ((t_sf + t_sb) / 1e3),
+                         "hbm_frac": {"fwd": b_sf / (t_sf / 1e3) / 1e9 / hbm, "bwd": b_sb / (t_sb / 1e3) / 1e9 / hbm},
+                         "fp32_frac": {"fwd": f_f / (t_sf / 1e3) / 1e12 / FP32_PEAK_TFLOPS,
+                                       "bwd": f_b / (t_sb / 1e3) / 1e12 / FP32_PEAK_TFLOPS}})
+            del wsh, gws
             # double backward (adjoint of the backward) with all three cotangents
             ggx, ggw, ggr = torch.randn_like(x), torch.randn_like(W), torch.randn((E, 3), device=dev)
             dws = torch.empty(plan.conv_double_backward_workspace_bytes(E) // 4 + 64, dtype=torch.float32,

@@ -39,6 +39,8 @@ SIGNATURES = {
     "cgtp_uvw_backward_workspace_size": (_i, [_p, _i, _i, _i, ctypes.POINTER(_sz)]),
     "cgtp_uvw_backward": (_i, [_p, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _p, _p, _p, _p, _p, _p,
                                _sz, _p]),
+    "cgtp_conv_forward_shared_weights": (_i, [_p, _i, _i, _p, _p, _p, _p, _p, _p, _p]),
+    "cgtp_conv_backward_shared_weights": (_i, [_p, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "cgtp_forces": (_i, [_i, _i, _p, _p, _p, _p, _p, _p]),
     "cgtp_radial_forward": (_i, [_p, _i, _p, _f, _p, _p, _p, _p]),
     "cgtp_radial_backward": (_i, [_p, _i, _p, _f, _p, _p, _p, _p, _p]),

@@ -274,6 +274,33 @@ class Plan:
              workspace.numel() * 4, _stream())
         return gx, gw, gm, gr
 
+    def conv_forward_shared(self, graph, x, w, out=None):
+        """Convolution with one weight row per edge for every path: w [E][mult]."""
+        _check(x, torch.float32, "x")
+        _check(w, torch.float32, "w")
+        if out is None:
+            out = torch.empty((graph.n_nodes, self.no, self.mult), dtype=torch.float32, device=x.device)
+        call("cgtp_conv_forward_shared_weights", self._h, graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr),
+             _ptr(graph.col), _ptr(graph.edge_vec), _ptr(x), _ptr(w), _ptr(out), _stream())
+        return out
+
+    def conv_backward_shared(self, graph, x, w, grad_out, want_x=True, want_w=True, want_r=True, workspace=None):
+        """Adjoint of conv_forward_shared: (grad_x, grad_w [E][mult], grad_edge_vec)."""
+        for t, nm in ((x, "x"), (w, "w"), (grad_out, "grad_out")):
+            _check(t, torch.float32, nm)
+        dev, E = x.device, graph.n_edges
+        gx = torch.empty_like(x) if want_x else None
+        gw = torch.empty((E, self.mult), dtype=torch.float32, device=dev) if want_w else None
+        gr = torch.empty((E, 3), dtype=torch.float32, device=dev) if want_r else None
+        nb = self.conv_backward_workspace_bytes(E) if want_r else 0
+        if want_r and workspace is None:
+            workspace = torch.empty(max(nb // 4, 64), dtype=torch.float32, device=dev)
+        call("cgtp_conv_backward_shared_weights", self._h, graph.n_nodes, E, _ptr(graph.csc_ptr),
+             _ptr(graph.csc_edge), _ptr(graph.csc_dst), _ptr(graph.edge_vec), _ptr(x), _ptr(w), _ptr(grad_out),
+             _ptr(gx), _ptr(gw), _ptr(gr), _ptr(workspace if want_r else None),
+             workspace.numel() * 4 if (want_r and workspace is not None) else 0, _stream())
+        return gx, gw, gr
+
     # ------------------------------------------------------------ radial network
     def radial_forward(self, edge_vec, rc, W1, W2, out=None):
         _check(edge_vec, torch.float32, "edge_vec")

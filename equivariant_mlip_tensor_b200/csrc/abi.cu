@@ -602,6 +602,62 @@ cgtp_status cgtp_uvw_backward(cgtp_plan p, int n_nodes, int n_edges, const int* 
   return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
 }
 
+// ---- weights shared by every path (path stride 0) ----
+cgtp_status cgtp_conv_forward_shared_weights(cgtp_plan p, int n_nodes, int n_edges, const int* row_ptr,
+                                             const int* col, const float* edge_vec, const float* x, const float* w,
+                                             float* out, void* stream) {
+  if (p == nullptr || n_nodes < 0 || n_edges < 0 || row_ptr == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (n_nodes > 0 && (x == nullptr || out == nullptr)) return CGTP_ERR_INVALID_ARG;
+  if (n_edges > 0 && (col == nullptr || edge_vec == nullptr || w == nullptr)) return CGTP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(out)) return CGTP_ERR_INVALID_ARG;
+  if (n_nodes == 0) return CGTP_OK;
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  ConvFwdArgs a{n_nodes, row_ptr, col, edge_vec, x, w, out, p->mult};
+  cudaError_t e = cudaErrorNotSupported;
+#define CGTP_SFWD_ENTRY(A, B, C) \
+  if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_fwd_shared<A, B, C>(a, sms, (cudaStream_t)stream);
+  CGTP_CONFIGS(CGTP_SFWD_ENTRY)
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
+cgtp_status cgtp_conv_backward_shared_weights(cgtp_plan p, int n_nodes, int n_edges, const int* csc_ptr,
+                                              const int* csc_edge, const int* csc_dst, const float* edge_vec,
+                                              const float* x, const float* w, const float* grad_out, float* grad_x,
+                                              float* grad_w, float* grad_edge_vec, void* workspace,
+                                              size_t workspace_bytes, void* stream) {
+  if (p == nullptr || n_nodes < 0 || n_edges < 0 || csc_ptr == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (n_nodes > 0 && (x == nullptr || grad_out == nullptr)) return CGTP_ERR_INVALID_ARG;
+  if (n_edges > 0 && (csc_edge == nullptr || csc_dst == nullptr || edge_vec == nullptr || w == nullptr))
+    return CGTP_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(grad_out) || !aligned16(grad_x) || !aligned16(grad_w))
+    return CGTP_ERR_INVALID_ARG;
+  if (grad_edge_vec != nullptr && n_edges > 0) {
+    size_t need = 0;
+    cgtp_conv_backward_workspace_size(p, n_edges, &need);  // same chunks, same partials
+    if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
+      return CGTP_ERR_WORKSPACE;
+  }
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (n_nodes == 0) return CGTP_OK;
+  if (n_edges == 0) {
+    cudaError_t e = cudaSuccess;
+    if (grad_x) e = cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)n_nodes * (p->li + 1) * (p->li + 1) * p->mult, s);
+    return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+  }
+  ConvBwdArgs a{n_nodes, n_edges, csc_ptr, csc_edge, csc_dst, edge_vec, x, w, grad_out,
+                grad_x, grad_w, grad_edge_vec, (float*)workspace, p->mult};
+  cudaError_t e = cudaErrorNotSupported;
+#define CGTP_SBWD_ENTRY(A, B, C) \
+  if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_bwd_shared<A, B, C>(a, sms, s);
+  CGTP_CONFIGS(CGTP_SBWD_ENTRY)
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
 cgtp_status cgtp_forces(int n_nodes, int n_edges, const int* row_ptr, const int* csc_ptr, const int* csc_edge,
                         const float* grad_edge_vec, float* forces, void* stream) {
   if (n_nodes < 0 || n_edges < 0 || row_ptr == nullptr || csc_ptr == nullptr) return CGTP_ERR_INVALID_ARG;

@@ -15,6 +15,10 @@ cudaError_t launch_conv_paths(const ConvFwdArgs& a, int num_sms, cudaStream_t st
 template <int LI, int LS, int LO>
 void conv_path_order(int* order, int* count_l3);
 template <int LI, int LS, int LO>
+cudaError_t launch_conv_fwd_shared(const ConvFwdArgs& a, int num_sms, cudaStream_t stream);
+template <int LI, int LS, int LO>
+cudaError_t launch_conv_bwd_shared(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);
+template <int LI, int LS, int LO>
 cudaError_t launch_conv_bwd_paths(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);
 template <int LI, int LS, int LO>
 cudaError_t launch_conv_bwd(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);

@@ -260,6 +260,27 @@ cgtp_status cgtp_uvw_backward(cgtp_plan plan, int n_nodes, int n_edges, const in
                               size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Convolution with weights shared by every path (path stride 0,
+ * W_e[p][u] = w[e][u]; "Tensor Decomposition Networks ...", reply to reviewer
+ * oXft: one weight set for all paths), forward and backward.  w and grad_w
+ * are [n_edges][mult]; grad_w[e] is the sum over paths of the per-path weight
+ * gradients.  Everything else as cgtp_conv_forward / cgtp_conv_backward
+ * (grad_edge_vec needs cgtp_conv_backward_workspace_size bytes of workspace).
+ * One weight row per edge instead of n_paths: the weight stream shrinks by
+ * n_paths and the kernels become FP32-bound.
+ * ------------------------------------------------------------------------- */
+cgtp_status cgtp_conv_forward_shared_weights(cgtp_plan plan, int n_nodes, int n_edges,
+                                             const int* row_ptr, const int* col,
+                                             const float* edge_vec, const float* x, const float* w,
+                                             float* out, void* stream);
+cgtp_status cgtp_conv_backward_shared_weights(cgtp_plan plan, int n_nodes, int n_edges,
+                                              const int* csc_ptr, const int* csc_edge,
+                                              const int* csc_dst, const float* edge_vec,
+                                              const float* x, const float* w, const float* grad_out,
+                                              float* grad_x, float* grad_w, float* grad_edge_vec,
+                                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * Per-atom forces from edge-vector gradients, F = -dE/dpos with
  * r_e = pos_src - pos_dst:  F[n] = sum_{e: dst=n} g[e] - sum_{e: src=n} g[e].
  * Segmented sums over the CSR row and the CSC row of each node; no atomics.
