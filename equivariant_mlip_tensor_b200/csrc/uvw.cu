@@ -11,6 +11,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <map>
+#include <mutex>
+
 #include "launch.h"
 
 #if !defined(CGTP_NO_CUTLASS)
@@ -77,6 +80,59 @@ __global__ void uvw_unpack_kernel(PathOrder po, int mult, int mult_out, int rank
     const int uu = int(ku % mult), rank = int(ku / mult);
     grad_mix[((long long)po.order[rank0 + rank] * mult + uu) * mult_out + v] = s;
   }
+}
+
+// The GEMMs of the l3 blocks are independent (disjoint outputs): they run
+// concurrently, block l3 on lane l3 % kLanes of a fork from the caller's
+// stream (lane 0 is the caller's stream itself) and join back before the
+// call returns, so the caller sees ordinary stream order.  The side streams
+// and events are created once per device and thread-safely cached.
+constexpr int kLanes = 3;
+struct Lanes {
+  cudaStream_t side[kLanes - 1];
+  cudaEvent_t fork, join[kLanes - 1];
+};
+static cudaError_t lanes_for_device(Lanes** out) {
+  static std::mutex mu;
+  static std::map<int, Lanes> per_dev;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = per_dev.find(dev);
+  if (it == per_dev.end()) {
+    Lanes L{};
+    for (int k = 0; k < kLanes - 1 && e == cudaSuccess; ++k) {
+      e = cudaStreamCreateWithFlags(&L.side[k], cudaStreamNonBlocking);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L.join[k], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L.fork, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+    it = per_dev.emplace(dev, L).first;
+  }
+  *out = &it->second;
+  return cudaSuccess;
+}
+// fork: lanes 1.. wait for the caller's stream; join: the caller's stream waits for them
+static cudaError_t lanes_fork(Lanes* L, cudaStream_t s) {
+  cudaError_t e = cudaEventRecord(L->fork, s);
+  for (int k = 0; k < kLanes - 1 && e == cudaSuccess; ++k) e = cudaStreamWaitEvent(L->side[k], L->fork, 0);
+  return e;
+}
+static cudaError_t lanes_join(Lanes* L, cudaStream_t s) {
+  cudaError_t e = cudaSuccess;
+  for (int k = 0; k < kLanes - 1 && e == cudaSuccess; ++k) {
+    e = cudaEventRecord(L->join[k], L->side[k]);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, L->join[k], 0);
+  }
+  return e;
+}
+static cudaStream_t lane(Lanes* L, cudaStream_t s, int l3) { return l3 % kLanes == 0 ? s : L->side[l3 % kLanes - 1]; }
+// Host threads that enqueue on the shared lanes take turns (the fork and join
+// events are shared too).
+static std::mutex& lanes_use_mutex() {
+  static std::mutex mu;
+  return mu;
 }
 
 #if !defined(CGTP_NO_CUTLASS)
@@ -217,7 +273,7 @@ size_t uvw_gemm_workspace(int n_nodes, int lmax_out, const int* count_l3, int mu
         block_args(n_nodes, l3, lmax_out, count_l3[l3] * mult, mult_out, nullptr, nullptr, nullptr));
     w = b > w ? b : w;
   }
-  return (w + 255) & ~(size_t)255;
+  return kLanes * ((w + 255) & ~(size_t)255);  // one slice per lane
 #endif
 }
 
@@ -226,21 +282,31 @@ cudaError_t launch_uvw_gemm(int n_nodes, int lmax_out, const int* count_l3, int 
 #if defined(CGTP_NO_CUTLASS)
   return cudaErrorNotSupported;
 #else
+  std::lock_guard<std::mutex> turn(lanes_use_mutex());
+  Lanes* Ls = nullptr;
+  cudaError_t e = lanes_for_device(&Ls);
+  if (e == cudaSuccess) e = lanes_fork(Ls, stream);
+  if (e != cudaSuccess) return e;
+  const size_t slice = (ws_bytes / kLanes) & ~(size_t)255;
   size_t t_off = 0, p_off = 0;
-  for (int l3 = 0; l3 <= lmax_out; ++l3) {
+  for (int l3 = 0; l3 <= lmax_out && e == cudaSuccess; ++l3) {
     const int npk = count_l3[l3], n3 = 2 * l3 + 1, K = npk * mult;
     if (npk > 0) {
+      cudaStream_t st = lane(Ls, stream, l3);
+      void* w = (char*)ws + (size_t)(l3 % kLanes) * slice;
       Gemm g;
       auto args = block_args(n_nodes, l3, lmax_out, K, mult_out, t + t_off, packed + p_off, out);
-      if (g.can_implement(args) != cutlass::Status::kSuccess) return cudaErrorNotSupported;
-      if (Gemm::get_workspace_size(args) > ws_bytes) return cudaErrorInvalidValue;
-      if (g.initialize(args, ws, stream) != cutlass::Status::kSuccess) return cudaErrorLaunchFailure;
-      if (g.run(stream) != cutlass::Status::kSuccess) return cudaErrorLaunchFailure;
+      if (g.can_implement(args) != cutlass::Status::kSuccess) e = cudaErrorNotSupported;
+      else if (Gemm::get_workspace_size(args) > slice) e = cudaErrorInvalidValue;
+      else if (g.initialize(args, w, st) != cutlass::Status::kSuccess) e = cudaErrorLaunchFailure;
+      else if (g.run(st) != cutlass::Status::kSuccess) e = cudaErrorLaunchFailure;
     }
     t_off += (size_t)n_nodes * n3 * K;
     p_off += (size_t)n3 * K * mult_out;
   }
-  return cudaGetLastError();
+  const cudaError_t ej = lanes_join(Ls, stream);
+  if (e != cudaSuccess) return e;
+  return ej != cudaSuccess ? ej : cudaGetLastError();
 #endif
 }
 
@@ -278,7 +344,7 @@ size_t uvw_bwd_gemm_workspace(int n_nodes, int lmax_out, const int* count_l3, in
     w = a > w ? a : w;
     w = b > w ? b : w;
   }
-  return (w + 255) & ~(size_t)255;
+  return kLanes * ((w + 255) & ~(size_t)255);  // one slice per lane
 #endif
 }
 
@@ -288,21 +354,31 @@ cudaError_t launch_uvw_gt(int n_nodes, int lmax_out, const int* count_l3, int mu
 #if defined(CGTP_NO_CUTLASS)
   return cudaErrorNotSupported;
 #else
+  std::lock_guard<std::mutex> turn(lanes_use_mutex());
+  Lanes* Ls = nullptr;
+  cudaError_t e = lanes_for_device(&Ls);
+  if (e == cudaSuccess) e = lanes_fork(Ls, stream);
+  if (e != cudaSuccess) return e;
+  const size_t slice = (ws_bytes / kLanes) & ~(size_t)255;
   size_t t_off = 0, p_off = 0;
-  for (int l3 = 0; l3 <= lmax_out; ++l3) {
+  for (int l3 = 0; l3 <= lmax_out && e == cudaSuccess; ++l3) {
     const int npk = count_l3[l3], n3 = 2 * l3 + 1, K = npk * mult;
     if (npk > 0) {
+      cudaStream_t st = lane(Ls, stream, l3);
+      void* w = (char*)ws + (size_t)(l3 % kLanes) * slice;
       Gemm gm;
       auto args = block_args_gt(n_nodes, l3, lmax_out, K, mult_out, g, packed_t + p_off, gt + t_off);
-      if (gm.can_implement(args) != cutlass::Status::kSuccess) return cudaErrorNotSupported;
-      if (Gemm::get_workspace_size(args) > ws_bytes) return cudaErrorInvalidValue;
-      if (gm.initialize(args, ws, stream) != cutlass::Status::kSuccess) return cudaErrorLaunchFailure;
-      if (gm.run(stream) != cutlass::Status::kSuccess) return cudaErrorLaunchFailure;
+      if (gm.can_implement(args) != cutlass::Status::kSuccess) e = cudaErrorNotSupported;
+      else if (Gemm::get_workspace_size(args) > slice) e = cudaErrorInvalidValue;
+      else if (gm.initialize(args, w, st) != cutlass::Status::kSuccess) e = cudaErrorLaunchFailure;
+      else if (gm.run(st) != cutlass::Status::kSuccess) e = cudaErrorLaunchFailure;
     }
     t_off += (size_t)n_nodes * n3 * K;
     p_off += (size_t)n3 * K * mult_out;
   }
-  return cudaGetLastError();
+  const cudaError_t ej = lanes_join(Ls, stream);
+  if (e != cudaSuccess) return e;
+  return ej != cudaSuccess ? ej : cudaGetLastError();
 #endif
 }
 
@@ -316,26 +392,37 @@ cudaError_t launch_uvw_grad_mix(int n_nodes, int n_paths, int lmax_out, const in
 #else
   PathOrder po{};
   for (int k = 0; k < n_paths && k < kMaxPaths; ++k) po.order[k] = order[k];
+  std::lock_guard<std::mutex> turn(lanes_use_mutex());
+  Lanes* Ls = nullptr;
+  cudaError_t e = lanes_for_device(&Ls);
+  if (e == cudaSuccess) e = lanes_fork(Ls, stream);
+  if (e != cudaSuccess) return e;
+  const size_t slice = (ws_bytes / kLanes) & ~(size_t)255;
   size_t t_off = 0, p_off = 0;
   int rank0 = 0;
-  for (int l3 = 0; l3 <= lmax_out; ++l3) {
+  for (int l3 = 0; l3 <= lmax_out && e == cudaSuccess; ++l3) {
     const int npk = count_l3[l3], n3 = 2 * l3 + 1, K = npk * mult;
     if (npk > 0) {
+      cudaStream_t st = lane(Ls, stream, l3);
+      void* w = (char*)ws + (size_t)(l3 % kLanes) * slice;
       GemmT gm;
       auto args = block_args_mix(n_nodes, l3, lmax_out, K, mult_out, t + t_off, g, part + p_off);
-      if (gm.can_implement(args) != cutlass::Status::kSuccess) return cudaErrorNotSupported;
-      if (GemmT::get_workspace_size(args) > ws_bytes) return cudaErrorInvalidValue;
-      if (gm.initialize(args, ws, stream) != cutlass::Status::kSuccess) return cudaErrorLaunchFailure;
-      if (gm.run(stream) != cutlass::Status::kSuccess) return cudaErrorLaunchFailure;
-      uvw_unpack_kernel<<<256, 256, 0, stream>>>(po, mult, mult_out, rank0, npk, n3, part + p_off, grad_mix);
-      const cudaError_t e = cudaGetLastError();
-      if (e != cudaSuccess) return e;
+      if (gm.can_implement(args) != cutlass::Status::kSuccess) e = cudaErrorNotSupported;
+      else if (GemmT::get_workspace_size(args) > slice) e = cudaErrorInvalidValue;
+      else if (gm.initialize(args, w, st) != cutlass::Status::kSuccess) e = cudaErrorLaunchFailure;
+      else if (gm.run(st) != cutlass::Status::kSuccess) e = cudaErrorLaunchFailure;
+      if (e == cudaSuccess) {
+        uvw_unpack_kernel<<<256, 256, 0, st>>>(po, mult, mult_out, rank0, npk, n3, part + p_off, grad_mix);
+        e = cudaGetLastError();
+      }
     }
     t_off += (size_t)n_nodes * n3 * K;
     p_off += (size_t)n3 * K * mult_out;
     rank0 += npk;
   }
-  return cudaGetLastError();
+  const cudaError_t ej = lanes_join(Ls, stream);
+  if (e != cudaSuccess) return e;
+  return ej != cudaSuccess ? ej : cudaGetLastError();
 #endif
 }
 
