@@ -137,7 +137,14 @@ static std::mutex& lanes_use_mutex() {
 
 #if !defined(CGTP_NO_CUTLASS)
 using namespace cute;
-using TileShape = Shape<_128, _128, _32>;
+#ifndef CGTP_UVW_TILE_N
+#define CGTP_UVW_TILE_N 128  // output-channel tile of the mixing GEMMs
+#endif
+#ifndef CGTP_UVW_TILE_N_MIX
+#define CGTP_UVW_TILE_N_MIX 64  // mixing-gradient GEMM: few, long tiles, so narrower ones
+#endif
+using TileShape = Shape<_128, Int<CGTP_UVW_TILE_N>, _32>;
+using TileShapeT = Shape<_128, Int<CGTP_UVW_TILE_N_MIX>, _32>;
 using ClusterShape = Shape<_1, _1, _1>;
 constexpr int kAlign = 4;  // floats: 16-byte rows and strides
 using Layout = cutlass::layout::RowMajor;
@@ -159,10 +166,13 @@ using Gemm = cutlass::gemm::device::GemmUniversalAdapter<Kernel>;
 // stride NO mult_out, batch stride mult_out).
 // D = A^T B with A stored K-major (column-major A): the mixing-matrix gradient.
 using LayoutCol = cutlass::layout::ColumnMajor;
-using EpilogueT = Epilogue;
+using EpilogueT = typename cutlass::epilogue::collective::CollectiveBuilder<
+    cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, TileShapeT, ClusterShape,
+    cutlass::epilogue::collective::EpilogueTileAuto, float, float, float, Layout, kAlign, float, Layout, kAlign,
+    cutlass::epilogue::collective::EpilogueScheduleAuto>::CollectiveOp;
 using MainloopT = typename cutlass::gemm::collective::CollectiveBuilder<
     cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, float, LayoutCol, kAlign, float, Layout, kAlign, float,
-    TileShape, ClusterShape,
+    TileShapeT, ClusterShape,
     cutlass::gemm::collective::StageCountAutoCarveout<static_cast<int>(sizeof(typename EpilogueT::SharedStorage))>,
     cutlass::gemm::KernelTmaWarpSpecialized1SmFastFP32Sm100>::CollectiveOp;
 using KernelT = cutlass::gemm::kernel::GemmUniversal<Shape<int, int, int, int>, MainloopT, EpilogueT>;
