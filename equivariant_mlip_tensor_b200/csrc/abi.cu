@@ -679,7 +679,8 @@ cgtp_status cgtp_radial_forward(cgtp_plan p, int n_edges, const float* edge_vec,
   int sms = 0;
   cgtp_status st = ensure_device(&sms);
   if (st != CGTP_OK) return st;
-  cudaError_t e = launch_radial_fwd(n_edges, p->n_paths * p->mult, edge_vec, rc, W1, W2, w, (cudaStream_t)stream);
+  cudaError_t e =
+      launch_radial_fwd(n_edges, p->n_paths * p->mult, edge_vec, rc, W1, W2, w, sms, (cudaStream_t)stream);
   return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
 }
 
@@ -693,7 +694,7 @@ cgtp_status cgtp_radial_backward(cgtp_plan p, int n_edges, const float* edge_vec
   int sms = 0;
   cgtp_status st = ensure_device(&sms);
   if (st != CGTP_OK) return st;
-  cudaError_t e = launch_radial_bwd(n_edges, p->n_paths * p->mult, edge_vec, rc, W1, W2, grad_w, grad_edge_vec,
+  cudaError_t e = launch_radial_bwd(n_edges, p->n_paths * p->mult, edge_vec, rc, W1, W2, grad_w, grad_edge_vec, sms,
                                     (cudaStream_t)stream);
   return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
 }

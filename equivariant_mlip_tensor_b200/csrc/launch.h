@@ -38,9 +38,9 @@ cudaError_t launch_csr_transpose(int n, int n_edges, const int* row_ptr, const i
 cudaError_t launch_graph_check(int n, int n_edges, const int* row_ptr, const int* col, const float* edge_vec,
                                int* flags, int num_sms, cudaStream_t stream);
 cudaError_t launch_radial_fwd(int n_edges, int N, const float* ev, float rc, const float* W1, const float* W2,
-                              float* w, cudaStream_t stream);
+                              float* w, int num_sms, cudaStream_t stream);
 cudaError_t launch_radial_bwd(int n_edges, int N, const float* ev, float rc, const float* W1, const float* W2,
-                              const float* gw, float* gev, cudaStream_t stream);
+                              const float* gw, float* gev, int num_sms, cudaStream_t stream);
 cudaError_t launch_forces(int n, const int* row_ptr, const int* csc_ptr, const int* csc_edge, const float* g,
                           float* F, int num_sms, cudaStream_t stream);
 cudaError_t launch_sh(int lmax_sh, int n_edges, const float* ev, float* Y, float* dY, int num_sms,
