@@ -109,12 +109,12 @@ class ClockSampler:
 # family at the molecules workload (97 480 edges), from an ncu capture
 # (profiles/conv_molecules_traffic.md), with a hash of the kernel sources it
 # was taken on: traffic is reported only while the sources are unchanged.
-KERNEL_HEADERS = ("common.cuh", "conv_common.cuh", "sh.cuh", "structure.h")
+KERNEL_HEADERS = ("common.cuh", "conv_common.cuh", "sh.cuh", "structure.h", "vec2.cuh")
 MEASURED_TRAFFIC = {
-    "conv_fwd": {"bytes": 1022236160, "n_edges": 97480, "sources": ("conv_fwd.cu",) + KERNEL_HEADERS,
-                 "sha256_16": "e371af1a1d48edcc"},
-    "conv_bwd": {"bytes": 2062439424, "n_edges": 97480, "sources": ("conv_bwd.cu",) + KERNEL_HEADERS,
-                 "sha256_16": "64f00dd54890ea3c"},
+    "conv_fwd": {"bytes": 1022903552, "n_edges": 97480, "sources": ("conv_fwd.cu",) + KERNEL_HEADERS,
+                 "sha256_16": "41535c1d242146e5"},
+    "conv_bwd": {"bytes": 2065300480, "n_edges": 97480, "sources": ("conv_bwd.cu",) + KERNEL_HEADERS,
+                 "sha256_16": "71fa7efaae53e6a0"},
 }
 
 

@@ -23,6 +23,7 @@ CGTP_DEFINE_CONSTANT_TABLES()
 }  // namespace cgtp
 
 #include "conv_common.cuh"
+#include "vec2.cuh"
 #include "sh.cuh"
 
 namespace cgtp {
@@ -101,9 +102,7 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
     float xw[2 * l1 + 1][VEC];  // W x, for the grad_Y channel sums
     if constexpr (NEED_GY) {
 #pragma unroll
-      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1)
-#pragma unroll
-        for (int c = 0; c < VEC; ++c) xw[m1][c] = wv[c] * xr[m1][c];
+      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) vmul<VEC>(xw[m1], wv, xr[m1]);
     }
     static_for<0, (tc + 3) / 4>([&](auto Qc) {
       constexpr int q = decltype(Qc)::value;
@@ -114,12 +113,9 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
         if constexpr (k < tc) {
           constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
           const float tv = tv4[decltype(Rc)::value];
-#pragma unroll
-          for (int c = 0; c < VEC; ++c) h[m1 + l1][c] = fmaf(tv, gv[m3 + l3][c], h[m1 + l1][c]);
+          axpy<VEC>(h[m1 + l1], tv, gv[m3 + l3]);
           if constexpr (NEED_GY) {
-            float av = 0.f;
-#pragma unroll
-            for (int c = 0; c < VEC; ++c) av = fmaf(xw[m1 + l1][c], gv[m3 + l3][c], av);
+            const float av = vdot<VEC>(xw[m1 + l1], gv[m3 + l3]);
             static_for<0, 2 * l2 + 1>([&](auto M2c) {
               constexpr int m2 = decltype(M2c)::value - l2;
               if constexpr (cg_allowed(l1, l2, l3, m1, m2, m3)) {
@@ -134,12 +130,10 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
 #pragma unroll
     for (int c = 0; c < VEC; ++c) gw[c] = 0.f;
 #pragma unroll
-    for (int m1 = 0; m1 < 2 * l1 + 1; ++m1)
-#pragma unroll
-      for (int c = 0; c < VEC; ++c) {
-        gx[m1][c] = fmaf(wv[c], h[m1][c], gx[m1][c]);
-        gw[c] = fmaf(xr[m1][c], h[m1][c], gw[c]);
-      }
+    for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) {
+      vfma<VEC>(gx[m1], wv, h[m1]);
+      vfma<VEC>(gw, xr[m1], h[m1]);
+    }
     if (gwrow != nullptr) {
       if (acc) {
         float prev[VEC];

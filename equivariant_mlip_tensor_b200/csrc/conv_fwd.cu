@@ -27,6 +27,7 @@ CGTP_DEFINE_CONSTANT_TABLES()
 }  // namespace cgtp
 
 #include "conv_common.cuh"
+#include "vec2.cuh"
 #include "sh.cuh"
 
 namespace cgtp {
@@ -115,22 +116,17 @@ __device__ __forceinline__ void fwd_edge(const float* __restrict__ T, const floa
           if constexpr (k < tc) {
             constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
             constexpr int rx = l1 * l1 + l1 + m1 - GR::D.rlo;
-#pragma unroll
-            for (int c = 0; c < kFwdVec; ++c) t[m3 + l3][c] = fmaf(tv4[decltype(Rc)::value], xr[rx][c], t[m3 + l3][c]);
+            axpy<kFwdVec>(t[m3 + l3], tv4[decltype(Rc)::value], xr[rx]);
           }
         });
       });
 #pragma unroll
-      for (int m3 = 0; m3 < 2 * l3 + 1; ++m3)
-#pragma unroll
-        for (int c = 0; c < kFwdVec; ++c) acc[o3 + m3][c] = fmaf(wv[c], t[m3][c], acc[o3 + m3][c]);
+      for (int m3 = 0; m3 < 2 * l3 + 1; ++m3) vfma<kFwdVec>(acc[o3 + m3], wv, t[m3]);
     } else {
       // xw[m1] = W x[m1], then out[m3] += sum_m1 T xw[m1]
       float xw[2 * l1 + 1][kFwdVec];
 #pragma unroll
-      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1)
-#pragma unroll
-        for (int c = 0; c < kFwdVec; ++c) xw[m1][c] = wv[c] * xr[l1 * l1 + m1 - GR::D.rlo][c];
+      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) vmul<kFwdVec>(xw[m1], wv, xr[l1 * l1 + m1 - GR::D.rlo]);
       static_for<0, (tc + 3) / 4>([&](auto Qc) {
         constexpr int q = decltype(Qc)::value;
         const float4 v4 = *reinterpret_cast<const float4*>(T + tb + 4 * q);
@@ -139,9 +135,7 @@ __device__ __forceinline__ void fwd_edge(const float* __restrict__ T, const floa
           constexpr int k = 4 * q + decltype(Rc)::value;
           if constexpr (k < tc) {
             constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
-#pragma unroll
-            for (int c = 0; c < kFwdVec; ++c)
-              acc[o3 + m3 + l3][c] = fmaf(tv4[decltype(Rc)::value], xw[m1 + l1][c], acc[o3 + m3 + l3][c]);
+            axpy<kFwdVec>(acc[o3 + m3 + l3], tv4[decltype(Rc)::value], xw[m1 + l1]);
           }
         });
       });
