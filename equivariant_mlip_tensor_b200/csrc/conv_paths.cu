@@ -12,6 +12,7 @@ CGTP_DEFINE_CONSTANT_TABLES()
 }  // namespace cgtp
 
 #include "conv_common.cuh"
+#include "vec2.cuh"
 #include "paths_common.cuh"
 #include "sh.cuh"
 
@@ -108,22 +109,17 @@ __device__ __forceinline__ void fwd_edge(const float* __restrict__ T, const floa
           if constexpr (k < tc) {
             constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
             constexpr int rx = l1 * l1 + l1 + m1 - GR::D.rlo;
-#pragma unroll
-            for (int c = 0; c < kFwdVec; ++c) t[m3 + l3][c] = fmaf(tv4[decltype(Rc)::value], xr[rx][c], t[m3 + l3][c]);
+            axpy<kFwdVec>(t[m3 + l3], tv4[decltype(Rc)::value], xr[rx]);
           }
         });
       });
 #pragma unroll
-      for (int m3 = 0; m3 < 2 * l3 + 1; ++m3)
-#pragma unroll
-        for (int c = 0; c < kFwdVec; ++c) acc[o3 + m3][c] = fmaf(wv[c], t[m3][c], acc[o3 + m3][c]);
+      for (int m3 = 0; m3 < 2 * l3 + 1; ++m3) vfma<kFwdVec>(acc[o3 + m3], wv, t[m3]);
     } else {
       // xw[m1] = W x[m1], then out[m3] += sum_m1 T xw[m1]
       float xw[2 * l1 + 1][kFwdVec];
 #pragma unroll
-      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1)
-#pragma unroll
-        for (int c = 0; c < kFwdVec; ++c) xw[m1][c] = wv[c] * xr[l1 * l1 + m1 - GR::D.rlo][c];
+      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) vmul<kFwdVec>(xw[m1], wv, xr[l1 * l1 + m1 - GR::D.rlo]);
       static_for<0, (tc + 3) / 4>([&](auto Qc) {
         constexpr int q = decltype(Qc)::value;
         const float4 v4 = *reinterpret_cast<const float4*>(T + tb + 4 * q);
@@ -132,9 +128,7 @@ __device__ __forceinline__ void fwd_edge(const float* __restrict__ T, const floa
           constexpr int k = 4 * q + decltype(Rc)::value;
           if constexpr (k < tc) {
             constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
-#pragma unroll
-            for (int c = 0; c < kFwdVec; ++c)
-              acc[o3 + m3 + l3][c] = fmaf(tv4[decltype(Rc)::value], xw[m1 + l1][c], acc[o3 + m3 + l3][c]);
+            axpy<kFwdVec>(acc[o3 + m3 + l3], tv4[decltype(Rc)::value], xw[m1 + l1]);
           }
         });
       });
@@ -494,9 +488,7 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
     float xw[2 * l1 + 1][VEC];  // W x, for the grad_Y channel sums
     if constexpr (NEED_GY) {
 #pragma unroll
-      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1)
-#pragma unroll
-        for (int c = 0; c < VEC; ++c) xw[m1][c] = wv[c] * xr[m1][c];
+      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) vmul<VEC>(xw[m1], wv, xr[m1]);
     }
     static_for<0, (tc + 3) / 4>([&](auto Qc) {
       constexpr int q = decltype(Qc)::value;
@@ -507,12 +499,9 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
         if constexpr (k < tc) {
           constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
           const float tv = tv4[decltype(Rc)::value];
-#pragma unroll
-          for (int c = 0; c < VEC; ++c) h[m1 + l1][c] = fmaf(tv, gv[m3 + l3][c], h[m1 + l1][c]);
+          axpy<VEC>(h[m1 + l1], tv, gv[m3 + l3]);
           if constexpr (NEED_GY) {
-            float av = 0.f;
-#pragma unroll
-            for (int c = 0; c < VEC; ++c) av = fmaf(xw[m1 + l1][c], gv[m3 + l3][c], av);
+            const float av = vdot<VEC>(xw[m1 + l1], gv[m3 + l3]);
             static_for<0, 2 * l2 + 1>([&](auto M2c) {
               constexpr int m2 = decltype(M2c)::value - l2;
               if constexpr (cg_allowed(l1, l2, l3, m1, m2, m3)) {
@@ -527,12 +516,10 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
 #pragma unroll
     for (int c = 0; c < VEC; ++c) gw[c] = 0.f;
 #pragma unroll
-    for (int m1 = 0; m1 < 2 * l1 + 1; ++m1)
-#pragma unroll
-      for (int c = 0; c < VEC; ++c) {
-        gx[m1][c] = fmaf(wv[c], h[m1][c], gx[m1][c]);
-        gw[c] = fmaf(xr[m1][c], h[m1][c], gw[c]);
-      }
+    for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) {
+      vfma<VEC>(gx[m1], wv, h[m1]);
+      vfma<VEC>(gw, xr[m1], h[m1]);
+    }
     if (gwrow != nullptr) {
       if (acc) {
         float prev[VEC];
