@@ -30,6 +30,10 @@ What it computes, and the passage each part follows:
 * ``tp``      -- the edge-free channelwise tensor product of batched pairs
                  ("Tensor Decomposition Networks ...", reply to reviewer S6y1,
                  timing at batch 1000 and multiplicity 128) and its adjoints.
+* ``cp``      -- the CP-decomposed surrogate z = A (B^T x (*) C^T y) of that
+                 product, its input and factor gradients, and the fit of the
+                 factors by least squares on standard-normal batches (same
+                 pages, reply to reviewer S6y1 on the backward and on Figure 3).
 
 Every function is pinned by tests under ``tests/`` against closed forms,
 library routines (sympy's Clebsch-Gordan values, scipy's spherical
