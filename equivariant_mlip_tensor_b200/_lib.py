@@ -48,6 +48,9 @@ SIGNATURES = {
     "cgtp_tp_backward_workspace_size": (_i, [_p, _i, ctypes.POINTER(_sz)]),
     "cgtp_tp_backward": (_i, [_p, _i, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "cgtp_tp_backward_noalloc": (_i, [_p, _i, _p, _p, _p, _p, _p, _p, _p, _p]),
+    "cgtp_cp_forward": (_i, [_p, _i, _i, _p, _p, _p, _p, _p, _p, _p]),
+    "cgtp_cp_backward_workspace_size": (_i, [_p, _i, _i, ctypes.POINTER(_sz)]),
+    "cgtp_cp_backward": (_i, [_p, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
 }
 
 STATUS = {0: "CGTP_OK", 1: "CGTP_ERR_INVALID_ARG", 2: "CGTP_ERR_UNSUPPORTED", 3: "CGTP_ERR_BAD_GRAPH",

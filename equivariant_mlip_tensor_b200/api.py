@@ -347,3 +347,36 @@ class Plan:
         call("cgtp_tp_backward", self._h, B, _ptr(x), _ptr(y), _ptr(w), _ptr(grad_z), _ptr(gx), _ptr(gy),
              _ptr(gw), _ptr(ws), nb, _stream())
         return gx, gy, gw
+
+    # ------------------------------------------------------------ CP-decomposed product
+    def cp_forward(self, A, B, C, x, y, out=None):
+        """z = A (B^T x (*) C^T y) per (pair, channel); A [d3][R], B [d1][R], C [d2][R]."""
+        for t, nm in ((A, "A"), (B, "B"), (C, "C"), (x, "x"), (y, "y")):
+            _check(t, torch.float32, nm)
+        R, batch = A.shape[1], x.shape[0]
+        if out is None:
+            out = torch.empty((batch, (self.lmax_out + 1) ** 2, self.mult), dtype=torch.float32, device=x.device)
+        call("cgtp_cp_forward", self._h, R, batch, _ptr(A), _ptr(B), _ptr(C), _ptr(x), _ptr(y), _ptr(out),
+             _stream())
+        return out
+
+    def cp_backward_workspace_bytes(self, rank, batch):
+        b = ctypes.c_size_t()
+        call("cgtp_cp_backward_workspace_size", self._h, rank, batch, ctypes.byref(b))
+        return b.value
+
+    def cp_backward(self, A, B, C, x, y, grad_z, want_x=True, want_y=True, want_factors=True):
+        """(grad_x, grad_y, grad_A, grad_B, grad_C); the unrequested ones are None."""
+        for t, nm in ((A, "A"), (B, "B"), (C, "C"), (x, "x"), (y, "y"), (grad_z, "grad_z")):
+            _check(t, torch.float32, nm)
+        R, batch = A.shape[1], x.shape[0]
+        gx = torch.empty_like(x) if want_x else None
+        gy = torch.empty_like(y) if want_y else None
+        gA, gB, gC = (torch.empty_like(v) if want_factors else None for v in (A, B, C))
+        ws, nb = None, 0
+        if want_factors:
+            nb = self.cp_backward_workspace_bytes(R, batch)
+            ws = torch.empty(max(nb // 4, 64), dtype=torch.float32, device=x.device)
+        call("cgtp_cp_backward", self._h, R, batch, _ptr(A), _ptr(B), _ptr(C), _ptr(x), _ptr(y), _ptr(grad_z),
+             _ptr(gx), _ptr(gy), _ptr(gA), _ptr(gB), _ptr(gC), _ptr(ws), nb, _stream())
+        return gx, gy, gA, gB, gC

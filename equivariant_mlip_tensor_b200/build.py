@@ -23,7 +23,7 @@ INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
                      "-Xcompiler", "-fPIC", "-I", CSRC, "-I", INCLUDE]
-PER_SHAPE = ["conv_fwd.cu", "conv_bwd.cu", "conv_paths.cu", "conv_shared.cu", "tp.cu"]
+PER_SHAPE = ["conv_fwd.cu", "conv_bwd.cu", "conv_paths.cu", "conv_shared.cu", "tp.cu", "cp.cu"]
 SHAPE_FREE = ["graph.cu", "radial.cu", "misc.cu", "abi.cu", "cg_table.cpp", "uvw.cu"]
 
 

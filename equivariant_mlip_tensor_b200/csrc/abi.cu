@@ -742,6 +742,74 @@ cgtp_status cgtp_tp_backward(cgtp_plan p, int batch, const float* x, const float
   return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
 }
 
+static size_t cp_device_smem_limit() {
+  int dev = 0, v = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
+  return (size_t)v;
+}
+
+static size_t cp_smem_for(cgtp_plan p, int rank, bool factor_grads) {
+  size_t b = 0;
+#define CGTP_CPS_ENTRY(A, B, C) \
+  if (p->li == A && p->ls == B && p->lo == C) b = cp_smem_bytes<A, B, C>(rank, factor_grads);
+  CGTP_CONFIGS(CGTP_CPS_ENTRY)
+  return b;
+}
+
+cgtp_status cgtp_cp_forward(cgtp_plan p, int rank, int batch, const float* A, const float* B, const float* C,
+                            const float* x, const float* y, float* z, void* stream) {
+  if (p == nullptr || rank < 1 || batch < 0) return CGTP_ERR_INVALID_ARG;
+  if (A == nullptr || B == nullptr || C == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (batch > 0 && (x == nullptr || y == nullptr || z == nullptr)) return CGTP_ERR_INVALID_ARG;
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  const size_t need = cp_smem_for(p, rank, false);
+  if (need == 0 || need > cp_device_smem_limit()) return CGTP_ERR_UNSUPPORTED;
+  CPArgs a{batch, p->mult, rank, A, B, C, x, y, nullptr, z, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr};
+  cudaError_t e = cudaErrorNotSupported;
+#define CGTP_CPF_ENTRY(LA, LB, LC) \
+  if (p->li == LA && p->ls == LB && p->lo == LC) e = launch_cp_fwd<LA, LB, LC>(a, (cudaStream_t)stream);
+  CGTP_CONFIGS(CGTP_CPF_ENTRY)
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
+cgtp_status cgtp_cp_backward_workspace_size(cgtp_plan p, int rank, int batch, size_t* bytes) {
+  if (p == nullptr || rank < 1 || batch < 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
+  const int d1 = (p->li + 1) * (p->li + 1), d2 = (p->ls + 1) * (p->ls + 1), d3 = (p->lo + 1) * (p->lo + 1);
+  const size_t b = sizeof(float) * (size_t)cp_bwd_blocks(batch, p->mult) * (size_t)(d1 + d2 + d3) * (size_t)rank;
+  *bytes = (b + 255) & ~(size_t)255;
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_cp_backward(cgtp_plan p, int rank, int batch, const float* A, const float* B, const float* C,
+                             const float* x, const float* y, const float* grad_z, float* grad_x, float* grad_y,
+                             float* grad_A, float* grad_B, float* grad_C, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  if (p == nullptr || rank < 1 || batch < 0) return CGTP_ERR_INVALID_ARG;
+  if (A == nullptr || B == nullptr || C == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (batch > 0 && (x == nullptr || y == nullptr || grad_z == nullptr)) return CGTP_ERR_INVALID_ARG;
+  const bool gf = grad_A != nullptr || grad_B != nullptr || grad_C != nullptr;
+  if (gf && batch > 0) {
+    size_t need = 0;
+    cgtp_cp_backward_workspace_size(p, rank, batch, &need);
+    if (workspace == nullptr || workspace_bytes < need) return CGTP_ERR_WORKSPACE;
+  }
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  const size_t need = cp_smem_for(p, rank, gf);
+  if (need == 0 || need > cp_device_smem_limit()) return CGTP_ERR_UNSUPPORTED;
+  CPArgs a{batch, p->mult, rank, A, B, C, x, y, grad_z, nullptr, grad_x, grad_y, grad_A, grad_B, grad_C,
+           gf ? (float*)workspace : nullptr};
+  cudaError_t e = cudaErrorNotSupported;
+#define CGTP_CPB_ENTRY(LA, LB, LC) \
+  if (p->li == LA && p->ls == LB && p->lo == LC) e = launch_cp_bwd<LA, LB, LC>(a, (cudaStream_t)stream);
+  CGTP_CONFIGS(CGTP_CPB_ENTRY)
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------

@@ -8,6 +8,25 @@
 
 namespace cgtp {
 
+// Arguments of the CP-decomposed tensor product (cp.cu): factors A [d3][R],
+// B [d1][R], C [d2][R]; features [batch][d][mult]; partial: the backward's
+// per-block factor-gradient partials (cp_bwd_blocks x (d1 + d2 + d3) x R floats).
+struct CPArgs {
+  int batch, mult, rank;
+  const float *A, *B, *C, *x, *y, *grad_z;
+  float *z, *grad_x, *grad_y, *grad_A, *grad_B, *grad_C, *partial;
+};
+constexpr int kCpItemsPerPartial = 64;  // (pair, channel) items per factor-gradient partial
+inline long long cp_bwd_blocks(int batch, int mult) {
+  return ((long long)batch * mult + kCpItemsPerPartial - 1) / kCpItemsPerPartial;
+}
+template <int LI, int LS, int LO>
+size_t cp_smem_bytes(int rank, bool factor_grads);
+template <int LI, int LS, int LO>
+cudaError_t launch_cp_fwd(const CPArgs& a, cudaStream_t stream);
+template <int LI, int LS, int LO>
+cudaError_t launch_cp_bwd(const CPArgs& a, cudaStream_t stream);
+
 template <int LI, int LS, int LO>
 cudaError_t launch_conv_fwd(const ConvFwdArgs& a, int num_sms, cudaStream_t stream);
 template <int LI, int LS, int LO>

@@ -347,6 +347,46 @@ cgtp_status cgtp_tp_backward_noalloc(cgtp_plan plan, int batch, const float* x, 
                                      const float* w, const float* grad_z, float* grad_x, float* grad_y,
                                      float* grad_w, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * CP-decomposed tensor product ("Tensor Decomposition Networks for
+ * Accelerating Machine Learning Force Field Computations", reply to reviewer
+ * S6y1 on the backward's complexity): the low-rank surrogate
+ *   z = A (B^T x (*) C^T y)                  ((*) = elementwise product)
+ * of the plan's CG product, applied channelwise with factors shared by every
+ * pair and channel:
+ *   z[b][k][u] = sum_r A[k][r] (sum_i B[i][r] x[b][i][u]) (sum_j C[j][r] y[b][j][u]).
+ * d1 = (lmax_in+1)^2, d2 = (lmax_sh+1)^2, d3 = (lmax_out+1)^2 from the plan;
+ * mult from the plan.  A: [d3][rank], B: [d1][rank], C: [d2][rank] (row-major,
+ * device, caller-owned); x: [batch][d1][mult], y: [batch][d2][mult],
+ * z: [batch][d3][mult] (overwritten).  The factors are inputs: they are fitted
+ * offline (the reply on Figure 3 fits them once, before training, by least
+ * squares on batches of standard-normal inputs).
+ * Errors: CGTP_ERR_INVALID_ARG for a null plan, rank < 1, batch < 0 or a null
+ * pointer that the call needs; CGTP_ERR_UNSUPPORTED when the factors (and, in
+ * the backward with factor gradients, the per-block staging) exceed the
+ * device's shared memory per block (rank <= 256 fits every compiled shape in
+ * the forward).  Nothing is launched on error.
+ * ------------------------------------------------------------------------- */
+cgtp_status cgtp_cp_forward(cgtp_plan plan, int rank, int batch, const float* A, const float* B,
+                            const float* C, const float* x, const float* y, float* z, void* stream);
+
+/* Workspace of cgtp_cp_backward when a factor gradient is requested:
+ * ceil(batch * mult / 64) * (d1 + d2 + d3) * rank floats, rounded up to 256 bytes. */
+cgtp_status cgtp_cp_backward_workspace_size(cgtp_plan plan, int rank, int batch, size_t* bytes);
+
+/* Gradients for grad_z [batch][d3][mult]:
+ *   grad_x = (g_z^T A (*) C^T y) B^T,  grad_y = (g_z^T A (*) B^T x) C^T   (per pair and channel),
+ *   grad_A = sum g_z (s (*) t)^T, grad_B = sum x (q (*) t)^T, grad_C = sum y (q (*) s)^T
+ * (sums over pairs and channels; s = B^T x, t = C^T y, q = A^T g_z).  Every
+ * output is nullable and overwritten; the factor gradients need the workspace
+ * of cgtp_cp_backward_workspace_size (CGTP_ERR_WORKSPACE otherwise) and are
+ * reduced in a fixed order (bit-reproducible).  An empty batch gives zero
+ * factor gradients. */
+cgtp_status cgtp_cp_backward(cgtp_plan plan, int rank, int batch, const float* A, const float* B,
+                             const float* C, const float* x, const float* y, const float* grad_z,
+                             float* grad_x, float* grad_y, float* grad_A, float* grad_B, float* grad_C,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
