@@ -359,6 +359,27 @@ def config_table(torch, api, dev, hbm, reps=20):
     rows.append({"workload": "tp_batch (edge-free tensor product)", "L": list(L), "mult": u, "batch": B,
                  "fwd_ms": t_f, "bwd_ms": t_b, "pairs_per_s_fwd_bwd": B / ((t_f + t_b) / 1e3),
                  "hbm_frac": {"fwd": b_f / (t_f / 1e3) / 1e9 / hbm, "bwd": b_b / (t_b / 1e3) / 1e9 / hbm}})
+    # CP-decomposed product of the same pairs, rank 40 (factors N(0,1)/sqrt(R): the
+    # kernels' cost does not depend on their values)
+    R = 40
+    gen = torch.Generator(device="cpu").manual_seed(7)
+    fA, fB, fC = (torch.randn(sh, generator=gen).div_(R ** 0.5).to(dev) for sh in ((no, R), (ni, R), (ns, R)))
+    zc = torch.empty_like(gz)
+    t_cf = _time_ms(torch, lambda: plan.cp_forward(fA, fB, fC, xs, ys, out=zc), reps)
+    t_cb = _time_ms(torch, lambda: plan.cp_backward(fA, fB, fC, xs, ys, gz, want_factors=False), reps)
+    t_cg = _time_ms(torch, lambda: plan.cp_backward(fA, fB, fC, xs, ys, gz), reps)
+    items = B * u
+    fl_f = items * (2 * R * (ni + ns + no) + R)
+    fl_b = items * (2 * R * (ni + ns + no) + 2 * R * (ni + ns) + 3 * R)
+    fl_g = fl_b + items * 2 * R * (ni + ns + no)
+    rows.append({"workload": "cp_batch (CP-decomposed product of the tp_batch pairs, rank 40)", "L": list(L),
+                 "mult": u, "batch": B, "rank": R, "fwd_ms": t_cf, "bwd_ms": t_cb, "bwd_with_factor_grads_ms": t_cg,
+                 "pairs_per_s_fwd_bwd": B / ((t_cf + t_cb) / 1e3),
+                 "hbm_frac": {"fwd": 4 * items * (ni + ns + no) / (t_cf / 1e3) / 1e9 / hbm,
+                              "bwd": 4 * items * (2 * ni + 2 * ns + no) / (t_cb / 1e3) / 1e9 / hbm},
+                 "fp32_frac": {"fwd": fl_f / (t_cf / 1e3) / 1e12 / FP32_PEAK_TFLOPS,
+                               "bwd": fl_b / (t_cb / 1e3) / 1e12 / FP32_PEAK_TFLOPS,
+                               "bwd_with_factor_grads": fl_g / (t_cg / 1e3) / 1e12 / FP32_PEAK_TFLOPS}})
     return rows
 
 

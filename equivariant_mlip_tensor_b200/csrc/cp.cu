@@ -17,10 +17,12 @@
 // of four floats), so that one rank component is a few broadcast float4 loads.
 // The rank loop is a runtime loop; the row loops are unrolled at the shape's
 // compile-time dimensions.  The factor gradients are reduced without atomics:
-// each block of 64 (pair, channel) items stages its per-item rank vectors
-// (s (*) t, q (*) t, q (*) s) and inputs in shared memory, contracts them over
-// its items into one partial of every factor entry, and a second kernel sums
-// the block partials in block order (bit-reproducible).
+// a block of 64 threads walks a fixed run of 64-item tiles; per tile it stages
+// the items' rank vectors (s (*) t, q (*) t, q (*) s) and inputs in shared
+// memory and adds their contraction over the tile's items into its own
+// partial of every factor entry (each thread owns fixed entries); a second
+// kernel sums the at most 512 block partials with a fixed reduction tree
+// (bit-reproducible).
 #include "common.cuh"
 #include "launch.h"
 
@@ -28,7 +30,7 @@ namespace cgtp {
 namespace {
 
 constexpr int kCpFwdThreads = 128;
-constexpr int kCpBwdItems = kCpItemsPerPartial;  // items (and threads) per backward block with factor gradients
+constexpr int kCpBwdItems = kCpItemsPerTile;  // items (and threads) per backward block with factor gradients
 constexpr int kCpBwdThreads = 128;
 constexpr int kCpItemStride = kCpBwdItems + 1;  // staged rows padded against bank conflicts
 
@@ -41,26 +43,20 @@ struct CpShape {
   static constexpr int PT = P1 + P2 + P3;  // transposed factor floats per rank component
 };
 
-// Factors into shared memory as [r][row] with rows padded by zeros.
+// Factors into shared memory as [r][row] with rows padded by zeros (reads in
+// the global row-major order, so that a warp reads consecutive floats).
+template <int D, int P>
+__device__ __forceinline__ void load_factor(const float* __restrict__ F, int R, float* Ft) {
+  for (int idx = threadIdx.x; idx < D * R; idx += blockDim.x) Ft[(idx % R) * P + idx / R] = F[idx];
+  if constexpr (P > D)
+    for (int idx = threadIdx.x; idx < (P - D) * R; idx += blockDim.x) Ft[(idx / (P - D)) * P + D + idx % (P - D)] = 0.f;
+}
 template <class S>
 __device__ __forceinline__ void load_factors(const float* __restrict__ A, const float* __restrict__ B,
                                              const float* __restrict__ C, int R, float* Bt, float* Ct, float* At) {
-  for (int idx = threadIdx.x; idx < R * S::PT; idx += blockDim.x) {
-    const int r = idx / S::PT, c = idx % S::PT;
-    float v = 0.f;
-    if (c < S::P1) {
-      if (c < S::D1) v = B[c * R + r];
-      Bt[r * S::P1 + c] = v;
-    } else if (c < S::P1 + S::P2) {
-      const int j = c - S::P1;
-      if (j < S::D2) v = C[j * R + r];
-      Ct[r * S::P2 + j] = v;
-    } else {
-      const int k = c - S::P1 - S::P2;
-      if (k < S::D3) v = A[k * R + r];
-      At[r * S::P3 + k] = v;
-    }
-  }
+  load_factor<S::D1, S::P1>(B, R, Bt);
+  load_factor<S::D2, S::P2>(C, R, Ct);
+  load_factor<S::D3, S::P3>(A, R, At);
 }
 
 // sum_i f[i] v[i] over D entries of a padded factor row.
@@ -124,27 +120,14 @@ __global__ void __launch_bounds__(kCpFwdThreads) cp_fwd_kernel(CPArgs a) {
   for (int k = 0; k < S::D3; ++k) a.z[(b * S::D3 + k) * a.mult + u] = z[k];
 }
 
-// Backward.  GF: also the block partials of the factor gradients.
+// Backward of one item (pair, channel), and, with GF, the staging of its rank
+// vectors and inputs for the factor gradients (column t of the tile buffers).
 template <class S, bool GF>
-__global__ void __launch_bounds__(GF ? kCpBwdItems : kCpBwdThreads) cp_bwd_kernel(CPArgs a) {
-  constexpr int T = GF ? kCpBwdItems : kCpBwdThreads;
-  extern __shared__ float4 cps4[];
-  float* Bt = reinterpret_cast<float*>(cps4);
-  float* Ct = Bt + a.rank * S::P1;
-  float* At = Ct + a.rank * S::P2;
-  float* Pst = At + a.rank * S::P3;             // GF: [R][65] s (*) t
-  float* Pqt = Pst + a.rank * kCpItemStride;     // GF: [R][65] q (*) t
-  float* Pqs = Pqt + a.rank * kCpItemStride;     // GF: [R][65] q (*) s
-  float* Xs = Pqs + a.rank * kCpItemStride;      // GF: [D1][65] x
-  float* Ys = Xs + S::D1 * kCpItemStride;        // GF: [D2][65] y
-  float* Gs = Ys + S::D2 * kCpItemStride;        // GF: [D3][65] g_z
-  load_factors<S>(a.A, a.B, a.C, a.rank, Bt, Ct, At);
-  __syncthreads();
-  const int t = threadIdx.x;
-  const long long item = (long long)blockIdx.x * T + t;
+__device__ __forceinline__ void cp_bwd_item(const CPArgs& a, long long item, int t, const float* Bt, const float* Ct,
+                                            const float* At, float* Pst, float* Pqt, float* Pqs, float* Xs,
+                                            float* Ys, float* Gs) {
   const long long items = (long long)a.batch * a.mult;
   const bool ok = item < items;
-  if (!GF && !ok) return;
   const long long b = ok ? item / a.mult : 0;
   const int u = ok ? (int)(item % a.mult) : 0;
   float x[S::D1], y[S::D2], g[S::D3], gx[S::D1], gy[S::D2];
@@ -185,11 +168,50 @@ __global__ void __launch_bounds__(GF ? kCpBwdItems : kCpBwdThreads) cp_bwd_kerne
     for (int j = 0; j < S::D2; ++j) Ys[j * kCpItemStride + t] = y[j];
 #pragma unroll
     for (int k = 0; k < S::D3; ++k) Gs[k * kCpItemStride + t] = g[k];
-    __syncthreads();
-    // block partial of every factor entry: [g_A (D3 x R) | g_B (D1 x R) | g_C (D2 x R)]
-    const int R = a.rank;
-    const int n_out = (S::D3 + S::D1 + S::D2) * R;
-    float* part = a.partial + (long long)blockIdx.x * n_out;
+  }
+}
+
+// Input gradients only: one thread per item.
+template <class S>
+__global__ void __launch_bounds__(kCpBwdThreads) cp_bwd_kernel(CPArgs a) {
+  extern __shared__ float4 cps4[];
+  float* Bt = reinterpret_cast<float*>(cps4);
+  float* Ct = Bt + a.rank * S::P1;
+  float* At = Ct + a.rank * S::P2;
+  load_factors<S>(a.A, a.B, a.C, a.rank, Bt, Ct, At);
+  __syncthreads();
+  const long long item = (long long)blockIdx.x * kCpBwdThreads + threadIdx.x;
+  if (item >= (long long)a.batch * a.mult) return;
+  cp_bwd_item<S, false>(a, item, threadIdx.x, Bt, Ct, At, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+}
+
+// Input gradients and the block's partial of every factor-gradient entry,
+// [g_A (D3 x R) | g_B (D1 x R) | g_C (D2 x R)], over the block's run of tiles.
+template <class S>
+__global__ void __launch_bounds__(kCpBwdItems) cp_bwd_factors_kernel(CPArgs a, long long tiles, long long tpb) {
+  constexpr int T = kCpBwdItems;
+  extern __shared__ float4 cps4[];
+  const int R = a.rank;
+  const int n_out = (S::D3 + S::D1 + S::D2) * R;
+  float* Bt = reinterpret_cast<float*>(cps4);
+  float* Ct = Bt + R * S::P1;
+  float* At = Ct + R * S::P2;
+  float* Pst = At + R * S::P3;            // [R][65] s (*) t
+  float* Pqt = Pst + R * kCpItemStride;    // [R][65] q (*) t
+  float* Pqs = Pqt + R * kCpItemStride;    // [R][65] q (*) s
+  float* Xs = Pqs + R * kCpItemStride;     // [D1][65] x
+  float* Ys = Xs + S::D1 * kCpItemStride;  // [D2][65] y
+  float* Gs = Ys + S::D2 * kCpItemStride;  // [D3][65] g_z
+  float* Acc = Gs + S::D3 * kCpItemStride; // [n_out] this block's partial
+  load_factors<S>(a.A, a.B, a.C, R, Bt, Ct, At);
+  const int t = threadIdx.x;
+  for (int o = t; o < n_out; o += T) Acc[o] = 0.f;  // entries o = t (mod 64) belong to thread t
+  __syncthreads();
+  const long long t0 = (long long)blockIdx.x * tpb;
+  const long long t1 = t0 + tpb < tiles ? t0 + tpb : tiles;
+  for (long long tile = t0; tile < t1; ++tile) {
+    cp_bwd_item<S, true>(a, tile * T + t, t, Bt, Ct, At, Pst, Pqt, Pqs, Xs, Ys, Gs);
+    __syncthreads();  // the tile's columns are staged
     for (int o = t; o < n_out; o += T) {
       const float* lhs;
       const float* rhs;
@@ -205,27 +227,46 @@ __global__ void __launch_bounds__(GF ? kCpBwdItems : kCpBwdThreads) cp_bwd_kerne
         lhs = Ys + (o2 / R) * kCpItemStride;
         rhs = Pqs + (o2 % R) * kCpItemStride;
       }
-      float v = 0.f;
-#pragma unroll 8
-      for (int it = 0; it < T; ++it) v = fmaf(lhs[it], rhs[it], v);
-      part[o] = v;
+      float v[4] = {0.f, 0.f, 0.f, 0.f};  // four interleaved partial sums over the tile's items
+#pragma unroll 4
+      for (int it = 0; it < T; it += 4) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) v[c] = fmaf(lhs[it + c], rhs[it + c], v[c]);
+      }
+      Acc[o] += (v[0] + v[1]) + (v[2] + v[3]);
     }
+    __syncthreads();  // the tile's columns are consumed
   }
+  float* part = a.partial + (long long)blockIdx.x * n_out;
+  for (int o = t; o < n_out; o += T) part[o] = Acc[o];
 }
 
-// g_A, g_B, g_C = the block partials summed in block order.
-__global__ void cp_reduce_kernel(int blocks, int d1, int d2, int d3, int R, const float* __restrict__ partial,
-                                 float* __restrict__ gA, float* __restrict__ gB, float* __restrict__ gC) {
+// g_A, g_B, g_C = the sum of the block partials.  A block of 256 threads takes
+// 32 entries: warp w sums the partials k = w (mod 8) in increasing k, then
+// warp 0 adds the eight warp sums in warp order.
+constexpr int kCpRedEntries = 32, kCpRedWarps = 8;
+__global__ void __launch_bounds__(32 * kCpRedWarps)
+    cp_reduce_kernel(int blocks, int d1, int d2, int d3, int R, const float* __restrict__ partial,
+                     float* __restrict__ gA, float* __restrict__ gB, float* __restrict__ gC) {
+  __shared__ float part[kCpRedWarps][kCpRedEntries];
   const int n_out = (d1 + d2 + d3) * R;
-  for (int o = blockIdx.x * blockDim.x + threadIdx.x; o < n_out; o += gridDim.x * blockDim.x) {
-    float v = 0.f;
-    for (int k = 0; k < blocks; ++k) v += partial[(long long)k * n_out + o];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int o = blockIdx.x * kCpRedEntries + lane;
+  float v = 0.f;
+  if (o < n_out)
+    for (int k = w; k < blocks; k += kCpRedWarps) v += partial[(long long)k * n_out + o];
+  part[w][lane] = v;
+  __syncthreads();
+  if (w == 0 && o < n_out) {
+    float s = 0.f;
+#pragma unroll
+    for (int q = 0; q < kCpRedWarps; ++q) s += part[q][lane];
     if (o < d3 * R) {
-      if (gA) gA[o] = v;
+      if (gA) gA[o] = s;
     } else if (o < (d3 + d1) * R) {
-      if (gB) gB[o - d3 * R] = v;
+      if (gB) gB[o - d3 * R] = s;
     } else {
-      if (gC) gC[o - (d3 + d1) * R] = v;
+      if (gC) gC[o - (d3 + d1) * R] = s;
     }
   }
 }
@@ -236,7 +277,8 @@ template <int LI, int LS, int LO>
 size_t cp_smem_bytes(int rank, bool factor_grads) {
   using S = CpShape<LI, LS, LO>;
   size_t n = (size_t)rank * S::PT;
-  if (factor_grads) n += (size_t)(3 * rank + S::D1 + S::D2 + S::D3) * kCpItemStride;
+  if (factor_grads)
+    n += (size_t)(3 * rank + S::D1 + S::D2 + S::D3) * kCpItemStride + (size_t)(S::D1 + S::D2 + S::D3) * rank;
   return sizeof(float) * n;
 }
 
@@ -257,30 +299,29 @@ cudaError_t launch_cp_bwd(const CPArgs& a, cudaStream_t stream) {
   using S = CpShape<LI, LS, LO>;
   const long long items = (long long)a.batch * a.mult;
   const bool gf = a.grad_A != nullptr || a.grad_B != nullptr || a.grad_C != nullptr;
-  if (items > 0 && (gf || a.grad_x != nullptr || a.grad_y != nullptr)) {
-    const size_t smem = cp_smem_bytes<LI, LS, LO>(a.rank, gf);
-    cudaError_t e;
-    if (gf) {
-      e = cudaFuncSetAttribute(cp_bwd_kernel<S, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = cp_smem_bytes<LI, LS, LO>(a.rank, gf);
+  cudaError_t e;
+  if (gf) {
+    if (items > 0) {
+      e = cudaFuncSetAttribute(cp_bwd_factors_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
-      cp_bwd_kernel<S, true><<<(unsigned)cp_bwd_blocks(a.batch, a.mult), kCpBwdItems, smem, stream>>>(a);
-    } else {
-      e = cudaFuncSetAttribute(cp_bwd_kernel<S, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cp_bwd_factors_kernel<S><<<(unsigned)cp_bwd_blocks(a.batch, a.mult), kCpBwdItems, smem, stream>>>(
+          a, cp_bwd_tiles(a.batch, a.mult), cp_bwd_tiles_per_block(a.batch, a.mult));
+      e = cudaGetLastError();
       if (e != cudaSuccess) return e;
-      cp_bwd_kernel<S, false>
-          <<<(unsigned)((items + kCpBwdThreads - 1) / kCpBwdThreads), kCpBwdThreads, smem, stream>>>(a);
     }
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
-  if (gf) {  // also for an empty batch: the gradients are then zero
+    // also for an empty batch: the gradients are then zero
     const int n_out = (S::D1 + S::D2 + S::D3) * a.rank;
-    cp_reduce_kernel<<<(n_out + 255) / 256, 256, 0, stream>>>((int)cp_bwd_blocks(a.batch, a.mult), S::D1, S::D2,
-                                                             S::D3, a.rank, a.partial, a.grad_A, a.grad_B,
-                                                             a.grad_C);
+    const int blocks = items > 0 ? (int)cp_bwd_blocks(a.batch, a.mult) : 0;
+    cp_reduce_kernel<<<(n_out + kCpRedEntries - 1) / kCpRedEntries, 32 * kCpRedWarps, 0, stream>>>(
+        blocks, S::D1, S::D2, S::D3, a.rank, a.partial, a.grad_A, a.grad_B, a.grad_C);
     return cudaGetLastError();
   }
-  return cudaSuccess;
+  if (items == 0 || (a.grad_x == nullptr && a.grad_y == nullptr)) return cudaSuccess;
+  e = cudaFuncSetAttribute(cp_bwd_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cp_bwd_kernel<S><<<(unsigned)((items + kCpBwdThreads - 1) / kCpBwdThreads), kCpBwdThreads, smem, stream>>>(a);
+  return cudaGetLastError();
 }
 
 // One translation unit per shape (the build passes CGTP_CFG_LI/LS/LO).

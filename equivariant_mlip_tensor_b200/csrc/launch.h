@@ -16,9 +16,22 @@ struct CPArgs {
   const float *A, *B, *C, *x, *y, *grad_z;
   float *z, *grad_x, *grad_y, *grad_A, *grad_B, *grad_C, *partial;
 };
-constexpr int kCpItemsPerPartial = 64;  // (pair, channel) items per factor-gradient partial
+// The backward with factor gradients walks (pair, channel) items in tiles of
+// 64; each block takes cp_bwd_tiles_per_block consecutive tiles (at most 512
+// blocks), a fixed function of the problem size, so the partials and their
+// summation order do not depend on the device.
+constexpr int kCpItemsPerTile = 64;
+constexpr long long kCpMaxPartials = 512;
+inline long long cp_bwd_tiles(int batch, int mult) {
+  return ((long long)batch * mult + kCpItemsPerTile - 1) / kCpItemsPerTile;
+}
+inline long long cp_bwd_tiles_per_block(int batch, int mult) {
+  const long long t = cp_bwd_tiles(batch, mult);
+  return t <= kCpMaxPartials ? 1 : (t + kCpMaxPartials - 1) / kCpMaxPartials;
+}
 inline long long cp_bwd_blocks(int batch, int mult) {
-  return ((long long)batch * mult + kCpItemsPerPartial - 1) / kCpItemsPerPartial;
+  const long long tpb = cp_bwd_tiles_per_block(batch, mult);
+  return (cp_bwd_tiles(batch, mult) + tpb - 1) / tpb;
 }
 template <int LI, int LS, int LO>
 size_t cp_smem_bytes(int rank, bool factor_grads);
