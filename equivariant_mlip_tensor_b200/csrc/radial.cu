@@ -15,7 +15,7 @@
 // instruction, rounded like two fmaf), which halves the issue slots the
 // products take.
 // Backward: grad_h = grad_W W2^T is a GEMM with M = edges, N = 64, K = P*mult;
-// each block owns 128 edges and all 64 hidden units, streams grad_W once
+// each block owns 96 edges and all 64 hidden units, streams grad_W once
 // through a two-stage cp.async pipeline, and its epilogue folds grad_h
 // through SiLU', W1 and dphi/dr into dL/d|r| per edge, added to
 // grad_edge_vec along r/|r| (one owner per edge, no atomics).
@@ -166,18 +166,22 @@ cudaError_t launch_radial_fwd(int n_edges, int N, const float* ev, float rc, con
 }
 
 // ---------------------------------------------------------------- backward
-// grad_h [128 edges][64 hidden] = grad_W [128][N] W2^T, K = N in chunks of 32
+// grad_h [96 edges][64 hidden] = grad_W [96][N] W2^T, K = N in chunks of 32
 // staged by cp.async in two stages.  Shared rows are padded to 36 floats so
 // that the per-thread float4 reads fall in distinct banks; thread (ty, tx)
-// owns edges ty + 16 i and hidden units tx + 8 j, an 8 x 8 register tile.
-constexpr int kBwdBM = 128, kBwdBK = 32, kBwdStride = kBwdBK + 4, kBwdThreads = 128;
+// owns edges ty + 16 i and hidden units tx + 8 j, a 6 x 8 register tile.
+// Edges per thread: 96-edge tiles (6 per thread) fill the 4 resident blocks per
+// SM in 1.7 waves at 97 480 edges where 128-edge tiles leave a 1.3-wave tail
+// (0.69 vs 0.76 ms measured; 112-edge tiles 0.72 ms).
+constexpr int kEPT = 6;
+constexpr int kBwdBM = 16 * kEPT, kBwdBK = 32, kBwdStride = kBwdBK + 4, kBwdThreads = 128;
 constexpr int kBwdSmem = (int)sizeof(float) * 2 * (kBwdBM + kRH) * kBwdStride;
 
 static __global__ void __launch_bounds__(kBwdThreads, 4)
     radial_bwd_kernel(int n_edges, int N, const float* __restrict__ ev, float rc, const float* __restrict__ W1,
                       const float* __restrict__ W2, const float* __restrict__ gw, float* __restrict__ gev) {
   extern __shared__ float4 rsm4[];
-  float* As = reinterpret_cast<float*>(rsm4);  // 2 x [128][36]  grad_W chunk, [edge][n]
+  float* As = reinterpret_cast<float*>(rsm4);  // 2 x [96][36]   grad_W chunk, [edge][n]
   float* Bs = As + 2 * kBwdBM * kBwdStride;    // 2 x [64][36]   W2 chunk, [hidden][n]
   const int t = threadIdx.x;
   const int tx = t & 7, ty = t >> 3;
@@ -204,9 +208,9 @@ static __global__ void __launch_bounds__(kBwdThreads, 4)
     }
     cp_commit();
   };
-  float acc[8][8];
+  float acc[kEPT][8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < kEPT; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
   const int n_chunks = (N + kBwdBK - 1) / kBwdBK;
@@ -225,14 +229,14 @@ static __global__ void __launch_bounds__(kBwdThreads, 4)
     const float* b = Bs + s * kRH * kBwdStride;
 #pragma unroll 1
     for (int q = 0; q < kBwdBK / 4; ++q) {
-      float4 av[8];
+      float4 av[kEPT];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) av[i] = *reinterpret_cast<const float4*>(a + (ty + 16 * i) * kBwdStride + 4 * q);
+      for (int i = 0; i < kEPT; ++i) av[i] = *reinterpret_cast<const float4*>(a + (ty + 16 * i) * kBwdStride + 4 * q);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const float4 bv = *reinterpret_cast<const float4*>(b + (tx + 8 * j) * kBwdStride + 4 * q);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < kEPT; ++i) {
           acc[i][j] = fmaf(av[i].x, bv.x, acc[i][j]);
           acc[i][j] = fmaf(av[i].y, bv.y, acc[i][j]);
           acc[i][j] = fmaf(av[i].z, bv.z, acc[i][j]);
@@ -243,7 +247,7 @@ static __global__ void __launch_bounds__(kBwdThreads, 4)
   }
   // epilogue: dL/dr = sum_k grad_h[k] SiLU'(a_k) (dphi W1)_k, per edge
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < kEPT; ++i) {
     const long long e = m0 + ty + 16 * i;
     float x = 0.f, y = 0.f, z = 0.f, r = 0.f;
     if (e < n_edges) {
