@@ -385,8 +385,9 @@ def config_table(torch, api, dev, hbm, reps=20):
 
 def run_op(args):
     """A short loop of one operation at the molecules workload, for profiling
-    (ncu launch lists): 'uvw' (fully connected forward) or 'double' (double
-    backward)."""
+    (ncu launch lists): 'uvw' (fully connected forward), 'uvw_bwd' (its
+    backward), 'double' (double backward) or 'cp' (CP-decomposed product of
+    the tp_batch pairs, rank 40, forward and backward with factor gradients)."""
     import torch
 
     from equivariant_mlip_tensor_b200 import api
@@ -403,6 +404,21 @@ def run_op(args):
     if args.op == "uvw":
         mix = torch.randn((plan.n_paths, u, 128), device=dev) / u ** 0.5
         fn = lambda: plan.uvw_forward(g, x, W, mix)
+    elif args.op == "uvw_bwd":
+        mix = torch.randn((plan.n_paths, u, 128), device=dev) / u ** 0.5
+        ugo = torch.randn((n, (L[2] + 1) ** 2, 128), device=dev)
+        fn = lambda: plan.uvw_backward(g, x, W, mix, ugo)
+    elif args.op == "cp":
+        t = synthetic.tp_batch()
+        Lt = (t.lmax_in, t.lmax_sh, t.lmax_out)
+        tplan = api.Plan(*Lt, t.mult)
+        xs, ys, gz = (torch.from_numpy(a).to(dev) for a in (t.x, t.y, t.grad_z))
+        d1, d2, d3 = ((l + 1) ** 2 for l in Lt)
+        fA, fB, fC = (torch.randn((d, 40), device=dev) / 40 ** 0.5 for d in (d3, d1, d2))
+
+        def fn():
+            tplan.cp_forward(fA, fB, fC, xs, ys)
+            tplan.cp_backward(fA, fB, fC, xs, ys, gz)
     else:
         ggx, ggw, ggr = torch.randn_like(x), torch.randn_like(W), torch.randn((g.n_edges, 3), device=dev)
         fn = lambda: plan.conv_double_backward(g, x, W, go, gg_x=ggx, gg_w=ggw, gg_edge_vec=ggr)
@@ -662,7 +678,7 @@ def main():
     ap.add_argument("--impl", choices=["cgtp", "reference"], default="cgtp")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-workload table")
-    ap.add_argument("--op", choices=["uvw", "double"], default=None,
+    ap.add_argument("--op", choices=["uvw", "uvw_bwd", "double", "cp"], default=None,
                     help="time one other operation alone (for profiling) instead of the benchmark")
     ap.add_argument("--graphs", type=int, default=256, help="molecules per rank (profiling uses fewer)")
     ap.add_argument("--conv-only", action="store_true",

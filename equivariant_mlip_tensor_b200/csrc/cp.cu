@@ -32,7 +32,7 @@ namespace {
 constexpr int kCpFwdThreads = 128;
 constexpr int kCpBwdItems = kCpItemsPerTile;  // items (and threads) per backward block with factor gradients
 constexpr int kCpBwdThreads = 128;
-constexpr int kCpItemStride = kCpBwdItems + 1;  // staged rows padded against bank conflicts
+constexpr int kCpItemStride = kCpBwdItems + 4;  // staged rows: 16-byte aligned, rows r and r+1 in distinct banks
 
 constexpr int pad4(int d) { return (d + 3) & ~3; }
 
@@ -196,12 +196,12 @@ __global__ void __launch_bounds__(kCpBwdItems) cp_bwd_factors_kernel(CPArgs a, l
   float* Bt = reinterpret_cast<float*>(cps4);
   float* Ct = Bt + R * S::P1;
   float* At = Ct + R * S::P2;
-  float* Pst = At + R * S::P3;            // [R][65] s (*) t
-  float* Pqt = Pst + R * kCpItemStride;    // [R][65] q (*) t
-  float* Pqs = Pqt + R * kCpItemStride;    // [R][65] q (*) s
-  float* Xs = Pqs + R * kCpItemStride;     // [D1][65] x
-  float* Ys = Xs + S::D1 * kCpItemStride;  // [D2][65] y
-  float* Gs = Ys + S::D2 * kCpItemStride;  // [D3][65] g_z
+  float* Pst = At + R * S::P3;            // [R][68] s (*) t
+  float* Pqt = Pst + R * kCpItemStride;    // [R][68] q (*) t
+  float* Pqs = Pqt + R * kCpItemStride;    // [R][68] q (*) s
+  float* Xs = Pqs + R * kCpItemStride;     // [D1][68] x
+  float* Ys = Xs + S::D1 * kCpItemStride;  // [D2][68] y
+  float* Gs = Ys + S::D2 * kCpItemStride;  // [D3][68] g_z
   float* Acc = Gs + S::D3 * kCpItemStride; // [n_out] this block's partial
   load_factors<S>(a.A, a.B, a.C, R, Bt, Ct, At);
   const int t = threadIdx.x;
@@ -230,8 +230,12 @@ __global__ void __launch_bounds__(kCpBwdItems) cp_bwd_factors_kernel(CPArgs a, l
       float v[4] = {0.f, 0.f, 0.f, 0.f};  // four interleaved partial sums over the tile's items
 #pragma unroll 4
       for (int it = 0; it < T; it += 4) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) v[c] = fmaf(lhs[it + c], rhs[it + c], v[c]);
+        const float4 l4 = *reinterpret_cast<const float4*>(lhs + it);
+        const float4 r4 = *reinterpret_cast<const float4*>(rhs + it);
+        v[0] = fmaf(l4.x, r4.x, v[0]);
+        v[1] = fmaf(l4.y, r4.y, v[1]);
+        v[2] = fmaf(l4.z, r4.z, v[2]);
+        v[3] = fmaf(l4.w, r4.w, v[3]);
       }
       Acc[o] += (v[0] + v[1]) + (v[2] + v[3]);
     }
@@ -253,8 +257,17 @@ __global__ void __launch_bounds__(32 * kCpRedWarps)
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int o = blockIdx.x * kCpRedEntries + lane;
   float v = 0.f;
-  if (o < n_out)
-    for (int k = w; k < blocks; k += kCpRedWarps) v += partial[(long long)k * n_out + o];
+  if (o < n_out) {
+    int k = w;
+    for (; k + 7 * kCpRedWarps < blocks; k += 8 * kCpRedWarps) {  // eight loads in flight, added in k order
+      float q[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) q[c] = partial[(long long)(k + c * kCpRedWarps) * n_out + o];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) v += q[c];
+    }
+    for (; k < blocks; k += kCpRedWarps) v += partial[(long long)k * n_out + o];
+  }
   part[w][lane] = v;
   __syncthreads();
   if (w == 0 && o < n_out) {
