@@ -300,6 +300,22 @@ static cudaError_t dispatch_fwd(cgtp_plan p, const ConvFwdArgs& a, int sms, cuda
   CGTP_CONFIGS(CGTP_DFWD_ENTRY)
   return e;
 }
+static cudaError_t dispatch_bwd(cgtp_plan p, const ConvBwdArgs& a, int sms, cudaStream_t s);
+// Harmonic-gradient-only backward pass (no grad_x / grad_W) when its partial
+// slices fit the plain backward's workspace, else the plain backward.
+static cudaError_t dispatch_bwd_gy(cgtp_plan p, const ConvBwdArgs& a, int sms, cudaStream_t s) {
+  cudaError_t e = cudaErrorNotSupported;
+  bool done = false;
+#define CGTP_BWD_GY_ENTRY(A, B, C)                                                     \
+  if (!done && p->li == A && p->ls == B && p->lo == C &&                                \
+      paths_bwd_slices<A, B, C>(p->mult) <= conv_bwd_slices<A, B, C>(p->mult)) {        \
+    e = launch_conv_bwd_gy<A, B, C>(a, sms, s);                                         \
+    done = true;                                                                        \
+  }
+  CGTP_CONFIGS(CGTP_BWD_GY_ENTRY)
+  return done ? e : dispatch_bwd(p, a, sms, s);
+}
+
 static cudaError_t dispatch_bwd(cgtp_plan p, const ConvBwdArgs& a, int sms, cudaStream_t s) {
   cudaError_t e = cudaErrorNotSupported;
 #define CGTP_DBWD_ENTRY(A, B, C) \
@@ -419,7 +435,7 @@ cgtp_status cgtp_conv_double_backward(cgtp_plan p, int n_nodes, int n_edges, con
                     nullptr, nullptr, d_edge_vec, gsh, p->mult};
       a.gr_mode = init ? mode_add : mode_set;
       a.gr_dir = gg_edge_vec;
-      e = dispatch_bwd(p, a, sms, s);
+      e = dispatch_bwd_gy(p, a, sms, s);
       init = true;
     };
     if (gg_x) gy(gg_x, w, 0, 1);

@@ -460,7 +460,7 @@ constexpr int pp_rowoff(int K) {
 // finished block goes to this lane's column of the shared reduction buffer
 // (gyrow, row stride rs).  The edge's weight rows and its destination's output-gradient
 // rows come from this lane's pipeline stage.
-template <class PS, class GR, int VEC, bool NEED_GY, bool PP>
+template <class PS, class GR, int VEC, bool NEED_GY, bool PP, bool HX>
 __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const float* __restrict__ stage, int rowf,
                                          const float (&xr)[GR::NOWN][VEC], float* __restrict__ gwrow, bool acc, int mult,
                                          float (&gx)[GR::NOWN][VEC], float* __restrict__ gyrow, int rs) {
@@ -499,7 +499,7 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
         if constexpr (k < tc) {
           constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
           const float tv = tv4[decltype(Rc)::value];
-          axpy<VEC>(h[m1 + l1], tv, gv[m3 + l3]);
+          if constexpr (HX) axpy<VEC>(h[m1 + l1], tv, gv[m3 + l3]);
           if constexpr (NEED_GY) {
             const float av = vdot<VEC>(xw[m1 + l1], gv[m3 + l3]);
             static_for<0, 2 * l2 + 1>([&](auto M2c) {
@@ -512,22 +512,24 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
         }
       });
     });
-    float gw[VEC];
+    if constexpr (HX) {
+      float gw[VEC];
 #pragma unroll
-    for (int c = 0; c < VEC; ++c) gw[c] = 0.f;
+      for (int c = 0; c < VEC; ++c) gw[c] = 0.f;
 #pragma unroll
-    for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) {
-      vfma<VEC>(gx[m1], wv, h[m1]);
-      vfma<VEC>(gw, xr[m1], h[m1]);
-    }
-    if (gwrow != nullptr) {
-      if (acc) {
-        float prev[VEC];
-        VecIO<VEC>::ld(prev, gwrow + P * mult);
-#pragma unroll
-        for (int c = 0; c < VEC; ++c) gw[c] += prev[c];
+      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) {
+        vfma<VEC>(gx[m1], wv, h[m1]);
+        vfma<VEC>(gw, xr[m1], h[m1]);
       }
-      VecIO<VEC>::st_stream(gwrow + P * mult, gw);
+      if (gwrow != nullptr) {
+        if (acc) {
+          float prev[VEC];
+          VecIO<VEC>::ld(prev, gwrow + P * mult);
+#pragma unroll
+          for (int c = 0; c < VEC; ++c) gw[c] += prev[c];
+        }
+        VecIO<VEC>::st_stream(gwrow + P * mult, gw);
+      }
     }
     if constexpr (NEED_GY && GR::D.last_l2[K]) {
 #pragma unroll
@@ -558,7 +560,9 @@ using BwdPlan = Plan<PS, kByL1, VEC, NEED_GY, bwd_budget<PS>()>;
 // results added onto the outputs); the plain variant compiles without either.
 // PP: grad_out is the per-path message layout of the fully connected
 // convolution (each path reads its own rows).
-template <class PS, int VEC, bool NEED_GY, int CH, int KMULT, bool EXT, bool PP>
+// HX = false: only the harmonic gradient (no grad_x, no grad_W, and none of
+// the T^T g products they need), for passes that want grad_Y alone.
+template <class PS, int VEC, bool NEED_GY, int CH, int KMULT, bool EXT, bool PP, bool HX>
 __global__ void CGTP_BWD_BOUNDS
 conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt) {
   // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x VEC
@@ -678,8 +682,8 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
         int e = 0;
         if (valid) {
           e = Eg[k];
-          bwd_edge<PS, GR, VEC, NEED_GY, PP>(Tg + k * NT, St + (k & 1) * stage_floats + gl * VEC, rowf, xr,
-                                         a.grad_w ? a.grad_w + (long long)e * PS::NP * mult + c0 : nullptr,
+          bwd_edge<PS, GR, VEC, NEED_GY, PP, HX>(Tg + k * NT, St + (k & 1) * stage_floats + gl * VEC, rowf, xr,
+                                         HX && a.grad_w ? a.grad_w + (long long)e * PS::NP * mult + c0 : nullptr,
                                          EXT && a.accumulate != 0, mult, gx, red + gl, rs);
         }
         if constexpr (NEED_GY) {
@@ -712,7 +716,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
       }
       __syncwarp();
     }
-    if (active && a.grad_x != nullptr) {
+    if (HX && active && a.grad_x != nullptr) {
       if (!GR::FIRST || (EXT && a.accumulate)) {
         // rows of an l1 block that an earlier chunk of this call wrote (wait
         // for that grid, the preceding launch), or the caller's values
@@ -841,14 +845,14 @@ int paths_bwd_slices(int mult) {
   return S * BwdPlan<PS, paths_bwd_vec<PS>(), true>::N;  // one partial grad_Y per (chunk, channel slice)
 }
 
-template <class PS, bool NEED_GY, int CH>
+template <class PS, bool NEED_GY, int CH, bool PP = true, bool HX = true, int KMULT = 0>
 cudaError_t paths_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
   constexpr int VEC = paths_bwd_vec<PS>();
   using GR = ChunkGrp<PS, BwdPlan<PS, VEC, NEED_GY>, CH, kByL1>;
   int G, lg_G, S;
   paths_bwd_geometry<PS>(a.mult, G, lg_G, S);
   const int gpw = 32 / G;
-  const int ng = pp_rowoff<PS, GR>(GR::NP);
+  const int ng = PP ? pp_rowoff<PS, GR>(GR::NP) : GR::NROW;
   const int stage_floats = (GR::NP + ng) * G * VEC;
   const int BT = pick_batch(gpw, GR::NT, stage_floats, CGTP_BWD_BATCH_FLOATS, CGTP_BWD_MAX_BATCH);
   const int group_floats = BT * GR::NT + 2 * stage_floats + 2 * ((BT + 3) & ~3);
@@ -858,7 +862,7 @@ cudaError_t paths_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t stre
   const long long groups_per_block = (long long)gpw * (kBwdThreads / 32);
   const long long blocks = (items + groups_per_block - 1) / groups_per_block;
   if (a.sh != nullptr || a.accumulate) return cudaErrorInvalidValue;
-  auto kern = conv_bwd_kernel<PS, VEC, NEED_GY, CH, 0, false, true>;
+  auto kern = conv_bwd_kernel<PS, VEC, NEED_GY, CH, KMULT, false, PP, HX>;
   cudaError_t e2 = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e2 != cudaSuccess) return e2;
   long long cap = 0x7fffffffLL;  // the kernel loops over items beyond the grid
@@ -925,7 +929,44 @@ cudaError_t launch_conv_bwd_paths(const ConvBwdArgs& a, int num_sms, cudaStream_
   return cudaGetLastError();
 }
 
+// The harmonic gradient alone (grad_x and grad_W not wanted): the chunks of
+// the plain backward without the T^T g products, then the Jacobian epilogue
+// of a.gr_mode.  Partials go to a.grad_sh as in the plain backward.
+template <int LI, int LS, int LO>
+cudaError_t launch_conv_bwd_gy(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
+  using PS = PathSet<LI, LS, LO>;
+  constexpr int VEC = paths_bwd_vec<PS>();
+  constexpr int NCH = BwdPlan<PS, VEC, true>::N;
+  if (a.grad_edge_vec == nullptr || a.grad_sh == nullptr) return cudaErrorInvalidValue;
+  if (a.n_edges == 0) return cudaSuccess;
+  const bool k128 = a.mult == 128 && 128 % (32 * VEC) == 0;
+  cudaError_t err = cudaSuccess;
+  static_for_host<0, NCH>([&](auto Cc) {
+    constexpr int CH = decltype(Cc)::value;
+    if (err != cudaSuccess) return;
+    err = k128 ? paths_bwd_chunk<PS, true, CH, false, false, 128>(a, num_sms, stream)
+               : paths_bwd_chunk<PS, true, CH, false, false, 0>(a, num_sms, stream);
+  });
+  if (err != cudaSuccess) return err;
+  const int threads = 256;
+  long long nbk = (a.n_edges + threads - 1) / threads;
+  if (nbk > (long long)num_sms * 16) nbk = (long long)num_sms * 16;
+  const int S = paths_bwd_slices<LI, LS, LO>(a.mult);
+  if (a.gr_mode >= 2) {
+    if (a.gr_dir == nullptr) return cudaErrorInvalidValue;
+    sh_backward_hess_kernel<LS><<<(unsigned)nbk, threads, 0, stream>>>(a.n_edges, S, a.edge_vec, a.grad_sh, a.gr_dir,
+                                                                      a.grad_edge_vec, a.gr_mode == 2);
+  } else {
+    sh_backward_kernel<LS><<<(unsigned)nbk, threads, 0, stream>>>(a.n_edges, S, a.edge_vec, a.grad_sh,
+                                                                 a.grad_edge_vec, a.gr_mode == 1);
+  }
+  return cudaGetLastError();
+}
+
 // One translation unit per shape (the build passes CGTP_CFG_LI/LS/LO).
+template cudaError_t launch_conv_bwd_gy<CGTP_CFG_LI, CGTP_CFG_LS, CGTP_CFG_LO>(const ConvBwdArgs&, int,
+                                                                             cudaStream_t);
+template int paths_bwd_slices<CGTP_CFG_LI, CGTP_CFG_LS, CGTP_CFG_LO>(int);
 template cudaError_t launch_conv_paths<CGTP_CFG_LI, CGTP_CFG_LS, CGTP_CFG_LO>(const ConvFwdArgs&, int,
                                                                            cudaStream_t);
 template void conv_path_order<CGTP_CFG_LI, CGTP_CFG_LS, CGTP_CFG_LO>(int*, int*);

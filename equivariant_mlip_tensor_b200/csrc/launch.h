@@ -52,6 +52,13 @@ template <int LI, int LS, int LO>
 cudaError_t launch_conv_bwd_shared(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);
 template <int LI, int LS, int LO>
 cudaError_t launch_conv_bwd_paths(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);
+// The harmonic gradient alone (grad_Y partials and the Jacobian epilogue of
+// a.gr_mode; no grad_x / grad_W work), and the number of grad_Y partial slices
+// it writes.
+template <int LI, int LS, int LO>
+cudaError_t launch_conv_bwd_gy(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);
+template <int LI, int LS, int LO>
+int paths_bwd_slices(int mult);
 template <int LI, int LS, int LO>
 cudaError_t launch_conv_bwd(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);
 template <int LI, int LS, int LO>
