@@ -26,6 +26,9 @@ CGTP_DEFINE_CONSTANT_TABLES()
 #include "vec2.cuh"
 #include "sh.cuh"
 
+#include <map>
+#include <mutex>
+
 namespace cgtp {
 
 namespace {
@@ -432,7 +435,7 @@ int conv_bwd_slices(int mult) {
 }
 
 template <class PS, bool NEED_GY, int CH>
-cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
+cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t stream, bool pdl) {
   constexpr int VEC = bwd_vec<PS>();
   using GR = ChunkGrp<PS, BwdPlan<PS, VEC, NEED_GY>, CH, kByL1>;
   int G, lg_G, S;
@@ -461,7 +464,7 @@ cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t str
   long long nb = blocks > cap ? cap : blocks;
   if (nb < 1) nb = 1;
   // Every chunk but the call's first may overlap the one before it.
-  return launch_kernel(kern, dim3((unsigned)nb), dim3(kBwdThreads), smem, stream, CGTP_BWD_PDL && CH > 0, a, lg_G,
+  return launch_kernel(kern, dim3((unsigned)nb), dim3(kBwdThreads), smem, stream, CGTP_BWD_PDL && pdl, a, lg_G,
                        S, BT, CH * S);
 }
 
@@ -484,13 +487,79 @@ cudaError_t zero_unreached_grad_x(const ConvBwdArgs& a, cudaStream_t stream) {
   return err;
 }
 
+// Chunks of different l1 blocks write disjoint outputs (their own grad_x rows,
+// their own paths' grad_W rows, their own grad_Y partial slices), so each l1
+// block's chunks run on a lane of their own, forked from the caller's stream
+// and joined back before the call's next launch: the latency-bound small
+// blocks then fill the SMs beside the large ones.  Within a lane, a chunk that
+// continues an l1 block overlaps its predecessor through programmatic
+// dependent launch and waits for it before adding to its rows.
+#ifndef CGTP_BWD_LANES
+#define CGTP_BWD_LANES 1
+#endif
+constexpr int kBwdMaxLanes = kLmaxTab + 1;
+struct BwdLanes {
+  cudaStream_t side[kBwdMaxLanes - 1];
+  cudaEvent_t fork, join[kBwdMaxLanes - 1];
+};
+static cudaError_t bwd_lanes_for_device(BwdLanes** out) {
+  static std::mutex mu;
+  static std::map<int, BwdLanes> per_dev;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = per_dev.find(dev);
+  if (it == per_dev.end()) {
+    BwdLanes L{};
+    for (int k = 0; k < kBwdMaxLanes - 1 && e == cudaSuccess; ++k) {
+      e = cudaStreamCreateWithFlags(&L.side[k], cudaStreamNonBlocking);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L.join[k], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L.fork, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+    it = per_dev.emplace(dev, L).first;
+  }
+  *out = &it->second;
+  return cudaSuccess;
+}
+// Host threads that enqueue on the shared lanes take turns (the events are shared).
+static std::mutex& bwd_lanes_mutex() {
+  static std::mutex mu;
+  return mu;
+}
+
 template <class PS, bool NEED_GY>
 cudaError_t launch_bwd_chunks(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
-  constexpr int NCH = BwdPlan<PS, bwd_vec<PS>(), NEED_GY>::N;
+  using PL = BwdPlan<PS, bwd_vec<PS>(), NEED_GY>;
+  constexpr int NCH = PL::N;
+  constexpr int NKEYS = PL::P.key[NCH - 1] - PL::P.key[0] + 1;
   cudaError_t err = a.accumulate ? cudaSuccess : zero_unreached_grad_x<PS>(a, stream);
+  if (!CGTP_BWD_LANES || NKEYS <= 1) {
+    static_for_host<0, NCH>([&](auto Cc) {
+      constexpr int CH = decltype(Cc)::value;
+      if (err == cudaSuccess) err = launch_bwd_chunk<PS, NEED_GY, CH>(a, num_sms, stream, CH > 0);
+    });
+    return err;
+  }
+  if (err != cudaSuccess) return err;
+  std::lock_guard<std::mutex> turn(bwd_lanes_mutex());
+  BwdLanes* L = nullptr;
+  err = bwd_lanes_for_device(&L);
+  if (err == cudaSuccess) err = cudaEventRecord(L->fork, stream);
+  for (int k = 0; k < NKEYS - 1 && err == cudaSuccess; ++k) err = cudaStreamWaitEvent(L->side[k], L->fork, 0);
   static_for_host<0, NCH>([&](auto Cc) {
-    if (err == cudaSuccess) err = launch_bwd_chunk<PS, NEED_GY, decltype(Cc)::value>(a, num_sms, stream);
+    constexpr int CH = decltype(Cc)::value;
+    constexpr int lane = PL::P.key[CH] - PL::P.key[0];  // the key's lane; lane 0 is the caller's stream
+    if (err == cudaSuccess)
+      err = launch_bwd_chunk<PS, NEED_GY, CH>(a, num_sms, lane == 0 ? stream : L->side[lane - 1],
+                                              !PL::P.first_of_key[CH]);
   });
+  for (int k = 0; k < NKEYS - 1; ++k) {  // join even after an error, so no lane is left forked
+    cudaError_t e = cudaEventRecord(L->join[k], L->side[k]);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(stream, L->join[k], 0);
+    if (err == cudaSuccess) err = e;
+  }
   return err;
 }
 
