@@ -167,6 +167,11 @@ cgtp_status cgtp_conv_backward_workspace_size(cgtp_plan plan, int n_edges, size_
  * grad_x, grad_w, grad_edge_vec are nullable (not computed when NULL) and
  * overwritten.  grad_edge_vec needs workspace of the size reported by
  * cgtp_conv_backward_workspace_size (device, 256-byte aligned).
+ * Streams: the launches of different l1 blocks run on side streams of the
+ * library, forked from `stream` with an event and joined back before the call
+ * returns, so the call is ordered on `stream` like a single launch.  The first
+ * call on a device creates those streams and events: make it before any
+ * stream capture.
  * ------------------------------------------------------------------------- */
 cgtp_status cgtp_conv_backward(cgtp_plan plan, int n_nodes, int n_edges,
                                const int* csc_ptr, const int* csc_edge, const int* csc_dst,
@@ -228,7 +233,10 @@ cgtp_status cgtp_uvw_forward_workspace_size(cgtp_plan plan, int n_nodes, int mul
  * mult_out must be multiples of 4 (CGTP_ERR_UNSUPPORTED otherwise, and when
  * the library was built without the CUTLASS headers).  workspace: device,
  * 256-byte aligned, of the size cgtp_uvw_forward_workspace_size reports
- * (CGTP_ERR_WORKSPACE otherwise).
+ * (CGTP_ERR_WORKSPACE otherwise).  The GEMMs of different l3 blocks run on
+ * side streams of the library, forked from `stream` and joined back before
+ * the call returns; the first call on a device creates them (make it before
+ * any stream capture).
  * ------------------------------------------------------------------------- */
 cgtp_status cgtp_uvw_forward(cgtp_plan plan, int n_nodes, int n_edges, const int* row_ptr,
                              const int* col, const float* edge_vec, const float* x, const float* w,
@@ -249,7 +257,8 @@ cgtp_status cgtp_uvw_backward_workspace_size(cgtp_plan plan, int n_nodes, int n_
  * grad_x [n_nodes][(lmax_in+1)^2][mult], grad_w [n_edges][n_paths][mult],
  * grad_edge_vec [n_edges][3].  Every output is nullable (not computed) and
  * overwritten.  Needs both graph views; workspace as reported by
- * cgtp_uvw_backward_workspace_size (device, 256-byte aligned).
+ * cgtp_uvw_backward_workspace_size (device, 256-byte aligned).  Side streams
+ * as in cgtp_uvw_forward.
  * ------------------------------------------------------------------------- */
 cgtp_status cgtp_uvw_backward(cgtp_plan plan, int n_nodes, int n_edges, const int* row_ptr,
                               const int* col, const int* csc_ptr, const int* csc_edge,
