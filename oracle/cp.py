@@ -19,6 +19,9 @@ minimising the Frobenius norm between the exact and the approximate product
 on batches of standard-normal inputs.  The reply to reviewer S6y1 on the
 low-rank structure bounds the rank of the CG tensor by (L+1)^4.
 
+The same reply (on Figure 3) reports the surrogate's SO(3)-equivariance error
+against its rank; ``equivariance_error`` measures it for given factors.
+
 Readings (the pages fix none of these):
 
 * R-cp1: the exact map is the plan's channelwise CG product with unit path
@@ -42,6 +45,7 @@ import numpy as np
 from .cg import paths
 from .conv import path_nonzeros
 from .tp import tp_forward
+from .wigner import block_rotation, random_rotation
 
 
 def dims(lmax_in, lmax_sh, lmax_out):
@@ -135,3 +139,22 @@ def batch_loss(A, B, C, lmax_in, lmax_sh, lmax_out, rng, batch):
     Z = _exact_pairs(X, Y, lmax_in, lmax_sh, lmax_out)
     Zc = cp_forward(A, B, C, X[:, :, None], Y[:, :, None])[:, :, 0]
     return float(np.mean(np.sum((Z - Zc) ** 2, axis=1)))
+
+
+def equivariance_error(A, B, C, lmax_in, lmax_sh, lmax_out, rng, n_rot=8, batch=64):
+    """Relative SO(3)-equivariance error of the CP map: for Haar-random rotations
+    R with block Wigner-D matrices D_in, D_sh, D_out,
+    ||CP(D_in x, D_sh y) - D_out CP(x, y)|| / ||CP(x, y)|| over N(0,1) pairs
+    (zero for any exactly equivariant map, such as the exact CG product)."""
+    d1, d2, _ = dims(lmax_in, lmax_sh, lmax_out)
+    num = den = 0.0
+    for _ in range(n_rot):
+        R = random_rotation(rng)
+        D1, D2, D3 = (block_rotation(l, R) for l in (lmax_in, lmax_sh, lmax_out))
+        x = rng.standard_normal((batch, d1, 1))
+        y = rng.standard_normal((batch, d2, 1))
+        z = cp_forward(A, B, C, x, y)
+        zr = cp_forward(A, B, C, np.einsum("ab,nbu->nau", D1, x), np.einsum("ab,nbu->nau", D2, y))
+        num += float(np.sum((zr - np.einsum("ab,nbu->nau", D3, z)) ** 2))
+        den += float(np.sum(z ** 2))
+    return float(np.sqrt(num / den))

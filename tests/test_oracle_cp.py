@@ -3,8 +3,9 @@ the exact tensor reproduce the oracle's exact edge-free product, the dot-product
 path's closed form in the dense tensor, the adjoints against Euler's identity
 for a map linear in each argument and against central differences, and the
 batch least-squares fit against exactly representable tensors, the
-Eckart-Young bound of a matrix-shaped tensor, and the expected N(0,1) batch
-loss = squared Frobenius distance."""
+Eckart-Young bound of a matrix-shaped tensor, the expected N(0,1) batch
+loss = squared Frobenius distance, and the equivariance error (zero for the
+exact factorisation, shrinking with the fit's error)."""
 import numpy as np
 import pytest
 
@@ -119,3 +120,19 @@ def test_batch_loss_estimates_the_frobenius_distance():
     frob2 = float(np.sum((M - cp.cp_tensor(A, B, C)) ** 2))
     est = cp.batch_loss(A, B, C, *L, np.random.default_rng(10), 40000)
     assert abs(est - frob2) <= 0.03 * frob2
+
+
+def test_equivariance_error_of_exact_and_fitted_factors():
+    """The exact factorisation is equivariant to rounding; random factors are
+    not; a fit's equivariance error shrinks with its Frobenius error (both vanish
+    together), here at (1,1,1) ranks 6 and 10."""
+    L = (1, 1, 1)
+    rng = np.random.default_rng(20)
+    assert cp.equivariance_error(*_exact_factors(L), *L, rng) <= 1e-13
+    A, B, C, _, _, _ = _random_problem(L, 6, 21)
+    assert cp.equivariance_error(A, B, C, *L, rng) > 0.1
+    e6 = cp.equivariance_error(*cp.fit_als(*L, 6, np.random.default_rng(22)), *L, rng)
+    f10 = cp.fit_als(*L, 10, np.random.default_rng(23))
+    e10 = cp.equivariance_error(*f10, *L, rng)
+    assert e10 < e6
+    assert e10 <= 4 * cp.rel_error(*f10, *L) + 1e-12
