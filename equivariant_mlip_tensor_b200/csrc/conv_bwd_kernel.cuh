@@ -1,0 +1,657 @@
+// CGTP convolution backward, node-centric over sources (CSC), for sm_100a:
+// the one kernel template every backward variant of the library is built
+// from.
+//
+// For edge e = (j -> i) with T_e^p[m1][m3] = sum_m2 C^p[m1,m2,m3] Y_e[l2,m2]:
+//   h_p[m1][u]      = sum_m3 T_e^p[m1][m3] g[i][l3,m3][u]
+//   grad_x[j][l1,m1][u] += W_e[p][u] h_p[m1][u]
+//   grad_W[e][p][u] = sum_m1 x[j][l1,m1][u] h_p[m1][u]
+//   grad_Y[e][l2,m2] = sum_p sum_{m1,m3} C^p[m1,m2,m3] sum_u W_e[p][u] x[j][l1,m1][u] g[i][l3,m3][u]
+// (the adjoints of the bilinear convolution; cf. the closed-form gradients
+// of a bilinear tensor product in "Tensor Decomposition Networks ...",
+// reply to reviewer S6y1, and the derivative computation of "LunaTP ...",
+// abstract).
+//
+// A group of G lanes owns one (source node j, channel slice); it keeps x[j]
+// and the grad_x[j] accumulator in registers for the whole CSC row, so W is
+// read once, grad_W is written once and grad_x needs no atomics.  grad_Y is
+// reduced over the group's channels through shared memory and written, per
+// channel slice, to a workspace [slices][E][NS]; sh_backward then sums the
+// slices and applies the harmonic Jacobian to give grad_edge_vec.
+//
+// Variants (compile-time flags VAR):
+//  - kVarExt: per-edge harmonics given by the caller and results added onto
+//    the outputs (the double backward's first-order passes);
+//  - kVarPerPath: grad_out holds one gradient block per path (the per-path
+//    message layout of the fully connected convolution);
+//  - kVarGyOnly: only the harmonic gradient (no grad_x, no grad_W, and none
+//    of the T^T g products they need);
+//  - kVarWShared: one weight row per edge shared by every path; grad_w[e] is
+//    the sum over paths (chunks then run in plain stream order, each adding
+//    onto the row the previous chunks wrote).
+//
+// Include after CGTP_DEFINE_CONSTANT_TABLES, conv_common.cuh, vec2.cuh and
+// sh.cuh.
+#pragma once
+
+namespace cgtp {
+
+enum : int { kVarExt = 1, kVarPerPath = 2, kVarGyOnly = 4, kVarWShared = 8 };
+
+namespace {
+
+// Warps per block, persistent grid or one group of lanes per item, and the
+// shared-memory budget per warp (floats) that sizes the edge batch (as in
+// the forward: one-warp blocks let the block scheduler balance the rows).
+#ifndef CGTP_BWD_WARPS
+#define CGTP_BWD_WARPS 1
+#endif
+#ifndef CGTP_BWD_PERSISTENT
+#define CGTP_BWD_PERSISTENT 0
+#endif
+#ifndef CGTP_BWD_BATCH_FLOATS
+#define CGTP_BWD_BATCH_FLOATS 6144
+#endif
+#ifndef CGTP_BWD_MAX_BATCH
+#define CGTP_BWD_MAX_BATCH 16
+#endif
+#ifndef CGTP_BWD_MINB
+#define CGTP_BWD_MINB 0
+#endif
+constexpr int kBwdThreads = 32 * CGTP_BWD_WARPS;
+#if CGTP_BWD_MINB > 0
+#define CGTP_BWD_BOUNDS __launch_bounds__(kBwdThreads, CGTP_BWD_MINB)
+#else
+#define CGTP_BWD_BOUNDS __launch_bounds__(kBwdThreads)
+#endif
+// Channels per lane (float4: measured faster than 2 at every shape with
+// one-warp blocks and budgeted chunks).
+#ifndef CGTP_BWD_VEC
+#define CGTP_BWD_VEC 4
+#endif
+constexpr int kBwdVec = CGTP_BWD_VEC;
+// Programmatic dependent launch between the chunks of one backward call
+// (1) or plain stream order (0).
+#ifndef CGTP_BWD_PDL
+#define CGTP_BWD_PDL 1
+#endif
+
+// Unrolled instructions per edge and lane allowed in one backward launch.
+#ifndef CGTP_BWD_BUDGET
+#define CGTP_BWD_BUDGET 1100
+#endif
+#ifndef CGTP_BWD_BUDGET_L3
+#define CGTP_BWD_BUDGET_L3 800  // l = 3 chunks carry more registers per path
+#endif
+template <class PS>
+constexpr int bwd_budget() {
+  return PS::LI >= 3 || PS::LO >= 3 ? CGTP_BWD_BUDGET_L3 : CGTP_BWD_BUDGET;
+}
+
+template <class PS, bool NEED_GY>
+using BwdPlan = Plan<PS, kByL1, kBwdVec, NEED_GY, bwd_budget<PS>()>;
+
+template <class PS, class GR>
+constexpr unsigned touched_sh_mask() {
+  unsigned m = 0;
+  for (int k = 0; k < GR::D.n; ++k) {
+    const int l2 = PS::D.l2[GR::D.path[k]];
+    for (int b = l2 * l2; b < (l2 + 1) * (l2 + 1); ++b) m |= 1u << b;
+  }
+  return m;
+}
+
+// Per-path output gradients: staged rows of path K of the group start at
+// pp_rowoff(K) (each path has its own 2 l3 + 1 rows).
+template <class PS, class GR>
+constexpr int pp_rowoff(int K) {
+  int r = 0;
+  for (int k = 0; k < K; ++k) r += 2 * PS::D.l3[GR::D.path[k]] + 1;
+  return r;
+}
+
+// Staged rows per edge: weight rows (one per path, or the one shared row)
+// and output-gradient rows (the chunk's l3 range, or every path's own block).
+template <class PS, class GR, int VAR>
+constexpr int bwd_staged_rows() {
+  return ((VAR & kVarWShared) ? 1 : GR::NP) + ((VAR & kVarPerPath) ? pp_rowoff<PS, GR>(GR::NP) : GR::NROW);
+}
+
+// Shared memory (floats), the same functions on both sides of the launch:
+// per group of lanes BT edges of T matrices, two pipeline stages and two
+// index arrays of BT ints rounded up to a float4; after all groups, one
+// grad_Y reduction buffer of NS rows of G + 4 floats per group.
+__host__ __device__ constexpr int bwd_group_floats(int BT, int nt, int stage_floats) {
+  return BT * nt + 2 * stage_floats + 2 * ((BT + 3) & ~3);
+}
+__host__ __device__ constexpr int bwd_red_floats(int ns, int G) { return ns * (G + 4); }
+
+// One edge of the CSC row, the paths of one group (l1 = GR's value).  Per
+// path, with h[m1] = sum_m3 T[m1][m3] g[m3] (one pass over the structural
+// nonzeros of T):
+//   grad_x[m1] += W h[m1],   grad_W = sum_m1 x[m1] h[m1],
+// and, for grad_Y, the channel sums sum_u W x[m1] g[m3] of every T entry
+// contracted with the CG coefficients.  Paths are visited in (l2, ...) order
+// so that only one l2 block of the grad_Y partial is live at a time; each
+// finished block goes to this lane's column of the shared reduction buffer
+// (gyrow, row stride rs).  The edge's weight rows and its destination's
+// output-gradient rows come from this lane's pipeline stage.
+template <class PS, class GR, int VEC, bool NEED_GY, int VAR>
+__device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const float* __restrict__ stage, int rowf,
+                                         const float (&xr)[GR::NOWN][VEC], float* __restrict__ gwrow, bool acc, int mult,
+                                         float (&gx)[GR::NOWN][VEC], float* __restrict__ gyrow, int rs) {
+  constexpr bool PP = (VAR & kVarPerPath) != 0, HX = (VAR & kVarGyOnly) == 0, WSH = (VAR & kVarWShared) != 0;
+  constexpr int NW = WSH ? 1 : GR::NP;  // staged weight rows
+  float gy[PS::NS];
+  float gws[VEC];  // WSH: grad of the shared weight row, summed over this chunk's paths
+#pragma unroll
+  for (int c = 0; c < VEC; ++c) gws[c] = 0.f;
+  static_for<0, GR::NP>([&](auto Kc) {
+    constexpr int K = decltype(Kc)::value;
+    constexpr int P = GR::D.path[K];
+    constexpr int l1 = PS::D.l1[P], l3 = PS::D.l3[P];
+    [[maybe_unused]] constexpr int l2 = PS::D.l2[P];
+    constexpr int tb = GR::D.lt[K], tc = PS::D.tcount[P];
+    // staged row of grad_out[l3, m3 = -l3] (of this path's own rows when PP)
+    constexpr int g0 = NW + (PP ? pp_rowoff<PS, GR>(K) : l3 * l3 - GR::D.rlo);
+    if constexpr (NEED_GY && GR::D.first_l2[K]) {
+#pragma unroll
+      for (int m2 = 0; m2 < 2 * l2 + 1; ++m2) gy[l2 * l2 + m2] = 0.f;
+    }
+    float wv[VEC];
+    VecIO<VEC>::lds(wv, stage + (WSH ? 0 : K) * rowf);
+    float gv[2 * l3 + 1][VEC], h[2 * l1 + 1][VEC];
+#pragma unroll
+    for (int m3 = 0; m3 < 2 * l3 + 1; ++m3) VecIO<VEC>::lds(gv[m3], stage + (g0 + m3) * rowf);
+#pragma unroll
+    for (int m1 = 0; m1 < 2 * l1 + 1; ++m1)
+#pragma unroll
+      for (int c = 0; c < VEC; ++c) h[m1][c] = 0.f;
+    [[maybe_unused]] float xw[2 * l1 + 1][VEC];  // W x, for the grad_Y channel sums
+    if constexpr (NEED_GY) {
+#pragma unroll
+      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) vmul<VEC>(xw[m1], wv, xr[m1]);
+    }
+    static_for<0, (tc + 3) / 4>([&](auto Qc) {
+      constexpr int q = decltype(Qc)::value;
+      const float4 v4 = *reinterpret_cast<const float4*>(T + tb + 4 * q);
+      const float tv4[4] = {v4.x, v4.y, v4.z, v4.w};
+      static_for<0, 4>([&](auto Rc) {
+        constexpr int k = 4 * q + decltype(Rc)::value;
+        if constexpr (k < tc) {
+          constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
+          const float tv = tv4[decltype(Rc)::value];
+          if constexpr (HX) axpy<VEC>(h[m1 + l1], tv, gv[m3 + l3]);
+          if constexpr (NEED_GY) {
+            const float av = vdot<VEC>(xw[m1 + l1], gv[m3 + l3]);
+            static_for<0, 2 * l2 + 1>([&](auto M2c) {
+              constexpr int m2 = decltype(M2c)::value - l2;
+              if constexpr (cg_allowed(l1, l2, l3, m1, m2, m3)) {
+                gy[l2 * l2 + l2 + m2] = fmaf(c_cg[table_index(l1, l2, l3, m1, m2, m3)], av, gy[l2 * l2 + l2 + m2]);
+              }
+            });
+          }
+        }
+      });
+    });
+    if constexpr (HX) {
+      if constexpr (WSH) {
+#pragma unroll
+        for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) {
+          vfma<VEC>(gx[m1], wv, h[m1]);
+          vfma<VEC>(gws, xr[m1], h[m1]);
+        }
+      } else {
+        float gw[VEC];
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) gw[c] = 0.f;
+#pragma unroll
+        for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) {
+          vfma<VEC>(gx[m1], wv, h[m1]);
+          vfma<VEC>(gw, xr[m1], h[m1]);
+        }
+        if (gwrow != nullptr) {
+          if (acc) {
+            float prev[VEC];
+            VecIO<VEC>::ld(prev, gwrow + P * mult);
+#pragma unroll
+            for (int c = 0; c < VEC; ++c) gw[c] += prev[c];
+          }
+          VecIO<VEC>::st_stream(gwrow + P * mult, gw);
+        }
+      }
+    }
+    if constexpr (NEED_GY && GR::D.last_l2[K]) {
+#pragma unroll
+      for (int m2 = 0; m2 < 2 * l2 + 1; ++m2) gyrow[(l2 * l2 + m2) * rs] = gy[l2 * l2 + m2];
+    }
+  });
+  if constexpr (HX && WSH) {
+    if (gwrow != nullptr) {
+      if (acc) {  // an earlier chunk of this call wrote the row: add onto it
+        float prev[VEC];
+        VecIO<VEC>::ld(prev, gwrow);
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) gws[c] += prev[c];
+      }
+      VecIO<VEC>::st_stream(gwrow, gws);
+    }
+  }
+}
+
+// One launch per chunk (paths of one l1 block): grad_x rows of that block
+// (written by the block's first chunk, accumulated by the others), grad_W
+// of the chunk's paths and a partial grad_Y over them.
+template <class PS, bool NEED_GY, int CH, int KMULT, int VAR>
+__global__ void CGTP_BWD_BOUNDS
+conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt) {
+  constexpr int VEC = kBwdVec;
+  constexpr bool EXT = (VAR & kVarExt) != 0, PP = (VAR & kVarPerPath) != 0;
+  constexpr bool HX = (VAR & kVarGyOnly) == 0, WSH = (VAR & kVarWShared) != 0;
+  // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x VEC
+  // channels, so every row offset below folds into an immediate.
+  const int mult = KMULT ? KMULT : a.mult;
+  const int lg_G = KMULT ? 5 : lg_G_rt;
+  const int S = KMULT ? KMULT / (32 * VEC) : S_rt;
+  const int slice_base = KMULT ? CH * S : slice_base_rt;
+  using GR = ChunkGrp<PS, BwdPlan<PS, NEED_GY>, CH, kByL1>;
+  constexpr int L1 = GR::KEY;
+  constexpr int NI = PS::NI, NO = PS::NO, NS = PS::NS, NR = GR::NOWN, NT = GR::NT;
+  constexpr int NW = WSH ? 1 : GR::NP;                       // staged weight rows
+  constexpr int NROWS = bwd_staged_rows<PS, GR, VAR>();
+  constexpr unsigned GY_MASK = touched_sh_mask<PS, GR>();  // harmonics this chunk's paths reach
+  extern __shared__ float4 smem_f4[];
+  float* smem = reinterpret_cast<float*>(smem_f4);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int G = 1 << lg_G, gpw = 32 >> lg_G;
+  const int grp = lane >> lg_G, gl = lane & (G - 1);
+  const int rowf = G * VEC;
+  const int stage_floats = NROWS * rowf;
+  const int group_floats = bwd_group_floats(BT, NT, stage_floats);
+  float* Tg = smem + (warp * gpw + grp) * group_floats;
+  float* St = Tg + BT * NT;
+  int* Eg = reinterpret_cast<int*>(St + 2 * stage_floats);
+  int* Ig = Eg + ((BT + 3) & ~3);
+  // grad_Y reduction buffer, per group of lanes: NS rows (one per harmonic)
+  // of G lane partials, row stride rs = G + 4 (float4 aligned, and rows read
+  // by the 8 lanes of one 128-bit access phase fall in distinct banks)
+  const int rs = G + 4;
+  float* red = smem + (kBwdThreads / 32) * gpw * group_floats + (warp * gpw + grp) * bwd_red_floats(NS, G);
+
+  // The next chunk of this call may start on SMs this grid leaves idle: no
+  // chunk reads what another writes, except a chunk that adds onto an
+  // earlier chunk's grad_x rows, and that one waits for it below.
+  grid_dependents_launch();
+  if (a.abort_flag != nullptr && (*a.abort_flag & kGraphUnsafeBits)) {  // checked mode, invalid graph
+    grid_dependency_wait();
+    return;
+  }
+  const long long n_items = (long long)a.n_nodes * S;
+  const long long warps_total = (long long)gridDim.x * (kBwdThreads / 32);
+  for (long long base = ((long long)blockIdx.x * (kBwdThreads / 32) + warp) * gpw; base < n_items;
+       base += warps_total * gpw) {
+    const long long item = base + grp;
+    const bool active = item < n_items;
+    const long long node = active ? item / S : 0;
+    const int slice = active ? int(item % S) : 0;
+    const int c0 = (slice * G + gl) * VEC;
+    int k0 = 0, k1 = 0;
+    if (active) {
+      k0 = __ldg(a.csc_ptr + node);
+      k1 = __ldg(a.csc_ptr + node + 1);
+    }
+    const int maxdeg = __reduce_max_sync(0xffffffffu, k1 - k0);
+    float xr[NR][VEC], gx[NR][VEC];
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      if (active) VecIO<VEC>::ld(xr[r], a.x + (node * NI + L1 * L1 + r) * mult + c0);
+      else {
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) xr[r][c] = 0.f;
+      }
+#pragma unroll
+      for (int c = 0; c < VEC; ++c) gx[r][c] = 0.f;
+    }
+
+    // copies of edge slot k of the current batch into stage s (this lane's channels only)
+    auto issue = [&](int b0, int k, int s) {
+      if (!(active && k0 + b0 + k < k1)) return;
+      float* dst = St + s * stage_floats + gl * VEC;
+      if constexpr (WSH) {
+        VecIO<VEC>::cp_async(dst, a.w + (long long)Eg[k] * mult + c0);
+      } else {
+        const float* wrow = a.w + (long long)Eg[k] * PS::NP * mult + c0;
+        static_for<0, GR::NP>([&](auto Kc) {
+          constexpr int K = decltype(Kc)::value;
+          constexpr int P = GR::D.path[K];
+          VecIO<VEC>::cp_async(dst + K * rowf, wrow + P * mult);
+        });
+      }
+      if constexpr (PP) {
+        // block l3 of the per-path layout: [node][m3][rank][u]
+        static_for<0, GR::NP>([&](auto Kc) {
+          constexpr int K = decltype(Kc)::value;
+          constexpr int P = GR::D.path[K];
+          constexpr int l3 = PS::D.l3[P], n3 = 2 * l3 + 1;
+          constexpr int npk = l3_count<PS>(l3), rank = l3_rank<PS>(P), pre = l3_prefix_rows<PS>(l3);
+          constexpr int ro = pp_rowoff<PS, GR>(K);
+          const float* base = a.grad_out + (long long)a.n_nodes * mult * pre +
+                              ((long long)Ig[k] * n3 * npk + rank) * mult + c0;
+#pragma unroll
+          for (int m3 = 0; m3 < n3; ++m3)
+            VecIO<VEC>::cp_async(dst + (NW + ro + m3) * rowf, base + (long long)m3 * npk * mult);
+        });
+      } else {
+        constexpr int rlo = GR::D.rlo;
+        const float* grow = a.grad_out + ((long long)Ig[k] * NO + rlo) * mult + c0;
+#pragma unroll
+        for (int r = 0; r < GR::NROW; ++r) VecIO<VEC>::cp_async(dst + (NW + r) * rowf, grow + r * mult);
+      }
+    };
+
+    for (int b0 = 0; b0 < maxdeg; b0 += BT) {
+      for (int k = gl; k < BT; k += G) {
+        const int kk = k0 + b0 + k;
+        if (active && kk < k1) {
+          const int e = __ldg(a.csc_edge + kk);
+          float Y[NS];
+          edge_sh<PS::LS>(EXT ? a.sh : nullptr, a.edge_vec, e, Y);
+          compute_T_grp<PS, GR>(Y, Tg + k * NT);
+          Eg[k] = e;
+          Ig[k] = __ldg(a.csc_dst + kk);
+        }
+      }
+      __syncwarp();
+      const int nb = min(BT, maxdeg - b0);
+      issue(b0, 0, 0);
+      cp_async_commit();
+      for (int k = 0; k < nb; ++k) {
+        if (k + 1 < nb) issue(b0, k + 1, (k + 1) & 1);
+        cp_async_commit();
+        cp_async_wait<1>();  // this lane's copies of edge k have landed
+        const bool valid = active && (k0 + b0 + k) < k1;
+        int e = 0;
+        if (valid) {
+          e = Eg[k];
+          float* gwrow = nullptr;
+          if (HX && a.grad_w != nullptr) gwrow = a.grad_w + (long long)e * (WSH ? 1 : PS::NP) * mult + c0;
+          // WSH: every chunk after the first adds onto the row (plain stream order)
+          const bool acc = (WSH && CH > 0) || (EXT && a.accumulate != 0);
+          bwd_edge<PS, GR, VEC, NEED_GY, VAR>(Tg + k * NT, St + (k & 1) * stage_floats + gl * VEC, rowf, xr, gwrow,
+                                               acc, mult, gx, red + gl, rs);
+        }
+        if constexpr (NEED_GY) {
+          __syncwarp();
+          if (valid) {
+            float* dst = a.grad_sh + ((long long)(slice_base + slice) * a.n_edges + e) * NS;
+            for (int b = gl; b < NS; b += G) {  // column sums; harmonics the chunk never reaches get 0
+              float v = 0.f;
+              if ((GY_MASK >> b) & 1u) {
+                const float* row = red + b * rs;
+                if (G % 4 == 0) {
+                  float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                  for (int r = 0; r < G; r += 4) {
+                    const float4 q4 = *reinterpret_cast<const float4*>(row + r);
+                    s4.x += q4.x;
+                    s4.y += q4.y;
+                    s4.z += q4.z;
+                    s4.w += q4.w;
+                  }
+                  v = (s4.x + s4.y) + (s4.z + s4.w);
+                } else {
+                  for (int r = 0; r < G; ++r) v += row[r];
+                }
+              }
+              dst[b] = v;
+            }
+          }
+          __syncwarp();
+        }
+      }
+      __syncwarp();
+    }
+    if (HX && active && a.grad_x != nullptr) {
+      if (!GR::FIRST || (EXT && a.accumulate)) {
+        // rows of an l1 block that an earlier chunk of this call wrote (wait
+        // for that grid, the preceding launch), or the caller's values
+        if constexpr (!GR::FIRST) grid_dependency_wait();
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          float prev[VEC];
+          VecIO<VEC>::ld(prev, a.grad_x + (node * NI + L1 * L1 + r) * mult + c0);
+#pragma unroll
+          for (int c = 0; c < VEC; ++c) gx[r][c] += prev[c];
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < NR; ++r) VecIO<VEC>::st(a.grad_x + (node * NI + L1 * L1 + r) * mult + c0, gx[r]);
+    }
+  }
+  // Complete only after the preceding launch: a grid launched with
+  // programmatic stream serialization that never waited (no grad_x rows to
+  // add onto, or no grad_x at all) could otherwise complete before its
+  // predecessor, and what the stream runs after the chain would overlap a
+  // launch that is still running.  A no-op in plain stream order.
+  grid_dependency_wait();
+}
+
+// grad_edge_vec[e] (= or +=) (dY_e/dr_e)^T sum_s grad_sh[s][e]
+template <int LS>
+__global__ void sh_backward_kernel(int n_edges, int S, const float* __restrict__ edge_vec,
+                                   const float* __restrict__ grad_sh, float* __restrict__ grad_edge_vec, int add) {
+  constexpr int NS = (LS + 1) * (LS + 1);
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n_edges;
+       e += (long long)gridDim.x * blockDim.x) {
+    float g[NS];
+#pragma unroll
+    for (int b = 0; b < NS; ++b) g[b] = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float* src = grad_sh + ((long long)s * n_edges + e) * NS;
+#pragma unroll
+      for (int b = 0; b < NS; ++b) g[b] += src[b];
+    }
+    Dual3 Y[NS];
+    sh_grad_of_vec<LS>(edge_vec[3 * e], edge_vec[3 * e + 1], edge_vec[3 * e + 2], Y);
+    float d0 = 0.f, d1 = 0.f, d2 = 0.f;
+#pragma unroll
+    for (int b = 0; b < NS; ++b) {
+      d0 = fmaf(g[b], Y[b].d0, d0);
+      d1 = fmaf(g[b], Y[b].d1, d1);
+      d2 = fmaf(g[b], Y[b].d2, d2);
+    }
+    if (add) {
+      d0 += grad_edge_vec[3 * e];
+      d1 += grad_edge_vec[3 * e + 1];
+      d2 += grad_edge_vec[3 * e + 2];
+    }
+    grad_edge_vec[3 * e] = d0;
+    grad_edge_vec[3 * e + 1] = d1;
+    grad_edge_vec[3 * e + 2] = d2;
+  }
+}
+
+// grad_edge_vec[e] (= or +=) sum_b G_b (d2Y_b/dr2) q_e with G = sum_s grad_sh[s][e]:
+// the second-order term of the double backward (q = the cotangent of grad_edge_vec).
+template <int LS>
+__global__ void sh_backward_hess_kernel(int n_edges, int S, const float* __restrict__ edge_vec,
+                                        const float* __restrict__ grad_sh, const float* __restrict__ q,
+                                        float* __restrict__ grad_edge_vec, int add) {
+  constexpr int NS = (LS + 1) * (LS + 1);
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n_edges;
+       e += (long long)gridDim.x * blockDim.x) {
+    float g[NS];
+#pragma unroll
+    for (int b = 0; b < NS; ++b) g[b] = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float* src = grad_sh + ((long long)s * n_edges + e) * NS;
+#pragma unroll
+      for (int b = 0; b < NS; ++b) g[b] += src[b];
+    }
+    HDual Y[NS];
+    sh_hess_of_vec<LS>(edge_vec[3 * e], edge_vec[3 * e + 1], edge_vec[3 * e + 2], q[3 * e], q[3 * e + 1],
+                       q[3 * e + 2], Y);
+    float d0 = 0.f, d1 = 0.f, d2 = 0.f;
+#pragma unroll
+    for (int b = 0; b < NS; ++b) {
+      d0 = fmaf(g[b], Y[b].d0.e, d0);
+      d1 = fmaf(g[b], Y[b].d1.e, d1);
+      d2 = fmaf(g[b], Y[b].d2.e, d2);
+    }
+    if (add) {
+      d0 += grad_edge_vec[3 * e];
+      d1 += grad_edge_vec[3 * e + 1];
+      d2 += grad_edge_vec[3 * e + 2];
+    }
+    grad_edge_vec[3 * e] = d0;
+    grad_edge_vec[3 * e + 1] = d1;
+    grad_edge_vec[3 * e + 2] = d2;
+  }
+}
+
+// channel lanes per group (G) and channel slices (S) of the backward
+inline void bwd_geometry(int mult, int& G, int& lg_G, int& S) { lane_geometry(mult, kBwdVec, G, lg_G, S); }
+
+// One partial grad_Y per (chunk, channel slice).
+template <class PS>
+int bwd_slices(int mult) {
+  int G, lg_G, S;
+  bwd_geometry(mult, G, lg_G, S);
+  return S * BwdPlan<PS, true>::N;
+}
+
+// Launch chunk CH of variant VAR (the double backward's harmonics input or
+// accumulate mode selects the kExt kernel at run time).
+template <class PS, bool NEED_GY, int CH, int VAR>
+cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t stream, bool pdl) {
+  using GR = ChunkGrp<PS, BwdPlan<PS, NEED_GY>, CH, kByL1>;
+  int G, lg_G, S;
+  bwd_geometry(a.mult, G, lg_G, S);
+  const int gpw = 32 / G;
+  const int stage_floats = bwd_staged_rows<PS, GR, VAR>() * G * kBwdVec;
+  const int BT = pick_batch(gpw, GR::NT, stage_floats, CGTP_BWD_BATCH_FLOATS, CGTP_BWD_MAX_BATCH);
+  // the kernel's indexing reaches gpw groups x warps of group_floats, then
+  // (with NEED_GY) as many reduction buffers
+  const size_t groups = (size_t)gpw * (kBwdThreads / 32);
+  const size_t smem = sizeof(float) * (groups * bwd_group_floats(BT, GR::NT, stage_floats) +
+                                       (NEED_GY ? groups * bwd_red_floats(PS::NS, G) : 0));
+  cudaError_t err = check_smem(smem);
+  if (err != cudaSuccess) return err;
+  const long long items = (long long)a.n_nodes * S;
+  const long long blocks = (items + (long long)groups - 1) / (long long)groups;
+  const bool ext = a.sh != nullptr || a.accumulate;
+  if (ext && (VAR & (kVarPerPath | kVarWShared))) return cudaErrorInvalidValue;  // not built
+  // the compile-time multiplicity for the common case; the per-path layout
+  // keeps the run-time one
+  constexpr bool kAllow128 = (VAR & kVarPerPath) == 0;
+  auto kern = ext ? conv_bwd_kernel<PS, NEED_GY, CH, 0, VAR | kVarExt>
+              : (kAllow128 && a.mult == 128) ? conv_bwd_kernel<PS, NEED_GY, CH, kAllow128 ? 128 : 0, VAR>
+                                             : conv_bwd_kernel<PS, NEED_GY, CH, 0, VAR>;
+  err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  long long cap = 0x7fffffffLL;  // the kernel loops over items beyond the grid
+  if (CGTP_BWD_PERSISTENT) {
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBwdThreads, smem);
+    if (err != cudaSuccess) return err;
+    cap = (long long)num_sms * (per_sm < 1 ? 1 : per_sm);
+  }
+  long long nb = blocks > cap ? cap : blocks;
+  if (nb < 1) nb = 1;
+  return launch_kernel(kern, dim3((unsigned)nb), dim3(kBwdThreads), smem, stream, CGTP_BWD_PDL && pdl, a, lg_G,
+                       S, BT, CH * S);
+}
+
+// grad_x blocks that no path reaches (l1 with no path) are zero.
+template <class PS>
+cudaError_t zero_unreached_grad_x(const ConvBwdArgs& a, cudaStream_t stream) {
+  if (a.grad_x == nullptr) return cudaSuccess;
+  cudaError_t err = cudaSuccess;
+  static_for_host<0, PS::LI + 1>([&](auto Lc) {
+    constexpr int l1 = decltype(Lc)::value;
+    constexpr bool reached = [] {
+      for (int p = 0; p < PS::D.np; ++p)
+        if (PS::D.l1[p] == l1) return true;
+      return false;
+    }();
+    if (!reached && err == cudaSuccess)
+      err = cudaMemset2DAsync(a.grad_x + (size_t)l1 * l1 * a.mult, sizeof(float) * PS::NI * a.mult, 0,
+                              sizeof(float) * (2 * l1 + 1) * a.mult, a.n_nodes, stream);
+  });
+  return err;
+}
+
+// Every chunk of variant VAR.  LANES: chunks of different l1 blocks write
+// disjoint outputs (their own grad_x rows, their own paths' grad_W rows,
+// their own grad_Y partial slices), so each l1 block's chunks run on a lane
+// of their own, forked from the caller's stream and joined back before the
+// call's next launch: the latency-bound small blocks then fill the SMs beside
+// the large ones.  Within a lane (and without lanes), a chunk that continues
+// an l1 block overlaps its predecessor through programmatic dependent launch
+// and waits for it before adding to its rows.  Shared-weight chunks all add
+// onto one gradient row per edge, so they run in plain stream order.
+template <class PS, bool NEED_GY, int VAR, bool LANES>
+cudaError_t launch_bwd_chunks(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
+  using PL = BwdPlan<PS, NEED_GY>;
+  constexpr int NCH = PL::N;
+  constexpr int NKEYS = PL::P.key[NCH - 1] - PL::P.key[0] + 1;
+  constexpr bool kPdl = (VAR & kVarWShared) == 0;
+  cudaError_t err = (a.accumulate || (VAR & kVarGyOnly)) ? cudaSuccess : zero_unreached_grad_x<PS>(a, stream);
+  if (err != cudaSuccess) return err;
+  if constexpr (!LANES || NKEYS <= 1 || !kPdl) {
+    static_for_host<0, NCH>([&](auto Cc) {
+      constexpr int CH = decltype(Cc)::value;
+      if (err == cudaSuccess) err = launch_bwd_chunk<PS, NEED_GY, CH, VAR>(a, num_sms, stream, kPdl && CH > 0);
+    });
+    return err;
+  } else {
+    std::lock_guard<std::mutex> turn(side_lanes_mutex(kLanesBwd));
+    SideLanes* L = nullptr;
+    err = side_lanes(kLanesBwd, &L);
+    if (err == cudaSuccess) err = lanes_fork(L, NKEYS - 1, stream);
+    static_for_host<0, NCH>([&](auto Cc) {
+      constexpr int CH = decltype(Cc)::value;
+      constexpr int lane = PL::P.key[CH] - PL::P.key[0];  // the key's lane; lane 0 is the caller's stream
+      if (err == cudaSuccess)
+        err = launch_bwd_chunk<PS, NEED_GY, CH, VAR>(a, num_sms, lane == 0 ? stream : L->side[lane - 1],
+                                                     !PL::P.first_of_key[CH]);
+    });
+    if (L != nullptr) {  // join even after an error, so no lane is left forked
+      const cudaError_t e = lanes_join(L, NKEYS - 1, stream);
+      if (err == cudaSuccess) err = e;
+    }
+    return err;
+  }
+}
+
+// The harmonic Jacobian epilogue: grad_edge_vec from the summed partials
+// (gr_mode 0/1), or the double backward's Hessian-vector term (gr_mode 2/3).
+template <int LS>
+cudaError_t launch_sh_backward(const ConvBwdArgs& a, int slices, int num_sms, cudaStream_t stream) {
+  const int threads = 256;
+  long long nbk = (a.n_edges + threads - 1) / threads;
+  if (nbk > (long long)num_sms * 16) nbk = (long long)num_sms * 16;
+  if (a.gr_mode >= 2) {
+    if (a.gr_dir == nullptr) return cudaErrorInvalidValue;
+    sh_backward_hess_kernel<LS><<<(unsigned)nbk, threads, 0, stream>>>(a.n_edges, slices, a.edge_vec, a.grad_sh,
+                                                                      a.gr_dir, a.grad_edge_vec, a.gr_mode == 2);
+  } else {
+    sh_backward_kernel<LS><<<(unsigned)nbk, threads, 0, stream>>>(a.n_edges, slices, a.edge_vec, a.grad_sh,
+                                                                 a.grad_edge_vec, a.gr_mode == 1);
+  }
+  return cudaGetLastError();
+}
+
+// The whole backward of variant VAR: the chunks (with grad_Y partials when
+// grad_edge_vec is wanted), then the harmonic Jacobian epilogue.
+template <class PS, int VAR, bool LANES>
+cudaError_t launch_bwd_all(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
+  if ((VAR & kVarGyOnly) && (a.grad_edge_vec == nullptr || a.grad_sh == nullptr)) return cudaErrorInvalidValue;
+  if ((VAR & kVarGyOnly) && a.n_edges == 0) return cudaSuccess;
+  const cudaError_t err = a.grad_edge_vec != nullptr ? launch_bwd_chunks<PS, true, VAR, LANES>(a, num_sms, stream)
+                                                     : launch_bwd_chunks<PS, false, VAR, LANES>(a, num_sms, stream);
+  if (err != cudaSuccess || a.grad_edge_vec == nullptr || a.n_edges == 0) return err;
+  return launch_sh_backward<PS::LS>(a, bwd_slices<PS>(a.mult), num_sms, stream);
+}
+
+}  // namespace
+}  // namespace cgtp

@@ -91,6 +91,8 @@ struct Grp {
   static constexpr int NOWN = KIND == kAll ? PS::NO : 2 * V + 1;
   static constexpr int OWN0 = KIND == kAll ? 0 : V * V;    // first own row
   static constexpr bool FIRST = true;                      // initialises its rows
+  static constexpr bool PERPATH = false;  // paths of one l3 summed into one block of rows
+  static constexpr int NPK = 0, PL0 = 0;  // per-path layout only (see PathRowsGrp)
 };
 
 // T^p[m1][m3] = sum_m2 C^p[m1,m2,m3] Y[l2,m2] for the group's paths, packed
@@ -118,6 +120,32 @@ __device__ __forceinline__ void compute_T_grp(const float (&Y)[PS::NS], float* _
   });
 }
 
+// ---- per-path messages (the fully connected convolution) ----
+// The messages of each path are kept apart in blocks by l3: block l3 holds
+// [node][m3][rank][u] for the paths of that l3 in (l2, path number) order
+// (the order in which the chunk planner visits them), and the blocks follow
+// one another in increasing l3.
+template <class PS>
+constexpr int l3_rank(int p) {  // place of path p among the paths of its l3 block
+  int r = 0;
+  for (int q = 0; q < PS::D.np; ++q)
+    if (PS::D.l3[q] == PS::D.l3[p] && (PS::D.l2[q] < PS::D.l2[p] || (PS::D.l2[q] == PS::D.l2[p] && q < p))) ++r;
+  return r;
+}
+template <class PS>
+constexpr int l3_count(int l3) {
+  int n = 0;
+  for (int q = 0; q < PS::D.np; ++q) n += PS::D.l3[q] == l3;
+  return n;
+}
+// rows per node (paths x (2 l3 + 1)) of the blocks before block l3
+template <class PS>
+constexpr int l3_prefix_rows(int l3) {
+  int r = 0;
+  for (int l = 0; l < l3; ++l) r += l3_count<PS>(l) * (2 * l + 1);
+  return r;
+}
+
 // ---- chunks: the launches of a kernel family ----
 // Paths sorted by (key, l2, lexicographic), key = l1 (backward) or l3
 // (forward), are cut into runs with one key value whose unrolled code per
@@ -143,8 +171,11 @@ constexpr int path_cost(int p, int kind, int vec, bool gy) {
          (tc + 3) / 4 + n3 + 2 * n1 * vec + 6;
 }
 
+// max_rows (forward by l3 only): at most this many output rows (sum of
+// 2 l3 + 1 over the chunk's paths), for kernels that keep one block of
+// accumulators per path.
 template <class PS>
-constexpr ChunkPlan make_chunk_plan(int kind, int vec, bool gy, int budget) {
+constexpr ChunkPlan make_chunk_plan(int kind, int vec, bool gy, int budget, int max_rows = 1 << 30) {
   ChunkPlan c{};
   int k = 0;
   const int kmax = kind == kByL1 ? PS::LI : PS::LO;
@@ -155,11 +186,13 @@ constexpr ChunkPlan make_chunk_plan(int kind, int vec, bool gy, int budget) {
   int start = 0;
   while (start < k) {
     const int key = kind == kByL1 ? PS::D.l1[c.order[start]] : PS::D.l3[c.order[start]];
-    int end = start, cost = 0;
+    int end = start, cost = 0, rows = 0;
     while (end < k && (kind == kByL1 ? PS::D.l1[c.order[end]] : PS::D.l3[c.order[end]]) == key) {
       const int pc = path_cost<PS>(c.order[end], kind, vec, gy);
-      if (end > start && cost + pc > budget) break;
+      const int pr = 2 * PS::D.l3[c.order[end]] + 1;
+      if (end > start && (cost + pc > budget || rows + pr > max_rows)) break;
       cost += pc;
+      rows += pr;
       ++end;
     }
     c.key[c.n] = key;
@@ -172,9 +205,9 @@ constexpr ChunkPlan make_chunk_plan(int kind, int vec, bool gy, int budget) {
   return c;
 }
 
-template <class PS, int KIND, int VEC, bool GY, int BUDGET>
+template <class PS, int KIND, int VEC, bool GY, int BUDGET, int MAX_ROWS = (1 << 30)>
 struct Plan {
-  static constexpr ChunkPlan P = make_chunk_plan<PS>(KIND, VEC, GY, BUDGET);
+  static constexpr ChunkPlan P = make_chunk_plan<PS>(KIND, VEC, GY, BUDGET, MAX_ROWS);
   static constexpr int N = P.n;
 };
 
@@ -214,7 +247,24 @@ struct ChunkGrp : Chunk<PS, PL, CH> {
   static constexpr int NROW = D.rhi - D.rlo;
   static constexpr int NOWN = 2 * Base::KEY + 1;
   static constexpr int OWN0 = Base::KEY * Base::KEY;
+  static constexpr bool PERPATH = false;
+  static constexpr int NPK = 0, PL0 = 0;
 };
+
+// Checks a launch's dynamic shared memory against the device's per-block
+// opt-in limit before the attribute is set (a request beyond it is refused
+// here rather than by the launch).
+inline cudaError_t check_smem(size_t smem) {
+  static int limit = -1;  // the same for every B200 in the process
+  if (limit < 0) {
+    int dev = 0, v = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    limit = v;
+  }
+  return smem <= (size_t)limit ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
 
 // Edges per batch: T matrices of BT edges per group of lanes, sized so that a
 // group's shared memory stays near 24 KB.

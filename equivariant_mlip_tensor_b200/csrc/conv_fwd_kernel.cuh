@@ -1,0 +1,404 @@
+// CGTP convolution forward, node-centric over CSR rows, for sm_100a: the one
+// kernel template every forward variant of the library is built from.
+//
+//   out[i][l3,m3][u] = sum_{e in row i} sum_p W_e[p][u] sum_m1 T_e^p[m1][m3] x[j_e][l1,m1][u]
+//   T_e^p[m1][m3]    = sum_m2 C^p[m1,m2,m3] Y_e[l2,m2]
+//
+// ("LunaTP: Enabling Efficient and Scalable Tensor Product for Equivariant
+// MLIPs", abstract: node-centric execution, path-group parallelism and reuse;
+// the kernel below is our own design for the B200.)
+//
+// Mapping.  A group of G lanes (G a power of two <= 32) owns one
+// (row, channel slice) work item; each lane owns 4 consecutive channels.
+// (Optionally one launch per chunk of same-l3 paths.)  The lanes walk the
+// row's edges in batches of BT: first every lane computes the harmonics and
+// the group's packed T matrices of one edge of the batch (channel
+// independent; coefficients are constant-memory operands) into shared
+// memory; then the lanes sweep the batch with a two-stage pipeline: while
+// edge k is computed, each lane's cp.async copies of edge k+1's weight rows
+// (the HBM stream, read once) and of its source's feature rows (L2 resident)
+// land in shared memory.  The output rows accumulate in registers and are
+// written once; there are no atomics.  Loops over paths and over the
+// structural nonzeros of T are unrolled at compile time, so every register
+// index is static.
+//
+// Variants (compile-time):
+//  - WSH: one weight row per edge shared by every path (path stride 0;
+//    "Tensor Decomposition Networks ...", reply to reviewer oXft) instead of
+//    one row per path;
+//  - GR::PERPATH: one block of 2 l3 + 1 output rows per path (the per-path
+//    messages of the fully connected convolution) instead of summing the
+//    paths of one l3.
+//
+// Include after CGTP_DEFINE_CONSTANT_TABLES, conv_common.cuh, vec2.cuh and
+// sh.cuh.
+#pragma once
+
+namespace cgtp {
+namespace {
+
+// Warps per block, whether the grid is persistent (one wave that loops over
+// the work items) or one group of lanes per item, and the shared-memory
+// budget per warp (floats) that sizes the edge batch.  One-warp blocks over
+// one item each let the block scheduler balance rows of unequal degree: an
+// SM takes a new row as soon as any of its warps finishes one.
+#ifndef CGTP_FWD_WARPS
+#define CGTP_FWD_WARPS 1
+#endif
+#ifndef CGTP_FWD_PERSISTENT
+#define CGTP_FWD_PERSISTENT 0
+#endif
+#ifndef CGTP_FWD_BATCH_FLOATS
+#define CGTP_FWD_BATCH_FLOATS 12288
+#endif
+#ifndef CGTP_FWD_MAX_BATCH
+#define CGTP_FWD_MAX_BATCH 16
+#endif
+#ifndef CGTP_FWD_MINB
+#define CGTP_FWD_MINB 1
+#endif
+constexpr int kFwdThreads = 32 * CGTP_FWD_WARPS;
+#if CGTP_FWD_MINB > 0
+#define CGTP_FWD_BOUNDS __launch_bounds__(kFwdThreads, CGTP_FWD_MINB)
+#else
+#define CGTP_FWD_BOUNDS __launch_bounds__(kFwdThreads)
+#endif
+#ifndef CGTP_FWD_VEC
+#define CGTP_FWD_VEC 4
+#endif
+constexpr int kFwdVec = CGTP_FWD_VEC;  // channels per lane
+
+// Stage x rows through the cp.async pipeline (1) or gather them with cached
+// loads after an L2 prefetch (0).
+#ifndef CGTP_FWD_STAGE_X
+#define CGTP_FWD_STAGE_X 1
+#endif
+constexpr bool kStageX = CGTP_FWD_STAGE_X != 0;
+
+// One launch over all paths while their unrolled code per edge and lane stays
+// within CGTP_FWD_SINGLE_MAX instructions; otherwise one launch per chunk of
+// paths with one l3, each within CGTP_FWD_BUDGET (the instruction cache).
+#ifndef CGTP_FWD_SINGLE_MAX
+#define CGTP_FWD_SINGLE_MAX 1600
+#endif
+#ifndef CGTP_FWD_BUDGET
+#define CGTP_FWD_BUDGET 1100
+#endif
+
+// Shared memory of one group of lanes (floats), the same function on both
+// sides of the launch: BT edges of T matrices, two pipeline stages, and BT
+// source indices rounded up to a float4.
+__host__ __device__ constexpr int fwd_stage_floats(int nw, int nrow, int G) {
+  return (nw + (kStageX ? nrow : 0)) * G * kFwdVec;
+}
+__host__ __device__ constexpr int fwd_group_floats(int BT, int nt, int stage_floats) {
+  return BT * nt + 2 * stage_floats + ((BT + 3) & ~3);
+}
+
+// One edge: acc[rows of path K][c] += W[p][c] sum_m1 T[p][m1][m3] x[l1,m1][c] for the group's paths.
+template <class PS, class GR, bool WSH>
+__device__ __forceinline__ void fwd_edge(const float* __restrict__ T, const float* __restrict__ stage, int rowf,
+                                         const float* __restrict__ xg, int mult,
+                                         float (&acc)[GR::NOWN][kFwdVec]) {
+  constexpr int NW = WSH ? 1 : GR::NP;  // staged weight rows
+  float xr[GR::NROW][kFwdVec];
+#pragma unroll
+  for (int r = 0; r < GR::NROW; ++r) {
+    if constexpr (kStageX) VecIO<kFwdVec>::lds(xr[r], stage + (NW + r) * rowf);
+    else VecIO<kFwdVec>::ld(xr[r], xg + r * mult);
+  }
+  float wsh[kFwdVec];
+  if constexpr (WSH) VecIO<kFwdVec>::lds(wsh, stage);  // the one weight row, shared by every path
+  static_for<0, GR::NP>([&](auto Kc) {
+    constexpr int K = decltype(Kc)::value;
+    constexpr int P = GR::D.path[K];
+    constexpr int l1 = PS::D.l1[P], l3 = PS::D.l3[P];
+    constexpr int tc = PS::D.tcount[P], tb = GR::D.lt[K];
+    float wv[kFwdVec];
+    if constexpr (WSH) {
+#pragma unroll
+      for (int c = 0; c < kFwdVec; ++c) wv[c] = wsh[c];
+    } else {
+      VecIO<kFwdVec>::lds(wv, stage + K * rowf);
+    }
+    // first own row of this path's output: its l3 block, or its own block of
+    // 2 l3 + 1 rows when the launch keeps the paths apart
+    constexpr int o3 = GR::PERPATH ? K * (2 * l3 + 1) : l3 * l3 - GR::OWN0;
+    if constexpr (2 * l3 + 1 <= 2 * l1 + 1) {
+      // t[m3] = sum_m1 T x[m1], then out[m3] += W t[m3]
+      float t[2 * l3 + 1][kFwdVec];
+#pragma unroll
+      for (int m3 = 0; m3 < 2 * l3 + 1; ++m3)
+#pragma unroll
+        for (int c = 0; c < kFwdVec; ++c) t[m3][c] = 0.f;
+      static_for<0, (tc + 3) / 4>([&](auto Qc) {
+        constexpr int q = decltype(Qc)::value;
+        const float4 v4 = *reinterpret_cast<const float4*>(T + tb + 4 * q);
+        const float tv4[4] = {v4.x, v4.y, v4.z, v4.w};
+        static_for<0, 4>([&](auto Rc) {
+          constexpr int k = 4 * q + decltype(Rc)::value;
+          if constexpr (k < tc) {
+            constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
+            constexpr int rx = l1 * l1 + l1 + m1 - GR::D.rlo;
+            axpy<kFwdVec>(t[m3 + l3], tv4[decltype(Rc)::value], xr[rx]);
+          }
+        });
+      });
+#pragma unroll
+      for (int m3 = 0; m3 < 2 * l3 + 1; ++m3) vfma<kFwdVec>(acc[o3 + m3], wv, t[m3]);
+    } else {
+      // xw[m1] = W x[m1], then out[m3] += sum_m1 T xw[m1]
+      float xw[2 * l1 + 1][kFwdVec];
+#pragma unroll
+      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) vmul<kFwdVec>(xw[m1], wv, xr[l1 * l1 + m1 - GR::D.rlo]);
+      static_for<0, (tc + 3) / 4>([&](auto Qc) {
+        constexpr int q = decltype(Qc)::value;
+        const float4 v4 = *reinterpret_cast<const float4*>(T + tb + 4 * q);
+        const float tv4[4] = {v4.x, v4.y, v4.z, v4.w};
+        static_for<0, 4>([&](auto Rc) {
+          constexpr int k = 4 * q + decltype(Rc)::value;
+          if constexpr (k < tc) {
+            constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
+            axpy<kFwdVec>(acc[o3 + m3 + l3], tv4[decltype(Rc)::value], xw[m1 + l1]);
+          }
+        });
+      });
+    }
+  });
+}
+
+// GR: the launch's paths (all of them, or one chunk of one l3 block).  A
+// chunk that continues an l3 block another chunk of the call started adds
+// onto that chunk's rows (GR::FIRST false).
+template <class PS, class GR, int KMULT, bool WSH>
+__global__ void CGTP_FWD_BOUNDS
+conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
+  // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x 4
+  // channels, so every row offset below folds into an immediate.
+  const int mult = KMULT ? KMULT : a.mult;
+  const int lg_G = KMULT ? 5 : lg_G_rt;
+  const int S = KMULT ? KMULT / (32 * kFwdVec) : S_rt;
+  constexpr int NI = PS::NI, NO = PS::NO, NS = PS::NS, NT = GR::NT;
+  constexpr int NW = WSH ? 1 : GR::NP;  // staged weight rows
+  extern __shared__ float4 smem_f4[];
+  float* smem = reinterpret_cast<float*>(smem_f4);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int G = 1 << lg_G, gpw = 32 >> lg_G;
+  const int grp = lane >> lg_G, gl = lane & (G - 1);
+  const int rowf = G * kFwdVec;                    // floats per staged row
+  const int stage_floats = fwd_stage_floats(NW, GR::NROW, G);
+  const int group_floats = fwd_group_floats(BT, NT, stage_floats);
+  float* Tg = smem + (warp * gpw + grp) * group_floats;
+  float* St = Tg + BT * NT;                        // two pipeline stages
+  int* Jg = reinterpret_cast<int*>(St + 2 * stage_floats);
+
+  // The next launch of this call may start on SMs this grid leaves idle
+  // (chunks write disjoint rows unless one continues another, and that one
+  // waits below).
+  grid_dependents_launch();
+  if (a.abort_flag != nullptr && (*a.abort_flag & kGraphUnsafeBits)) {  // checked mode, invalid graph
+    grid_dependency_wait();
+    return;
+  }
+  const long long n_items = (long long)a.n_nodes * S;
+  const long long warps_total = (long long)gridDim.x * (kFwdThreads / 32);
+  for (long long base = ((long long)blockIdx.x * (kFwdThreads / 32) + warp) * gpw; base < n_items;
+       base += warps_total * gpw) {
+    const long long item = base + grp;
+    const bool active = item < n_items;
+    const int node = active ? int(item / S) : 0;
+    const int slice = active ? int(item % S) : 0;
+    const int c0 = (slice * G + gl) * kFwdVec;
+    int e0 = 0, e1 = 0;
+    if (active) {
+      e0 = __ldg(a.row_ptr + node);
+      e1 = __ldg(a.row_ptr + node + 1);
+    }
+    const int maxdeg = __reduce_max_sync(0xffffffffu, e1 - e0);
+    float acc[GR::NOWN][kFwdVec];
+#pragma unroll
+    for (int r = 0; r < GR::NOWN; ++r)
+#pragma unroll
+      for (int c = 0; c < kFwdVec; ++c) acc[r][c] = 0.f;
+
+    // copies of edge slot k of the current batch into stage s (this lane's channels only)
+    auto issue = [&](int b0, int k, int s) {
+      const int e = e0 + b0 + k;
+      if (!(active && e < e1)) return;
+      float* dst = St + s * stage_floats + gl * kFwdVec;
+      if constexpr (WSH) {
+        VecIO<kFwdVec>::cp_async(dst, a.w + (long long)e * mult + c0);
+      } else {
+        const float* wrow = a.w + (long long)e * PS::NP * mult + c0;
+        static_for<0, GR::NP>([&](auto Kc) {
+          constexpr int K = decltype(Kc)::value;
+          constexpr int P = GR::D.path[K];
+          VecIO<kFwdVec>::cp_async(dst + K * rowf, wrow + P * mult);
+        });
+      }
+      if constexpr (kStageX) {
+        constexpr int rlo = GR::D.rlo;
+        const float* xrow = a.x + ((long long)Jg[k] * NI + rlo) * mult + c0;
+#pragma unroll
+        for (int r = 0; r < GR::NROW; ++r) VecIO<kFwdVec>::cp_async(dst + (NW + r) * rowf, xrow + r * mult);
+      }
+    };
+
+    for (int b0 = 0; b0 < maxdeg; b0 += BT) {
+      // sources of every slot, then the first slot's copies, so that they fly
+      // while the T matrices of the batch are computed
+      for (int k = gl; k < BT; k += G) {
+        const int e = e0 + b0 + k;
+        if (active && e < e1) {
+          const int j = __ldg(a.col + e);
+          if constexpr (!kStageX) {
+            constexpr int rlo = GR::D.rlo;
+            prefetch_l2(a.x + ((long long)j * NI + rlo) * mult, (unsigned)(GR::NROW * mult * 4));
+          }
+          Jg[k] = j;
+        }
+      }
+      __syncwarp();
+      const int nb = min(BT, maxdeg - b0);
+      issue(b0, 0, 0);
+      cp_async_commit();
+      for (int k = gl; k < BT; k += G) {
+        const int e = e0 + b0 + k;
+        if (active && e < e1) {
+          float Y[NS];
+          edge_sh<PS::LS>(a.sh, a.edge_vec, e, Y);
+          compute_T_grp<PS, GR>(Y, Tg + k * NT);
+        }
+      }
+      __syncwarp();
+      for (int k = 0; k < nb; ++k) {
+        if (k + 1 < nb) issue(b0, k + 1, (k + 1) & 1);
+        cp_async_commit();
+        cp_async_wait<1>();  // this lane's copies of edge k have landed
+        if (active && e0 + b0 + k < e1) {
+          constexpr int rlo = GR::D.rlo;
+          fwd_edge<PS, GR, WSH>(Tg + k * NT, St + (k & 1) * stage_floats + gl * kFwdVec, rowf,
+                                a.x + ((long long)Jg[k] * NI + rlo) * mult + c0, mult, acc);
+        }
+      }
+      __syncwarp();
+    }
+    if constexpr (GR::PERPATH) {
+      // t[node][m3][rank][u] of this l3 block, rank = the path's place among
+      // the block's paths
+      if (active) {
+        constexpr int n3 = 2 * GR::KEY + 1;
+        static_for<0, GR::NP>([&](auto Kc) {
+          constexpr int K = decltype(Kc)::value;
+#pragma unroll
+          for (int m3 = 0; m3 < n3; ++m3)
+            VecIO<kFwdVec>::st(a.out + (((long long)node * n3 + m3) * GR::NPK + GR::PL0 + K) * mult + c0,
+                               acc[K * n3 + m3]);
+        });
+      }
+    } else if (active) {
+      if (!GR::FIRST || a.accumulate) {
+        // rows of an l3 block that the preceding launch wrote (wait for it),
+        // or the caller's values to add onto
+        if constexpr (!GR::FIRST) grid_dependency_wait();
+#pragma unroll
+        for (int r = 0; r < GR::NOWN; ++r) {
+          float prev[kFwdVec];
+          VecIO<kFwdVec>::ld(prev, a.out + ((long long)node * NO + GR::OWN0 + r) * mult + c0);
+#pragma unroll
+          for (int c = 0; c < kFwdVec; ++c) acc[r][c] += prev[c];
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < GR::NOWN; ++r)
+        VecIO<kFwdVec>::st(a.out + ((long long)node * NO + GR::OWN0 + r) * mult + c0, acc[r]);
+    }
+  }
+  // Complete only after the preceding launch: a grid launched with
+  // programmatic stream serialization that never waited could otherwise
+  // complete before its predecessor, and whatever the stream runs after the
+  // last launch of the chain (the next call, or a caller's kernel writing
+  // into memory this call has finished with) would then overlap a launch that
+  // is still running.  A no-op for a grid launched in plain stream order.
+  grid_dependency_wait();
+}
+
+template <class PS, class GR, bool WSH>
+cudaError_t launch_fwd_group(const ConvFwdArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
+  int G, lg_G, S;
+  lane_geometry(a.mult, kFwdVec, G, lg_G, S);
+  const int gpw = 32 / G;
+  const int stage_floats = fwd_stage_floats(WSH ? 1 : GR::NP, GR::NROW, G);
+  const int BT = pick_batch(gpw, GR::NT, stage_floats, CGTP_FWD_BATCH_FLOATS, CGTP_FWD_MAX_BATCH);
+  // the kernel's indexing reaches gpw groups x warps of group_floats each
+  const size_t smem = sizeof(float) * (size_t)fwd_group_floats(BT, GR::NT, stage_floats) * gpw * (kFwdThreads / 32);
+  cudaError_t err = check_smem(smem);
+  if (err != cudaSuccess) return err;
+  auto kern = a.mult == 128 ? conv_fwd_kernel<PS, GR, 128, WSH> : conv_fwd_kernel<PS, GR, 0, WSH>;
+  err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  const long long items = (long long)a.n_nodes * S;
+  const long long groups_per_block = (long long)gpw * (kFwdThreads / 32);
+  long long blocks = (items + groups_per_block - 1) / groups_per_block;
+  long long cap = 0x7fffffffLL;  // the kernel loops over items beyond the grid
+  if (CGTP_FWD_PERSISTENT) {
+    int per_sm = 0;
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFwdThreads, smem);
+    if (err != cudaSuccess) return err;
+    cap = (long long)num_sms * (per_sm < 1 ? 1 : per_sm);
+  }
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return launch_kernel(kern, dim3((unsigned)blocks), dim3(kFwdThreads), smem, stream, pdl, a, lg_G, S, BT);
+}
+
+// Unrolled instructions per edge and lane of all paths in one launch.
+template <class PS>
+constexpr int fwd_all_cost() {
+  int c = 0;
+  for (int p = 0; p < PS::D.np; ++p) c += path_cost<PS>(p, kByL3, kFwdVec, false);
+  return c;
+}
+
+template <class PS>
+using FwdPlan = Plan<PS, kByL3, kFwdVec, false, CGTP_FWD_BUDGET>;
+
+// Output blocks l3 that no path reaches are zero.
+template <class PS>
+cudaError_t zero_unreached_out(const ConvFwdArgs& a, cudaStream_t stream) {
+  cudaError_t err = cudaSuccess;
+  static_for_host<0, PS::LO + 1>([&](auto Lc) {
+    constexpr int l3 = decltype(Lc)::value;
+    constexpr bool reached = [] {
+      for (int p = 0; p < PS::D.np; ++p)
+        if (PS::D.l3[p] == l3) return true;
+      return false;
+    }();
+    if (!reached && err == cudaSuccess)
+      err = cudaMemset2DAsync(a.out + (size_t)l3 * l3 * a.mult, sizeof(float) * PS::NO * a.mult, 0,
+                              sizeof(float) * (2 * l3 + 1) * a.mult, a.n_nodes, stream);
+  });
+  return err;
+}
+
+// The forward over every path (summed by l3 blocks): one launch when all
+// paths fit one unrolled edge body, else one launch per chunk of same-l3
+// paths, every chunk after the first overlapping its predecessor.
+template <class PS, bool WSH>
+cudaError_t launch_fwd_all(const ConvFwdArgs& a, int num_sms, cudaStream_t stream) {
+  if constexpr (fwd_all_cost<PS>() <= CGTP_FWD_SINGLE_MAX) {
+    // all paths in one launch (it writes every output row, reached or not)
+    return launch_fwd_group<PS, Grp<PS, kAll, 0>, WSH>(a, num_sms, false, stream);
+  } else {
+    cudaError_t err = a.accumulate ? cudaSuccess : zero_unreached_out<PS>(a, stream);
+    static_for_host<0, FwdPlan<PS>::N>([&](auto Cc) {
+      constexpr int CH = decltype(Cc)::value;
+      if (err == cudaSuccess)
+        err = launch_fwd_group<PS, ChunkGrp<PS, FwdPlan<PS>, CH, kByL3>, WSH>(a, num_sms, CH > 0, stream);
+    });
+    return err;
+  }
+}
+
+}  // namespace
+}  // namespace cgtp

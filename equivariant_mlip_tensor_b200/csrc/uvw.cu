@@ -11,7 +11,6 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include <map>
 #include <mutex>
 
 #include "launch.h"
@@ -86,54 +85,16 @@ __global__ void uvw_unpack_kernel(PathOrder po, int mult, int mult_out, int rank
 // concurrently, block l3 on lane l3 % kLanes of a fork from the caller's
 // stream (lane 0 is the caller's stream itself) and join back before the
 // call returns, so the caller sees ordinary stream order.  The side streams
-// and events are created once per device and thread-safely cached.
+// and events are the library's per-device pool (lanes.cu).
 constexpr int kLanes = 3;
-struct Lanes {
-  cudaStream_t side[kLanes - 1];
-  cudaEvent_t fork, join[kLanes - 1];
-};
-static cudaError_t lanes_for_device(Lanes** out) {
-  static std::mutex mu;
-  static std::map<int, Lanes> per_dev;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  std::lock_guard<std::mutex> lock(mu);
-  auto it = per_dev.find(dev);
-  if (it == per_dev.end()) {
-    Lanes L{};
-    for (int k = 0; k < kLanes - 1 && e == cudaSuccess; ++k) {
-      e = cudaStreamCreateWithFlags(&L.side[k], cudaStreamNonBlocking);
-      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L.join[k], cudaEventDisableTiming);
-    }
-    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&L.fork, cudaEventDisableTiming);
-    if (e != cudaSuccess) return e;
-    it = per_dev.emplace(dev, L).first;
-  }
-  *out = &it->second;
-  return cudaSuccess;
-}
-// fork: lanes 1.. wait for the caller's stream; join: the caller's stream waits for them
-static cudaError_t lanes_fork(Lanes* L, cudaStream_t s) {
-  cudaError_t e = cudaEventRecord(L->fork, s);
-  for (int k = 0; k < kLanes - 1 && e == cudaSuccess; ++k) e = cudaStreamWaitEvent(L->side[k], L->fork, 0);
-  return e;
-}
-static cudaError_t lanes_join(Lanes* L, cudaStream_t s) {
-  cudaError_t e = cudaSuccess;
-  for (int k = 0; k < kLanes - 1 && e == cudaSuccess; ++k) {
-    e = cudaEventRecord(L->join[k], L->side[k]);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, L->join[k], 0);
-  }
-  return e;
-}
+using Lanes = SideLanes;
+static cudaError_t lanes_for_device(Lanes** out) { return side_lanes(kLanesUvw, out); }
+static cudaError_t lanes_fork(Lanes* L, cudaStream_t s) { return lanes_fork(L, kLanes - 1, s); }
+static cudaError_t lanes_join(Lanes* L, cudaStream_t s) { return lanes_join(L, kLanes - 1, s); }
 static cudaStream_t lane(Lanes* L, cudaStream_t s, int l3) { return l3 % kLanes == 0 ? s : L->side[l3 % kLanes - 1]; }
 // Host threads that enqueue on the shared lanes take turns (the fork and join
 // events are shared too).
-static std::mutex& lanes_use_mutex() {
-  static std::mutex mu;
-  return mu;
-}
+static std::mutex& lanes_use_mutex() { return side_lanes_mutex(kLanesUvw); }
 
 #if !defined(CGTP_NO_CUTLASS)
 using namespace cute;
