@@ -19,9 +19,11 @@ _sz = ctypes.c_size_t
 SIGNATURES = {
     "cgtp_status_string": (ctypes.c_char_p, [_i]),
     "cgtp_last_cuda_error": (_i, []),
-    "cgtp_plan_create": (_i, [_i, _i, _i, _i, ctypes.POINTER(_p)]),
+    "cgtp_plan_create": (_i, [_i, _i, _i, _i, _i, ctypes.POINTER(_p)]),
     "cgtp_plan_destroy": (_i, [_p]),
-    "cgtp_supported": (_i, [_i, _i, _i]),
+    "cgtp_supported": (_i, [_i, _i, _i, _i]),
+    "cgtp_plan_set_checked": (_i, [_p, _i]),
+    "cgtp_plan_check": (_i, [_p, ctypes.POINTER(_i)]),
     "cgtp_plan_info": (_i, [_p, ctypes.POINTER(_i), _p, ctypes.POINTER(_i)]),
     "cgtp_cg_block": (_i, [_i, _i, _i, _p]),
     "cgtp_graph_build": (_i, [_p, _i, _f, _f, _p, _i, _p, _p, _p, _p, _p, _p, _i, _p, _p]),
@@ -39,9 +41,9 @@ SIGNATURES = {
     "cgtp_uvw_backward_workspace_size": (_i, [_p, _i, _i, _i, ctypes.POINTER(_sz)]),
     "cgtp_uvw_backward": (_i, [_p, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _i, _p, _p, _p, _p, _p, _p,
                                _sz, _p]),
-    "cgtp_conv_forward_shared_weights": (_i, [_p, _i, _i, _p, _p, _p, _p, _p, _p, _p]),
-    "cgtp_conv_backward_shared_weights": (_i, [_p, _i, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
     "cgtp_forces": (_i, [_i, _i, _p, _p, _p, _p, _p, _p]),
+    "cgtp_gather_rows": (_i, [_i, _i, _p, _p, _p, _p]),
+    "cgtp_scatter_add_rows": (_i, [_i, _i, _p, _p, _p, _p]),
     "cgtp_radial_forward": (_i, [_p, _i, _p, _f, _p, _p, _p, _p]),
     "cgtp_radial_backward": (_i, [_p, _i, _p, _f, _p, _p, _p, _p, _p]),
     "cgtp_tp_forward": (_i, [_p, _i, _p, _p, _p, _p, _p]),

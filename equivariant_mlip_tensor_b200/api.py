@@ -9,6 +9,7 @@ import ctypes
 from dataclasses import dataclass
 from typing import Optional
 
+import numpy as np
 import torch
 
 from ._lib import call, lib
@@ -38,8 +39,12 @@ def n_paths(lmax_in, lmax_sh, lmax_out):
                for l3 in range(abs(l1 - l2), min(l1 + l2, lmax_out) + 1))
 
 
-def supported(lmax_in, lmax_sh, lmax_out):
-    return bool(lib().cgtp_supported(lmax_in, lmax_sh, lmax_out))
+# plan modes of the C ABI (cgtp_mode)
+MODES = {"conv": 0, "pair": 1, "conv_shared": 2, "uvw": 3}
+
+
+def supported(lmax_in, lmax_sh, lmax_out, mode="conv"):
+    return bool(lib().cgtp_supported(lmax_in, lmax_sh, lmax_out, MODES[mode]))
 
 
 def cg_block(l1, l2, l3):
@@ -130,14 +135,44 @@ def forces(graph, grad_edge_vec, out=None):
     return out
 
 
-class Plan:
-    """Paths and CG coefficients of one irreps shape (lmax_in, lmax_sh, lmax_out, mult)."""
+def gather_rows(idx, src, out=None):
+    """out[k] = src[idx[k]] (rows of src's trailing shape)."""
+    _check(idx, torch.int32, "idx")
+    _check(src, torch.float32, "src")
+    n, rf = idx.numel(), int(np.prod(src.shape[1:]))
+    if out is None:
+        out = torch.empty((n,) + tuple(src.shape[1:]), dtype=torch.float32, device=src.device)
+    call("cgtp_gather_rows", n, rf, _ptr(idx), _ptr(src), _ptr(out), _stream())
+    return out
 
-    def __init__(self, lmax_in, lmax_sh, lmax_out, mult):
+
+def scatter_add_rows(idx, src, dst):
+    """dst[idx[k]] += src[k] (idx without repeats); returns dst."""
+    _check(idx, torch.int32, "idx")
+    _check(src, torch.float32, "src")
+    _check(dst, torch.float32, "dst")
+    n = idx.numel()
+    rf = int(np.prod(dst.shape[1:])) if dst.dim() > 1 else 1
+    call("cgtp_scatter_add_rows", n, rf, _ptr(idx), _ptr(src), _ptr(dst), _stream())
+    return dst
+
+
+class Plan:
+    """Paths and CG coefficients of one irreps shape (lmax_in, lmax_sh, lmax_out, mult).
+
+    The C library takes one plan per mode (what the plan computes: "conv", the
+    channelwise convolution; "pair", the edge-free product and its CP
+    surrogate; "conv_shared", the convolution with one weight row per edge
+    for every path; "uvw", the fully connected convolution).  This object
+    holds the plan of ``mode`` and creates the plan of another mode of the
+    same shape the first time one of that mode's methods is called."""
+
+    def __init__(self, lmax_in, lmax_sh, lmax_out, mult, mode="conv"):
         self.lmax_in, self.lmax_sh, self.lmax_out, self.mult = lmax_in, lmax_sh, lmax_out, mult
-        h = ctypes.c_void_p()
-        call("cgtp_plan_create", lmax_in, lmax_sh, lmax_out, mult, ctypes.byref(h))
-        self._h = h
+        self.mode = mode
+        self._handles = {}
+        self._checked = False
+        h = self.handle(mode)
         n = ctypes.c_int()
         nnz = ctypes.c_int()
         call("cgtp_plan_info", h, ctypes.byref(n), None, ctypes.byref(nnz))
@@ -148,14 +183,49 @@ class Plan:
         self.paths = [tuple(buf[3 * k:3 * k + 3]) for k in range(n.value)]
         self.ni, self.ns, self.no = (lmax_in + 1) ** 2, (lmax_sh + 1) ** 2, (lmax_out + 1) ** 2
 
+    def handle(self, mode=None):
+        """The C plan (cgtp_plan) of ``mode`` (default: this plan's own)."""
+        mode = self.mode if mode is None else mode
+        h = self._handles.get(mode)
+        if h is None:
+            h = ctypes.c_void_p()
+            call("cgtp_plan_create", self.lmax_in, self.lmax_sh, self.lmax_out, self.mult, MODES[mode],
+                 ctypes.byref(h))
+            self._handles[mode] = h
+            if self._checked:
+                call("cgtp_plan_set_checked", h, 1)
+        return h
+
+    @property
+    def _h(self):
+        return self.handle()
+
+    def set_checked(self, on=True):
+        """Checked mode for every plan of this object (see cgtp_plan_set_checked)."""
+        self._checked = bool(on)
+        for h in self._handles.values():
+            call("cgtp_plan_set_checked", h, 1 if on else 0)
+
+    def check(self):
+        """Flags recorded by checked-mode calls (0 = every graph was valid);
+        synchronises the device and clears them."""
+        flags = 0
+        for h in self._handles.values():
+            f = ctypes.c_int()
+            st = lib().cgtp_plan_check(h, ctypes.byref(f))
+            if st not in (0, 3):  # CGTP_OK, CGTP_ERR_BAD_GRAPH
+                call("cgtp_plan_check", h, None)  # raises with the status
+            flags |= f.value
+        return flags
+
     def __del__(self):
-        h = getattr(self, "_h", None)
-        if h is not None and h.value:
-            try:
-                lib().cgtp_plan_destroy(h)
-            except Exception:
-                pass
-            self._h = None
+        for h in getattr(self, "_handles", {}).values():
+            if h is not None and h.value:
+                try:
+                    lib().cgtp_plan_destroy(h)
+                except Exception:
+                    pass
+        self._handles = {}
 
     # ------------------------------------------------------------ convolution
     def conv_forward(self, graph, x, w, out=None):
@@ -163,13 +233,13 @@ class Plan:
         _check(w, torch.float32, "w")
         if out is None:
             out = torch.empty((graph.n_nodes, self.no, self.mult), dtype=torch.float32, device=x.device)
-        call("cgtp_conv_forward", self._h, graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr), _ptr(graph.col),
+        call("cgtp_conv_forward", self.handle("conv"), graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr), _ptr(graph.col),
              _ptr(graph.edge_vec), _ptr(x), _ptr(w), _ptr(out), _stream())
         return out
 
     def conv_backward_workspace_bytes(self, n_edges):
         b = ctypes.c_size_t()
-        call("cgtp_conv_backward_workspace_size", self._h, n_edges, ctypes.byref(b))
+        call("cgtp_conv_backward_workspace_size", self.handle("conv"), n_edges, ctypes.byref(b))
         return b.value
 
     def conv_backward(self, graph, x, w, grad_out, want_x=True, want_w=True, want_r=True,
@@ -190,7 +260,7 @@ class Plan:
             ws_bytes = self.conv_backward_workspace_bytes(E)
             if workspace is None:
                 workspace = torch.empty(max(ws_bytes // 4, 64), dtype=torch.float32, device=dev)
-        call("cgtp_conv_backward", self._h, graph.n_nodes, E, _ptr(graph.csc_ptr), _ptr(graph.csc_edge),
+        call("cgtp_conv_backward", self.handle("conv"), graph.n_nodes, E, _ptr(graph.csc_ptr), _ptr(graph.csc_edge),
              _ptr(graph.csc_dst), _ptr(graph.edge_vec), _ptr(x), _ptr(w), _ptr(grad_out),
              _ptr(grad_x if want_x else None), _ptr(grad_w if want_w else None),
              _ptr(grad_edge_vec if want_r else None), _ptr(workspace if want_r else None),
@@ -199,7 +269,7 @@ class Plan:
 
     def conv_double_backward_workspace_bytes(self, n_edges):
         b = ctypes.c_size_t()
-        call("cgtp_conv_double_backward_workspace_size", self._h, n_edges, ctypes.byref(b))
+        call("cgtp_conv_double_backward_workspace_size", self.handle("conv"), n_edges, ctypes.byref(b))
         return b.value
 
     def conv_double_backward(self, graph, x, w, grad_out, gg_x=None, gg_w=None, gg_edge_vec=None,
@@ -222,7 +292,7 @@ class Plan:
             nb = self.conv_double_backward_workspace_bytes(E)
             if workspace is None:
                 workspace = torch.empty(max(nb // 4, 64), dtype=torch.float32, device=dev)
-        call("cgtp_conv_double_backward", self._h, graph.n_nodes, E, _ptr(graph.row_ptr), _ptr(graph.col),
+        call("cgtp_conv_double_backward", self.handle("conv"), graph.n_nodes, E, _ptr(graph.row_ptr), _ptr(graph.col),
              _ptr(graph.csc_ptr), _ptr(graph.csc_edge), _ptr(graph.csc_dst), _ptr(graph.edge_vec), _ptr(x),
              _ptr(w), _ptr(grad_out), _ptr(gg_x), _ptr(gg_w), _ptr(gg_edge_vec), _ptr(d_x), _ptr(d_w), _ptr(d_g),
              _ptr(d_r), _ptr(workspace if nb else None), workspace.numel() * 4 if (nb and workspace is not None) else 0,
@@ -231,7 +301,7 @@ class Plan:
 
     def uvw_forward_workspace_bytes(self, n_nodes, mult_out):
         b = ctypes.c_size_t()
-        call("cgtp_uvw_forward_workspace_size", self._h, n_nodes, mult_out, ctypes.byref(b))
+        call("cgtp_uvw_forward_workspace_size", self.handle("uvw"), n_nodes, mult_out, ctypes.byref(b))
         return b.value
 
     def uvw_forward(self, graph, x, w, mix, out=None, workspace=None):
@@ -244,14 +314,14 @@ class Plan:
         nb = self.uvw_forward_workspace_bytes(graph.n_nodes, mult_out)
         if workspace is None:
             workspace = torch.empty(max(nb // 4, 64), dtype=torch.float32, device=x.device)
-        call("cgtp_uvw_forward", self._h, graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr), _ptr(graph.col),
+        call("cgtp_uvw_forward", self.handle("uvw"), graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr), _ptr(graph.col),
              _ptr(graph.edge_vec), _ptr(x), _ptr(w), _ptr(mix), mult_out, _ptr(out), _ptr(workspace),
              workspace.numel() * 4, _stream())
         return out
 
     def uvw_backward_workspace_bytes(self, n_nodes, n_edges, mult_out):
         b = ctypes.c_size_t()
-        call("cgtp_uvw_backward_workspace_size", self._h, n_nodes, n_edges, mult_out, ctypes.byref(b))
+        call("cgtp_uvw_backward_workspace_size", self.handle("uvw"), n_nodes, n_edges, mult_out, ctypes.byref(b))
         return b.value
 
     def uvw_backward(self, graph, x, w, mix, grad_out, want_x=True, want_w=True, want_mix=True, want_r=True,
@@ -268,7 +338,7 @@ class Plan:
         nb = self.uvw_backward_workspace_bytes(graph.n_nodes, E, mult_out)
         if workspace is None:
             workspace = torch.empty(max(nb // 4, 64), dtype=torch.float32, device=dev)
-        call("cgtp_uvw_backward", self._h, graph.n_nodes, E, _ptr(graph.row_ptr), _ptr(graph.col),
+        call("cgtp_uvw_backward", self.handle("uvw"), graph.n_nodes, E, _ptr(graph.row_ptr), _ptr(graph.col),
              _ptr(graph.csc_ptr), _ptr(graph.csc_edge), _ptr(graph.csc_dst), _ptr(graph.edge_vec), _ptr(x), _ptr(w),
              _ptr(mix), mult_out, _ptr(grad_out), _ptr(gx), _ptr(gw), _ptr(gm), _ptr(gr), _ptr(workspace),
              workspace.numel() * 4, _stream())
@@ -280,7 +350,7 @@ class Plan:
         _check(w, torch.float32, "w")
         if out is None:
             out = torch.empty((graph.n_nodes, self.no, self.mult), dtype=torch.float32, device=x.device)
-        call("cgtp_conv_forward_shared_weights", self._h, graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr),
+        call("cgtp_conv_forward", self.handle("conv_shared"), graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr),
              _ptr(graph.col), _ptr(graph.edge_vec), _ptr(x), _ptr(w), _ptr(out), _stream())
         return out
 
@@ -292,24 +362,34 @@ class Plan:
         gx = torch.empty_like(x) if want_x else None
         gw = torch.empty((E, self.mult), dtype=torch.float32, device=dev) if want_w else None
         gr = torch.empty((E, 3), dtype=torch.float32, device=dev) if want_r else None
-        nb = self.conv_backward_workspace_bytes(E) if want_r else 0
+        nb = 0
+        if want_r:
+            b = ctypes.c_size_t()
+            call("cgtp_conv_backward_workspace_size", self.handle("conv_shared"), E, ctypes.byref(b))
+            nb = b.value
         if want_r and workspace is None:
             workspace = torch.empty(max(nb // 4, 64), dtype=torch.float32, device=dev)
-        call("cgtp_conv_backward_shared_weights", self._h, graph.n_nodes, E, _ptr(graph.csc_ptr),
+        call("cgtp_conv_backward", self.handle("conv_shared"), graph.n_nodes, E, _ptr(graph.csc_ptr),
              _ptr(graph.csc_edge), _ptr(graph.csc_dst), _ptr(graph.edge_vec), _ptr(x), _ptr(w), _ptr(grad_out),
              _ptr(gx), _ptr(gw), _ptr(gr), _ptr(workspace if want_r else None),
              workspace.numel() * 4 if (want_r and workspace is not None) else 0, _stream())
         return gx, gw, gr
 
     # ------------------------------------------------------------ radial network
+    def _radial_mode(self):
+        return self.mode if self.mode in ("conv", "conv_shared", "uvw") else "conv"
+
     def radial_forward(self, edge_vec, rc, W1, W2, out=None):
+        """Per-edge weights of the plan's mode: [E][n_paths][mult], or [E][mult]
+        for "conv_shared"."""
         _check(edge_vec, torch.float32, "edge_vec")
         _check(W1, torch.float32, "W1")
         _check(W2, torch.float32, "W2")
         E = edge_vec.shape[0]
         if out is None:
-            out = torch.empty((E, self.n_paths, self.mult), dtype=torch.float32, device=edge_vec.device)
-        call("cgtp_radial_forward", self._h, E, _ptr(edge_vec), ctypes.c_float(float(rc)), _ptr(W1), _ptr(W2),
+            shape = (E, self.mult) if self._radial_mode() == "conv_shared" else (E, self.n_paths, self.mult)
+            out = torch.empty(shape, dtype=torch.float32, device=edge_vec.device)
+        call("cgtp_radial_forward", self.handle(self._radial_mode()), E, _ptr(edge_vec), ctypes.c_float(float(rc)), _ptr(W1), _ptr(W2),
              _ptr(out), _stream())
         return out
 
@@ -317,7 +397,7 @@ class Plan:
         """Adds dL/d edge_vec through the weights into grad_edge_vec (in place)."""
         _check(grad_w, torch.float32, "grad_w")
         _check(grad_edge_vec, torch.float32, "grad_edge_vec")
-        call("cgtp_radial_backward", self._h, edge_vec.shape[0], _ptr(edge_vec), ctypes.c_float(float(rc)),
+        call("cgtp_radial_backward", self.handle(self._radial_mode()), edge_vec.shape[0], _ptr(edge_vec), ctypes.c_float(float(rc)),
              _ptr(W1), _ptr(W2), _ptr(grad_w), _ptr(grad_edge_vec), _stream())
         return grad_edge_vec
 
@@ -328,7 +408,7 @@ class Plan:
         B = x.shape[0]
         if out is None:
             out = torch.empty((B, self.no, self.mult), dtype=torch.float32, device=x.device)
-        call("cgtp_tp_forward", self._h, B, _ptr(x), _ptr(y), _ptr(w), _ptr(out), _stream())
+        call("cgtp_tp_forward", self.handle("pair"), B, _ptr(x), _ptr(y), _ptr(w), _ptr(out), _stream())
         return out
 
     def tp_backward(self, x, y, w, grad_z, want_x=True, want_y=True, want_w=True):
@@ -341,10 +421,10 @@ class Plan:
         nb = 0
         if want_w:
             b = ctypes.c_size_t()
-            call("cgtp_tp_backward_workspace_size", self._h, B, ctypes.byref(b))
+            call("cgtp_tp_backward_workspace_size", self.handle("pair"), B, ctypes.byref(b))
             nb = b.value
             ws = torch.empty(max(nb // 4, 64), dtype=torch.float32, device=dev)
-        call("cgtp_tp_backward", self._h, B, _ptr(x), _ptr(y), _ptr(w), _ptr(grad_z), _ptr(gx), _ptr(gy),
+        call("cgtp_tp_backward", self.handle("pair"), B, _ptr(x), _ptr(y), _ptr(w), _ptr(grad_z), _ptr(gx), _ptr(gy),
              _ptr(gw), _ptr(ws), nb, _stream())
         return gx, gy, gw
 
@@ -356,13 +436,13 @@ class Plan:
         R, batch = A.shape[1], x.shape[0]
         if out is None:
             out = torch.empty((batch, (self.lmax_out + 1) ** 2, self.mult), dtype=torch.float32, device=x.device)
-        call("cgtp_cp_forward", self._h, R, batch, _ptr(A), _ptr(B), _ptr(C), _ptr(x), _ptr(y), _ptr(out),
+        call("cgtp_cp_forward", self.handle("pair"), R, batch, _ptr(A), _ptr(B), _ptr(C), _ptr(x), _ptr(y), _ptr(out),
              _stream())
         return out
 
     def cp_backward_workspace_bytes(self, rank, batch):
         b = ctypes.c_size_t()
-        call("cgtp_cp_backward_workspace_size", self._h, rank, batch, ctypes.byref(b))
+        call("cgtp_cp_backward_workspace_size", self.handle("pair"), rank, batch, ctypes.byref(b))
         return b.value
 
     def cp_backward(self, A, B, C, x, y, grad_z, want_x=True, want_y=True, want_factors=True):
@@ -377,6 +457,6 @@ class Plan:
         if want_factors:
             nb = self.cp_backward_workspace_bytes(R, batch)
             ws = torch.empty(max(nb // 4, 64), dtype=torch.float32, device=x.device)
-        call("cgtp_cp_backward", self._h, R, batch, _ptr(A), _ptr(B), _ptr(C), _ptr(x), _ptr(y), _ptr(grad_z),
+        call("cgtp_cp_backward", self.handle("pair"), R, batch, _ptr(A), _ptr(B), _ptr(C), _ptr(x), _ptr(y), _ptr(grad_z),
              _ptr(gx), _ptr(gy), _ptr(gA), _ptr(gB), _ptr(gC), _ptr(ws), nb, _stream())
         return gx, gy, gA, gB, gC

@@ -1,10 +1,13 @@
 """Build libcgtp.so (sm_100a) in-tree.
 
-Every per-shape kernel family (conv forward, conv backward, edge-free tensor
-product) is compiled once per shape listed in csrc/configs.h, each as its
-own translation unit so that the compiles run in parallel; the shape-free
-parts (graph, radial network, forces, harmonics, C ABI, host CG tables) are
-one unit each.  Objects go to _build/, the library to the package directory.
+Every per-shape kernel family (convolution forward, backward and
+harmonic-gradient passes, edge-free tensor product, CP product) is compiled
+once per shape of CGTP_CONFIGS in csrc/configs.h, and the weight-structure
+variants (path-shared weights, fully connected convolution) once per shape of
+CGTP_VARIANT_CONFIGS, each as its own translation unit so that the compiles
+run in parallel; the shape-free parts (graph, radial network, forces,
+harmonics, C ABI, host CG tables, tensor-core GEMMs, side streams) are one
+unit each.  Objects go to _build/, the library to the package directory.
 Objects newer than their sources and headers are reused.
 """
 import os
@@ -23,8 +26,11 @@ INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
                      "-Xcompiler", "-fPIC", "-I", CSRC, "-I", INCLUDE]
-PER_SHAPE = ["conv_fwd.cu", "conv_bwd.cu", "conv_paths.cu", "conv_shared.cu", "tp.cu", "cp.cu"]
-SHAPE_FREE = ["graph.cu", "radial.cu", "misc.cu", "abi.cu", "cg_table.cpp", "uvw.cu"]
+# per-shape units: every shape of CGTP_CONFIGS, and the weight-structure
+# variants for the shapes of CGTP_VARIANT_CONFIGS
+PER_SHAPE = ["conv_fwd.cu", "conv_bwd.cu", "conv_gy.cu", "tp.cu", "cp.cu"]
+PER_VARIANT_SHAPE = ["conv_paths.cu", "conv_shared.cu"]
+SHAPE_FREE = ["graph.cu", "radial.cu", "misc.cu", "abi.cu", "cg_table.cpp", "uvw.cu", "lanes.cu"]
 
 
 def cutlass_include():
@@ -51,9 +57,11 @@ def nvcc():
     return cand
 
 
-def shapes():
+def shapes(macro="CGTP_CONFIGS"):
+    """(lmax_in, lmax_sh, lmax_out) entries of one list of csrc/configs.h."""
     text = open(os.path.join(CSRC, "configs.h")).read()
-    return [tuple(int(v) for v in m) for m in re.findall(r"X\((\d+),\s*(\d+),\s*(\d+)\)", text)]
+    body = text.split("#define " + macro + "(X)", 1)[1].split("\n\n", 1)[0]
+    return [tuple(int(v) for v in m) for m in re.findall(r"X\((\d+),\s*(\d+),\s*(\d+)\)", body)]
 
 
 def _headers():
@@ -70,17 +78,20 @@ def _stale(obj, src, deps):
 
 def _jobs():
     jobs = []
-    for src in PER_SHAPE:
-        for li, ls, lo in shapes():
-            obj = os.path.join(BUILD, f"{src.split('.')[0]}_{li}{ls}{lo}.o")
-            defs = [f"-DCGTP_CFG_LI={li}", f"-DCGTP_CFG_LS={ls}", f"-DCGTP_CFG_LO={lo}"]
-            jobs.append((os.path.join(CSRC, src), obj, defs))
     for src in SHAPE_FREE:
         obj = os.path.join(BUILD, src.rsplit(".", 1)[0] + ".o")
         defs = []
         if src == "uvw.cu":
             inc = cutlass_include()
             defs = (sum((["-I", d] for d in inc), []) + ["-diag-suppress", "20012,177"]) if inc else ["-DCGTP_NO_CUTLASS"]
+        jobs.append((os.path.join(CSRC, src), obj, defs))
+    units = [(src, shp) for src in PER_SHAPE for shp in shapes()]
+    units += [(src, shp) for src in PER_VARIANT_SHAPE for shp in shapes("CGTP_VARIANT_CONFIGS")]
+    # the largest shapes first, so that the long compiles start early
+    units.sort(key=lambda u: -(u[1][0] + 1) * (u[1][1] + 1) * (u[1][2] + 1))
+    for src, (li, ls, lo) in units:
+        obj = os.path.join(BUILD, f"{src.split('.')[0]}_{li}{ls}{lo}.o")
+        defs = [f"-DCGTP_CFG_LI={li}", f"-DCGTP_CFG_LS={ls}", f"-DCGTP_CFG_LO={lo}"]
         jobs.append((os.path.join(CSRC, src), obj, defs))
     return jobs
 

@@ -84,6 +84,14 @@ struct Shape {
   int li, ls, lo;
 };
 const Shape kShapes[] = {CGTP_CONFIGS(CGTP_LIST_ENTRY)};
+const Shape kVariantShapes[] = {CGTP_VARIANT_CONFIGS(CGTP_LIST_ENTRY)};
+
+template <size_t N>
+bool listed(const Shape (&list)[N], int li, int ls, int lo) {
+  for (const Shape& s : list)
+    if (s.li == li && s.ls == ls && s.lo == lo) return true;
+  return false;
+}
 
 }  // namespace
 }  // namespace cgtp
@@ -92,10 +100,40 @@ using namespace cgtp;
 
 struct cgtp_plan_s {
   int li, ls, lo, mult;
+  cgtp_mode mode;
   int n_paths;
   int nnz;
   std::vector<int> paths;
+  // checked mode: validation flags on the device of cgtp_plan_set_checked
+  int checked = 0;
+  int* d_flags = nullptr;
+  int flags_device = -1;
 };
+
+namespace {
+
+bool mode_is(cgtp_plan p, cgtp_mode m) { return p != nullptr && p->mode == m; }
+bool conv_mode(cgtp_plan p) {  // plans whose convolution takes one weight row per path or one shared row
+  return p != nullptr && (p->mode == CGTP_MODE_CONV_UVU || p->mode == CGTP_MODE_CONV_UVU_SHARED);
+}
+
+// Checked mode: OR the validation bits of the graph arrays a call uses into
+// the plan's flags (same stream, before the call's kernels) and hand the
+// flags to the kernels, which do nothing when they mark the graph unsafe.
+cudaError_t validate_graph(cgtp_plan p, int n, int E, const int* row_ptr, const int* col, const float* edge_vec,
+                           const int* csc_ptr, const int* csc_edge, const int* csc_dst, int sms, cudaStream_t s,
+                           const int** abort_flag) {
+  *abort_flag = nullptr;
+  if (!p->checked) return cudaSuccess;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev != p->flags_device) return cudaErrorInvalidDevice;
+  *abort_flag = p->d_flags;
+  return launch_graph_validate(n, E, row_ptr, col, edge_vec, csc_ptr, csc_edge, csc_dst, p->d_flags, sms, s);
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -115,9 +153,13 @@ const char* cgtp_status_string(cgtp_status s) {
 
 int cgtp_last_cuda_error(void) { return g_last_cuda_error; }
 
-int cgtp_supported(int li, int ls, int lo) {
-  for (const Shape& s : kShapes)
-    if (s.li == li && s.ls == ls && s.lo == lo) return 1;
+int cgtp_supported(int li, int ls, int lo, cgtp_mode mode) {
+  switch (mode) {
+    case CGTP_MODE_CONV_UVU:
+    case CGTP_MODE_PAIR_UVU: return listed(kShapes, li, ls, lo) ? 1 : 0;
+    case CGTP_MODE_CONV_UVU_SHARED:
+    case CGTP_MODE_CONV_UVW: return listed(kVariantShapes, li, ls, lo) ? 1 : 0;
+  }
   return 0;
 }
 
@@ -129,11 +171,14 @@ cgtp_status cgtp_cg_block(int l1, int l2, int l3, double* out) {
   return disc > 1e-12 ? CGTP_ERR_TABLE : CGTP_OK;
 }
 
-cgtp_status cgtp_plan_create(int li, int ls, int lo, int mult, cgtp_plan* plan) {
+cgtp_status cgtp_plan_create(int li, int ls, int lo, int mult, cgtp_mode mode, cgtp_plan* plan) {
   if (plan == nullptr) return CGTP_ERR_INVALID_ARG;
   *plan = nullptr;
   if (li < 0 || ls < 0 || lo < 0 || mult <= 0 || mult % 4 != 0) return CGTP_ERR_INVALID_ARG;
-  if (!cgtp_supported(li, ls, lo)) return CGTP_ERR_UNSUPPORTED;
+  if (mode != CGTP_MODE_CONV_UVU && mode != CGTP_MODE_PAIR_UVU && mode != CGTP_MODE_CONV_UVU_SHARED &&
+      mode != CGTP_MODE_CONV_UVW)
+    return CGTP_ERR_INVALID_ARG;
+  if (!cgtp_supported(li, ls, lo, mode)) return CGTP_ERR_UNSUPPORTED;
   if (host_tables().status != 0) return CGTP_ERR_TABLE;
   int sms = 0;
   cgtp_status st = ensure_device(&sms);
@@ -145,6 +190,7 @@ cgtp_status cgtp_plan_create(int li, int ls, int lo, int mult, cgtp_plan* plan) 
   p->ls = ls;
   p->lo = lo;
   p->mult = mult;
+  p->mode = mode;
   p->n_paths = d.np;
   p->nnz = d.nnz;
   for (int k = 0; k < d.np; ++k) {
@@ -157,8 +203,50 @@ cgtp_status cgtp_plan_create(int li, int ls, int lo, int mult, cgtp_plan* plan) 
 }
 
 cgtp_status cgtp_plan_destroy(cgtp_plan plan) {
+  if (plan != nullptr && plan->d_flags != nullptr) {
+    int cur = 0;
+    if (cudaGetDevice(&cur) == cudaSuccess && cudaSetDevice(plan->flags_device) == cudaSuccess) {
+      cudaFree(plan->d_flags);
+      cudaSetDevice(cur);
+    }
+  }
   delete plan;
   return CGTP_OK;
+}
+
+cgtp_status cgtp_plan_set_checked(cgtp_plan plan, int checked) {
+  if (plan == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (checked && plan->d_flags == nullptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaMalloc(&plan->d_flags, 16);
+    if (e == cudaSuccess) e = cudaMemset(plan->d_flags, 0, 16);
+    if (e != cudaSuccess) {
+      if (plan->d_flags) cudaFree(plan->d_flags);
+      plan->d_flags = nullptr;
+      return e == cudaErrorMemoryAllocation ? CGTP_ERR_OOM : cuda_fail(e);
+    }
+    plan->flags_device = dev;
+  }
+  plan->checked = checked ? 1 : 0;
+  return CGTP_OK;
+}
+
+cgtp_status cgtp_plan_check(cgtp_plan plan, int* flags) {
+  if (plan == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (flags) *flags = 0;
+  if (plan->d_flags == nullptr) return CGTP_OK;  // never in checked mode: nothing recorded
+  int cur = 0;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e == cudaSuccess) e = cudaSetDevice(plan->flags_device);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  int f = 0;
+  if (e == cudaSuccess) e = cudaMemcpy(&f, plan->d_flags, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(plan->d_flags, 0, sizeof(int));
+  cudaSetDevice(cur);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (flags) *flags = f;
+  return f ? CGTP_ERR_BAD_GRAPH : CGTP_OK;
 }
 
 cgtp_status cgtp_plan_info(cgtp_plan plan, int* n_paths, int* paths, int* n_nonzero) {
@@ -225,7 +313,7 @@ cgtp_status cgtp_spherical_harmonics(int lmax_sh, int n_edges, const float* edge
 
 cgtp_status cgtp_conv_forward(cgtp_plan p, int n_nodes, int n_edges, const int* row_ptr, const int* col,
                               const float* edge_vec, const float* x, const float* w, float* out, void* stream) {
-  if (p == nullptr || n_nodes < 0 || n_edges < 0 || row_ptr == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (!conv_mode(p) || n_nodes < 0 || n_edges < 0 || row_ptr == nullptr) return CGTP_ERR_INVALID_ARG;
   if (n_nodes > 0 && (x == nullptr || out == nullptr)) return CGTP_ERR_INVALID_ARG;
   if (n_edges > 0 && (col == nullptr || edge_vec == nullptr || w == nullptr)) return CGTP_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w) || !aligned16(out)) return CGTP_ERR_INVALID_ARG;
@@ -233,11 +321,21 @@ cgtp_status cgtp_conv_forward(cgtp_plan p, int n_nodes, int n_edges, const int* 
   int sms = 0;
   cgtp_status st = ensure_device(&sms);
   if (st != CGTP_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
   ConvFwdArgs a{n_nodes, row_ptr, col, edge_vec, x, w, out, p->mult};
-  cudaError_t e = cudaErrorNotSupported;
+  cudaError_t e = validate_graph(p, n_nodes, n_edges, row_ptr, col, edge_vec, nullptr, nullptr, nullptr, sms, s,
+                                 &a.abort_flag);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaErrorNotSupported;
+  if (p->mode == CGTP_MODE_CONV_UVU_SHARED) {
+#define CGTP_SFWD_ENTRY(A, B, C) \
+    if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_fwd_shared<A, B, C>(a, sms, s);
+    CGTP_VARIANT_CONFIGS(CGTP_SFWD_ENTRY)
+  } else {
 #define CGTP_FWD_ENTRY(A, B, C) \
-  if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_fwd<A, B, C>(a, sms, (cudaStream_t)stream);
-  CGTP_CONFIGS(CGTP_FWD_ENTRY)
+    if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_fwd<A, B, C>(a, sms, s);
+    CGTP_CONFIGS(CGTP_FWD_ENTRY)
+  }
   return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
 }
 
@@ -250,7 +348,7 @@ static int bwd_slices(cgtp_plan p) {
 }
 
 cgtp_status cgtp_conv_backward_workspace_size(cgtp_plan p, int n_edges, size_t* bytes) {
-  if (p == nullptr || n_edges < 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (p == nullptr || p->mode == CGTP_MODE_PAIR_UVU || n_edges < 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
   const size_t ns = (size_t)(p->ls + 1) * (p->ls + 1);
   const size_t b = sizeof(float) * (size_t)bwd_slices(p) * (size_t)n_edges * ns;
   *bytes = (b + 255) & ~(size_t)255;
@@ -261,7 +359,7 @@ cgtp_status cgtp_conv_backward(cgtp_plan p, int n_nodes, int n_edges, const int*
                                const int* csc_dst, const float* edge_vec, const float* x, const float* w,
                                const float* grad_out, float* grad_x, float* grad_w, float* grad_edge_vec,
                                void* workspace, size_t workspace_bytes, void* stream) {
-  if (p == nullptr || n_nodes < 0 || n_edges < 0 || csc_ptr == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (!conv_mode(p) || n_nodes < 0 || n_edges < 0 || csc_ptr == nullptr) return CGTP_ERR_INVALID_ARG;
   if (n_nodes > 0 && (x == nullptr || grad_out == nullptr)) return CGTP_ERR_INVALID_ARG;
   if (n_edges > 0 && (csc_edge == nullptr || csc_dst == nullptr || edge_vec == nullptr || w == nullptr))
     return CGTP_ERR_INVALID_ARG;
@@ -285,10 +383,19 @@ cgtp_status cgtp_conv_backward(cgtp_plan p, int n_nodes, int n_edges, const int*
   }
   ConvBwdArgs a{n_nodes, n_edges, csc_ptr, csc_edge, csc_dst, edge_vec, x, w, grad_out,
                 grad_x, grad_w, grad_edge_vec, (float*)workspace, p->mult};
-  cudaError_t e = cudaErrorNotSupported;
+  cudaError_t e = validate_graph(p, n_nodes, n_edges, nullptr, nullptr, edge_vec, csc_ptr, csc_edge, csc_dst, sms, s,
+                                 &a.abort_flag);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaErrorNotSupported;
+  if (p->mode == CGTP_MODE_CONV_UVU_SHARED) {
+#define CGTP_SBWD_ENTRY(A, B, C) \
+    if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_bwd_shared<A, B, C>(a, sms, s);
+    CGTP_VARIANT_CONFIGS(CGTP_SBWD_ENTRY)
+  } else {
 #define CGTP_BWD_ENTRY(A, B, C) \
-  if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_bwd<A, B, C>(a, sms, s);
-  CGTP_CONFIGS(CGTP_BWD_ENTRY)
+    if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_bwd<A, B, C>(a, sms, s);
+    CGTP_CONFIGS(CGTP_BWD_ENTRY)
+  }
   return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
 }
 
@@ -300,20 +407,14 @@ static cudaError_t dispatch_fwd(cgtp_plan p, const ConvFwdArgs& a, int sms, cuda
   CGTP_CONFIGS(CGTP_DFWD_ENTRY)
   return e;
 }
-static cudaError_t dispatch_bwd(cgtp_plan p, const ConvBwdArgs& a, int sms, cudaStream_t s);
-// Harmonic-gradient-only backward pass (no grad_x / grad_W) when its partial
-// slices fit the plain backward's workspace, else the plain backward.
+// Harmonic-gradient-only backward pass (no grad_x / grad_W work); its
+// partials have the plain backward's layout, so they fit its workspace.
 static cudaError_t dispatch_bwd_gy(cgtp_plan p, const ConvBwdArgs& a, int sms, cudaStream_t s) {
   cudaError_t e = cudaErrorNotSupported;
-  bool done = false;
-#define CGTP_BWD_GY_ENTRY(A, B, C)                                                     \
-  if (!done && p->li == A && p->ls == B && p->lo == C &&                                \
-      paths_bwd_slices<A, B, C>(p->mult) <= conv_bwd_slices<A, B, C>(p->mult)) {        \
-    e = launch_conv_bwd_gy<A, B, C>(a, sms, s);                                         \
-    done = true;                                                                        \
-  }
+#define CGTP_BWD_GY_ENTRY(A, B, C) \
+  if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_bwd_gy<A, B, C>(a, sms, s);
   CGTP_CONFIGS(CGTP_BWD_GY_ENTRY)
-  return done ? e : dispatch_bwd(p, a, sms, s);
+  return e;
 }
 
 static cudaError_t dispatch_bwd(cgtp_plan p, const ConvBwdArgs& a, int sms, cudaStream_t s) {
@@ -325,7 +426,7 @@ static cudaError_t dispatch_bwd(cgtp_plan p, const ConvBwdArgs& a, int sms, cuda
 }
 
 cgtp_status cgtp_conv_double_backward_workspace_size(cgtp_plan p, int n_edges, size_t* bytes) {
-  if (p == nullptr || n_edges < 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (!mode_is(p, CGTP_MODE_CONV_UVU) || n_edges < 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
   const size_t ns = (size_t)(p->ls + 1) * (p->ls + 1);
   const size_t u = (sizeof(float) * (size_t)n_edges * ns + 255) & ~(size_t)255;
   size_t bw = 0;
@@ -340,7 +441,7 @@ cgtp_status cgtp_conv_double_backward(cgtp_plan p, int n_nodes, int n_edges, con
                                       const float* gg_x, const float* gg_w, const float* gg_edge_vec, float* d_x,
                                       float* d_w, float* d_grad_out, float* d_edge_vec, void* workspace,
                                       size_t workspace_bytes, void* stream) {
-  if (p == nullptr || n_nodes < 0 || n_edges < 0 || row_ptr == nullptr || csc_ptr == nullptr)
+  if (!mode_is(p, CGTP_MODE_CONV_UVU) || n_nodes < 0 || n_edges < 0 || row_ptr == nullptr || csc_ptr == nullptr)
     return CGTP_ERR_INVALID_ARG;
   if (n_nodes > 0 && (x == nullptr || grad_out == nullptr)) return CGTP_ERR_INVALID_ARG;
   if (n_edges > 0 && (col == nullptr || csc_edge == nullptr || csc_dst == nullptr || edge_vec == nullptr ||
@@ -378,7 +479,9 @@ cgtp_status cgtp_conv_double_backward(cgtp_plan p, int n_nodes, int n_edges, con
   float* uY = need_ws ? (float*)workspace : nullptr;                      // [E][NS] = (dY/dr) gg_edge_vec
   float* gsh = need_ws ? (float*)((char*)workspace + u_bytes) : nullptr;  // harmonic-gradient partials
   const bool gr = gg_edge_vec != nullptr;
-  if (gr) e = launch_sh_dir(p->ls, n_edges, edge_vec, gg_edge_vec, uY, sms, s);
+  const int* abort_flag = nullptr;
+  e = validate_graph(p, n_nodes, n_edges, row_ptr, col, edge_vec, csc_ptr, csc_edge, csc_dst, sms, s, &abort_flag);
+  if (gr && e == cudaSuccess) e = launch_sh_dir(p->ls, n_edges, edge_vec, gg_edge_vec, uY, sms, s);
 
   // d grad_out: forward convolutions with one argument replaced at a time
   //   (Y -> uY), (x -> gg_x), (W -> gg_w), summed
@@ -387,6 +490,7 @@ cgtp_status cgtp_conv_double_backward(cgtp_plan p, int n_nodes, int n_edges, con
     auto fwd = [&](const float* xx, const float* ww, const float* sh) {
       if (e != cudaSuccess) return;
       ConvFwdArgs a{n_nodes, row_ptr, col, edge_vec, xx, ww, d_grad_out, p->mult};
+      a.abort_flag = abort_flag;
       a.sh = sh;
       a.accumulate = init ? 1 : 0;
       e = dispatch_fwd(p, a, sms, s);
@@ -405,6 +509,7 @@ cgtp_status cgtp_conv_double_backward(cgtp_plan p, int n_nodes, int n_edges, con
     if (gr && e == cudaSuccess) {
       ConvBwdArgs a{n_nodes, n_edges, csc_ptr, csc_edge, csc_dst, edge_vec, x, w, grad_out,
                     d_x, d_w, nullptr, nullptr, p->mult};
+      a.abort_flag = abort_flag;
       a.sh = uY;
       e = dispatch_bwd(p, a, sms, s);
       init_x = d_x != nullptr;
@@ -416,6 +521,7 @@ cgtp_status cgtp_conv_double_backward(cgtp_plan p, int n_nodes, int n_edges, con
       // the two outputs accumulate together: both were written above or neither
       ConvBwdArgs a{n_nodes, n_edges, csc_ptr, csc_edge, csc_dst, edge_vec, gg_x ? gg_x : x, gg_w ? gg_w : w,
                     grad_out, ox, ow, nullptr, nullptr, p->mult};
+      a.abort_flag = abort_flag;
       a.accumulate = gr ? 1 : 0;
       e = dispatch_bwd(p, a, sms, s);
       init_x = init_x || ox != nullptr;
@@ -433,6 +539,7 @@ cgtp_status cgtp_conv_double_backward(cgtp_plan p, int n_nodes, int n_edges, con
       if (e != cudaSuccess) return;
       ConvBwdArgs a{n_nodes, n_edges, csc_ptr, csc_edge, csc_dst, edge_vec, xx, ww, grad_out,
                     nullptr, nullptr, d_edge_vec, gsh, p->mult};
+      a.abort_flag = abort_flag;
       a.gr_mode = init ? mode_add : mode_set;
       a.gr_dir = gg_edge_vec;
       e = dispatch_bwd_gy(p, a, sms, s);
@@ -456,7 +563,7 @@ static bool uvw_layout(cgtp_plan p, int n_nodes, int mult_out, UvwLayout* L) {
   bool found = false;
 #define CGTP_UVW_ORDER_ENTRY(A, B, C) \
   if (p->li == A && p->ls == B && p->lo == C) { conv_path_order<A, B, C>(L->order, L->count_l3); found = true; }
-  CGTP_CONFIGS(CGTP_UVW_ORDER_ENTRY)
+  CGTP_VARIANT_CONFIGS(CGTP_UVW_ORDER_ENTRY)
   if (!found) return false;
   L->t_floats = L->packed_floats = 0;
   for (int l3 = 0; l3 <= p->lo; ++l3) {
@@ -468,7 +575,8 @@ static bool uvw_layout(cgtp_plan p, int n_nodes, int mult_out, UvwLayout* L) {
 static size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 cgtp_status cgtp_uvw_forward_workspace_size(cgtp_plan p, int n_nodes, int mult_out, size_t* bytes) {
-  if (p == nullptr || n_nodes < 0 || mult_out <= 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (!mode_is(p, CGTP_MODE_CONV_UVW) || n_nodes < 0 || mult_out <= 0 || bytes == nullptr)
+    return CGTP_ERR_INVALID_ARG;
   UvwLayout L;
   if (!uvw_layout(p, n_nodes, mult_out, &L)) return CGTP_ERR_UNSUPPORTED;
   *bytes = round256(sizeof(float) * L.t_floats) + round256(sizeof(float) * L.packed_floats) +
@@ -479,7 +587,8 @@ cgtp_status cgtp_uvw_forward_workspace_size(cgtp_plan p, int n_nodes, int mult_o
 cgtp_status cgtp_uvw_forward(cgtp_plan p, int n_nodes, int n_edges, const int* row_ptr, const int* col,
                              const float* edge_vec, const float* x, const float* w, const float* mix, int mult_out,
                              float* out, void* workspace, size_t workspace_bytes, void* stream) {
-  if (p == nullptr || n_nodes < 0 || n_edges < 0 || row_ptr == nullptr || mult_out <= 0 || mix == nullptr)
+  if (!mode_is(p, CGTP_MODE_CONV_UVW) || n_nodes < 0 || n_edges < 0 || row_ptr == nullptr || mult_out <= 0 ||
+      mix == nullptr)
     return CGTP_ERR_INVALID_ARG;
   if (n_nodes > 0 && (x == nullptr || out == nullptr)) return CGTP_ERR_INVALID_ARG;
   if (n_edges > 0 && (col == nullptr || edge_vec == nullptr || w == nullptr)) return CGTP_ERR_INVALID_ARG;
@@ -504,10 +613,13 @@ cgtp_status cgtp_uvw_forward(cgtp_plan p, int n_nodes, int n_edges, const int* r
                            round256(sizeof(float) * L.packed_floats);
   // stage 1: per-path messages t (channelwise convolution, paths kept apart)
   ConvFwdArgs a{n_nodes, row_ptr, col, edge_vec, x, w, t, p->mult};
-  cudaError_t e = cudaErrorNotSupported;
+  cudaError_t e = validate_graph(p, n_nodes, n_edges, row_ptr, col, edge_vec, nullptr, nullptr, nullptr, sms, s,
+                                 &a.abort_flag);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaErrorNotSupported;
 #define CGTP_UVW_PATHS_ENTRY(A, B, C) \
   if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_paths<A, B, C>(a, sms, s);
-  CGTP_CONFIGS(CGTP_UVW_PATHS_ENTRY)
+  CGTP_VARIANT_CONFIGS(CGTP_UVW_PATHS_ENTRY)
   if (e != cudaSuccess) return cuda_fail(e);
   // stage 2: per-l3 mixing GEMMs; output blocks no path reaches are zero
   e = launch_uvw_pack(p->n_paths, p->mult, mult_out, p->lo, L.order, L.count_l3, mix, packed, s);
@@ -543,7 +655,8 @@ static bool uvw_bwd_parts(cgtp_plan p, int n_nodes, int n_edges, int mult_out, b
 }
 
 cgtp_status cgtp_uvw_backward_workspace_size(cgtp_plan p, int n_nodes, int n_edges, int mult_out, size_t* bytes) {
-  if (p == nullptr || n_nodes < 0 || n_edges < 0 || mult_out <= 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (!mode_is(p, CGTP_MODE_CONV_UVW) || n_nodes < 0 || n_edges < 0 || mult_out <= 0 || bytes == nullptr)
+    return CGTP_ERR_INVALID_ARG;
   UvwLayout L;
   UvwBwdParts W;
   if (!uvw_bwd_parts(p, n_nodes, n_edges, mult_out, true, true, &L, &W)) return CGTP_ERR_UNSUPPORTED;
@@ -556,8 +669,8 @@ cgtp_status cgtp_uvw_backward(cgtp_plan p, int n_nodes, int n_edges, const int* 
                               const float* x, const float* w, const float* mix, int mult_out, const float* grad_out,
                               float* grad_x, float* grad_w, float* grad_mix, float* grad_edge_vec, void* workspace,
                               size_t workspace_bytes, void* stream) {
-  if (p == nullptr || n_nodes < 0 || n_edges < 0 || row_ptr == nullptr || csc_ptr == nullptr || mult_out <= 0 ||
-      mix == nullptr)
+  if (!mode_is(p, CGTP_MODE_CONV_UVW) || n_nodes < 0 || n_edges < 0 || row_ptr == nullptr || csc_ptr == nullptr ||
+      mult_out <= 0 || mix == nullptr)
     return CGTP_ERR_INVALID_ARG;
   if (n_nodes > 0 && (x == nullptr || grad_out == nullptr)) return CGTP_ERR_INVALID_ARG;
   if (n_edges > 0 && (col == nullptr || csc_edge == nullptr || csc_dst == nullptr || edge_vec == nullptr ||
@@ -586,8 +699,12 @@ cgtp_status cgtp_uvw_backward(cgtp_plan p, int n_nodes, int n_edges, const int* 
   float* part = (float*)(ws + W.gt + W.t + W.packed);
   void* gws = ws + W.gt + W.t + W.packed + W.part;
   float* bws = (float*)(ws + W.gt + W.t + W.packed + W.part + W.gemm);
+  const int* abort_flag = nullptr;
+  cudaError_t e = validate_graph(p, n_nodes, n_edges, row_ptr, col, edge_vec, csc_ptr, csc_edge, csc_dst, sms, s,
+                                 &abort_flag);
+  if (e != cudaSuccess) return cuda_fail(e);
   // per-path output gradients gt (tensor cores)
-  cudaError_t e = launch_uvw_pack_t(p->n_paths, p->mult, mult_out, p->lo, L.order, L.count_l3, mix, packed_t, s);
+  e = launch_uvw_pack_t(p->n_paths, p->mult, mult_out, p->lo, L.order, L.count_l3, mix, packed_t, s);
   if (e == cudaSuccess)
     e = launch_uvw_gt(n_nodes, p->lo, L.count_l3, p->mult, mult_out, grad_out, packed_t, gt, gws, W.gemm, s);
   // channelwise backward with one output gradient per path
@@ -597,80 +714,26 @@ cgtp_status cgtp_uvw_backward(cgtp_plan p, int n_nodes, int n_edges, const int* 
     } else {
       ConvBwdArgs a{n_nodes, n_edges, csc_ptr, csc_edge, csc_dst, edge_vec, x, w, gt,
                     grad_x, grad_w, grad_edge_vec, bws, p->mult};
+      a.abort_flag = abort_flag;
       e = cudaErrorNotSupported;
 #define CGTP_UVWB_BWD_ENTRY(A, B, C) \
       if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_bwd_paths<A, B, C>(a, sms, s);
-      CGTP_CONFIGS(CGTP_UVWB_BWD_ENTRY)
+      CGTP_VARIANT_CONFIGS(CGTP_UVWB_BWD_ENTRY)
     }
   }
   // grad_mix from the recomputed per-path messages t (tensor cores)
   if (e == cudaSuccess && grad_mix != nullptr) {
     ConvFwdArgs a{n_nodes, row_ptr, col, edge_vec, x, w, t, p->mult};
+    a.abort_flag = abort_flag;
     e = cudaErrorNotSupported;
 #define CGTP_UVWB_PATHS_ENTRY(A, B, C) \
     if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_paths<A, B, C>(a, sms, s);
-    CGTP_CONFIGS(CGTP_UVWB_PATHS_ENTRY)
+    CGTP_VARIANT_CONFIGS(CGTP_UVWB_PATHS_ENTRY)
     if (e == cudaSuccess)
       e = launch_uvw_grad_mix(n_nodes, p->n_paths, p->lo, L.order, L.count_l3, p->mult, mult_out, t, grad_out, part,
                               grad_mix, gws, W.gemm, s);
   }
   if (e == cudaErrorNotSupported) return CGTP_ERR_UNSUPPORTED;
-  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
-}
-
-// ---- weights shared by every path (path stride 0) ----
-cgtp_status cgtp_conv_forward_shared_weights(cgtp_plan p, int n_nodes, int n_edges, const int* row_ptr,
-                                             const int* col, const float* edge_vec, const float* x, const float* w,
-                                             float* out, void* stream) {
-  if (p == nullptr || n_nodes < 0 || n_edges < 0 || row_ptr == nullptr) return CGTP_ERR_INVALID_ARG;
-  if (n_nodes > 0 && (x == nullptr || out == nullptr)) return CGTP_ERR_INVALID_ARG;
-  if (n_edges > 0 && (col == nullptr || edge_vec == nullptr || w == nullptr)) return CGTP_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(w) || !aligned16(out)) return CGTP_ERR_INVALID_ARG;
-  if (n_nodes == 0) return CGTP_OK;
-  int sms = 0;
-  cgtp_status st = ensure_device(&sms);
-  if (st != CGTP_OK) return st;
-  ConvFwdArgs a{n_nodes, row_ptr, col, edge_vec, x, w, out, p->mult};
-  cudaError_t e = cudaErrorNotSupported;
-#define CGTP_SFWD_ENTRY(A, B, C) \
-  if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_fwd_shared<A, B, C>(a, sms, (cudaStream_t)stream);
-  CGTP_CONFIGS(CGTP_SFWD_ENTRY)
-  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
-}
-
-cgtp_status cgtp_conv_backward_shared_weights(cgtp_plan p, int n_nodes, int n_edges, const int* csc_ptr,
-                                              const int* csc_edge, const int* csc_dst, const float* edge_vec,
-                                              const float* x, const float* w, const float* grad_out, float* grad_x,
-                                              float* grad_w, float* grad_edge_vec, void* workspace,
-                                              size_t workspace_bytes, void* stream) {
-  if (p == nullptr || n_nodes < 0 || n_edges < 0 || csc_ptr == nullptr) return CGTP_ERR_INVALID_ARG;
-  if (n_nodes > 0 && (x == nullptr || grad_out == nullptr)) return CGTP_ERR_INVALID_ARG;
-  if (n_edges > 0 && (csc_edge == nullptr || csc_dst == nullptr || edge_vec == nullptr || w == nullptr))
-    return CGTP_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(w) || !aligned16(grad_out) || !aligned16(grad_x) || !aligned16(grad_w))
-    return CGTP_ERR_INVALID_ARG;
-  if (grad_edge_vec != nullptr && n_edges > 0) {
-    size_t need = 0;
-    cgtp_conv_backward_workspace_size(p, n_edges, &need);  // same chunks, same partials
-    if (workspace == nullptr || workspace_bytes < need || ((uintptr_t)workspace & 255u) != 0)
-      return CGTP_ERR_WORKSPACE;
-  }
-  int sms = 0;
-  cgtp_status st = ensure_device(&sms);
-  if (st != CGTP_OK) return st;
-  cudaStream_t s = (cudaStream_t)stream;
-  if (n_nodes == 0) return CGTP_OK;
-  if (n_edges == 0) {
-    cudaError_t e = cudaSuccess;
-    if (grad_x) e = cudaMemsetAsync(grad_x, 0, sizeof(float) * (size_t)n_nodes * (p->li + 1) * (p->li + 1) * p->mult, s);
-    return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
-  }
-  ConvBwdArgs a{n_nodes, n_edges, csc_ptr, csc_edge, csc_dst, edge_vec, x, w, grad_out,
-                grad_x, grad_w, grad_edge_vec, (float*)workspace, p->mult};
-  cudaError_t e = cudaErrorNotSupported;
-#define CGTP_SBWD_ENTRY(A, B, C) \
-  if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_bwd_shared<A, B, C>(a, sms, s);
-  CGTP_CONFIGS(CGTP_SBWD_ENTRY)
   return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
 }
 
@@ -686,9 +749,33 @@ cgtp_status cgtp_forces(int n_nodes, int n_edges, const int* row_ptr, const int*
   return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
 }
 
+// Weights per edge of a convolution plan: one row per path, or one shared row.
+static int edge_weights(cgtp_plan p) { return p->mode == CGTP_MODE_CONV_UVU_SHARED ? p->mult : p->n_paths * p->mult; }
+
+cgtp_status cgtp_gather_rows(int n, int row_floats, const int* idx, const float* src, float* dst, void* stream) {
+  if (n < 0 || row_floats < 0) return CGTP_ERR_INVALID_ARG;
+  if (n > 0 && row_floats > 0 && (idx == nullptr || src == nullptr || dst == nullptr)) return CGTP_ERR_INVALID_ARG;
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  cudaError_t e = launch_rows(false, n, row_floats, idx, src, dst, sms, (cudaStream_t)stream);
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
+cgtp_status cgtp_scatter_add_rows(int n, int row_floats, const int* idx, const float* src, float* dst,
+                                  void* stream) {
+  if (n < 0 || row_floats < 0) return CGTP_ERR_INVALID_ARG;
+  if (n > 0 && row_floats > 0 && (idx == nullptr || src == nullptr || dst == nullptr)) return CGTP_ERR_INVALID_ARG;
+  int sms = 0;
+  cgtp_status st = ensure_device(&sms);
+  if (st != CGTP_OK) return st;
+  cudaError_t e = launch_rows(true, n, row_floats, idx, src, dst, sms, (cudaStream_t)stream);
+  return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+}
+
 cgtp_status cgtp_radial_forward(cgtp_plan p, int n_edges, const float* edge_vec, float rc, const float* W1,
                                 const float* W2, float* w, void* stream) {
-  if (p == nullptr || n_edges < 0 || !(rc > 0.f)) return CGTP_ERR_INVALID_ARG;
+  if (p == nullptr || p->mode == CGTP_MODE_PAIR_UVU || n_edges < 0 || !(rc > 0.f)) return CGTP_ERR_INVALID_ARG;
   if (n_edges > 0 && (edge_vec == nullptr || W1 == nullptr || W2 == nullptr || w == nullptr))
     return CGTP_ERR_INVALID_ARG;
   if (!aligned16(W2) || !aligned16(w)) return CGTP_ERR_INVALID_ARG;
@@ -696,13 +783,13 @@ cgtp_status cgtp_radial_forward(cgtp_plan p, int n_edges, const float* edge_vec,
   cgtp_status st = ensure_device(&sms);
   if (st != CGTP_OK) return st;
   cudaError_t e =
-      launch_radial_fwd(n_edges, p->n_paths * p->mult, edge_vec, rc, W1, W2, w, sms, (cudaStream_t)stream);
+      launch_radial_fwd(n_edges, edge_weights(p), edge_vec, rc, W1, W2, w, sms, (cudaStream_t)stream);
   return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
 }
 
 cgtp_status cgtp_radial_backward(cgtp_plan p, int n_edges, const float* edge_vec, float rc, const float* W1,
                                  const float* W2, const float* grad_w, float* grad_edge_vec, void* stream) {
-  if (p == nullptr || n_edges < 0 || !(rc > 0.f)) return CGTP_ERR_INVALID_ARG;
+  if (p == nullptr || p->mode == CGTP_MODE_PAIR_UVU || n_edges < 0 || !(rc > 0.f)) return CGTP_ERR_INVALID_ARG;
   if (n_edges > 0 && (edge_vec == nullptr || W1 == nullptr || W2 == nullptr || grad_w == nullptr ||
                       grad_edge_vec == nullptr))
     return CGTP_ERR_INVALID_ARG;
@@ -710,14 +797,14 @@ cgtp_status cgtp_radial_backward(cgtp_plan p, int n_edges, const float* edge_vec
   int sms = 0;
   cgtp_status st = ensure_device(&sms);
   if (st != CGTP_OK) return st;
-  cudaError_t e = launch_radial_bwd(n_edges, p->n_paths * p->mult, edge_vec, rc, W1, W2, grad_w, grad_edge_vec, sms,
+  cudaError_t e = launch_radial_bwd(n_edges, edge_weights(p), edge_vec, rc, W1, W2, grad_w, grad_edge_vec, sms,
                                     (cudaStream_t)stream);
   return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
 }
 
 cgtp_status cgtp_tp_forward(cgtp_plan p, int batch, const float* x, const float* y, const float* w, float* z,
                             void* stream) {
-  if (p == nullptr || batch < 0) return CGTP_ERR_INVALID_ARG;
+  if (!mode_is(p, CGTP_MODE_PAIR_UVU) || batch < 0) return CGTP_ERR_INVALID_ARG;
   if (batch > 0 && (x == nullptr || y == nullptr || w == nullptr || z == nullptr)) return CGTP_ERR_INVALID_ARG;
   int sms = 0;
   cgtp_status st = ensure_device(&sms);
@@ -731,7 +818,7 @@ cgtp_status cgtp_tp_forward(cgtp_plan p, int batch, const float* x, const float*
 }
 
 cgtp_status cgtp_tp_backward_workspace_size(cgtp_plan p, int batch, size_t* bytes) {
-  if (p == nullptr || batch < 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (!mode_is(p, CGTP_MODE_PAIR_UVU) || batch < 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
   const size_t b = sizeof(float) * (size_t)tp_chunks(batch) * p->n_paths * p->mult;
   *bytes = (b + 255) & ~(size_t)255;
   return CGTP_OK;
@@ -740,7 +827,7 @@ cgtp_status cgtp_tp_backward_workspace_size(cgtp_plan p, int batch, size_t* byte
 cgtp_status cgtp_tp_backward(cgtp_plan p, int batch, const float* x, const float* y, const float* w,
                              const float* grad_z, float* grad_x, float* grad_y, float* grad_w, void* workspace,
                              size_t workspace_bytes, void* stream) {
-  if (p == nullptr || batch < 0) return CGTP_ERR_INVALID_ARG;
+  if (!mode_is(p, CGTP_MODE_PAIR_UVU) || batch < 0) return CGTP_ERR_INVALID_ARG;
   if (batch > 0 && (x == nullptr || y == nullptr || w == nullptr || grad_z == nullptr)) return CGTP_ERR_INVALID_ARG;
   if (grad_w != nullptr) {
     size_t need = 0;
@@ -775,7 +862,7 @@ static size_t cp_smem_for(cgtp_plan p, int rank, bool factor_grads) {
 
 cgtp_status cgtp_cp_forward(cgtp_plan p, int rank, int batch, const float* A, const float* B, const float* C,
                             const float* x, const float* y, float* z, void* stream) {
-  if (p == nullptr || rank < 1 || batch < 0) return CGTP_ERR_INVALID_ARG;
+  if (!mode_is(p, CGTP_MODE_PAIR_UVU) || rank < 1 || batch < 0) return CGTP_ERR_INVALID_ARG;
   if (A == nullptr || B == nullptr || C == nullptr) return CGTP_ERR_INVALID_ARG;
   if (batch > 0 && (x == nullptr || y == nullptr || z == nullptr)) return CGTP_ERR_INVALID_ARG;
   int sms = 0;
@@ -792,7 +879,7 @@ cgtp_status cgtp_cp_forward(cgtp_plan p, int rank, int batch, const float* A, co
 }
 
 cgtp_status cgtp_cp_backward_workspace_size(cgtp_plan p, int rank, int batch, size_t* bytes) {
-  if (p == nullptr || rank < 1 || batch < 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
+  if (!mode_is(p, CGTP_MODE_PAIR_UVU) || rank < 1 || batch < 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
   const int d1 = (p->li + 1) * (p->li + 1), d2 = (p->ls + 1) * (p->ls + 1), d3 = (p->lo + 1) * (p->lo + 1);
   const size_t b = sizeof(float) * (size_t)cp_bwd_blocks(batch, p->mult) * (size_t)(d1 + d2 + d3) * (size_t)rank;
   *bytes = (b + 255) & ~(size_t)255;
@@ -803,7 +890,7 @@ cgtp_status cgtp_cp_backward(cgtp_plan p, int rank, int batch, const float* A, c
                              const float* x, const float* y, const float* grad_z, float* grad_x, float* grad_y,
                              float* grad_A, float* grad_B, float* grad_C, void* workspace, size_t workspace_bytes,
                              void* stream) {
-  if (p == nullptr || rank < 1 || batch < 0) return CGTP_ERR_INVALID_ARG;
+  if (!mode_is(p, CGTP_MODE_PAIR_UVU) || rank < 1 || batch < 0) return CGTP_ERR_INVALID_ARG;
   if (A == nullptr || B == nullptr || C == nullptr) return CGTP_ERR_INVALID_ARG;
   if (batch > 0 && (x == nullptr || y == nullptr || grad_z == nullptr)) return CGTP_ERR_INVALID_ARG;
   const bool gf = grad_A != nullptr || grad_B != nullptr || grad_C != nullptr;
@@ -874,7 +961,7 @@ cgtp_status noalloc_scratch(float** out) {
 extern "C" cgtp_status cgtp_tp_backward_noalloc(cgtp_plan p, int batch, const float* x, const float* y,
                                                 const float* w, const float* grad_z, float* grad_x,
                                                 float* grad_y, float* grad_w, void* stream) {
-  if (p == nullptr || batch < 0) return CGTP_ERR_INVALID_ARG;
+  if (!mode_is(p, CGTP_MODE_PAIR_UVU) || batch < 0) return CGTP_ERR_INVALID_ARG;
   if (batch > 0 && (x == nullptr || y == nullptr || w == nullptr || grad_z == nullptr)) return CGTP_ERR_INVALID_ARG;
   float* scratch = nullptr;
   if (grad_w != nullptr) {

@@ -99,6 +99,11 @@ __device__ __forceinline__ void f4_to(float (&a)[4], float4 v) {
 }
 __device__ __forceinline__ float4 to_f4(const float (&a)[4]) { return make_float4(a[0], a[1], a[2], a[3]); }
 
+// Bits of the graph validation (graph.cu) that make a launch unsafe (offsets
+// and indices out of range): a kernel given a flag word with any of them set
+// does no work.
+constexpr int kGraphUnsafeBits = 1 | 2 | 16 | 32;
+
 // ---- launch arguments ----
 struct ConvFwdArgs {
   int n_nodes;
@@ -113,6 +118,9 @@ struct ConvFwdArgs {
   // Y(edge_vec) (the double backward substitutes directional derivatives)
   const float* sh = nullptr;
   int accumulate = 0;  // add onto out instead of overwriting it
+  // checked mode: the plan's validation flags, written by a validation
+  // launch earlier in the stream; the kernel does nothing if they are unsafe
+  const int* abort_flag = nullptr;
 };
 
 struct ConvBwdArgs {
@@ -137,6 +145,7 @@ struct ConvBwdArgs {
   // 3: = sum_b G_b (d2Y_b/dr2) gr_dir
   int gr_mode = 0;
   const float* gr_dir = nullptr;  // [n_edges][3], for gr_mode 2 and 3
+  const int* abort_flag = nullptr;  // checked mode, as in ConvFwdArgs
 };
 
 struct TPArgs {

@@ -293,31 +293,64 @@ cudaError_t launch_csr_transpose(int n, int n_edges, const int* row_ptr, const i
 }
 
 // ---------------------------------------------------------------- validation
-static __global__ void graph_check_kernel(int n, int n_edges, const int* __restrict__ row_ptr,
-                                   const int* __restrict__ col, const float* __restrict__ edge_vec,
-                                   int* __restrict__ flags) {
+// Flag bits (OR-ed into *flags): 1 CSR offsets (row_ptr[0] != 0,
+// row_ptr[n] != n_edges or decreasing), 2 CSR source out of range,
+// 4 zero-length edge vector, 8 non-finite edge vector, 16 CSC offsets,
+// 32 CSC edge number or destination out of range.  Any array may be null
+// (not checked).
+static __global__ void graph_validate_kernel(int n, int n_edges, const int* __restrict__ row_ptr,
+                                             const int* __restrict__ col, const float* __restrict__ edge_vec,
+                                             const int* __restrict__ csc_ptr, const int* __restrict__ csc_edge,
+                                             const int* __restrict__ csc_dst, int* __restrict__ flags) {
   const long long stride = (long long)gridDim.x * blockDim.x;
   const long long t0 = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   int f = 0;
-  if (t0 == 0 && (row_ptr[0] != 0 || row_ptr[n] != n_edges)) f |= 1;
-  for (long long i = t0; i < n; i += stride)
-    if (row_ptr[i + 1] < row_ptr[i]) f |= 1;
+  if (row_ptr != nullptr) {
+    if (t0 == 0 && (row_ptr[0] != 0 || row_ptr[n] != n_edges)) f |= 1;
+    for (long long i = t0; i < n; i += stride)
+      if (row_ptr[i + 1] < row_ptr[i]) f |= 1;
+  }
+  if (csc_ptr != nullptr) {
+    if (t0 == 0 && (csc_ptr[0] != 0 || csc_ptr[n] != n_edges)) f |= 16;
+    for (long long i = t0; i < n; i += stride)
+      if (csc_ptr[i + 1] < csc_ptr[i]) f |= 16;
+  }
   for (long long e = t0; e < n_edges; e += stride) {
-    const int j = col[e];
-    if (j < 0 || j >= n) f |= 2;
-    const float x = edge_vec[3 * e], y = edge_vec[3 * e + 1], z = edge_vec[3 * e + 2];
-    if (!(isfinite(x) && isfinite(y) && isfinite(z))) f |= 8;
-    else if (x == 0.f && y == 0.f && z == 0.f) f |= 4;
+    if (col != nullptr) {
+      const int j = col[e];
+      if (j < 0 || j >= n) f |= 2;
+    }
+    if (csc_edge != nullptr) {
+      const int k = csc_edge[e];
+      if (k < 0 || k >= n_edges) f |= 32;
+    }
+    if (csc_dst != nullptr) {
+      const int d = csc_dst[e];
+      if (d < 0 || d >= n) f |= 32;
+    }
+    if (edge_vec != nullptr) {
+      const float x = edge_vec[3 * e], y = edge_vec[3 * e + 1], z = edge_vec[3 * e + 2];
+      if (!(isfinite(x) && isfinite(y) && isfinite(z))) f |= 8;
+      else if (x == 0.f && y == 0.f && z == 0.f) f |= 4;
+    }
   }
   if (f) atomicOr(flags, f);
+}
+
+cudaError_t launch_graph_validate(int n, int n_edges, const int* row_ptr, const int* col, const float* edge_vec,
+                                  const int* csc_ptr, const int* csc_edge, const int* csc_dst, int* flags,
+                                  int num_sms, cudaStream_t stream) {
+  graph_validate_kernel<<<num_sms * 4, 256, 0, stream>>>(n, n_edges, row_ptr, col, edge_vec, csc_ptr, csc_edge,
+                                                          csc_dst, flags);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_graph_check(int n, int n_edges, const int* row_ptr, const int* col, const float* edge_vec,
                                int* flags, int num_sms, cudaStream_t stream) {
   cudaError_t e = cudaMemsetAsync(flags, 0, sizeof(int), stream);
   if (e != cudaSuccess) return e;
-  graph_check_kernel<<<num_sms * 4, 256, 0, stream>>>(n, n_edges, row_ptr, col, edge_vec, flags);
-  return cudaGetLastError();
+  return launch_graph_validate(n, n_edges, row_ptr, col, edge_vec, nullptr, nullptr, nullptr, flags, num_sms,
+                               stream);
 }
 
 }  // namespace cgtp

@@ -4,9 +4,27 @@
 
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace cgtp {
+
+// ---- side streams (lanes.cu) ----
+// Launches of one call that write disjoint outputs run on lanes forked from
+// the caller's stream (lanes_fork: lanes 0..n-1 wait for it) and joined back
+// (lanes_join: the caller's stream waits for them).  A host thread holds
+// side_lanes_mutex(pool) from the fork to the join (the events are shared).
+constexpr int kMaxSideLanes = 4;
+enum { kLanesBwd = 0, kLanesUvw = 1, kLanePools = 2 };
+struct SideLanes {
+  cudaStream_t side[kMaxSideLanes];
+  cudaEvent_t fork, join[kMaxSideLanes];
+};
+cudaError_t side_lanes(int pool, SideLanes** out);
+std::mutex& side_lanes_mutex(int pool);
+cudaError_t lanes_fork(SideLanes* L, int n, cudaStream_t s);
+cudaError_t lanes_join(SideLanes* L, int n, cudaStream_t s);
 
 // Arguments of the CP-decomposed tensor product (cp.cu): factors A [d3][R],
 // B [d1][R], C [d2][R]; features [batch][d][mult]; partial: the backward's
@@ -58,8 +76,6 @@ cudaError_t launch_conv_bwd_paths(const ConvBwdArgs& a, int num_sms, cudaStream_
 template <int LI, int LS, int LO>
 cudaError_t launch_conv_bwd_gy(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);
 template <int LI, int LS, int LO>
-int paths_bwd_slices(int mult);
-template <int LI, int LS, int LO>
 cudaError_t launch_conv_bwd(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);
 template <int LI, int LS, int LO>
 int conv_bwd_slices(int mult);
@@ -76,6 +92,10 @@ cudaError_t launch_csr_transpose(int n, int n_edges, const int* row_ptr, const i
                                  int* csc_edge, int* csc_dst, int* ws, int num_sms, cudaStream_t stream);
 cudaError_t launch_graph_check(int n, int n_edges, const int* row_ptr, const int* col, const float* edge_vec,
                                int* flags, int num_sms, cudaStream_t stream);
+// OR the validation bits of the given arrays (each nullable) into *flags.
+cudaError_t launch_graph_validate(int n, int n_edges, const int* row_ptr, const int* col, const float* edge_vec,
+                                  const int* csc_ptr, const int* csc_edge, const int* csc_dst, int* flags,
+                                  int num_sms, cudaStream_t stream);
 cudaError_t launch_radial_fwd(int n_edges, int N, const float* ev, float rc, const float* W1, const float* W2,
                               float* w, int num_sms, cudaStream_t stream);
 cudaError_t launch_radial_bwd(int n_edges, int N, const float* ev, float rc, const float* W1, const float* W2,
@@ -100,6 +120,10 @@ cudaError_t launch_uvw_gt(int n_nodes, int lmax_out, const int* count_l3, int mu
 cudaError_t launch_uvw_grad_mix(int n_nodes, int n_paths, int lmax_out, const int* order, const int* count_l3,
                                 int mult, int mult_out, const float* t, const float* g, float* part,
                                 float* grad_mix, void* ws, size_t ws_bytes, cudaStream_t stream);
+// dst[k] = src[idx[k]] (add = false) or dst[idx[k]] += src[k] (add = true)
+// for n rows of rf floats; idx unique within one call.
+cudaError_t launch_rows(bool add, int n, int rf, const int* idx, const float* src, float* dst, int num_sms,
+                        cudaStream_t stream);
 cudaError_t launch_sh_dir(int lmax_sh, int n_edges, const float* ev, const float* q, float* u, int num_sms,
                           cudaStream_t stream);
 

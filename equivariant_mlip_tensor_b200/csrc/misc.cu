@@ -1,4 +1,5 @@
-// Per-atom forces from edge gradients, and materialised spherical harmonics,
+// Per-atom forces from edge gradients, materialised spherical harmonics, and
+// the row gather / scatter-add of the domain decomposition's halo exchange,
 // for sm_100a.
 //
 // Forces: with r_e = pos_src - pos_dst, dE/dpos_n = sum_{e: src=n} g_e -
@@ -6,6 +7,7 @@
 // (contiguous) and its CSC row (through the edge permutation), so there are
 // no atomics and the summation order is fixed.
 #include <cuda_runtime.h>
+#include <stdint.h>
 
 #include "common.cuh"
 
@@ -78,7 +80,63 @@ __global__ void sh_dir_kernel(int n_edges, const float* __restrict__ ev, const f
   }
 }
 
+// Row gather and scatter-add (the pack and unpack of a halo exchange):
+// element t of the n x rf block is row t / rf, column t % rf; float4 steps
+// when every row is a whole number of 16-byte vectors.
+__global__ void gather_rows_kernel(long long total, int rf, int vec4, const int* __restrict__ idx,
+                                   const float* __restrict__ src, float* __restrict__ dst) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  if (vec4) {
+    const int rq = rf / 4;
+    for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < total / 4; t += stride) {
+      const long long r = t / rq, c = t % rq;
+      reinterpret_cast<float4*>(dst)[r * rq + c] = reinterpret_cast<const float4*>(src)[(long long)idx[r] * rq + c];
+    }
+  } else {
+    for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < total; t += stride) {
+      const long long r = t / rf, c = t % rf;
+      dst[r * rf + c] = src[(long long)idx[r] * rf + c];
+    }
+  }
+}
+
+__global__ void scatter_add_rows_kernel(long long total, int rf, int vec4, const int* __restrict__ idx,
+                                        const float* __restrict__ src, float* __restrict__ dst) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  if (vec4) {
+    const int rq = rf / 4;
+    for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < total / 4; t += stride) {
+      const long long r = t / rq, c = t % rq;
+      float4* d = reinterpret_cast<float4*>(dst) + (long long)idx[r] * rq + c;
+      const float4 v = reinterpret_cast<const float4*>(src)[r * rq + c];
+      float4 o = *d;
+      o.x += v.x;
+      o.y += v.y;
+      o.z += v.z;
+      o.w += v.w;
+      *d = o;
+    }
+  } else {
+    for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < total; t += stride) {
+      const long long r = t / rf, c = t % rf;
+      dst[(long long)idx[r] * rf + c] += src[r * rf + c];
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_rows(bool add, int n, int rf, const int* idx, const float* src, float* dst, int num_sms,
+                        cudaStream_t stream) {
+  if (n == 0 || rf == 0) return cudaSuccess;
+  const long long total = (long long)n * rf;
+  const int vec4 = (rf % 4 == 0 && ((uintptr_t)src & 15u) == 0 && ((uintptr_t)dst & 15u) == 0) ? 1 : 0;
+  long long b = ((vec4 ? total / 4 : total) + 255) / 256;
+  if (b > num_sms * 16LL) b = num_sms * 16LL;
+  if (add) scatter_add_rows_kernel<<<(int)b, 256, 0, stream>>>(total, rf, vec4, idx, src, dst);
+  else gather_rows_kernel<<<(int)b, 256, 0, stream>>>(total, rf, vec4, idx, src, dst);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_sh_dir(int lmax_sh, int n_edges, const float* ev, const float* q, float* u, int num_sms,
                           cudaStream_t stream) {

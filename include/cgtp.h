@@ -64,6 +64,30 @@ typedef enum {
 
 typedef struct cgtp_plan_s* cgtp_plan;
 
+/* What a plan computes.  Every entry point states the modes it accepts and
+ * returns CGTP_ERR_INVALID_ARG for a plan of another mode.
+ *  CGTP_MODE_CONV_UVU         the channelwise convolution over a graph, one
+ *                             weight per edge, path and channel (w [E][P][u]):
+ *                             cgtp_conv_forward / _backward / _double_backward,
+ *                             cgtp_radial_*;
+ *  CGTP_MODE_PAIR_UVU         the edge-free channelwise product of batched pairs
+ *                             and its CP-decomposed surrogate: cgtp_tp_*, cgtp_cp_*;
+ *  CGTP_MODE_CONV_UVU_SHARED  the channelwise convolution with one weight row per
+ *                             edge shared by every path (path stride 0, w [E][u];
+ *                             "Tensor Decomposition Networks ...", reply to
+ *                             reviewer oXft): cgtp_conv_forward / _backward,
+ *                             cgtp_radial_*;
+ *  CGTP_MODE_CONV_UVW         the fully connected convolution (channelwise
+ *                             messages mixed across channels per path;
+ *                             "Tensor Decomposition Networks ...", reply to
+ *                             reviewer cmnz): cgtp_uvw_*, cgtp_radial_*. */
+typedef enum {
+  CGTP_MODE_CONV_UVU = 0,
+  CGTP_MODE_PAIR_UVU = 1,
+  CGTP_MODE_CONV_UVU_SHARED = 2,
+  CGTP_MODE_CONV_UVW = 3
+} cgtp_mode;
+
 /* Human-readable name of a status code (static string). */
 const char* cgtp_status_string(cgtp_status s);
 
@@ -72,21 +96,50 @@ const char* cgtp_status_string(cgtp_status s);
 int cgtp_last_cuda_error(void);
 
 /* ---------------------------------------------------------------------------
- * Plan: the path list and the real CG coefficients for one irreps shape.
- * ("Tensor Decomposition Networks ...", reply to S6y1: only triples obeying
- * |l1-l2| <= l3 <= l1+l2 and m3 = m1+m2 are nonzero.)
+ * Plan: the path list and the real CG coefficients of one irreps shape, for
+ * one mode.  ("Tensor Decomposition Networks ...", reply to S6y1: only
+ * triples obeying |l1-l2| <= l3 <= l1+l2 and m3 = m1+m2 are nonzero.)
  * Builds the coefficients on the host (fp64, by the angular-momentum
  * lowering operator and the complex-to-real change of basis), checks them,
  * and uploads them once per device to constant memory (synchronous copy on
  * the current device).  mult must be a positive multiple of 4.
- * Supported (lmax_in, lmax_sh, lmax_out): see cgtp_supported().
- * Returns CGTP_ERR_UNSUPPORTED for shapes that are not compiled in.
+ * Returns CGTP_ERR_INVALID_ARG for a negative l, a bad mult or an unknown
+ * mode, and CGTP_ERR_UNSUPPORTED for a shape whose kernels are not compiled
+ * in for the mode (see cgtp_supported).  The plan owns its host path list
+ * and, in checked mode, 16 bytes of device memory; nothing else.
  * ------------------------------------------------------------------------- */
-cgtp_status cgtp_plan_create(int lmax_in, int lmax_sh, int lmax_out, int mult, cgtp_plan* plan);
+cgtp_status cgtp_plan_create(int lmax_in, int lmax_sh, int lmax_out, int mult, cgtp_mode mode,
+                             cgtp_plan* plan);
 cgtp_status cgtp_plan_destroy(cgtp_plan plan);
 
-/* 1 if kernels for this (lmax_in, lmax_sh, lmax_out) are compiled in. */
-int cgtp_supported(int lmax_in, int lmax_sh, int lmax_out);
+/* 1 if the kernels of (lmax_in, lmax_sh, lmax_out) are compiled in for the
+ * mode, else 0.  Compiled shapes, all with lmax_in, lmax_out <= 3 and
+ * lmax_sh <= 4:
+ *  CONV_UVU, PAIR_UVU: every interaction shape (lmax_in == lmax_out), every
+ *    embedding shape (lmax_in == 0) and every read-out shape (lmax_out == 0);
+ *  CONV_UVU_SHARED, CONV_UVW: (0,0,0), (1,1,1), (1,2,1), (2,2,2), (2,4,2),
+ *    (3,3,3).
+ * Host only. */
+int cgtp_supported(int lmax_in, int lmax_sh, int lmax_out, cgtp_mode mode);
+
+/* Checked mode (off by default).  With checked != 0, every convolution call
+ * of the plan first validates, on the device and in its stream, the graph
+ * arrays it is given, OR-ing the bits of cgtp_graph_check (plus 16 = CSC
+ * offsets not monotone or not ending at n_edges, 32 = a CSC edge number or
+ * destination out of range) into the plan's flags.  If an offset or index
+ * bit (1, 2, 16 or 32) is set, the call's convolution kernels do no work
+ * (their outputs are left unspecified), so an invalid graph cannot make them
+ * read or write out of bounds.  The first switch-on allocates the flags
+ * (16 bytes) on the current device; the plan's checked calls must then run
+ * on that device (CGTP_ERR_CUDA otherwise). */
+cgtp_status cgtp_plan_set_checked(cgtp_plan plan, int checked);
+
+/* Reads and clears the flags that the plan's checked-mode calls recorded:
+ * synchronises the device (every stream), stores the bits in *flags
+ * (nullable) and returns CGTP_ERR_BAD_GRAPH if any bit is set, CGTP_OK if
+ * none (also for a plan never put in checked mode).  Not for use during
+ * stream capture. */
+cgtp_status cgtp_plan_check(cgtp_plan plan, int* flags);
 
 /* Number of paths; if paths_l1l2l3 is not NULL it receives 3*n_paths ints
  * (l1, l2, l3 per path, lexicographic).  n_cg_nonzero (nullable) receives
@@ -100,7 +153,11 @@ cgtp_status cgtp_cg_block(int l1, int l2, int l3, double* out);
 
 /* ---------------------------------------------------------------------------
  * Neighbour list (CSR by destination + CSC by source), brute force over the
- * candidate pairs of each graph, bit-exact contract:
+ * candidate pairs of each graph.  (The convolution sums over the neighbours
+ * of each atom within a cutoff, as interatomic potentials do: "LunaTP ...",
+ * abstract, convolutions over atomic neighbourhoods; the machine review of
+ * "AccelNet", summary: sums over the neighbours within the cutoff.  The
+ * pages fix no algorithm; this one is exact.)  Bit-exact contract:
  *   d = p_j - p_i per axis in fp64 (positions upcast from fp32);
  *   periodic box (side box_len > 0): d <- d - L*rint(d/L), each operation
  *   rounded separately (rint: halves to even); box_len <= 0 means no box;
@@ -129,7 +186,8 @@ cgtp_status cgtp_csr_transpose(int n, int n_edges, const int* row_ptr, const int
                                int* csc_ptr, int* csc_edge, int* csc_dst,
                                void* workspace, size_t workspace_bytes, void* stream);
 
-/* Device-side validation of a CSR graph: sets bits of *flags (device int,
+/* Device-side validation of a CSR graph (the checks that checked-mode plans
+ * run; an addition of this library): sets bits of *flags (device int,
  * cleared by the call): 1 = row_ptr not monotone or row_ptr[0] != 0 or
  * row_ptr[n] != n_edges, 2 = col out of range, 4 = zero-length edge vector,
  * 8 = non-finite edge vector. */
@@ -147,7 +205,9 @@ cgtp_status cgtp_spherical_harmonics(int lmax_sh, int n_edges, const float* edge
 
 /* ---------------------------------------------------------------------------
  * Convolution forward (node-centric: one owner per destination row, no
- * atomics).  x: [n_nodes][(lmax_in+1)^2][mult]; w: [n_edges][n_paths][mult];
+ * atomics).  Modes CONV_UVU and CONV_UVU_SHARED.
+ * x: [n_nodes][(lmax_in+1)^2][mult]; w: [n_edges][n_paths][mult], or
+ * [n_edges][mult] (one row shared by every path) for CONV_UVU_SHARED;
  * out: [n_nodes][(lmax_out+1)^2][mult] (overwritten).
  * ------------------------------------------------------------------------- */
 cgtp_status cgtp_conv_forward(cgtp_plan plan, int n_nodes, int n_edges,
@@ -155,11 +215,15 @@ cgtp_status cgtp_conv_forward(cgtp_plan plan, int n_nodes, int n_edges,
                               const float* x, const float* w, float* out, void* stream);
 
 /* Bytes of device workspace cgtp_conv_backward needs when grad_edge_vec is
- * requested (0 otherwise is also accepted). */
+ * requested (0 otherwise is also accepted).  Modes CONV_UVU,
+ * CONV_UVU_SHARED, CONV_UVW. */
 cgtp_status cgtp_conv_backward_workspace_size(cgtp_plan plan, int n_edges, size_t* bytes);
 
 /* ---------------------------------------------------------------------------
- * Convolution backward, node-centric over sources (CSC), one read of W:
+ * Convolution backward, node-centric over sources (CSC), one read of W
+ * (modes CONV_UVU and CONV_UVU_SHARED; with the latter w and grad_w are
+ * [n_edges][mult] and grad_w[e] is the sum over paths of the per-path weight
+ * gradients):
  *   grad_x[j] = sum_{e: src=j} sum_p W_e[p] (T_e^p)^T grad_out[dst(e)]
  *   grad_w[e][p][u] = sum C x[j] Y_e grad_out[i]
  *   grad_edge_vec[e] = (dY_e/dr_e)^T sum_u sum_p W x grad_out C
@@ -181,13 +245,13 @@ cgtp_status cgtp_conv_backward(cgtp_plan plan, int n_nodes, int n_edges,
                                void* stream);
 
 /* Bytes of device workspace cgtp_conv_double_backward needs when
- * gg_edge_vec or d_edge_vec is given. */
+ * gg_edge_vec or d_edge_vec is given.  Mode CONV_UVU. */
 cgtp_status cgtp_conv_double_backward_workspace_size(cgtp_plan plan, int n_edges, size_t* bytes);
 
 /* ---------------------------------------------------------------------------
  * Double backward: the adjoint of cgtp_conv_backward, the higher-order
  * derivative that force training needs ("LunaTP ...", abstract: derivative
- * computation).  With (grad_x, grad_w, grad_edge_vec) the outputs of
+ * computation).  Mode CONV_UVU.  With (grad_x, grad_w, grad_edge_vec) the outputs of
  * cgtp_conv_backward for (x, w, grad_out, edge_vec) and cotangents gg_x
  * [n_nodes][(lmax_in+1)^2][mult], gg_w [n_edges][n_paths][mult] and
  * gg_edge_vec [n_edges][3] (each nullable = zero), the call returns the
@@ -215,13 +279,14 @@ cgtp_status cgtp_conv_double_backward(cgtp_plan plan, int n_nodes, int n_edges,
 
 /* Bytes of device workspace cgtp_uvw_forward needs for n_nodes nodes and
  * mult_out output channels (per-path messages, packed mixing matrices and
- * the GEMM's own scratch). */
+ * the GEMM's own scratch).  Mode CONV_UVW. */
 cgtp_status cgtp_uvw_forward_workspace_size(cgtp_plan plan, int n_nodes, int mult_out, size_t* bytes);
 
 /* ---------------------------------------------------------------------------
  * Fully connected ("uvw") convolution forward, the fully connected CG tensor
  * product of Equiformer ("Tensor Decomposition Networks ...", reply to
- * reviewer cmnz): the channelwise convolution's per-path messages, summed
+ * reviewer cmnz), mode CONV_UVW: the channelwise convolution's per-path
+ * messages, summed
  * over each row but kept per path, then mixed across channels by a dense
  * matrix per path and summed into l3 blocks:
  *   t[i][p][m3][u]   = sum_{e in row i} W_e[p][u] sum C^p x[j][l1,m1][u] Y_e[l2,m2]
@@ -243,12 +308,14 @@ cgtp_status cgtp_uvw_forward(cgtp_plan plan, int n_nodes, int n_edges, const int
                              const float* mix, int mult_out, float* out, void* workspace,
                              size_t workspace_bytes, void* stream);
 
-/* Bytes of device workspace cgtp_uvw_backward needs (with every output). */
+/* Bytes of device workspace cgtp_uvw_backward needs (with every output).
+ * Mode CONV_UVW. */
 cgtp_status cgtp_uvw_backward_workspace_size(cgtp_plan plan, int n_nodes, int n_edges, int mult_out,
                                              size_t* bytes);
 
 /* ---------------------------------------------------------------------------
- * Fully connected convolution backward, the adjoint of cgtp_uvw_forward for
+ * Fully connected convolution backward (mode CONV_UVW), the adjoint of
+ * cgtp_uvw_forward for
  * grad_out [n_nodes][(lmax_out+1)^2][mult_out]:
  *   gt[i][p][m3][u]    = sum_v grad_out[i][l3,m3][v] mix[p][u][v]      (tensor cores)
  *   grad_mix[p][u][v]  = sum_i sum_m3 t[i][p][m3][u] grad_out[i][l3,m3][v]  (tensor cores,
@@ -269,29 +336,12 @@ cgtp_status cgtp_uvw_backward(cgtp_plan plan, int n_nodes, int n_edges, const in
                               size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
- * Convolution with weights shared by every path (path stride 0,
- * W_e[p][u] = w[e][u]; "Tensor Decomposition Networks ...", reply to reviewer
- * oXft: one weight set for all paths), forward and backward.  w and grad_w
- * are [n_edges][mult]; grad_w[e] is the sum over paths of the per-path weight
- * gradients.  Everything else as cgtp_conv_forward / cgtp_conv_backward
- * (grad_edge_vec needs cgtp_conv_backward_workspace_size bytes of workspace).
- * One weight row per edge instead of n_paths: the weight stream shrinks by
- * n_paths and the kernels become FP32-bound.
- * ------------------------------------------------------------------------- */
-cgtp_status cgtp_conv_forward_shared_weights(cgtp_plan plan, int n_nodes, int n_edges,
-                                             const int* row_ptr, const int* col,
-                                             const float* edge_vec, const float* x, const float* w,
-                                             float* out, void* stream);
-cgtp_status cgtp_conv_backward_shared_weights(cgtp_plan plan, int n_nodes, int n_edges,
-                                              const int* csc_ptr, const int* csc_edge,
-                                              const int* csc_dst, const float* edge_vec,
-                                              const float* x, const float* w, const float* grad_out,
-                                              float* grad_x, float* grad_w, float* grad_edge_vec,
-                                              void* workspace, size_t workspace_bytes, void* stream);
-
-/* ---------------------------------------------------------------------------
  * Per-atom forces from edge-vector gradients, F = -dE/dpos with
  * r_e = pos_src - pos_dst:  F[n] = sum_{e: dst=n} g[e] - sum_{e: src=n} g[e].
+ * (Potentials predict energies and forces: "Tensor Decomposition Networks
+ * ...", reply to reviewer 7Mvd, the DFT energy and force labels; the machine
+ * review of "AccelNet", summary: analytic forces.  F is the negative gradient
+ * of the energy through the edge vectors.)
  * Segmented sums over the CSR row and the CSC row of each node; no atomics.
  * forces: device [n_nodes][3], overwritten.
  * ------------------------------------------------------------------------- */
@@ -300,9 +350,28 @@ cgtp_status cgtp_forces(int n_nodes, int n_edges, const int* row_ptr, const int*
                         void* stream);
 
 /* ---------------------------------------------------------------------------
- * Radial weight network: 8 Gaussians on [0, rc] (centres k*rc/7, width
- * rc/7) -> a = phi @ W1 [8][64] -> SiLU -> w = h @ W2 [64][n_paths*mult],
- * no biases.  w: [n_edges][n_paths][mult], overwritten.
+ * Row gather and scatter-add: the pack and unpack of the halo exchange of a
+ * graph partitioned over several GPUs (an addition of this library; the
+ * pages name multi-GPU scalability without a method: "LunaTP ...",
+ * abstract).  For n rows of row_floats floats (device arrays, idx int32):
+ *   cgtp_gather_rows:      dst[k][:] = src[idx[k]][:]
+ *   cgtp_scatter_add_rows: dst[idx[k]][:] += src[k][:]  (idx must not repeat
+ *                          within one call; no atomics)
+ * Float4 accesses when row_floats % 4 == 0 and src, dst are 16-byte aligned.
+ * ------------------------------------------------------------------------- */
+cgtp_status cgtp_gather_rows(int n, int row_floats, const int* idx, const float* src, float* dst,
+                             void* stream);
+cgtp_status cgtp_scatter_add_rows(int n, int row_floats, const int* idx, const float* src, float* dst,
+                                  void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Radial weight network (an addition of this library: the pages give none;
+ * this is the per-edge weight generator of the standard workloads, the
+ * Gaussian-basis MLP of NequIP-style potentials): 8 Gaussians on [0, rc]
+ * (centres k*rc/7, width rc/7) -> a = phi @ W1 [8][64] -> SiLU ->
+ * w = h @ W2 [64][K], no biases, K = the plan's weights per edge
+ * (n_paths*mult, or mult for CONV_UVU_SHARED).  Modes CONV_UVU,
+ * CONV_UVU_SHARED, CONV_UVW.  w: [n_edges][K], overwritten.
  * ------------------------------------------------------------------------- */
 cgtp_status cgtp_radial_forward(cgtp_plan plan, int n_edges, const float* edge_vec, float rc,
                                 const float* W1, const float* W2, float* w, void* stream);
@@ -314,9 +383,9 @@ cgtp_status cgtp_radial_backward(cgtp_plan plan, int n_edges, const float* edge_
                                  float* grad_edge_vec, void* stream);
 
 /* ---------------------------------------------------------------------------
- * Edge-free channelwise tensor product of batched pairs ("Tensor
- * Decomposition Networks ...", reply to S6y1: the exact CG product, timed at
- * batch 1000 and multiplicity 128):
+ * Edge-free channelwise tensor product of batched pairs, mode PAIR_UVU
+ * ("Tensor Decomposition Networks ...", reply to S6y1: the exact CG product,
+ * timed at batch 1000 and multiplicity 128):
  *   z[b][l3,m3][u] = sum_p w[p][u] sum C^p[m1,m2,m3] x[b][l1,m1][u] y[b][l2,m2][u]
  * x: [batch][(lmax_in+1)^2][mult], y: [batch][(lmax_sh+1)^2][mult],
  * w: [n_paths][mult], z: [batch][(lmax_out+1)^2][mult] (overwritten).
@@ -334,7 +403,7 @@ cgtp_status cgtp_tp_backward(cgtp_plan plan, int batch, const float* x, const fl
 
 /* ---------------------------------------------------------------------------
  * Allocation-free cgtp_tp_backward (an addition of this library; the paper
- * has no counterpart).  For callers that cannot allocate device memory when
+ * has no counterpart), mode PAIR_UVU.  For callers that cannot allocate device memory when
  * they call in: a host framework that owns all device memory through its own
  * allocator and forbids direct cudaMalloc, or a time-stepping loop that must
  * not allocate after set-up.  Same arguments and results as
@@ -359,7 +428,7 @@ cgtp_status cgtp_tp_backward_noalloc(cgtp_plan plan, int batch, const float* x, 
 /* ---------------------------------------------------------------------------
  * CP-decomposed tensor product ("Tensor Decomposition Networks for
  * Accelerating Machine Learning Force Field Computations", reply to reviewer
- * S6y1 on the backward's complexity): the low-rank surrogate
+ * S6y1 on the backward's complexity), mode PAIR_UVU: the low-rank surrogate
  *   z = A (B^T x (*) C^T y)                  ((*) = elementwise product)
  * of the plan's CG product, applied channelwise with factors shared by every
  * pair and channel:

@@ -89,7 +89,11 @@ def test_pipeline_with_radial_network_and_forces(api, name):
 
 @pytest.mark.parametrize("L,mult", [((0, 0, 0), 4), ((1, 1, 1), 8), ((1, 1, 1), 16), ((1, 2, 1), 32),
                                     ((2, 2, 2), 64), ((2, 2, 2), 96), ((2, 4, 2), 128), ((2, 4, 2), 256),
-                                    ((3, 3, 3), 64), ((3, 3, 3), 128)])
+                                    ((3, 3, 3), 64), ((3, 3, 3), 128),
+                                    # interaction, embedding and read-out shapes of the wider policy
+                                    ((2, 3, 2), 64), ((1, 4, 1), 32), ((3, 4, 3), 32), ((3, 4, 3), 128),
+                                    ((2, 0, 2), 16), ((0, 4, 3), 64), ((0, 1, 1), 8), ((3, 2, 0), 32),
+                                    ((1, 4, 0), 128)])
 def test_shapes_and_multiplicities(api, L, mult):
     rng = np.random.default_rng(30 + mult)
     n = 37  # ragged: not a multiple of any tile
@@ -185,8 +189,60 @@ def test_optional_gradients_and_errors(api):
         plan.conv_backward(g, cuda(w.x), cuda(W), cuda(w.grad_out), workspace=cuda(np.zeros(4, np.float32)))
     assert ei.value.status == 7
     with pytest.raises(CGTPError) as ei:
-        api.Plan(2, 3, 2, 128)
+        api.Plan(2, 3, 1, 128)  # outside the compiled shapes
     assert ei.value.status == 2
+    with pytest.raises(CGTPError) as ei:
+        api.Plan(2, 3, 2, 128, mode="uvw")  # a shape the fully connected mode is not built for
+    assert ei.value.status == 2
+    # an entry point given a plan of another mode
+    from equivariant_mlip_tensor_b200._lib import lib
+    import ctypes
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    z = cuda(np.zeros((2, 4, w.mult), np.float32))
+    assert lib().cgtp_tp_forward(plan.handle("conv"), 2, p(z), p(z), p(z), p(z), None) == 1
+    assert lib().cgtp_conv_forward(plan.handle("pair"), g.n_nodes, g.n_edges, p(g.row_ptr), p(g.col),
+                                   p(g.edge_vec), p(cuda(w.x)), p(cuda(W)), p(cuda(w.x)), None) == 1
     with pytest.raises(CGTPError) as ei:
         api.Plan(1, 1, 1, 6)
     assert ei.value.status == 1
+
+
+def test_checked_mode_reports_and_stops_invalid_graphs(api):
+    """Checked plans validate each call's graph on the device first; an index
+    out of range is reported by cgtp_plan_check and the kernels do no work
+    (the planted index is one past the last node, so even an unguarded read
+    would stay inside the caller's allocation)."""
+    w = synthetic.tiny()
+    L = (w.lmax_in, w.lmax_sh, w.lmax_out)
+    g, o = _graph_pair(api, w)
+    W = _random_w(o, w.n_paths, w.mult, 102)
+    plan = api.Plan(*L, w.mult)
+    plan.set_checked(True)
+    x, Wd, go = cuda(w.x), cuda(W), cuda(w.grad_out)
+    out = plan.conv_forward(g, x, Wd)
+    gx, gw, gr = plan.conv_backward(g, x, Wd, go)
+    assert plan.check() == 0
+    assert rel_err(host(out), oconv.conv_forward(o["row_ptr"], o["col"], o["edge_vec"], w.x, W, *L)) < FWD_TOL
+    rx, rw, rr = oconv.conv_backward(o["row_ptr"], o["col"], o["edge_vec"], w.x, W, w.grad_out, *L)
+    assert rel_err(host(gx), rx) < GRAD_TOL and rel_err(host(gw), rw) < GRAD_TOL
+    bad_col = g.col.clone()
+    bad_col[3] = w.n_nodes
+    gb = api.Graph(g.n_nodes, g.n_edges, g.row_ptr, bad_col, g.edge_vec, g.csc_ptr, g.csc_edge, g.csc_dst)
+    plan.conv_forward(gb, x, Wd)
+    assert plan.check() & 2
+    bad_dst = g.csc_dst.clone()
+    bad_dst[0] = w.n_nodes
+    gb = api.Graph(g.n_nodes, g.n_edges, g.row_ptr, g.col, g.edge_vec, g.csc_ptr, g.csc_edge, bad_dst)
+    plan.conv_backward(gb, x, Wd, go)
+    assert plan.check() & 32
+    bad_ptr = g.csc_ptr.clone()
+    bad_ptr[-1] = g.n_edges + 1
+    gb = api.Graph(g.n_nodes, g.n_edges, g.row_ptr, g.col, g.edge_vec, bad_ptr, g.csc_edge, g.csc_dst)
+    plan.conv_backward(gb, x, Wd, go)
+    assert plan.check() & 16
+    # the flags were cleared and a valid call computes as before
+    out2 = plan.conv_forward(g, x, Wd)
+    assert plan.check() == 0 and np.array_equal(host(out2), host(out))
+    plan.set_checked(False)
+    out3 = plan.conv_forward(g, x, Wd)
+    assert np.array_equal(host(out3), host(out))

@@ -120,16 +120,16 @@ def test_host_errors(api):
     Ad, Bd, Cd, xd, yd, gd = (cuda(v) for v in (A, B, C, x, y, g))
     z = torch.empty((batch, 4, mult), device="cuda")
     f = lib().cgtp_cp_forward
-    assert f(plan._h, 0, batch, p(Ad), p(Bd), p(Cd), p(xd), p(yd), p(z), None) == 1      # rank < 1
-    assert f(plan._h, R, -1, p(Ad), p(Bd), p(Cd), p(xd), p(yd), p(z), None) == 1     # negative batch
-    assert f(plan._h, R, batch, None, p(Bd), p(Cd), p(xd), p(yd), p(z), None) == 1   # missing factor
-    assert f(plan._h, 100000, batch, p(Ad), p(Bd), p(Cd), p(xd), p(yd), p(z), None) == 2  # factors exceed smem
+    assert f(plan.handle("pair"), 0, batch, p(Ad), p(Bd), p(Cd), p(xd), p(yd), p(z), None) == 1      # rank < 1
+    assert f(plan.handle("pair"), R, -1, p(Ad), p(Bd), p(Cd), p(xd), p(yd), p(z), None) == 1     # negative batch
+    assert f(plan.handle("pair"), R, batch, None, p(Bd), p(Cd), p(xd), p(yd), p(z), None) == 1   # missing factor
+    assert f(plan.handle("pair"), 100000, batch, p(Ad), p(Bd), p(Cd), p(xd), p(yd), p(z), None) == 2  # factors exceed smem
     gA = torch.empty_like(Ad)
     nb = plan.cp_backward_workspace_bytes(R, batch)
     ws = torch.empty(nb // 4 + 64, device="cuda")
     b = lib().cgtp_cp_backward
-    args = (plan._h, R, batch, p(Ad), p(Bd), p(Cd), p(xd), p(yd), p(gd), None, None, p(gA), None, None)
+    args = (plan.handle("pair"), R, batch, p(Ad), p(Bd), p(Cd), p(xd), p(yd), p(gd), None, None, p(gA), None, None)
     assert b(*args, None, 0, None) == 7              # factor gradient without workspace
     assert b(*args, p(ws), nb - 256, None) == 7      # workspace too small
     assert b(*args, p(ws), nb, None) == 0
-    assert f(plan._h, R, batch, p(Ad), p(Bd), p(Cd), p(xd), p(yd), p(z), None) == 0
+    assert f(plan.handle("pair"), R, batch, p(Ad), p(Bd), p(Cd), p(xd), p(yd), p(z), None) == 0

@@ -53,7 +53,7 @@ def _check(api, plan, d, L, cots):
 
 
 @pytest.mark.parametrize("L,mult", [((1, 1, 1), 8), ((2, 2, 2), 64), ((2, 4, 2), 128), ((3, 3, 3), 32),
-                                    ((3, 3, 3), 128)])
+                                    ((3, 3, 3), 128), ((2, 3, 2), 32), ((0, 2, 2), 16), ((3, 4, 3), 32)])
 def test_all_cotangents(api, L, mult):
     d = _case(api, L, mult, 40 + mult)
     _check(api, api.Plan(*L, mult), d, L, "xwr")

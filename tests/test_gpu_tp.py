@@ -36,7 +36,8 @@ def test_tp_batch_workload(api):
 
 
 @pytest.mark.parametrize("L,mult,batch", [((1, 1, 1), 8, 3), ((2, 2, 2), 96, 77), ((2, 4, 2), 32, 130),
-                                          ((3, 3, 3), 64, 9), ((0, 0, 0), 4, 1)])
+                                          ((3, 3, 3), 64, 9), ((0, 0, 0), 4, 1), ((3, 4, 3), 32, 19),
+                                          ((0, 3, 3), 16, 5), ((2, 1, 0), 8, 11)])
 def test_tp_shapes(api, L, mult, batch):
     rng = np.random.default_rng(40 + batch)
     P = len(ocg.paths(*L))

@@ -106,7 +106,7 @@ def test_host_errors(api):
     out = torch.empty((g.n_nodes, 4, 8), device="cuda")
     nb = plan.uvw_forward_workspace_bytes(g.n_nodes, 8)
     ws = torch.empty(nb // 4 + 64, device="cuda")
-    args = (plan._h, g.n_nodes, g.n_edges, p(g.row_ptr), p(g.col), p(g.edge_vec), p(xd), p(Wd), p(md))
+    args = (plan.handle("uvw"), g.n_nodes, g.n_edges, p(g.row_ptr), p(g.col), p(g.edge_vec), p(xd), p(Wd), p(md))
     f = lib().cgtp_uvw_forward
     assert f(*args, 6, p(out), p(ws), nb, None) == 2                # mult_out not a multiple of 4
     assert f(*args, 8, p(out), p(ws), nb - 256, None) == 7          # workspace too small
