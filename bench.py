@@ -109,11 +109,11 @@ class ClockSampler:
 # family at the molecules workload (97 480 edges), from an ncu capture
 # (profiles/conv_molecules_traffic.md), with a hash of the kernel sources it
 # was taken on: traffic is reported only while the sources are unchanged.
-KERNEL_HEADERS = ("common.cuh", "conv_common.cuh", "sh.cuh", "structure.h", "vec2.cuh")
+KERNEL_HEADERS = ("common.cuh", "conv_common.cuh", "sh.cuh", "structure.h", "vec2.cuh", "launch.h")
 MEASURED_TRAFFIC = {
-    "conv_fwd": {"bytes": 1022369024, "n_edges": 97480, "sources": ("conv_fwd.cu",) + KERNEL_HEADERS,
+    "conv_fwd": {"bytes": 1022369024, "n_edges": 97480, "sources": ("conv_fwd.cu", "conv_fwd_kernel.cuh") + KERNEL_HEADERS,
                  "sha256_16": "41535c1d242146e5"},
-    "conv_bwd": {"bytes": 2064909568, "n_edges": 97480, "sources": ("conv_bwd.cu",) + KERNEL_HEADERS,
+    "conv_bwd": {"bytes": 2064909568, "n_edges": 97480, "sources": ("conv_bwd.cu", "conv_bwd_kernel.cuh") + KERNEL_HEADERS,
                  "sha256_16": "5508022eb4546212"},
 }
 
@@ -135,12 +135,25 @@ def measured_traffic(kernel, n_edges):
 
 
 # ---------------------------------------------------------------- algorithmic bytes
-def conv_bytes(n, E, P, u, ni, ns, no, slices):
-    """Algorithmic bytes of one forward and one backward launch (fp32/int32)."""
-    fwd = 4 * (E * P * u + n * ni * u + n * no * u + 3 * E + E + (n + 1))
-    bwd = 4 * (2 * E * P * u + 2 * n * ni * u + n * no * u + 3 * E + 2 * E + (n + 1)
-               + slices * E * ns)
+def conv_bytes(n, E, P, u, ni, ns, no):
+    """Algorithmic bytes of one forward and one backward launch (fp32/int32),
+    what the method must move:
+      forward  4 [E P u (W) + 4E (edge vectors, sources) + (N+1) (row offsets)
+                  + N u ni (x) + N u no (out)]
+      backward 4 [2 E P u (W read, grad_W written) + N u (2 ni + no) (x, grad_x,
+                  grad_out) + 8E (edge vectors, grad_edge_vec, CSC edge and
+                  destination lists) + 2 (N+1) (CSR and CSC offsets)]
+    The backward's harmonic-gradient partials (a workspace of this design) are
+    not counted; partials_bytes gives them separately."""
+    fwd = 4 * (E * P * u + 4 * E + (n + 1) + n * u * ni + n * u * no)
+    bwd = 4 * (2 * E * P * u + n * u * (2 * ni + no) + 8 * E + 2 * (n + 1))
     return fwd, bwd
+
+
+def partials_bytes(E, ns, slices):
+    """Bytes of the backward's harmonic-gradient partials (written by the
+    chunks, read by the Jacobian epilogue)."""
+    return 4 * 2 * slices * E * ns
 
 
 def structural_counts(li, ls, lo):
@@ -280,7 +293,7 @@ def config_table(torch, api, dev, hbm, reps=20):
                                                           workspace=ws), k)
         t_frc = _time_ms(torch, lambda: api.forces(g, gr, out=F), k)
         slices = max(1, int(ws_bytes // (4 * E * ns))) if E else 1
-        b_f, b_b = conv_bytes(n, E, P, u, ni, ns, no, slices)
+        b_f, b_b = conv_bytes(n, E, P, u, ni, ns, no)
         nT, nnz, no_sum = structural_counts(*L)
         f_f, f_b = conv_flops(E, u, nT, nnz, no_sum, P)
         rows.append({"workload": name, "L": list(L), "mult": u, "n_nodes": n, "n_edges": E, "paths": P,
@@ -296,7 +309,7 @@ def config_table(torch, api, dev, hbm, reps=20):
             t_sf = _time_ms(torch, lambda: plan.conv_forward_shared(g, x, wsh, out=out), k)
             t_sb = _time_ms(torch, lambda: plan.conv_backward_shared(g, x, wsh, go, workspace=ws), k)
             b_sf = 4 * (E * u + n * ni * u + n * no * u + 4 * E + (n + 1))
-            b_sb = 4 * (2 * E * u + 2 * n * ni * u + n * no * u + 5 * E + (n + 1) + slices * E * ns)
+            b_sb = 4 * (2 * E * u + n * u * (2 * ni + no) + 8 * E + 2 * (n + 1))
             rows.append({"workload": "molecules, weights shared by every path (path stride 0)",
                          "L": list(L), "mult": u, "n_edges": E, "fwd_ms": t_sf, "bwd_ms": t_sb,
                          "edges_per_s_fwd_bwd": E / ((t_sf + t_sb) / 1e3),
@@ -626,7 +639,7 @@ def run_gpu(args):
     # roofline of the dominant kernel (the backward)
     hbm, peak_kind = _load_peaks()
     slices = max(1, int(ws_bytes // (4 * E * ns))) if E else 1
-    b_fwd, b_bwd = conv_bytes(n, E, P, u, ni, ns, no, slices)
+    b_fwd, b_bwd = conv_bytes(n, E, P, u, ni, ns, no)
     dominant = "conv_bwd" if t_bwd >= t_fwd else "conv_fwd"
     b_dom, t_dom = (b_bwd, t_bwd) if dominant == "conv_bwd" else (b_fwd, t_fwd)
     achieved = b_dom / (t_dom / 1e3) / 1e9
@@ -648,7 +661,9 @@ def run_gpu(args):
         "roofline": {"bound": "hbm", "kernel": dominant, "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
                      "alg_bytes_per_launch": b_dom,
-                     "traffic_over_alg": traffic / b_dom if traffic else None},
+                     "traffic_over_alg": traffic / b_dom if traffic else None,
+                     "frac_with_partials": ((b_dom + (partials_bytes(E, ns, slices) if dominant == "conv_bwd" else 0))
+                                            / (t_dom / 1e3) / 1e9 / hbm)},
         "kernels_ms": {"conv_fwd": t_fwd, "conv_bwd_incl_sh_jacobian": t_bwd, "forces": t_frc},
         "step_hbm_frac": (step_bytes / (ms_step / 1e3) / 1e9) / hbm,
         "fp32_tflops": {"conv_fwd": f_fwd / (t_fwd / 1e3) / 1e12, "conv_bwd": f_bwd / (t_bwd / 1e3) / 1e12},

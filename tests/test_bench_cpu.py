@@ -34,31 +34,37 @@ def test_reference_arm_json_line():
 
 
 def test_conv_bytes_are_the_arrays_a_launch_touches():
-    n, E, P, u, ni, ns, no, slices = 7, 40, 19, 128, 9, 25, 9, 4
-    fwd, bwd = bench.conv_bytes(n, E, P, u, ni, ns, no, slices)
+    n, E, P, u, ni, ns, no = 7, 40, 19, 128, 9, 25, 9
+    fwd, bwd = bench.conv_bytes(n, E, P, u, ni, ns, no)
     f32 = 4
     # forward: W, x, out, edge vectors, col, row_ptr
     W, x, out = E * P * u, n * ni * u, n * no * u
     assert fwd == f32 * (W + x + out + 3 * E + E + (n + 1))
-    # the backward reads at least W, x, grad_out and writes grad_W, grad_x
-    assert bwd >= f32 * (2 * W + 2 * x + out)
-    # it grows with the harmonic-gradient partials it writes and reads
-    _, bwd1 = bench.conv_bytes(n, E, P, u, ni, ns, no, 1)
-    assert bwd > bwd1
+    # backward: W read and grad_W written, x read and grad_x written, grad_out
+    # read, edge vectors read and their gradients written, the CSC edge and
+    # destination lists, and both offset arrays; no workspace partials
+    assert bwd == f32 * (2 * W + 2 * x + out + 3 * E + 3 * E + 2 * E + 2 * (n + 1))
+    assert bench.partials_bytes(E, ns, 4) == f32 * 2 * 4 * E * ns
 
 
 def test_measured_traffic_tracks_the_sources(tmp_path, monkeypatch):
-    rec = bench.MEASURED_TRAFFIC["conv_bwd"]
-    got = bench.measured_traffic("conv_bwd", rec["n_edges"])
-    assert got == rec["bytes"]  # the committed sources are the captured ones
+    import hashlib
+    rec = dict(bench.MEASURED_TRAFFIC["conv_bwd"])
+    # a record taken on the current sources scales with the edge count
+    m = hashlib.sha256()
+    for name in rec["sources"]:
+        with open(os.path.join(ROOT, "equivariant_mlip_tensor_b200", "csrc", name), "rb") as f:
+            m.update(f.read())
+    rec["sha256_16"] = m.hexdigest()[:16]
+    monkeypatch.setitem(bench.MEASURED_TRAFFIC, "conv_bwd", rec)
+    assert bench.measured_traffic("conv_bwd", rec["n_edges"]) == rec["bytes"]
     assert bench.measured_traffic("conv_bwd", 2 * rec["n_edges"]) == 2 * rec["bytes"]
     assert bench.measured_traffic("no_such_kernel", 10) is None
     # a copy of the sources with one kernel file changed no longer matches
     src = os.path.join(ROOT, "equivariant_mlip_tensor_b200", "csrc")
     dst = tmp_path / "equivariant_mlip_tensor_b200" / "csrc"
     shutil.copytree(src, dst)
-    with open(dst / "conv_bwd.cu", "a") as f:
+    with open(dst / "conv_bwd_kernel.cuh", "a") as f:
         f.write("\n// changed\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.measured_traffic("conv_bwd", rec["n_edges"]) is None
-    assert bench.measured_traffic("conv_fwd", rec["n_edges"]) == bench.MEASURED_TRAFFIC["conv_fwd"]["bytes"]

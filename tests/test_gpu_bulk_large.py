@@ -1,8 +1,12 @@
 """GPU parity at the large periodic workload (20,000 atoms, ~1.05M edges,
-L = 3, mult 128): the whole path runs at full size on the GPU; the oracle
-checks the full neighbour list bit for bit and a sample of outputs it can
-compute one by one (output rows, weight gradients of sampled edges, feature
-gradients of sampled sources, edge-vector gradients and forces)."""
+L = 3, mult 128), whole tensors: the whole path runs at full size on the GPU;
+the oracle checks the full neighbour list bit for bit and then recomputes
+every output row, every feature gradient, every weight gradient (18 GB,
+streamed from the device in chunks of whole source rows), every edge-vector
+gradient and every force, in fp64 on the host's cores, and the measure
+max|gpu - oracle| / max|oracle| is taken over each whole tensor."""
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import pytest
 
@@ -10,9 +14,11 @@ from equivariant_mlip_tensor_b200 import synthetic
 from oracle import conv as oconv
 from oracle import graph as ograph
 from oracle import radial as oradial
-from tests.gpu_common import FWD_TOL, GRAD_TOL, cuda, host, rel_err
+from tests.gpu_common import FWD_TOL, GRAD_TOL, THREADS, cuda, host
 
 pytestmark = pytest.mark.gpu
+
+CHUNK_EDGES = 4096  # edges per oracle work item (whole rows)
 
 
 @pytest.fixture(scope="module")
@@ -33,14 +39,100 @@ def run():
     plan.radial_backward(g.edge_vec, w.rc, W1, W2, gw, gr)
     F = api.forces(g, gr)
     torch.cuda.synchronize()
+    del Wg
     o = ograph.neighbour_list(w.pos, w.rc, w.box)
-    rng = np.random.default_rng(77)
-    nodes = np.sort(rng.choice(w.n_nodes, size=24, replace=False))
-    nodes = np.unique(np.concatenate([nodes, [0, w.n_nodes - 1]]))
-    res = dict(w=w, L=L, g=g, o=o, nodes=nodes, out=out, gx=gx, gw=gw, gr=gr, F=F, Wg=Wg)
+    res = dict(w=w, L=L, g=g, o=o, out=host(out), gx=host(gx), gw=gw, gr=host(gr), F=host(F))
     yield res
-    del res, Wg, gw, out, gx, gr, F
+    del res, gw, out, gx, gr, F
     torch.cuda.empty_cache()
+
+
+def _row_chunks(ptr, target):
+    """Consecutive node ranges [a, b) of about `target` edges each (whole rows)."""
+    ptr = np.asarray(ptr, dtype=np.int64)
+    n = ptr.size - 1
+    cuts = np.searchsorted(ptr, np.arange(0, ptr[-1], target), side="right") - 1
+    cuts = np.unique(np.concatenate([[0], cuts, [n]]))
+    return [(int(a), int(b)) for a, b in zip(cuts[:-1], cuts[1:]) if b > a]
+
+
+def _segment_sums(vals, starts, n_rows, n_vals):
+    """Row sums of consecutive segments (rows with no entries are zero)."""
+    out = np.zeros((n_rows,) + vals.shape[1:])
+    deg = np.diff(np.concatenate([starts, [n_vals]]))
+    nz = deg > 0
+    if n_vals:
+        out[nz] = np.add.reduceat(vals, starts[nz], axis=0)
+    return out
+
+
+def _bounded_map(fn, items, workers):
+    """fn over items on a thread pool, results in order, at most 2 x workers
+    in flight (each result holds a chunk of weight gradients)."""
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        pending = []
+        for it in items:
+            pending.append(ex.submit(fn, *it))
+            if len(pending) >= 2 * workers:
+                yield pending.pop(0).result()
+        for f in pending:
+            yield f.result()
+
+
+class _Err:
+    """max|got - want| and max|want| accumulated over chunks of one tensor."""
+
+    def __init__(self):
+        self.d = self.s = 0.0
+
+    def add(self, got, want):
+        got = np.asarray(got, dtype=np.float64)
+        self.d = max(self.d, float(np.max(np.abs(got - want), initial=0.0)))
+        self.s = max(self.s, float(np.max(np.abs(want), initial=0.0)))
+
+    def rel(self):
+        return self.d / self.s if self.s > 0 else self.d
+
+
+@pytest.fixture(scope="module")
+def whole(run):
+    """Oracle over the whole graph, compared chunk by chunk with the GPU."""
+    import torch
+    from threadpoolctl import threadpool_limits
+    w, L, o = run["w"], run["L"], run["o"]
+    rp, col, ev = o["row_ptr"].astype(np.int64), o["col"].astype(np.int64), o["edge_vec"]
+    cp, ce, cd = o["csc_ptr"].astype(np.int64), o["csc_edge"].astype(np.int64), o["csc_dst"].astype(np.int64)
+    n, E = w.n_nodes, col.size
+    workers = max(1, THREADS)
+
+    def fwd(a, b):
+        e0, e1 = rp[a], rp[b]
+        Wc = oradial.radial_forward(ev[e0:e1], w.W1, w.W2, w.rc, w.n_paths, w.mult)
+        m = oconv.edge_messages(col[e0:e1], ev[e0:e1], w.x, Wc, *L)
+        return a, b, _segment_sums(m, rp[a:b] - e0, b - a, e1 - e0)
+
+    def bwd(a, b):
+        k0, k1 = cp[a], cp[b]
+        edges = ce[k0:k1]
+        evk = ev[edges]
+        Wc = oradial.radial_forward(evk, w.W1, w.W2, w.rc, w.n_paths, w.mult)
+        mx, gw, gr = oconv.edge_backward(col[edges], cd[k0:k1], evk, w.x, Wc, w.grad_out, *L)
+        gr = gr + oradial.radial_backward(evk, w.W1, w.W2, w.rc, gw)
+        return a, b, edges, _segment_sums(mx, cp[a:b] - k0, b - a, k1 - k0), gw, gr
+
+    errs = {k: _Err() for k in ("out", "gx", "gw", "gr", "F")}
+    gr_ref = np.zeros((E, 3))
+    with threadpool_limits(1):
+        for a, b, ref in _bounded_map(fwd, _row_chunks(rp, CHUNK_EDGES), workers):
+            errs["out"].add(run["out"][a:b], ref)
+        for a, b, edges, gx_ref, gw_ref, gr_chunk in _bounded_map(bwd, _row_chunks(cp, CHUNK_EDGES), workers):
+            errs["gx"].add(run["gx"][a:b], gx_ref)
+            idx = torch.as_tensor(edges, device=run["gw"].device)
+            errs["gw"].add(host(run["gw"].index_select(0, idx)), gw_ref)
+            gr_ref[edges] = gr_chunk
+    errs["gr"].add(run["gr"], gr_ref)
+    errs["F"].add(run["F"], oconv.edge_forces(rp, col, gr_ref, n))
+    return {k: e.rel() for k, e in errs.items()}
 
 
 def test_graph_bit_exact(run):
@@ -53,53 +145,26 @@ def test_graph_bit_exact(run):
     assert np.array_equal(host(g.csc_dst), o["csc_dst"])
 
 
-def _edge_grads(w, L, o, edges):
-    """Oracle gradients of the sampled edges: weights, and edge vectors
-    including the radial network's contribution."""
-    dst = ograph.edge_dst(o["row_ptr"])
-    ev = o["edge_vec"][edges]
-    Wo = oradial.radial_forward(ev, w.W1, w.W2, w.rc, w.n_paths, w.mult)
-    mx, gw, gr = oconv.edge_backward(o["col"][edges], dst[edges], ev, w.x, Wo, w.grad_out, *L)
-    gr = gr + oradial.radial_backward(ev, w.W1, w.W2, w.rc, gw)
-    return mx, gw, gr
+def test_forward_whole_tensor(whole):
+    assert whole["out"] < FWD_TOL, whole
 
 
-def test_forward_rows(run):
-    w, L, o, nodes = run["w"], run["L"], run["o"], run["nodes"]
-    rp = o["row_ptr"].astype(np.int64)
-    Wrows = {}
-    ref = []
-    for i in nodes:
-        s, e = rp[i], rp[i + 1]
-        ev = o["edge_vec"][s:e]
-        Wo = oradial.radial_forward(ev, w.W1, w.W2, w.rc, w.n_paths, w.mult)
-        m = oconv.edge_messages(o["col"][s:e], ev, w.x, Wo, *L)
-        ref.append(m.sum(axis=0))
-    got = host(run["out"][nodes.tolist()])
-    assert rel_err(got, np.stack(ref)) < FWD_TOL
+def test_feature_and_weight_gradients_whole_tensors(whole):
+    assert whole["gx"] < GRAD_TOL, whole
+    assert whole["gw"] < GRAD_TOL, whole
 
 
-def test_weight_and_edge_gradients_of_sampled_edges(run):
-    w, L, o = run["w"], run["L"], run["o"]
-    rng = np.random.default_rng(78)
-    E = o["col"].size
-    edges = np.unique(np.concatenate([rng.choice(E, size=400, replace=False), [0, E - 1]]))
-    _, gw, gr = _edge_grads(w, L, o, edges)
-    assert rel_err(host(run["gw"][edges.tolist()]), gw) < GRAD_TOL
-    assert rel_err(host(run["gr"][edges.tolist()]), gr) < GRAD_TOL
+def test_edge_vector_gradients_and_forces_whole_tensors(whole):
+    assert whole["gr"] < GRAD_TOL, whole
+    assert whole["F"] < GRAD_TOL, whole
 
 
-def test_feature_gradients_and_forces_of_sampled_nodes(run):
-    w, L, o, nodes = run["w"], run["L"], run["o"], run["nodes"]
-    cp, ce = o["csc_ptr"].astype(np.int64), o["csc_edge"]
-    rp = o["row_ptr"].astype(np.int64)
-    gx_ref, F_ref = [], []
-    for j in nodes:
-        out_edges = ce[cp[j]:cp[j + 1]]          # edges leaving j (j is the source)
-        in_edges = np.arange(rp[j], rp[j + 1])   # edges arriving at j
-        mx, _, gr_out = _edge_grads(w, L, o, out_edges)
-        gx_ref.append(mx.sum(axis=0))
-        _, _, gr_in = _edge_grads(w, L, o, in_edges)
-        F_ref.append(gr_in.sum(axis=0) - gr_out.sum(axis=0))
-    assert rel_err(host(run["gx"][nodes.tolist()]), np.stack(gx_ref)) < GRAD_TOL
-    assert rel_err(host(run["F"][nodes.tolist()]), np.stack(F_ref)) < GRAD_TOL
+def test_chunking_helpers_cover_every_row_once():
+    assert _row_chunks(np.array([0, 0, 0, 5]), 2)[0][0] == 0  # leading empty rows are covered
+    ptr = np.array([0, 3, 3, 3, 10, 11, 11, 20])
+    chunks = _row_chunks(ptr, 4)
+    assert chunks[0][0] == 0 and chunks[-1][1] == 7
+    assert all(b0 == a1 for (_, b0), (a1, _) in zip(chunks[:-1], chunks[1:]))
+    vals = np.arange(20.0)[:, None]
+    sums = _segment_sums(vals, ptr[:-1], 7, 20)
+    assert np.array_equal(sums[:, 0], [0 + 1 + 2, 0, 0, sum(range(3, 10)), 10, 0, sum(range(11, 20))])
