@@ -326,10 +326,15 @@ def config_table(torch, api, dev, hbm, reps=20):
             # algorithmic bytes: read x, gg_x, W, gg_w, grad_out, gg_r, edge vectors; write d_x, d_W,
             # d_grad_out, d_edge_vec
             b_d = 4 * (3 * E * P * u + 3 * n * ni * u + 2 * n * no * u + 9 * E + 2 * (n + 1) + 2 * E)
+            # an atomic-free schedule reads W and gg_w twice (once by destination for d grad_out,
+            # once by source for d x and d W) and writes d W once: 5 weight-sized transfers
+            b_s = b_d + 4 * 2 * E * P * u
             rows.append({"workload": "molecules double backward (adjoint of the backward, all cotangents)",
                          "L": list(L), "mult": u, "n_edges": E, "ms": t_d, "edges_per_s": E / (t_d / 1e3),
                          "hbm_frac": b_d / (t_d / 1e3) / 1e9 / hbm,
-                         "launches": "3 forward + 2 backward + 3 harmonic-gradient passes + 1 directional harmonics"})
+                         "hbm_frac_of_atomic_free_schedule": b_s / (t_d / 1e3) / 1e9 / hbm,
+                         "launches": "fused: d grad_out by one forward pass (chunks by l3), d x / d W / edge terms "
+                                     "by one source-centric pass (chunks by l1), one Jacobian-and-Hessian epilogue"})
             del ggx, ggw, ggr, dws
             # fully connected (uvw) forward, 128 output channels: per-path messages, then one
             # tensor-core GEMM per l3 block

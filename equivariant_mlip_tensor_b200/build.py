@@ -1,7 +1,7 @@
 """Build libcgtp.so (sm_100a) in-tree.
 
-Every per-shape kernel family (convolution forward, backward and
-harmonic-gradient passes, edge-free tensor product, CP product) is compiled
+Every per-shape kernel family (convolution forward, backward, the double
+backward's fused passes, edge-free tensor product, CP product) is compiled
 once per shape of CGTP_CONFIGS in csrc/configs.h, and the weight-structure
 variants (path-shared weights, fully connected convolution) once per shape of
 CGTP_VARIANT_CONFIGS, each as its own translation unit so that the compiles
@@ -24,11 +24,16 @@ LIB = os.path.join(HERE, "libcgtp.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-NVCC_FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
+# Line information (for profiler source views) is compiled into the
+# shape-free units and the units of the standard workloads' shapes; the
+# fully unrolled kernels of the other policy shapes omit it, since their line
+# tables would be about 8x their code and the library several hundred MB.
+BASE_FLAGS = ARCH + ["-O3", "-std=c++17", "--expt-relaxed-constexpr",
                      "-Xcompiler", "-fPIC", "-I", CSRC, "-I", INCLUDE]
+NVCC_FLAGS = BASE_FLAGS + ["-lineinfo"]
 # per-shape units: every shape of CGTP_CONFIGS, and the weight-structure
 # variants for the shapes of CGTP_VARIANT_CONFIGS
-PER_SHAPE = ["conv_fwd.cu", "conv_bwd.cu", "conv_gy.cu", "tp.cu", "cp.cu"]
+PER_SHAPE = ["conv_fwd.cu", "conv_bwd.cu", "conv_dd.cu", "tp.cu", "cp.cu"]
 PER_VARIANT_SHAPE = ["conv_paths.cu", "conv_shared.cu"]
 SHAPE_FREE = ["graph.cu", "radial.cu", "misc.cu", "abi.cu", "cg_table.cpp", "uvw.cu", "lanes.cu"]
 
@@ -89,16 +94,20 @@ def _jobs():
     units += [(src, shp) for src in PER_VARIANT_SHAPE for shp in shapes("CGTP_VARIANT_CONFIGS")]
     # the largest shapes first, so that the long compiles start early
     units.sort(key=lambda u: -(u[1][0] + 1) * (u[1][1] + 1) * (u[1][2] + 1))
+    lined = set(shapes("CGTP_VARIANT_CONFIGS"))
     for src, (li, ls, lo) in units:
         obj = os.path.join(BUILD, f"{src.split('.')[0]}_{li}{ls}{lo}.o")
         defs = [f"-DCGTP_CFG_LI={li}", f"-DCGTP_CFG_LS={ls}", f"-DCGTP_CFG_LO={lo}"]
+        if (li, ls, lo) not in lined:
+            defs.append("--no-lineinfo")
         jobs.append((os.path.join(CSRC, src), obj, defs))
     return jobs
 
 
 def _compile(job, verbose):
     src, obj, defs = job
-    cmd = [nvcc()] + NVCC_FLAGS + defs + ["-c", src, "-o", obj]
+    flags = BASE_FLAGS if "--no-lineinfo" in defs else NVCC_FLAGS
+    cmd = [nvcc()] + flags + [d for d in defs if d != "--no-lineinfo"] + ["-c", src, "-o", obj]
     if src.endswith(".cpp"):
         cmd = [nvcc(), "-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-I", CSRC, "-x", "c++", "-c", src, "-o", obj]
     r = subprocess.run(cmd, capture_output=True, text=True)

@@ -407,14 +407,12 @@ static cudaError_t dispatch_fwd(cgtp_plan p, const ConvFwdArgs& a, int sms, cuda
   CGTP_CONFIGS(CGTP_DFWD_ENTRY)
   return e;
 }
-// Harmonic-gradient-only backward pass (no grad_x / grad_W work); its
-// partials have the plain backward's layout, so they fit its workspace.
+static cudaError_t dispatch_bwd(cgtp_plan p, const ConvBwdArgs& a, int sms, cudaStream_t s);
+// Harmonic-gradient pass of the first-order double backward: the plain
+// backward with neither grad_x nor grad_W requested (nothing but the grad_Y
+// partials and the Jacobian epilogue of a.gr_mode is written).
 static cudaError_t dispatch_bwd_gy(cgtp_plan p, const ConvBwdArgs& a, int sms, cudaStream_t s) {
-  cudaError_t e = cudaErrorNotSupported;
-#define CGTP_BWD_GY_ENTRY(A, B, C) \
-  if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_bwd_gy<A, B, C>(a, sms, s);
-  CGTP_CONFIGS(CGTP_BWD_GY_ENTRY)
-  return e;
+  return dispatch_bwd(p, a, sms, s);
 }
 
 static cudaError_t dispatch_bwd(cgtp_plan p, const ConvBwdArgs& a, int sms, cudaStream_t s) {
@@ -425,13 +423,24 @@ static cudaError_t dispatch_bwd(cgtp_plan p, const ConvBwdArgs& a, int sms, cuda
   return e;
 }
 
+static int dd_slices(cgtp_plan p) {
+  int s = 0;
+#define CGTP_DD_SLICES_ENTRY(A, B, C) \
+  if (p->li == A && p->ls == B && p->lo == C) s = conv_dd_slices<A, B, C>(p->mult);
+  CGTP_CONFIGS(CGTP_DD_SLICES_ENTRY)
+  return s;
+}
+
+// [E][NS] directional harmonics, then the harmonic-gradient partials: those
+// of the first-order passes, or the fused pass's two sets, whichever is larger.
 cgtp_status cgtp_conv_double_backward_workspace_size(cgtp_plan p, int n_edges, size_t* bytes) {
   if (!mode_is(p, CGTP_MODE_CONV_UVU) || n_edges < 0 || bytes == nullptr) return CGTP_ERR_INVALID_ARG;
   const size_t ns = (size_t)(p->ls + 1) * (p->ls + 1);
   const size_t u = (sizeof(float) * (size_t)n_edges * ns + 255) & ~(size_t)255;
   size_t bw = 0;
   cgtp_conv_backward_workspace_size(p, n_edges, &bw);
-  *bytes = u + bw;
+  const size_t dd = (sizeof(float) * 2 * (size_t)dd_slices(p) * (size_t)n_edges * ns + 255) & ~(size_t)255;
+  *bytes = u + (dd > bw ? dd : bw);
   return CGTP_OK;
 }
 
@@ -481,7 +490,40 @@ cgtp_status cgtp_conv_double_backward(cgtp_plan p, int n_nodes, int n_edges, con
   const bool gr = gg_edge_vec != nullptr;
   const int* abort_flag = nullptr;
   e = validate_graph(p, n_nodes, n_edges, row_ptr, col, edge_vec, csc_ptr, csc_edge, csc_dst, sms, s, &abort_flag);
-  if (gr && e == cudaSuccess) e = launch_sh_dir(p->ls, n_edges, edge_vec, gg_edge_vec, uY, sms, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+
+  // Every cotangent given: the fused passes.  d grad_out by one forward that
+  // reads W and gg_W once; d x, d W and the edge-vector term by one
+  // source-centric pass that reads them once more and writes d W once.
+  if (gg_x != nullptr && gg_w != nullptr && gr) {
+    if (d_grad_out != nullptr) {
+      ConvFwdArgs a{n_nodes, row_ptr, col, edge_vec, x, w, d_grad_out, p->mult};
+      a.abort_flag = abort_flag;
+      a.x2 = gg_x;
+      a.w2 = gg_w;
+      a.gr_dir = gg_edge_vec;
+      e = cudaErrorNotSupported;
+#define CGTP_DDF_ENTRY(A, B, C) \
+      if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_dd_fwd<A, B, C>(a, sms, s);
+      CGTP_CONFIGS(CGTP_DDF_ENTRY)
+    }
+    if (e == cudaSuccess && (d_x != nullptr || d_w != nullptr || d_edge_vec != nullptr)) {
+      ConvBwdArgs a{n_nodes, n_edges, csc_ptr, csc_edge, csc_dst, edge_vec, x, w, grad_out,
+                    d_x, d_w, d_edge_vec, gsh, p->mult};
+      a.abort_flag = abort_flag;
+      a.x2 = gg_x;
+      a.w2 = gg_w;
+      a.gr_dir = gg_edge_vec;
+      e = cudaErrorNotSupported;
+#define CGTP_DDB_ENTRY(A, B, C) \
+      if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_dd_bwd<A, B, C>(a, sms, s);
+      CGTP_CONFIGS(CGTP_DDB_ENTRY)
+    }
+    return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
+  }
+
+  // Otherwise a sum of first-order passes with one argument replaced.
+  if (gr) e = launch_sh_dir(p->ls, n_edges, edge_vec, gg_edge_vec, uY, sms, s);
 
   // d grad_out: forward convolutions with one argument replaced at a time
   //   (Y -> uY), (x -> gg_x), (W -> gg_w), summed

@@ -121,6 +121,11 @@ struct ConvFwdArgs {
   // checked mode: the plan's validation flags, written by a validation
   // launch earlier in the stream; the kernel does nothing if they are unsafe
   const int* abort_flag = nullptr;
+  // the double backward's fused forward: out = conv(x2, w, Y) + conv(x, w2, Y)
+  // + conv(x, w, (dY/dr) gr_dir)
+  const float* x2 = nullptr;
+  const float* w2 = nullptr;
+  const float* gr_dir = nullptr;
 };
 
 struct ConvBwdArgs {
@@ -146,6 +151,10 @@ struct ConvBwdArgs {
   int gr_mode = 0;
   const float* gr_dir = nullptr;  // [n_edges][3], for gr_mode 2 and 3
   const int* abort_flag = nullptr;  // checked mode, as in ConvFwdArgs
+  // the double backward's fused pass: second features and weights (the
+  // cotangents gg_x, gg_w); gr_dir is then the cotangent gg_r
+  const float* x2 = nullptr;
+  const float* w2 = nullptr;
 };
 
 struct TPArgs {

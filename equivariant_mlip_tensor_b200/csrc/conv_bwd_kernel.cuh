@@ -24,11 +24,12 @@
 //    the outputs (the double backward's first-order passes);
 //  - kVarPerPath: grad_out holds one gradient block per path (the per-path
 //    message layout of the fully connected convolution);
-//  - kVarGyOnly: only the harmonic gradient (no grad_x, no grad_W, and none
-//    of the T^T g products they need);
 //  - kVarWShared: one weight row per edge shared by every path; grad_w[e] is
 //    the sum over paths (chunks then run in plain stream order, each adding
-//    onto the row the previous chunks wrote).
+//    onto the row the previous chunks wrote);
+//  - kVarDD: the double backward's d x, d W and edge-vector terms in one pass
+//    (see bwd_edge_dd): W and gg_W staged per edge, x and gg_x held per
+//    source, T from Y and T' from Y' = (dY/dr) gg_r.
 //
 // Include after CGTP_DEFINE_CONSTANT_TABLES, conv_common.cuh, vec2.cuh and
 // sh.cuh.
@@ -36,7 +37,7 @@
 
 namespace cgtp {
 
-enum : int { kVarExt = 1, kVarPerPath = 2, kVarGyOnly = 4, kVarWShared = 8 };
+enum : int { kVarExt = 1, kVarPerPath = 2, kVarWShared = 8, kVarDD = 16 };
 
 namespace {
 
@@ -88,8 +89,11 @@ constexpr int bwd_budget() {
   return PS::LI >= 3 || PS::LO >= 3 ? CGTP_BWD_BUDGET_L3 : CGTP_BWD_BUDGET;
 }
 
-template <class PS, bool NEED_GY>
-using BwdPlan = Plan<PS, kByL1, kBwdVec, NEED_GY, bwd_budget<PS>()>;
+// The fused double-backward pass carries a little over twice the code per
+// path (two T products, two harmonic-gradient sums): chunks of 4/9 of the
+// budget.
+template <class PS, bool NEED_GY, int VAR = 0>
+using BwdPlan = Plan<PS, kByL1, kBwdVec, NEED_GY, (VAR & kVarDD) ? bwd_budget<PS>() * 4 / 9 : bwd_budget<PS>()>;
 
 template <class PS, class GR>
 constexpr unsigned touched_sh_mask() {
@@ -114,7 +118,8 @@ constexpr int pp_rowoff(int K) {
 // and output-gradient rows (the chunk's l3 range, or every path's own block).
 template <class PS, class GR, int VAR>
 constexpr int bwd_staged_rows() {
-  return ((VAR & kVarWShared) ? 1 : GR::NP) + ((VAR & kVarPerPath) ? pp_rowoff<PS, GR>(GR::NP) : GR::NROW);
+  return ((VAR & kVarWShared) ? 1 : GR::NP) * ((VAR & kVarDD) ? 2 : 1) +
+         ((VAR & kVarPerPath) ? pp_rowoff<PS, GR>(GR::NP) : GR::NROW);
 }
 
 // Shared memory (floats), the same functions on both sides of the launch:
@@ -140,7 +145,7 @@ template <class PS, class GR, int VEC, bool NEED_GY, int VAR>
 __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const float* __restrict__ stage, int rowf,
                                          const float (&xr)[GR::NOWN][VEC], float* __restrict__ gwrow, bool acc, int mult,
                                          float (&gx)[GR::NOWN][VEC], float* __restrict__ gyrow, int rs) {
-  constexpr bool PP = (VAR & kVarPerPath) != 0, HX = (VAR & kVarGyOnly) == 0, WSH = (VAR & kVarWShared) != 0;
+  constexpr bool PP = (VAR & kVarPerPath) != 0, WSH = (VAR & kVarWShared) != 0;
   constexpr int NW = WSH ? 1 : GR::NP;  // staged weight rows
   float gy[PS::NS];
   float gws[VEC];  // WSH: grad of the shared weight row, summed over this chunk's paths
@@ -181,7 +186,7 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
         if constexpr (k < tc) {
           constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
           const float tv = tv4[decltype(Rc)::value];
-          if constexpr (HX) axpy<VEC>(h[m1 + l1], tv, gv[m3 + l3]);
+          axpy<VEC>(h[m1 + l1], tv, gv[m3 + l3]);
           if constexpr (NEED_GY) {
             const float av = vdot<VEC>(xw[m1 + l1], gv[m3 + l3]);
             static_for<0, 2 * l2 + 1>([&](auto M2c) {
@@ -194,7 +199,7 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
         }
       });
     });
-    if constexpr (HX) {
+    {
       if constexpr (WSH) {
 #pragma unroll
         for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) {
@@ -226,7 +231,7 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
       for (int m2 = 0; m2 < 2 * l2 + 1; ++m2) gyrow[(l2 * l2 + m2) * rs] = gy[l2 * l2 + m2];
     }
   });
-  if constexpr (HX && WSH) {
+  if constexpr (WSH) {
     if (gwrow != nullptr) {
       if (acc) {  // an earlier chunk of this call wrote the row: add onto it
         float prev[VEC];
@@ -239,6 +244,99 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
   }
 }
 
+// One edge of the double backward's fused pass, per path, with
+// h[m1] = sum_m3 T[m1][m3] g[m3] and h'[m1] = sum_m3 T'[m1][m3] g[m3]:
+//   d_x[m1]  += gg_W h[m1] + W h'[m1]
+//   d_W       = sum_m1 gg_x[m1] h[m1] + x[m1] h'[m1]
+//   A[l2,m2] += C sum_u (W gg_x[m1] + gg_W x[m1]) g[m3]   (contracted with dY/dr)
+//   B[l2,m2] += C sum_u W x[m1] g[m3]                      (with d2Y/dr2 gg_r)
+// (the derivatives of <gg_x, grad_x> + <gg_W, grad_W> + <gg_r, grad_r>).
+// Stage layout: W rows (NP), gg_W rows (NP), grad_out rows (NROW).
+template <class PS, class GR, int VEC, bool NEED_GY>
+__device__ __forceinline__ void bwd_edge_dd(const float* __restrict__ T, const float* __restrict__ Td,
+                                            const float* __restrict__ stage, int rowf,
+                                            const float (&xr)[GR::NOWN][VEC], const float (&gxr)[GR::NOWN][VEC],
+                                            float* __restrict__ gwrow, int mult, float (&gx)[GR::NOWN][VEC],
+                                            float* __restrict__ gyrowA, float* __restrict__ gyrowB, int rs) {
+  constexpr int NP = GR::NP;
+  float gyA[PS::NS], gyB[PS::NS];
+  static_for<0, NP>([&](auto Kc) {
+    constexpr int K = decltype(Kc)::value;
+    constexpr int P = GR::D.path[K];
+    constexpr int l1 = PS::D.l1[P], l3 = PS::D.l3[P];
+    [[maybe_unused]] constexpr int l2 = PS::D.l2[P];
+    constexpr int tb = GR::D.lt[K], tc = PS::D.tcount[P];
+    constexpr int g0 = 2 * NP + l3 * l3 - GR::D.rlo;  // staged row of grad_out[l3, m3 = -l3]
+    if constexpr (NEED_GY && GR::D.first_l2[K]) {
+#pragma unroll
+      for (int m2 = 0; m2 < 2 * l2 + 1; ++m2) gyA[l2 * l2 + m2] = gyB[l2 * l2 + m2] = 0.f;
+    }
+    float wv[VEC], gwv[VEC];
+    VecIO<VEC>::lds(wv, stage + K * rowf);
+    VecIO<VEC>::lds(gwv, stage + (NP + K) * rowf);
+    float gv[2 * l3 + 1][VEC], h[2 * l1 + 1][VEC], hd[2 * l1 + 1][VEC];
+#pragma unroll
+    for (int m3 = 0; m3 < 2 * l3 + 1; ++m3) VecIO<VEC>::lds(gv[m3], stage + (g0 + m3) * rowf);
+#pragma unroll
+    for (int m1 = 0; m1 < 2 * l1 + 1; ++m1)
+#pragma unroll
+      for (int c = 0; c < VEC; ++c) h[m1][c] = hd[m1][c] = 0.f;
+    [[maybe_unused]] float pa[2 * l1 + 1][VEC], pb[2 * l1 + 1][VEC];
+    if constexpr (NEED_GY) {
+#pragma unroll
+      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) {
+        vmul<VEC>(pa[m1], wv, gxr[m1]);
+        vfma<VEC>(pa[m1], gwv, xr[m1]);
+        vmul<VEC>(pb[m1], wv, xr[m1]);
+      }
+    }
+    static_for<0, (tc + 3) / 4>([&](auto Qc) {
+      constexpr int q = decltype(Qc)::value;
+      const float4 v4 = *reinterpret_cast<const float4*>(T + tb + 4 * q);
+      const float4 d4 = *reinterpret_cast<const float4*>(Td + tb + 4 * q);
+      const float tv4[4] = {v4.x, v4.y, v4.z, v4.w}, td4[4] = {d4.x, d4.y, d4.z, d4.w};
+      static_for<0, 4>([&](auto Rc) {
+        constexpr int k = 4 * q + decltype(Rc)::value;
+        if constexpr (k < tc) {
+          constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
+          axpy<VEC>(h[m1 + l1], tv4[decltype(Rc)::value], gv[m3 + l3]);
+          axpy<VEC>(hd[m1 + l1], td4[decltype(Rc)::value], gv[m3 + l3]);
+          if constexpr (NEED_GY) {
+            const float aa = vdot<VEC>(pa[m1 + l1], gv[m3 + l3]);
+            const float ab = vdot<VEC>(pb[m1 + l1], gv[m3 + l3]);
+            static_for<0, 2 * l2 + 1>([&](auto M2c) {
+              constexpr int m2 = decltype(M2c)::value - l2;
+              if constexpr (cg_allowed(l1, l2, l3, m1, m2, m3)) {
+                constexpr int ti = table_index(l1, l2, l3, m1, m2, m3);
+                gyA[l2 * l2 + l2 + m2] = fmaf(c_cg[ti], aa, gyA[l2 * l2 + l2 + m2]);
+                gyB[l2 * l2 + l2 + m2] = fmaf(c_cg[ti], ab, gyB[l2 * l2 + l2 + m2]);
+              }
+            });
+          }
+        }
+      });
+    });
+    float gw[VEC];
+#pragma unroll
+    for (int c = 0; c < VEC; ++c) gw[c] = 0.f;
+#pragma unroll
+    for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) {
+      vfma<VEC>(gx[m1], gwv, h[m1]);
+      vfma<VEC>(gx[m1], wv, hd[m1]);
+      vfma<VEC>(gw, gxr[m1], h[m1]);
+      vfma<VEC>(gw, xr[m1], hd[m1]);
+    }
+    if (gwrow != nullptr) VecIO<VEC>::st_stream(gwrow + P * mult, gw);
+    if constexpr (NEED_GY && GR::D.last_l2[K]) {
+#pragma unroll
+      for (int m2 = 0; m2 < 2 * l2 + 1; ++m2) {
+        gyrowA[(l2 * l2 + m2) * rs] = gyA[l2 * l2 + m2];
+        gyrowB[(l2 * l2 + m2) * rs] = gyB[l2 * l2 + m2];
+      }
+    }
+  });
+}
+
 // One launch per chunk (paths of one l1 block): grad_x rows of that block
 // (written by the block's first chunk, accumulated by the others), grad_W
 // of the chunk's paths and a partial grad_Y over them.
@@ -247,17 +345,20 @@ __global__ void CGTP_BWD_BOUNDS
 conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt) {
   constexpr int VEC = kBwdVec;
   constexpr bool EXT = (VAR & kVarExt) != 0, PP = (VAR & kVarPerPath) != 0;
-  constexpr bool HX = (VAR & kVarGyOnly) == 0, WSH = (VAR & kVarWShared) != 0;
+  constexpr bool WSH = (VAR & kVarWShared) != 0, DD = (VAR & kVarDD) != 0;
+  static_assert(!DD || (VAR == kVarDD), "the fused double-backward pass is a variant of its own");
   // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x VEC
   // channels, so every row offset below folds into an immediate.
   const int mult = KMULT ? KMULT : a.mult;
   const int lg_G = KMULT ? 5 : lg_G_rt;
   const int S = KMULT ? KMULT / (32 * VEC) : S_rt;
   const int slice_base = KMULT ? CH * S : slice_base_rt;
-  using GR = ChunkGrp<PS, BwdPlan<PS, NEED_GY>, CH, kByL1>;
+  using PL = BwdPlan<PS, NEED_GY, VAR & kVarDD>;
+  using GR = ChunkGrp<PS, PL, CH, kByL1>;
   constexpr int L1 = GR::KEY;
   constexpr int NI = PS::NI, NO = PS::NO, NS = PS::NS, NR = GR::NOWN, NT = GR::NT;
-  constexpr int NW = WSH ? 1 : GR::NP;                       // staged weight rows
+  constexpr int NW = (WSH ? 1 : GR::NP) * (DD ? 2 : 1);     // staged weight rows (W, then gg_W)
+  constexpr int NTE = NT * (DD ? 2 : 1);                   // T floats per edge (T, then T')
   constexpr int NROWS = bwd_staged_rows<PS, GR, VAR>();
   constexpr unsigned GY_MASK = touched_sh_mask<PS, GR>();  // harmonics this chunk's paths reach
   extern __shared__ float4 smem_f4[];
@@ -267,16 +368,19 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
   const int grp = lane >> lg_G, gl = lane & (G - 1);
   const int rowf = G * VEC;
   const int stage_floats = NROWS * rowf;
-  const int group_floats = bwd_group_floats(BT, NT, stage_floats);
+  const int group_floats = bwd_group_floats(BT, NTE, stage_floats);
   float* Tg = smem + (warp * gpw + grp) * group_floats;
-  float* St = Tg + BT * NT;
+  float* St = Tg + BT * NTE;
   int* Eg = reinterpret_cast<int*>(St + 2 * stage_floats);
   int* Ig = Eg + ((BT + 3) & ~3);
   // grad_Y reduction buffer, per group of lanes: NS rows (one per harmonic)
   // of G lane partials, row stride rs = G + 4 (float4 aligned, and rows read
   // by the 8 lanes of one 128-bit access phase fall in distinct banks)
   const int rs = G + 4;
-  float* red = smem + (kBwdThreads / 32) * gpw * group_floats + (warp * gpw + grp) * bwd_red_floats(NS, G);
+  // (two such buffers in the fused double-backward pass: its A and B sums)
+  float* red = smem + (kBwdThreads / 32) * gpw * group_floats +
+               (warp * gpw + grp) * bwd_red_floats(NS, G) * (DD ? 2 : 1);
+  [[maybe_unused]] const int slices_total = S * PL::N;  // the B partials follow the A partials
 
   // The next chunk of this call may start on SMs this grid leaves idle: no
   // chunk reads what another writes, except a chunk that adds onto an
@@ -302,12 +406,18 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
     }
     const int maxdeg = __reduce_max_sync(0xffffffffu, k1 - k0);
     float xr[NR][VEC], gx[NR][VEC];
+    [[maybe_unused]] float gxr[NR][VEC];  // DD: gg_x of the source
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
-      if (active) VecIO<VEC>::ld(xr[r], a.x + (node * NI + L1 * L1 + r) * mult + c0);
-      else {
+      if (active) {
+        VecIO<VEC>::ld(xr[r], a.x + (node * NI + L1 * L1 + r) * mult + c0);
+        if constexpr (DD) VecIO<VEC>::ld(gxr[r], a.x2 + (node * NI + L1 * L1 + r) * mult + c0);
+      } else {
 #pragma unroll
-        for (int c = 0; c < VEC; ++c) xr[r][c] = 0.f;
+        for (int c = 0; c < VEC; ++c) {
+          xr[r][c] = 0.f;
+          if constexpr (DD) gxr[r][c] = 0.f;
+        }
       }
 #pragma unroll
       for (int c = 0; c < VEC; ++c) gx[r][c] = 0.f;
@@ -321,10 +431,12 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
         VecIO<VEC>::cp_async(dst, a.w + (long long)Eg[k] * mult + c0);
       } else {
         const float* wrow = a.w + (long long)Eg[k] * PS::NP * mult + c0;
+        [[maybe_unused]] const float* w2row = DD ? a.w2 + (long long)Eg[k] * PS::NP * mult + c0 : nullptr;
         static_for<0, GR::NP>([&](auto Kc) {
           constexpr int K = decltype(Kc)::value;
           constexpr int P = GR::D.path[K];
           VecIO<VEC>::cp_async(dst + K * rowf, wrow + P * mult);
+          if constexpr (DD) VecIO<VEC>::cp_async(dst + (GR::NP + K) * rowf, w2row + P * mult);
         });
       }
       if constexpr (PP) {
@@ -355,8 +467,24 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
         if (active && kk < k1) {
           const int e = __ldg(a.csc_edge + kk);
           float Y[NS];
-          edge_sh<PS::LS>(EXT ? a.sh : nullptr, a.edge_vec, e, Y);
-          compute_T_grp<PS, GR>(Y, Tg + k * NT);
+          if constexpr (DD) {
+            // Y and Y' = (dY/dr) gg_r in one evaluation
+            Dual1 yd[NS];
+            sh_dir_of_vec<PS::LS>(__ldg(a.edge_vec + 3 * e), __ldg(a.edge_vec + 3 * e + 1),
+                                  __ldg(a.edge_vec + 3 * e + 2), __ldg(a.gr_dir + 3 * e),
+                                  __ldg(a.gr_dir + 3 * e + 1), __ldg(a.gr_dir + 3 * e + 2), yd);
+            float Yd[NS];
+#pragma unroll
+            for (int b = 0; b < NS; ++b) {
+              Y[b] = yd[b].v;
+              Yd[b] = yd[b].e;
+            }
+            compute_T_grp<PS, GR>(Y, Tg + k * NT);
+            compute_T_grp<PS, GR>(Yd, Tg + (BT + k) * NT);
+          } else {
+            edge_sh<PS::LS>(EXT ? a.sh : nullptr, a.edge_vec, e, Y);
+            compute_T_grp<PS, GR>(Y, Tg + k * NT);
+          }
           Eg[k] = e;
           Ig[k] = __ldg(a.csc_dst + kk);
         }
@@ -374,43 +502,55 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
         if (valid) {
           e = Eg[k];
           float* gwrow = nullptr;
-          if (HX && a.grad_w != nullptr) gwrow = a.grad_w + (long long)e * (WSH ? 1 : PS::NP) * mult + c0;
-          // WSH: every chunk after the first adds onto the row (plain stream order)
-          const bool acc = (WSH && CH > 0) || (EXT && a.accumulate != 0);
-          bwd_edge<PS, GR, VEC, NEED_GY, VAR>(Tg + k * NT, St + (k & 1) * stage_floats + gl * VEC, rowf, xr, gwrow,
-                                               acc, mult, gx, red + gl, rs);
+          if (a.grad_w != nullptr) gwrow = a.grad_w + (long long)e * (WSH ? 1 : PS::NP) * mult + c0;
+          if constexpr (DD) {
+            bwd_edge_dd<PS, GR, VEC, NEED_GY>(Tg + k * NT, Tg + (BT + k) * NT,
+                                               St + (k & 1) * stage_floats + gl * VEC, rowf, xr, gxr, gwrow,
+                                               mult, gx, red + gl, red + NS * rs + gl, rs);
+          } else {
+            // WSH: every chunk after the first adds onto the row (plain stream order)
+            const bool acc = (WSH && CH > 0) || (EXT && a.accumulate != 0);
+            bwd_edge<PS, GR, VEC, NEED_GY, VAR>(Tg + k * NT, St + (k & 1) * stage_floats + gl * VEC, rowf, xr,
+                                                 gwrow, acc, mult, gx, red + gl, rs);
+          }
         }
         if constexpr (NEED_GY) {
           __syncwarp();
           if (valid) {
-            float* dst = a.grad_sh + ((long long)(slice_base + slice) * a.n_edges + e) * NS;
-            for (int b = gl; b < NS; b += G) {  // column sums; harmonics the chunk never reaches get 0
-              float v = 0.f;
-              if ((GY_MASK >> b) & 1u) {
-                const float* row = red + b * rs;
-                if (G % 4 == 0) {
-                  float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                  for (int r = 0; r < G; r += 4) {
-                    const float4 q4 = *reinterpret_cast<const float4*>(row + r);
-                    s4.x += q4.x;
-                    s4.y += q4.y;
-                    s4.z += q4.z;
-                    s4.w += q4.w;
+            // column sums; harmonics the chunk never reaches get 0
+            auto column_sums = [&](const float* rbuf, float* dst) {
+              for (int b = gl; b < NS; b += G) {
+                float v = 0.f;
+                if ((GY_MASK >> b) & 1u) {
+                  const float* row = rbuf + b * rs;
+                  if (G % 4 == 0) {
+                    float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int r = 0; r < G; r += 4) {
+                      const float4 q4 = *reinterpret_cast<const float4*>(row + r);
+                      s4.x += q4.x;
+                      s4.y += q4.y;
+                      s4.z += q4.z;
+                      s4.w += q4.w;
+                    }
+                    v = (s4.x + s4.y) + (s4.z + s4.w);
+                  } else {
+                    for (int r = 0; r < G; ++r) v += row[r];
                   }
-                  v = (s4.x + s4.y) + (s4.z + s4.w);
-                } else {
-                  for (int r = 0; r < G; ++r) v += row[r];
                 }
+                dst[b] = v;
               }
-              dst[b] = v;
-            }
+            };
+            column_sums(red, a.grad_sh + ((long long)(slice_base + slice) * a.n_edges + e) * NS);
+            if constexpr (DD)
+              column_sums(red + NS * rs,
+                          a.grad_sh + ((long long)(slices_total + slice_base + slice) * a.n_edges + e) * NS);
           }
           __syncwarp();
         }
       }
       __syncwarp();
     }
-    if (HX && active && a.grad_x != nullptr) {
+    if (active && a.grad_x != nullptr) {
       if (!GR::FIRST || (EXT && a.accumulate)) {
         // rows of an l1 block that an earlier chunk of this call wrote (wait
         // for that grid, the preceding launch), or the caller's values
@@ -511,39 +651,42 @@ __global__ void sh_backward_hess_kernel(int n_edges, int S, const float* __restr
 // channel lanes per group (G) and channel slices (S) of the backward
 inline void bwd_geometry(int mult, int& G, int& lg_G, int& S) { lane_geometry(mult, kBwdVec, G, lg_G, S); }
 
-// One partial grad_Y per (chunk, channel slice).
-template <class PS>
+// One partial grad_Y per (chunk, channel slice) (the fused double-backward
+// pass writes two such sets).
+template <class PS, int VAR = 0>
 int bwd_slices(int mult) {
   int G, lg_G, S;
   bwd_geometry(mult, G, lg_G, S);
-  return S * BwdPlan<PS, true>::N;
+  return S * BwdPlan<PS, true, VAR & kVarDD>::N;
 }
 
 // Launch chunk CH of variant VAR (the double backward's harmonics input or
 // accumulate mode selects the kExt kernel at run time).
 template <class PS, bool NEED_GY, int CH, int VAR>
 cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t stream, bool pdl) {
-  using GR = ChunkGrp<PS, BwdPlan<PS, NEED_GY>, CH, kByL1>;
+  using GR = ChunkGrp<PS, BwdPlan<PS, NEED_GY, VAR & kVarDD>, CH, kByL1>;
+  constexpr int mul = (VAR & kVarDD) ? 2 : 1;  // T and T', two reduction buffers
   int G, lg_G, S;
   bwd_geometry(a.mult, G, lg_G, S);
   const int gpw = 32 / G;
   const int stage_floats = bwd_staged_rows<PS, GR, VAR>() * G * kBwdVec;
-  const int BT = pick_batch(gpw, GR::NT, stage_floats, CGTP_BWD_BATCH_FLOATS, CGTP_BWD_MAX_BATCH);
+  const int BT = pick_batch(gpw, GR::NT * mul, stage_floats, CGTP_BWD_BATCH_FLOATS, CGTP_BWD_MAX_BATCH);
   // the kernel's indexing reaches gpw groups x warps of group_floats, then
   // (with NEED_GY) as many reduction buffers
   const size_t groups = (size_t)gpw * (kBwdThreads / 32);
-  const size_t smem = sizeof(float) * (groups * bwd_group_floats(BT, GR::NT, stage_floats) +
-                                       (NEED_GY ? groups * bwd_red_floats(PS::NS, G) : 0));
+  const size_t smem = sizeof(float) * (groups * bwd_group_floats(BT, GR::NT * mul, stage_floats) +
+                                       (NEED_GY ? groups * bwd_red_floats(PS::NS, G) * mul : 0));
   cudaError_t err = check_smem(smem);
   if (err != cudaSuccess) return err;
   const long long items = (long long)a.n_nodes * S;
   const long long blocks = (items + (long long)groups - 1) / (long long)groups;
   const bool ext = a.sh != nullptr || a.accumulate;
-  if (ext && (VAR & (kVarPerPath | kVarWShared))) return cudaErrorInvalidValue;  // not built
+  if (ext && (VAR & (kVarPerPath | kVarWShared | kVarDD))) return cudaErrorInvalidValue;  // not built
   // the compile-time multiplicity for the common case; the per-path layout
   // keeps the run-time one
   constexpr bool kAllow128 = (VAR & kVarPerPath) == 0;
-  auto kern = ext ? conv_bwd_kernel<PS, NEED_GY, CH, 0, VAR | kVarExt>
+  constexpr int kExtVar = (VAR & (kVarPerPath | kVarWShared | kVarDD)) ? VAR : (VAR | kVarExt);
+  auto kern = ext ? conv_bwd_kernel<PS, NEED_GY, CH, 0, kExtVar>
               : (kAllow128 && a.mult == 128) ? conv_bwd_kernel<PS, NEED_GY, CH, kAllow128 ? 128 : 0, VAR>
                                              : conv_bwd_kernel<PS, NEED_GY, CH, 0, VAR>;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -591,11 +734,11 @@ cudaError_t zero_unreached_grad_x(const ConvBwdArgs& a, cudaStream_t stream) {
 // onto one gradient row per edge, so they run in plain stream order.
 template <class PS, bool NEED_GY, int VAR, bool LANES>
 cudaError_t launch_bwd_chunks(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
-  using PL = BwdPlan<PS, NEED_GY>;
+  using PL = BwdPlan<PS, NEED_GY, VAR & kVarDD>;
   constexpr int NCH = PL::N;
   constexpr int NKEYS = PL::P.key[NCH - 1] - PL::P.key[0] + 1;
   constexpr bool kPdl = (VAR & kVarWShared) == 0;
-  cudaError_t err = (a.accumulate || (VAR & kVarGyOnly)) ? cudaSuccess : zero_unreached_grad_x<PS>(a, stream);
+  cudaError_t err = a.accumulate ? cudaSuccess : zero_unreached_grad_x<PS>(a, stream);
   if (err != cudaSuccess) return err;
   if constexpr (!LANES || NKEYS <= 1 || !kPdl) {
     static_for_host<0, NCH>([&](auto Cc) {
@@ -645,12 +788,70 @@ cudaError_t launch_sh_backward(const ConvBwdArgs& a, int slices, int num_sms, cu
 // grad_edge_vec is wanted), then the harmonic Jacobian epilogue.
 template <class PS, int VAR, bool LANES>
 cudaError_t launch_bwd_all(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
-  if ((VAR & kVarGyOnly) && (a.grad_edge_vec == nullptr || a.grad_sh == nullptr)) return cudaErrorInvalidValue;
-  if ((VAR & kVarGyOnly) && a.n_edges == 0) return cudaSuccess;
   const cudaError_t err = a.grad_edge_vec != nullptr ? launch_bwd_chunks<PS, true, VAR, LANES>(a, num_sms, stream)
                                                      : launch_bwd_chunks<PS, false, VAR, LANES>(a, num_sms, stream);
   if (err != cudaSuccess || a.grad_edge_vec == nullptr || a.n_edges == 0) return err;
   return launch_sh_backward<PS::LS>(a, bwd_slices<PS>(a.mult), num_sms, stream);
+}
+
+// The fused double backward's edge-vector term:
+//   d_r[e] = (dY/dr)^T A_e + sum_b B_e,b (d2Y_b/dr2) gg_r[e]
+// with A and B the two partial sets (each summed over its slices); one
+// evaluation gives the Jacobian and the Hessian-vector product.
+template <int LS>
+__global__ void sh_backward_dd_kernel(int n_edges, int S, const float* __restrict__ edge_vec,
+                                      const float* __restrict__ gsh, const float* __restrict__ q,
+                                      float* __restrict__ d_r) {
+  constexpr int NS = (LS + 1) * (LS + 1);
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n_edges;
+       e += (long long)gridDim.x * blockDim.x) {
+    float A[NS], B[NS];
+#pragma unroll
+    for (int b = 0; b < NS; ++b) A[b] = B[b] = 0.f;
+    for (int s = 0; s < S; ++s) {
+      const float* pa = gsh + ((long long)s * n_edges + e) * NS;
+      const float* pb = gsh + ((long long)(S + s) * n_edges + e) * NS;
+#pragma unroll
+      for (int b = 0; b < NS; ++b) {
+        A[b] += pa[b];
+        B[b] += pb[b];
+      }
+    }
+    HDual Y[NS];
+    sh_hess_of_vec<LS>(edge_vec[3 * e], edge_vec[3 * e + 1], edge_vec[3 * e + 2], q[3 * e], q[3 * e + 1],
+                       q[3 * e + 2], Y);
+    float d0 = 0.f, d1 = 0.f, d2 = 0.f;
+#pragma unroll
+    for (int b = 0; b < NS; ++b) {
+      d0 = fmaf(A[b], Y[b].d0.v, fmaf(B[b], Y[b].d0.e, d0));
+      d1 = fmaf(A[b], Y[b].d1.v, fmaf(B[b], Y[b].d1.e, d1));
+      d2 = fmaf(A[b], Y[b].d2.v, fmaf(B[b], Y[b].d2.e, d2));
+    }
+    d_r[3 * e] = d0;
+    d_r[3 * e + 1] = d1;
+    d_r[3 * e + 2] = d2;
+  }
+}
+
+// The fused double backward's source-centric pass: every chunk (the l1
+// blocks on forked lanes), then the edge-vector epilogue when
+// a.grad_edge_vec is wanted.  a.x2 = gg_x, a.w2 = gg_W, a.gr_dir = gg_r;
+// a.grad_x = d_x, a.grad_w = d_W, a.grad_edge_vec = d_r (each nullable);
+// a.grad_sh holds 2 x bwd_slices<PS, kVarDD> partial slices.
+template <class PS>
+cudaError_t launch_bwd_dd(const ConvBwdArgs& a, int num_sms, cudaStream_t stream) {
+  if (a.x2 == nullptr || a.w2 == nullptr || a.gr_dir == nullptr || a.sh != nullptr || a.accumulate)
+    return cudaErrorInvalidValue;
+  if (a.grad_edge_vec != nullptr && a.grad_sh == nullptr) return cudaErrorInvalidValue;
+  const cudaError_t err = a.grad_edge_vec != nullptr ? launch_bwd_chunks<PS, true, kVarDD, true>(a, num_sms, stream)
+                                                     : launch_bwd_chunks<PS, false, kVarDD, true>(a, num_sms, stream);
+  if (err != cudaSuccess || a.grad_edge_vec == nullptr || a.n_edges == 0) return err;
+  const int threads = 256;
+  long long nbk = (a.n_edges + threads - 1) / threads;
+  if (nbk > (long long)num_sms * 16) nbk = (long long)num_sms * 16;
+  sh_backward_dd_kernel<PS::LS><<<(unsigned)nbk, threads, 0, stream>>>(
+      a.n_edges, bwd_slices<PS, kVarDD>(a.mult), a.edge_vec, a.grad_sh, a.gr_dir, a.grad_edge_vec);
+  return cudaGetLastError();
 }
 
 }  // namespace

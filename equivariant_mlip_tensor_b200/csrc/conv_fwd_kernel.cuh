@@ -28,7 +28,12 @@
 //    one row per path;
 //  - GR::PERPATH: one block of 2 l3 + 1 output rows per path (the per-path
 //    messages of the fully connected convolution) instead of summing the
-//    paths of one l3.
+//    paths of one l3;
+//  - DD: the double backward's d grad_out in one pass,
+//      out = conv(gg_x, W, Y) + conv(x, gg_W, Y) + conv(x, W, Y'),
+//    Y' = (dY/dr) gg_r the harmonics' derivative along the edge-vector
+//    cotangent: each edge stages W, gg_W, x and gg_x rows and builds both
+//    T (from Y) and T' (from Y'), so W and gg_W are read once.
 //
 // Include after CGTP_DEFINE_CONSTANT_TABLES, conv_common.cuh, vec2.cuh and
 // sh.cuh.
@@ -167,10 +172,89 @@ __device__ __forceinline__ void fwd_edge(const float* __restrict__ T, const floa
   });
 }
 
+// One edge of the double backward's fused forward, per path:
+//   out[m3] += W (sum_m1 T gg_x[m1] + T' x[m1]) + gg_W sum_m1 T x[m1]
+// (T' has T's structural pattern: the same path with Y' in place of Y).
+// Stage layout: W rows (NP), gg_W rows (NP), x rows, gg_x rows (NROW each).
+template <class PS, class GR>
+__device__ __forceinline__ void fwd_edge_dd(const float* __restrict__ T, const float* __restrict__ Td,
+                                            const float* __restrict__ stage, int rowf,
+                                            float (&acc)[GR::NOWN][kFwdVec]) {
+  constexpr int NP = GR::NP, NR = GR::NROW;
+  float xr[NR][kFwdVec], gxr[NR][kFwdVec];
+#pragma unroll
+  for (int r = 0; r < NR; ++r) {
+    VecIO<kFwdVec>::lds(xr[r], stage + (2 * NP + r) * rowf);
+    VecIO<kFwdVec>::lds(gxr[r], stage + (2 * NP + NR + r) * rowf);
+  }
+  static_for<0, NP>([&](auto Kc) {
+    constexpr int K = decltype(Kc)::value;
+    constexpr int P = GR::D.path[K];
+    constexpr int l1 = PS::D.l1[P], l3 = PS::D.l3[P];
+    constexpr int tc = PS::D.tcount[P], tb = GR::D.lt[K];
+    float wv[kFwdVec], gwv[kFwdVec];
+    VecIO<kFwdVec>::lds(wv, stage + K * rowf);
+    VecIO<kFwdVec>::lds(gwv, stage + (NP + K) * rowf);
+    constexpr int o3 = l3 * l3 - GR::OWN0;
+    if constexpr (2 * l3 + 1 <= 2 * l1 + 1) {
+      // tw[m3] = sum T gg_x + T' x (multiplied by W), tg[m3] = sum T x (by gg_W)
+      float tw[2 * l3 + 1][kFwdVec], tg[2 * l3 + 1][kFwdVec];
+#pragma unroll
+      for (int m3 = 0; m3 < 2 * l3 + 1; ++m3)
+#pragma unroll
+        for (int c = 0; c < kFwdVec; ++c) tw[m3][c] = tg[m3][c] = 0.f;
+      static_for<0, (tc + 3) / 4>([&](auto Qc) {
+        constexpr int q = decltype(Qc)::value;
+        const float4 v4 = *reinterpret_cast<const float4*>(T + tb + 4 * q);
+        const float4 d4 = *reinterpret_cast<const float4*>(Td + tb + 4 * q);
+        const float tv4[4] = {v4.x, v4.y, v4.z, v4.w}, td4[4] = {d4.x, d4.y, d4.z, d4.w};
+        static_for<0, 4>([&](auto Rc) {
+          constexpr int k = 4 * q + decltype(Rc)::value;
+          if constexpr (k < tc) {
+            constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
+            constexpr int rx = l1 * l1 + l1 + m1 - GR::D.rlo;
+            axpy<kFwdVec>(tw[m3 + l3], tv4[decltype(Rc)::value], gxr[rx]);
+            axpy<kFwdVec>(tw[m3 + l3], td4[decltype(Rc)::value], xr[rx]);
+            axpy<kFwdVec>(tg[m3 + l3], tv4[decltype(Rc)::value], xr[rx]);
+          }
+        });
+      });
+#pragma unroll
+      for (int m3 = 0; m3 < 2 * l3 + 1; ++m3) {
+        vfma<kFwdVec>(acc[o3 + m3], wv, tw[m3]);
+        vfma<kFwdVec>(acc[o3 + m3], gwv, tg[m3]);
+      }
+    } else {
+      // qa[m1] = W gg_x + gg_W x (through T), qb[m1] = W x (through T')
+      float qa[2 * l1 + 1][kFwdVec], qb[2 * l1 + 1][kFwdVec];
+#pragma unroll
+      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) {
+        vmul<kFwdVec>(qa[m1], wv, gxr[l1 * l1 + m1 - GR::D.rlo]);
+        vfma<kFwdVec>(qa[m1], gwv, xr[l1 * l1 + m1 - GR::D.rlo]);
+        vmul<kFwdVec>(qb[m1], wv, xr[l1 * l1 + m1 - GR::D.rlo]);
+      }
+      static_for<0, (tc + 3) / 4>([&](auto Qc) {
+        constexpr int q = decltype(Qc)::value;
+        const float4 v4 = *reinterpret_cast<const float4*>(T + tb + 4 * q);
+        const float4 d4 = *reinterpret_cast<const float4*>(Td + tb + 4 * q);
+        const float tv4[4] = {v4.x, v4.y, v4.z, v4.w}, td4[4] = {d4.x, d4.y, d4.z, d4.w};
+        static_for<0, 4>([&](auto Rc) {
+          constexpr int k = 4 * q + decltype(Rc)::value;
+          if constexpr (k < tc) {
+            constexpr int m1 = PS::t_entry_m1(P, k), m3 = PS::t_entry_m3(P, k);
+            axpy<kFwdVec>(acc[o3 + m3 + l3], tv4[decltype(Rc)::value], qa[m1 + l1]);
+            axpy<kFwdVec>(acc[o3 + m3 + l3], td4[decltype(Rc)::value], qb[m1 + l1]);
+          }
+        });
+      });
+    }
+  });
+}
+
 // GR: the launch's paths (all of them, or one chunk of one l3 block).  A
 // chunk that continues an l3 block another chunk of the call started adds
 // onto that chunk's rows (GR::FIRST false).
-template <class PS, class GR, int KMULT, bool WSH>
+template <class PS, class GR, int KMULT, bool WSH, bool DD>
 __global__ void CGTP_FWD_BOUNDS
 conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
   // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x 4
@@ -179,17 +263,20 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
   const int lg_G = KMULT ? 5 : lg_G_rt;
   const int S = KMULT ? KMULT / (32 * kFwdVec) : S_rt;
   constexpr int NI = PS::NI, NO = PS::NO, NS = PS::NS, NT = GR::NT;
-  constexpr int NW = WSH ? 1 : GR::NP;  // staged weight rows
+  constexpr int NW = (WSH ? 1 : GR::NP) * (DD ? 2 : 1);  // staged weight rows (W, then gg_W)
+  constexpr int NXR = GR::NROW * (DD ? 2 : 1);            // staged feature rows (x, then gg_x)
+  constexpr int NTE = NT * (DD ? 2 : 1);                  // T floats per edge (T, then T')
+  static_assert(!DD || kStageX, "the fused double-backward pass stages its feature rows");
   extern __shared__ float4 smem_f4[];
   float* smem = reinterpret_cast<float*>(smem_f4);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int G = 1 << lg_G, gpw = 32 >> lg_G;
   const int grp = lane >> lg_G, gl = lane & (G - 1);
   const int rowf = G * kFwdVec;                    // floats per staged row
-  const int stage_floats = fwd_stage_floats(NW, GR::NROW, G);
-  const int group_floats = fwd_group_floats(BT, NT, stage_floats);
+  const int stage_floats = fwd_stage_floats(NW, NXR, G);
+  const int group_floats = fwd_group_floats(BT, NTE, stage_floats);
   float* Tg = smem + (warp * gpw + grp) * group_floats;
-  float* St = Tg + BT * NT;                        // two pipeline stages
+  float* St = Tg + BT * NTE;                       // two pipeline stages
   int* Jg = reinterpret_cast<int*>(St + 2 * stage_floats);
 
   // The next launch of this call may start on SMs this grid leaves idle
@@ -230,17 +317,25 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
         VecIO<kFwdVec>::cp_async(dst, a.w + (long long)e * mult + c0);
       } else {
         const float* wrow = a.w + (long long)e * PS::NP * mult + c0;
+        [[maybe_unused]] const float* w2row = DD ? a.w2 + (long long)e * PS::NP * mult + c0 : nullptr;
         static_for<0, GR::NP>([&](auto Kc) {
           constexpr int K = decltype(Kc)::value;
           constexpr int P = GR::D.path[K];
           VecIO<kFwdVec>::cp_async(dst + K * rowf, wrow + P * mult);
+          if constexpr (DD) VecIO<kFwdVec>::cp_async(dst + (GR::NP + K) * rowf, w2row + P * mult);
         });
       }
-      if constexpr (kStageX) {
+      if constexpr (kStageX || DD) {
         constexpr int rlo = GR::D.rlo;
         const float* xrow = a.x + ((long long)Jg[k] * NI + rlo) * mult + c0;
 #pragma unroll
         for (int r = 0; r < GR::NROW; ++r) VecIO<kFwdVec>::cp_async(dst + (NW + r) * rowf, xrow + r * mult);
+        if constexpr (DD) {
+          const float* x2row = a.x2 + ((long long)Jg[k] * NI + rlo) * mult + c0;
+#pragma unroll
+          for (int r = 0; r < GR::NROW; ++r)
+            VecIO<kFwdVec>::cp_async(dst + (NW + GR::NROW + r) * rowf, x2row + r * mult);
+        }
       }
     };
 
@@ -266,8 +361,24 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
         const int e = e0 + b0 + k;
         if (active && e < e1) {
           float Y[NS];
-          edge_sh<PS::LS>(a.sh, a.edge_vec, e, Y);
-          compute_T_grp<PS, GR>(Y, Tg + k * NT);
+          if constexpr (DD) {
+            // Y and Y' = (dY/dr) gg_r in one evaluation
+            Dual1 yd[NS];
+            sh_dir_of_vec<PS::LS>(__ldg(a.edge_vec + 3 * e), __ldg(a.edge_vec + 3 * e + 1),
+                                  __ldg(a.edge_vec + 3 * e + 2), __ldg(a.gr_dir + 3 * e),
+                                  __ldg(a.gr_dir + 3 * e + 1), __ldg(a.gr_dir + 3 * e + 2), yd);
+            float Yd[NS];
+#pragma unroll
+            for (int b = 0; b < NS; ++b) {
+              Y[b] = yd[b].v;
+              Yd[b] = yd[b].e;
+            }
+            compute_T_grp<PS, GR>(Y, Tg + k * NT);
+            compute_T_grp<PS, GR>(Yd, Tg + (BT + k) * NT);
+          } else {
+            edge_sh<PS::LS>(a.sh, a.edge_vec, e, Y);
+            compute_T_grp<PS, GR>(Y, Tg + k * NT);
+          }
         }
       }
       __syncwarp();
@@ -277,8 +388,12 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
         cp_async_wait<1>();  // this lane's copies of edge k have landed
         if (active && e0 + b0 + k < e1) {
           constexpr int rlo = GR::D.rlo;
-          fwd_edge<PS, GR, WSH>(Tg + k * NT, St + (k & 1) * stage_floats + gl * kFwdVec, rowf,
-                                a.x + ((long long)Jg[k] * NI + rlo) * mult + c0, mult, acc);
+          if constexpr (DD)
+            fwd_edge_dd<PS, GR>(Tg + k * NT, Tg + (BT + k) * NT, St + (k & 1) * stage_floats + gl * kFwdVec, rowf,
+                                acc);
+          else
+            fwd_edge<PS, GR, WSH>(Tg + k * NT, St + (k & 1) * stage_floats + gl * kFwdVec, rowf,
+                                  a.x + ((long long)Jg[k] * NI + rlo) * mult + c0, mult, acc);
         }
       }
       __syncwarp();
@@ -323,18 +438,20 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
   grid_dependency_wait();
 }
 
-template <class PS, class GR, bool WSH>
+template <class PS, class GR, bool WSH, bool DD = false>
 cudaError_t launch_fwd_group(const ConvFwdArgs& a, int num_sms, bool pdl, cudaStream_t stream) {
   int G, lg_G, S;
   lane_geometry(a.mult, kFwdVec, G, lg_G, S);
   const int gpw = 32 / G;
-  const int stage_floats = fwd_stage_floats(WSH ? 1 : GR::NP, GR::NROW, G);
-  const int BT = pick_batch(gpw, GR::NT, stage_floats, CGTP_FWD_BATCH_FLOATS, CGTP_FWD_MAX_BATCH);
+  const int mul = DD ? 2 : 1;  // the fused double-backward pass stages and builds everything twice
+  const int stage_floats = fwd_stage_floats((WSH ? 1 : GR::NP) * mul, GR::NROW * mul, G);
+  const int BT = pick_batch(gpw, GR::NT * mul, stage_floats, CGTP_FWD_BATCH_FLOATS, CGTP_FWD_MAX_BATCH);
   // the kernel's indexing reaches gpw groups x warps of group_floats each
-  const size_t smem = sizeof(float) * (size_t)fwd_group_floats(BT, GR::NT, stage_floats) * gpw * (kFwdThreads / 32);
+  const size_t smem =
+      sizeof(float) * (size_t)fwd_group_floats(BT, GR::NT * mul, stage_floats) * gpw * (kFwdThreads / 32);
   cudaError_t err = check_smem(smem);
   if (err != cudaSuccess) return err;
-  auto kern = a.mult == 128 ? conv_fwd_kernel<PS, GR, 128, WSH> : conv_fwd_kernel<PS, GR, 0, WSH>;
+  auto kern = a.mult == 128 ? conv_fwd_kernel<PS, GR, 128, WSH, DD> : conv_fwd_kernel<PS, GR, 0, WSH, DD>;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const long long items = (long long)a.n_nodes * S;
@@ -362,6 +479,10 @@ constexpr int fwd_all_cost() {
 
 template <class PS>
 using FwdPlan = Plan<PS, kByL3, kFwdVec, false, CGTP_FWD_BUDGET>;
+// the fused double-backward forward carries about three times the code per
+// path (three T products): chunks of a third of the budget
+template <class PS>
+using FwdPlanDD = Plan<PS, kByL3, kFwdVec, false, CGTP_FWD_BUDGET / 3>;
 
 // Output blocks l3 that no path reaches are zero.
 template <class PS>
@@ -395,6 +516,26 @@ cudaError_t launch_fwd_all(const ConvFwdArgs& a, int num_sms, cudaStream_t strea
       constexpr int CH = decltype(Cc)::value;
       if (err == cudaSuccess)
         err = launch_fwd_group<PS, ChunkGrp<PS, FwdPlan<PS>, CH, kByL3>, WSH>(a, num_sms, CH > 0, stream);
+    });
+    return err;
+  }
+}
+
+// The double backward's d grad_out in one pass per chunk of same-l3 paths
+// (a.x2 = gg_x, a.w2 = gg_W, a.gr_dir = gg_r); overwrites a.out.
+template <class PS>
+cudaError_t launch_fwd_dd(const ConvFwdArgs& a, int num_sms, cudaStream_t stream) {
+  if (a.x2 == nullptr || a.w2 == nullptr || a.gr_dir == nullptr || a.accumulate || a.sh != nullptr)
+    return cudaErrorInvalidValue;
+  if constexpr (3 * fwd_all_cost<PS>() <= CGTP_FWD_SINGLE_MAX) {
+    return launch_fwd_group<PS, Grp<PS, kAll, 0>, false, true>(a, num_sms, false, stream);
+  } else {
+    cudaError_t err = zero_unreached_out<PS>(a, stream);
+    static_for_host<0, FwdPlanDD<PS>::N>([&](auto Cc) {
+      constexpr int CH = decltype(Cc)::value;
+      if (err == cudaSuccess)
+        err = launch_fwd_group<PS, ChunkGrp<PS, FwdPlanDD<PS>, CH, kByL3>, false, true>(a, num_sms, CH > 0,
+                                                                                         stream);
     });
     return err;
   }

@@ -70,13 +70,16 @@ template <int LI, int LS, int LO>
 cudaError_t launch_conv_bwd_shared(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);
 template <int LI, int LS, int LO>
 cudaError_t launch_conv_bwd_paths(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);
-// The harmonic gradient alone (grad_Y partials and the Jacobian epilogue of
-// a.gr_mode; no grad_x / grad_W work), and the number of grad_Y partial slices
-// it writes.
-template <int LI, int LS, int LO>
-cudaError_t launch_conv_bwd_gy(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);
 template <int LI, int LS, int LO>
 cudaError_t launch_conv_bwd(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);
+// The double backward's fused passes (conv_dd.cu) and the number of partial
+// slices of each of the fused pass's two harmonic-gradient sets.
+template <int LI, int LS, int LO>
+cudaError_t launch_conv_dd_fwd(const ConvFwdArgs& a, int num_sms, cudaStream_t stream);
+template <int LI, int LS, int LO>
+cudaError_t launch_conv_dd_bwd(const ConvBwdArgs& a, int num_sms, cudaStream_t stream);
+template <int LI, int LS, int LO>
+int conv_dd_slices(int mult);
 template <int LI, int LS, int LO>
 int conv_bwd_slices(int mult);
 template <int LI, int LS, int LO>

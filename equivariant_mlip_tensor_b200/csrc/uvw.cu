@@ -104,7 +104,10 @@ using namespace cute;
 #ifndef CGTP_UVW_TILE_N_MIX
 #define CGTP_UVW_TILE_N_MIX 64  // mixing-gradient GEMM: few, long tiles, so narrower ones
 #endif
-using TileShape = Shape<_128, Int<CGTP_UVW_TILE_N>, _32>;
+#ifndef CGTP_UVW_TILE_M
+#define CGTP_UVW_TILE_M 128  // node-row tile of the mixing GEMMs
+#endif
+using TileShape = Shape<Int<CGTP_UVW_TILE_M>, Int<CGTP_UVW_TILE_N>, _32>;
 using TileShapeT = Shape<_128, Int<CGTP_UVW_TILE_N_MIX>, _32>;
 using ClusterShape = Shape<_1, _1, _1>;
 constexpr int kAlign = 4;  // floats: 16-byte rows and strides
