@@ -77,23 +77,43 @@ constexpr int kBwdVec = CGTP_BWD_VEC;
 #define CGTP_BWD_PDL 1
 #endif
 
-// Unrolled instructions per edge and lane allowed in one backward launch.
+// Unrolled instructions per edge and lane allowed in one backward launch
+// (measured at the molecules shape: 1100 -> 1400 took the backward from
+// 0.535 to 0.507 ms; 1700 and more lose again, and a launch near 3000
+// instructions doubles the time on instruction fetch), and in one launch of
+// the fused double-backward pass (two T products per path: 730 measured
+// best of 488 ... 2000).
 #ifndef CGTP_BWD_BUDGET
-#define CGTP_BWD_BUDGET 1100
+#define CGTP_BWD_BUDGET 1400
 #endif
 #ifndef CGTP_BWD_BUDGET_L3
 #define CGTP_BWD_BUDGET_L3 800  // l = 3 chunks carry more registers per path
+#endif
+#ifndef CGTP_DD_BWD_BUDGET
+#define CGTP_DD_BWD_BUDGET 730
 #endif
 template <class PS>
 constexpr int bwd_budget() {
   return PS::LI >= 3 || PS::LO >= 3 ? CGTP_BWD_BUDGET_L3 : CGTP_BWD_BUDGET;
 }
+template <class PS>
+constexpr int dd_bwd_budget() {  // l = 3: scaled like the plain backward's
+  return PS::LI >= 3 || PS::LO >= 3 ? CGTP_DD_BWD_BUDGET * CGTP_BWD_BUDGET_L3 / 1100 : CGTP_DD_BWD_BUDGET;
+}
 
 // The fused double-backward pass carries a little over twice the code per
-// path (two T products, two harmonic-gradient sums): chunks of 4/9 of the
-// budget.
+// path (two T products, two harmonic-gradient sums): its own budget.
+// Merge small l1 blocks into the next one's launch when the whole blocks fit
+// the budget (1), or one launch per block at least (0).
+#ifndef CGTP_BWD_MERGE
+#define CGTP_BWD_MERGE 1
+#endif
+// The fused double-backward pass plans its chunks as if the harmonic
+// gradient were always wanted, so that d x and d W come out of the same
+// chunks (and bit for bit the same) whichever outputs a call requests.
 template <class PS, bool NEED_GY, int VAR = 0>
-using BwdPlan = Plan<PS, kByL1, kBwdVec, NEED_GY, (VAR & kVarDD) ? bwd_budget<PS>() * 4 / 9 : bwd_budget<PS>()>;
+using BwdPlan = Plan<PS, kByL1, kBwdVec, ((VAR & kVarDD) != 0) || NEED_GY,
+                     (VAR & kVarDD) ? dd_bwd_budget<PS>() : bwd_budget<PS>(), (1 << 30), CGTP_BWD_MERGE != 0>;
 
 template <class PS, class GR>
 constexpr unsigned touched_sh_mask() {
@@ -157,6 +177,7 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
     constexpr int l1 = PS::D.l1[P], l3 = PS::D.l3[P];
     [[maybe_unused]] constexpr int l2 = PS::D.l2[P];
     constexpr int tb = GR::D.lt[K], tc = PS::D.tcount[P];
+    constexpr int o1 = l1 * l1 - GR::OWN0;  // the path's x / grad_x rows among the chunk's own
     // staged row of grad_out[l3, m3 = -l3] (of this path's own rows when PP)
     constexpr int g0 = NW + (PP ? pp_rowoff<PS, GR>(K) : l3 * l3 - GR::D.rlo);
     if constexpr (NEED_GY && GR::D.first_l2[K]) {
@@ -175,7 +196,7 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
     [[maybe_unused]] float xw[2 * l1 + 1][VEC];  // W x, for the grad_Y channel sums
     if constexpr (NEED_GY) {
 #pragma unroll
-      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) vmul<VEC>(xw[m1], wv, xr[m1]);
+      for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) vmul<VEC>(xw[m1], wv, xr[o1 + m1]);
     }
     static_for<0, (tc + 3) / 4>([&](auto Qc) {
       constexpr int q = decltype(Qc)::value;
@@ -203,8 +224,8 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
       if constexpr (WSH) {
 #pragma unroll
         for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) {
-          vfma<VEC>(gx[m1], wv, h[m1]);
-          vfma<VEC>(gws, xr[m1], h[m1]);
+          vfma<VEC>(gx[o1 + m1], wv, h[m1]);
+          vfma<VEC>(gws, xr[o1 + m1], h[m1]);
         }
       } else {
         float gw[VEC];
@@ -212,8 +233,8 @@ __device__ __forceinline__ void bwd_edge(const float* __restrict__ T, const floa
         for (int c = 0; c < VEC; ++c) gw[c] = 0.f;
 #pragma unroll
         for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) {
-          vfma<VEC>(gx[m1], wv, h[m1]);
-          vfma<VEC>(gw, xr[m1], h[m1]);
+          vfma<VEC>(gx[o1 + m1], wv, h[m1]);
+          vfma<VEC>(gw, xr[o1 + m1], h[m1]);
         }
         if (gwrow != nullptr) {
           if (acc) {
@@ -267,6 +288,7 @@ __device__ __forceinline__ void bwd_edge_dd(const float* __restrict__ T, const f
     [[maybe_unused]] constexpr int l2 = PS::D.l2[P];
     constexpr int tb = GR::D.lt[K], tc = PS::D.tcount[P];
     constexpr int g0 = 2 * NP + l3 * l3 - GR::D.rlo;  // staged row of grad_out[l3, m3 = -l3]
+    constexpr int o1 = l1 * l1 - GR::OWN0;             // the path's rows among the chunk's own
     if constexpr (NEED_GY && GR::D.first_l2[K]) {
 #pragma unroll
       for (int m2 = 0; m2 < 2 * l2 + 1; ++m2) gyA[l2 * l2 + m2] = gyB[l2 * l2 + m2] = 0.f;
@@ -285,9 +307,9 @@ __device__ __forceinline__ void bwd_edge_dd(const float* __restrict__ T, const f
     if constexpr (NEED_GY) {
 #pragma unroll
       for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) {
-        vmul<VEC>(pa[m1], wv, gxr[m1]);
-        vfma<VEC>(pa[m1], gwv, xr[m1]);
-        vmul<VEC>(pb[m1], wv, xr[m1]);
+        vmul<VEC>(pa[m1], wv, gxr[o1 + m1]);
+        vfma<VEC>(pa[m1], gwv, xr[o1 + m1]);
+        vmul<VEC>(pb[m1], wv, xr[o1 + m1]);
       }
     }
     static_for<0, (tc + 3) / 4>([&](auto Qc) {
@@ -321,10 +343,10 @@ __device__ __forceinline__ void bwd_edge_dd(const float* __restrict__ T, const f
     for (int c = 0; c < VEC; ++c) gw[c] = 0.f;
 #pragma unroll
     for (int m1 = 0; m1 < 2 * l1 + 1; ++m1) {
-      vfma<VEC>(gx[m1], gwv, h[m1]);
-      vfma<VEC>(gx[m1], wv, hd[m1]);
-      vfma<VEC>(gw, gxr[m1], h[m1]);
-      vfma<VEC>(gw, xr[m1], hd[m1]);
+      vfma<VEC>(gx[o1 + m1], gwv, h[m1]);
+      vfma<VEC>(gx[o1 + m1], wv, hd[m1]);
+      vfma<VEC>(gw, gxr[o1 + m1], h[m1]);
+      vfma<VEC>(gw, xr[o1 + m1], hd[m1]);
     }
     if (gwrow != nullptr) VecIO<VEC>::st_stream(gwrow + P * mult, gw);
     if constexpr (NEED_GY && GR::D.last_l2[K]) {
@@ -342,7 +364,7 @@ __device__ __forceinline__ void bwd_edge_dd(const float* __restrict__ T, const f
 // of the chunk's paths and a partial grad_Y over them.
 template <class PS, bool NEED_GY, int CH, int KMULT, int VAR>
 __global__ void CGTP_BWD_BOUNDS
-conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt) {
+conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt, int lg_Q) {
   constexpr int VEC = kBwdVec;
   constexpr bool EXT = (VAR & kVarExt) != 0, PP = (VAR & kVarPerPath) != 0;
   constexpr bool WSH = (VAR & kVarWShared) != 0, DD = (VAR & kVarDD) != 0;
@@ -355,7 +377,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
   const int slice_base = KMULT ? CH * S : slice_base_rt;
   using PL = BwdPlan<PS, NEED_GY, VAR & kVarDD>;
   using GR = ChunkGrp<PS, PL, CH, kByL1>;
-  constexpr int L1 = GR::KEY;
+  constexpr int OWN0 = GR::OWN0;  // first x / grad_x row of the chunk's l1 blocks
   constexpr int NI = PS::NI, NO = PS::NO, NS = PS::NS, NR = GR::NOWN, NT = GR::NT;
   constexpr int NW = (WSH ? 1 : GR::NP) * (DD ? 2 : 1);     // staged weight rows (W, then gg_W)
   constexpr int NTE = NT * (DD ? 2 : 1);                   // T floats per edge (T, then T')
@@ -390,28 +412,35 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
     grid_dependency_wait();
     return;
   }
+  // Row split: Q = 2^lg_Q groups of lanes share one work item (source row),
+  // group `part` taking the row's edges part, part + Q, ...; their grad_x
+  // accumulators are summed by shuffles at the end.
+  const int Q = 1 << lg_Q, part = grp & (Q - 1), ipw = gpw >> lg_Q;  // items per warp
+  const uint64_t wpol = stream_policy();
   const long long n_items = (long long)a.n_nodes * S;
   const long long warps_total = (long long)gridDim.x * (kBwdThreads / 32);
-  for (long long base = ((long long)blockIdx.x * (kBwdThreads / 32) + warp) * gpw; base < n_items;
-       base += warps_total * gpw) {
-    const long long item = base + grp;
+  for (long long base = ((long long)blockIdx.x * (kBwdThreads / 32) + warp) * ipw; base < n_items;
+       base += warps_total * ipw) {
+    const long long item = base + (grp >> lg_Q);
     const bool active = item < n_items;
     const long long node = active ? item / S : 0;
     const int slice = active ? int(item % S) : 0;
     const int c0 = (slice * G + gl) * VEC;
-    int k0 = 0, k1 = 0;
+    int k0 = 0, cnt = 0;  // this group's CSC slots: k0 + part + Q t, t < cnt
     if (active) {
       k0 = __ldg(a.csc_ptr + node);
-      k1 = __ldg(a.csc_ptr + node + 1);
+      const int deg = __ldg(a.csc_ptr + node + 1) - k0;
+      cnt = deg > part ? (deg - part + Q - 1) >> lg_Q : 0;
+      k0 += part;
     }
-    const int maxdeg = __reduce_max_sync(0xffffffffu, k1 - k0);
+    const int maxdeg = __reduce_max_sync(0xffffffffu, cnt);
     float xr[NR][VEC], gx[NR][VEC];
     [[maybe_unused]] float gxr[NR][VEC];  // DD: gg_x of the source
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
       if (active) {
-        VecIO<VEC>::ld(xr[r], a.x + (node * NI + L1 * L1 + r) * mult + c0);
-        if constexpr (DD) VecIO<VEC>::ld(gxr[r], a.x2 + (node * NI + L1 * L1 + r) * mult + c0);
+        VecIO<VEC>::ld(xr[r], a.x + (node * NI + OWN0 + r) * mult + c0);
+        if constexpr (DD) VecIO<VEC>::ld(gxr[r], a.x2 + (node * NI + OWN0 + r) * mult + c0);
       } else {
 #pragma unroll
         for (int c = 0; c < VEC; ++c) {
@@ -425,18 +454,18 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
 
     // copies of edge slot k of the current batch into stage s (this lane's channels only)
     auto issue = [&](int b0, int k, int s) {
-      if (!(active && k0 + b0 + k < k1)) return;
+      if (!(active && b0 + k < cnt)) return;
       float* dst = St + s * stage_floats + gl * VEC;
       if constexpr (WSH) {
-        VecIO<VEC>::cp_async(dst, a.w + (long long)Eg[k] * mult + c0);
+        cp_async_w<VEC>(dst, a.w + (long long)Eg[k] * mult + c0, wpol);
       } else {
         const float* wrow = a.w + (long long)Eg[k] * PS::NP * mult + c0;
         [[maybe_unused]] const float* w2row = DD ? a.w2 + (long long)Eg[k] * PS::NP * mult + c0 : nullptr;
         static_for<0, GR::NP>([&](auto Kc) {
           constexpr int K = decltype(Kc)::value;
           constexpr int P = GR::D.path[K];
-          VecIO<VEC>::cp_async(dst + K * rowf, wrow + P * mult);
-          if constexpr (DD) VecIO<VEC>::cp_async(dst + (GR::NP + K) * rowf, w2row + P * mult);
+          cp_async_w<VEC>(dst + K * rowf, wrow + P * mult, wpol);
+          if constexpr (DD) cp_async_w<VEC>(dst + (GR::NP + K) * rowf, w2row + P * mult, wpol);
         });
       }
       if constexpr (PP) {
@@ -463,8 +492,8 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
 
     for (int b0 = 0; b0 < maxdeg; b0 += BT) {
       for (int k = gl; k < BT; k += G) {
-        const int kk = k0 + b0 + k;
-        if (active && kk < k1) {
+        const int kk = k0 + ((b0 + k) << lg_Q);
+        if (active && b0 + k < cnt) {
           const int e = __ldg(a.csc_edge + kk);
           float Y[NS];
           if constexpr (DD) {
@@ -497,7 +526,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
         if (k + 1 < nb) issue(b0, k + 1, (k + 1) & 1);
         cp_async_commit();
         cp_async_wait<1>();  // this lane's copies of edge k have landed
-        const bool valid = active && (k0 + b0 + k) < k1;
+        const bool valid = active && b0 + k < cnt;
         int e = 0;
         if (valid) {
           e = Eg[k];
@@ -550,7 +579,14 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
       }
       __syncwarp();
     }
-    if (active && a.grad_x != nullptr) {
+    // the row's parts: sum the groups of one item (lanes gl + G part)
+    for (int sh = 1; sh < Q; sh <<= 1) {
+#pragma unroll
+      for (int r = 0; r < NR; ++r)
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) gx[r][c] += __shfl_xor_sync(0xffffffffu, gx[r][c], sh * G);
+    }
+    if (active && part == 0 && a.grad_x != nullptr) {
       if (!GR::FIRST || (EXT && a.accumulate)) {
         // rows of an l1 block that an earlier chunk of this call wrote (wait
         // for that grid, the preceding launch), or the caller's values
@@ -558,13 +594,13 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt)
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
           float prev[VEC];
-          VecIO<VEC>::ld(prev, a.grad_x + (node * NI + L1 * L1 + r) * mult + c0);
+          VecIO<VEC>::ld(prev, a.grad_x + (node * NI + OWN0 + r) * mult + c0);
 #pragma unroll
           for (int c = 0; c < VEC; ++c) gx[r][c] += prev[c];
         }
       }
 #pragma unroll
-      for (int r = 0; r < NR; ++r) VecIO<VEC>::st(a.grad_x + (node * NI + L1 * L1 + r) * mult + c0, gx[r]);
+      for (int r = 0; r < NR; ++r) VecIO<VEC>::st(a.grad_x + (node * NI + OWN0 + r) * mult + c0, gx[r]);
     }
   }
   // Complete only after the preceding launch: a grid launched with
@@ -679,7 +715,9 @@ cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t str
   cudaError_t err = check_smem(smem);
   if (err != cudaSuccess) return err;
   const long long items = (long long)a.n_nodes * S;
-  const long long blocks = (items + (long long)groups - 1) / (long long)groups;
+  const int lg_Q = row_split(items, gpw, num_sms);
+  const long long items_per_block = (long long)(gpw >> lg_Q) * (kBwdThreads / 32);
+  const long long blocks = (items + items_per_block - 1) / items_per_block;
   const bool ext = a.sh != nullptr || a.accumulate;
   if (ext && (VAR & (kVarPerPath | kVarWShared | kVarDD))) return cudaErrorInvalidValue;  // not built
   // the compile-time multiplicity for the common case; the per-path layout
@@ -701,7 +739,7 @@ cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t str
   long long nb = blocks > cap ? cap : blocks;
   if (nb < 1) nb = 1;
   return launch_kernel(kern, dim3((unsigned)nb), dim3(kBwdThreads), smem, stream, CGTP_BWD_PDL && pdl, a, lg_G,
-                       S, BT, CH * S);
+                       S, BT, CH * S, lg_Q);
 }
 
 // grad_x blocks that no path reaches (l1 with no path) are zero.

@@ -21,6 +21,12 @@ struct VecIO<4> {
     const unsigned sa = (unsigned)__cvta_generic_to_shared(s);
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(g) : "memory");
   }
+  // the same with an L2 eviction policy (streamed data: evict first)
+  static __device__ __forceinline__ void cp_async_hint(float* s, const float* g, uint64_t pol) {
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(s);
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(sa), "l"(g), "l"(pol)
+                 : "memory");
+  }
 };
 template <>
 struct VecIO<2> {
@@ -38,7 +44,30 @@ struct VecIO<2> {
     const unsigned sa = (unsigned)__cvta_generic_to_shared(s);
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(sa), "l"(g) : "memory");
   }
+  static __device__ __forceinline__ void cp_async_hint(float* s, const float* g, uint64_t pol) {
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(s);
+    asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 8, %2;" ::"r"(sa), "l"(g), "l"(pol)
+                 : "memory");
+  }
 };
+
+// Weight rows are streamed (each read once per pass).  With
+// CGTP_W_EVICT_FIRST their copies carry an L2 evict-first policy, so that
+// they do not push the gathered feature and output-gradient rows (read once
+// per edge, many times per pass) out of L2.
+#ifndef CGTP_W_EVICT_FIRST
+#define CGTP_W_EVICT_FIRST 0
+#endif
+__device__ __forceinline__ uint64_t stream_policy() {
+  uint64_t pol = 0;
+  if (CGTP_W_EVICT_FIRST) asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+template <int VEC>
+__device__ __forceinline__ void cp_async_w(float* s, const float* g, uint64_t pol) {
+  if constexpr (CGTP_W_EVICT_FIRST != 0) VecIO<VEC>::cp_async_hint(s, g, pol);
+  else VecIO<VEC>::cp_async(s, g);
+}
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
@@ -152,10 +181,15 @@ constexpr int l3_prefix_rows(int l3) {
 // edge stays below a budget: a loop body much larger than about 20 KB of
 // instructions stops fitting the instruction cache and the warps stall on
 // instruction fetch.  Every run is one launch; the first run of a key
-// initialises that key's block of rows, later runs add to it.
+// initialises that key's block of rows, later runs add to it.  With merge,
+// a run that holds a whole key may go on with the next keys while every one
+// of them fits whole within the budget: the launch then owns the rows of
+// keys key..key_hi (a small block, such as l1 = 0, rides along with the
+// next instead of costing a pass of its own).
 struct ChunkPlan {
   int n;                        // chunks
-  int key[kMaxPaths];           // key value (l1 or l3) of chunk c
+  int key[kMaxPaths];           // key value (l1 or l3) of chunk c (the first, when several)
+  int key_hi[kMaxPaths];        // last key of chunk c
   int first[kMaxPaths];         // chunk c is order[first[c] .. first[c] + count[c])
   int count[kMaxPaths];
   bool first_of_key[kMaxPaths];
@@ -175,7 +209,8 @@ constexpr int path_cost(int p, int kind, int vec, bool gy) {
 // 2 l3 + 1 over the chunk's paths), for kernels that keep one block of
 // accumulators per path.
 template <class PS>
-constexpr ChunkPlan make_chunk_plan(int kind, int vec, bool gy, int budget, int max_rows = 1 << 30) {
+constexpr ChunkPlan make_chunk_plan(int kind, int vec, bool gy, int budget, int max_rows = 1 << 30,
+                                   bool merge = false) {
   ChunkPlan c{};
   int k = 0;
   const int kmax = kind == kByL1 ? PS::LI : PS::LO;
@@ -195,19 +230,39 @@ constexpr ChunkPlan make_chunk_plan(int kind, int vec, bool gy, int budget, int 
       rows += pr;
       ++end;
     }
+    const bool whole = (start == 0 || (kind == kByL1 ? PS::D.l1[c.order[start - 1]] : PS::D.l3[c.order[start - 1]]) != key);
+    int key_hi = key;
+    if (merge && whole) {
+      // append the following keys while each fits whole
+      while (end < k) {
+        const int nk = kind == kByL1 ? PS::D.l1[c.order[end]] : PS::D.l3[c.order[end]];
+        int e2 = end, kc = 0, kr = 0;
+        while (e2 < k && (kind == kByL1 ? PS::D.l1[c.order[e2]] : PS::D.l3[c.order[e2]]) == nk) {
+          kc += path_cost<PS>(c.order[e2], kind, vec, gy);
+          kr += 2 * PS::D.l3[c.order[e2]] + 1;
+          ++e2;
+        }
+        if (cost + kc > budget || rows + kr > max_rows) break;
+        cost += kc;
+        rows += kr;
+        end = e2;
+        key_hi = nk;
+      }
+    }
     c.key[c.n] = key;
+    c.key_hi[c.n] = key_hi;
     c.first[c.n] = start;
     c.count[c.n] = end - start;
-    c.first_of_key[c.n] = c.n == 0 || c.key[c.n - 1] != key;
+    c.first_of_key[c.n] = c.n == 0 || c.key_hi[c.n - 1] != key;
     ++c.n;
     start = end;
   }
   return c;
 }
 
-template <class PS, int KIND, int VEC, bool GY, int BUDGET, int MAX_ROWS = (1 << 30)>
+template <class PS, int KIND, int VEC, bool GY, int BUDGET, int MAX_ROWS = (1 << 30), bool MERGE = false>
 struct Plan {
-  static constexpr ChunkPlan P = make_chunk_plan<PS>(KIND, VEC, GY, BUDGET, MAX_ROWS);
+  static constexpr ChunkPlan P = make_chunk_plan<PS>(KIND, VEC, GY, BUDGET, MAX_ROWS, MERGE);
   static constexpr int N = P.n;
 };
 
@@ -216,17 +271,24 @@ template <class PS, class PL, int CH>
 struct Chunk {
   using Data = typename Grp<PS, kAll, 0>::Data;
   static constexpr int KEY = PL::P.key[CH];
+  static constexpr int KEY_HI = PL::P.key_hi[CH];
   static constexpr bool FIRST = PL::P.first_of_key[CH];
   static constexpr Data make(bool by_l1) {
     Data d{};
     int lo = 99, hi = -1;
-    for (int k = 0; k < PL::P.count[CH]; ++k) {
-      const int p = PL::P.order[PL::P.first[CH] + k];
-      d.path[d.n++] = p;
-      const int other = by_l1 ? PS::D.l3[p] : PS::D.l1[p];
-      lo = other < lo ? other : lo;
-      hi = other > hi ? other : hi;
-    }
+    // the chunk's paths by l2 (stable): the backward keeps one l2 block of its
+    // harmonic-gradient partial live at a time, so all paths of one l2 must be
+    // adjacent, also when the chunk holds several keys (each key's run is
+    // already in l2 order)
+    for (int b = 0; b <= PS::LS; ++b)
+      for (int k = 0; k < PL::P.count[CH]; ++k) {
+        const int p = PL::P.order[PL::P.first[CH] + k];
+        if (PS::D.l2[p] != b) continue;
+        d.path[d.n++] = p;
+        const int other = by_l1 ? PS::D.l3[p] : PS::D.l1[p];
+        lo = other < lo ? other : lo;
+        hi = other > hi ? other : hi;
+      }
     d.lt[0] = 0;
     for (int k = 0; k < d.n; ++k) {
       d.lt[k + 1] = d.lt[k] + (PS::D.tcount[d.path[k]] + 3) / 4 * 4;
@@ -245,7 +307,8 @@ struct ChunkGrp : Chunk<PS, PL, CH> {
   static constexpr int NP = D.n;
   static constexpr int NT = D.lt[D.n] > 0 ? D.lt[D.n] : 4;
   static constexpr int NROW = D.rhi - D.rlo;
-  static constexpr int NOWN = 2 * Base::KEY + 1;
+  // own rows: the blocks of keys KEY..KEY_HI
+  static constexpr int NOWN = (Base::KEY_HI + 1) * (Base::KEY_HI + 1) - Base::KEY * Base::KEY;
   static constexpr int OWN0 = Base::KEY * Base::KEY;
   static constexpr bool PERPATH = false;
   static constexpr int NPK = 0, PL0 = 0;
@@ -273,6 +336,16 @@ inline int pick_batch(int gpw, int t_floats, int stage_floats, int budget_floats
   int bt = budget / (t_floats + 3);
   if (bt > max_bt) bt = max_bt;
   return bt < 1 ? 1 : bt;
+}
+
+// Row split (log2 of the groups of lanes that share one work item): with few
+// items, a warp holds one item instead of 32 / G, its groups taking every
+// Q-th edge of the row, until there are about 8 warps per SM.
+inline int row_split(long long items, int gpw, int num_sms) {
+  int lg_Q = 0;
+  const long long target = 8LL * num_sms;
+  while ((1 << (lg_Q + 1)) <= gpw && items * (1LL << lg_Q) / gpw < target) ++lg_Q;
+  return lg_Q;
 }
 
 // Channel lanes per group (G, a power of two <= 32) and channel slices S for

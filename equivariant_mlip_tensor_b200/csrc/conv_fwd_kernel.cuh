@@ -256,7 +256,7 @@ __device__ __forceinline__ void fwd_edge_dd(const float* __restrict__ T, const f
 // onto that chunk's rows (GR::FIRST false).
 template <class PS, class GR, int KMULT, bool WSH, bool DD>
 __global__ void CGTP_FWD_BOUNDS
-conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
+conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT, int lg_Q) {
   // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x 4
   // channels, so every row offset below folds into an immediate.
   const int mult = KMULT ? KMULT : a.mult;
@@ -287,21 +287,28 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
     grid_dependency_wait();
     return;
   }
+  // Row split: Q = 2^lg_Q groups of lanes share one work item, group `part`
+  // taking the row's edges part, part + Q, ...; their accumulators are summed
+  // by shuffles at the end (more warps for graphs with few rows).
+  const int Q = 1 << lg_Q, part = grp & (Q - 1), ipw = gpw >> lg_Q;  // items per warp
+  const uint64_t wpol = stream_policy();
   const long long n_items = (long long)a.n_nodes * S;
   const long long warps_total = (long long)gridDim.x * (kFwdThreads / 32);
-  for (long long base = ((long long)blockIdx.x * (kFwdThreads / 32) + warp) * gpw; base < n_items;
-       base += warps_total * gpw) {
-    const long long item = base + grp;
+  for (long long base = ((long long)blockIdx.x * (kFwdThreads / 32) + warp) * ipw; base < n_items;
+       base += warps_total * ipw) {
+    const long long item = base + (grp >> lg_Q);
     const bool active = item < n_items;
     const int node = active ? int(item / S) : 0;
     const int slice = active ? int(item % S) : 0;
     const int c0 = (slice * G + gl) * kFwdVec;
-    int e0 = 0, e1 = 0;
+    int e0 = 0, cnt = 0;  // this group's edges: e0 + part + Q t, t < cnt
     if (active) {
       e0 = __ldg(a.row_ptr + node);
-      e1 = __ldg(a.row_ptr + node + 1);
+      const int deg = __ldg(a.row_ptr + node + 1) - e0;
+      cnt = deg > part ? (deg - part + Q - 1) >> lg_Q : 0;
+      e0 += part;
     }
-    const int maxdeg = __reduce_max_sync(0xffffffffu, e1 - e0);
+    const int maxdeg = __reduce_max_sync(0xffffffffu, cnt);
     float acc[GR::NOWN][kFwdVec];
 #pragma unroll
     for (int r = 0; r < GR::NOWN; ++r)
@@ -310,19 +317,19 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
 
     // copies of edge slot k of the current batch into stage s (this lane's channels only)
     auto issue = [&](int b0, int k, int s) {
-      const int e = e0 + b0 + k;
-      if (!(active && e < e1)) return;
+      if (!(active && b0 + k < cnt)) return;
+      const int e = e0 + ((b0 + k) << lg_Q);
       float* dst = St + s * stage_floats + gl * kFwdVec;
       if constexpr (WSH) {
-        VecIO<kFwdVec>::cp_async(dst, a.w + (long long)e * mult + c0);
+        cp_async_w<kFwdVec>(dst, a.w + (long long)e * mult + c0, wpol);
       } else {
         const float* wrow = a.w + (long long)e * PS::NP * mult + c0;
         [[maybe_unused]] const float* w2row = DD ? a.w2 + (long long)e * PS::NP * mult + c0 : nullptr;
         static_for<0, GR::NP>([&](auto Kc) {
           constexpr int K = decltype(Kc)::value;
           constexpr int P = GR::D.path[K];
-          VecIO<kFwdVec>::cp_async(dst + K * rowf, wrow + P * mult);
-          if constexpr (DD) VecIO<kFwdVec>::cp_async(dst + (GR::NP + K) * rowf, w2row + P * mult);
+          cp_async_w<kFwdVec>(dst + K * rowf, wrow + P * mult, wpol);
+          if constexpr (DD) cp_async_w<kFwdVec>(dst + (GR::NP + K) * rowf, w2row + P * mult, wpol);
         });
       }
       if constexpr (kStageX || DD) {
@@ -343,8 +350,8 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
       // sources of every slot, then the first slot's copies, so that they fly
       // while the T matrices of the batch are computed
       for (int k = gl; k < BT; k += G) {
-        const int e = e0 + b0 + k;
-        if (active && e < e1) {
+        if (active && b0 + k < cnt) {
+          const int e = e0 + ((b0 + k) << lg_Q);
           const int j = __ldg(a.col + e);
           if constexpr (!kStageX) {
             constexpr int rlo = GR::D.rlo;
@@ -358,8 +365,8 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
       issue(b0, 0, 0);
       cp_async_commit();
       for (int k = gl; k < BT; k += G) {
-        const int e = e0 + b0 + k;
-        if (active && e < e1) {
+        if (active && b0 + k < cnt) {
+          const int e = e0 + ((b0 + k) << lg_Q);
           float Y[NS];
           if constexpr (DD) {
             // Y and Y' = (dY/dr) gg_r in one evaluation
@@ -386,7 +393,7 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
         if (k + 1 < nb) issue(b0, k + 1, (k + 1) & 1);
         cp_async_commit();
         cp_async_wait<1>();  // this lane's copies of edge k have landed
-        if (active && e0 + b0 + k < e1) {
+        if (active && b0 + k < cnt) {
           constexpr int rlo = GR::D.rlo;
           if constexpr (DD)
             fwd_edge_dd<PS, GR>(Tg + k * NT, Tg + (BT + k) * NT, St + (k & 1) * stage_floats + gl * kFwdVec, rowf,
@@ -398,10 +405,17 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
       }
       __syncwarp();
     }
+    // the row's parts: sum the groups of one item (lanes gl + G part)
+    for (int sh = 1; sh < Q; sh <<= 1) {
+#pragma unroll
+      for (int r = 0; r < GR::NOWN; ++r)
+#pragma unroll
+        for (int c = 0; c < kFwdVec; ++c) acc[r][c] += __shfl_xor_sync(0xffffffffu, acc[r][c], sh * G);
+    }
     if constexpr (GR::PERPATH) {
       // t[node][m3][rank][u] of this l3 block, rank = the path's place among
       // the block's paths
-      if (active) {
+      if (active && part == 0) {
         constexpr int n3 = 2 * GR::KEY + 1;
         static_for<0, GR::NP>([&](auto Kc) {
           constexpr int K = decltype(Kc)::value;
@@ -411,7 +425,7 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT) {
                                acc[K * n3 + m3]);
         });
       }
-    } else if (active) {
+    } else if (active && part == 0) {
       if (!GR::FIRST || a.accumulate) {
         // rows of an l3 block that the preceding launch wrote (wait for it),
         // or the caller's values to add onto
@@ -455,8 +469,9 @@ cudaError_t launch_fwd_group(const ConvFwdArgs& a, int num_sms, bool pdl, cudaSt
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   const long long items = (long long)a.n_nodes * S;
-  const long long groups_per_block = (long long)gpw * (kFwdThreads / 32);
-  long long blocks = (items + groups_per_block - 1) / groups_per_block;
+  const int lg_Q = row_split(items, gpw, num_sms);
+  const long long items_per_block = (long long)(gpw >> lg_Q) * (kFwdThreads / 32);
+  long long blocks = (items + items_per_block - 1) / items_per_block;
   long long cap = 0x7fffffffLL;  // the kernel loops over items beyond the grid
   if (CGTP_FWD_PERSISTENT) {
     int per_sm = 0;
@@ -466,7 +481,7 @@ cudaError_t launch_fwd_group(const ConvFwdArgs& a, int num_sms, bool pdl, cudaSt
   }
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  return launch_kernel(kern, dim3((unsigned)blocks), dim3(kFwdThreads), smem, stream, pdl, a, lg_G, S, BT);
+  return launch_kernel(kern, dim3((unsigned)blocks), dim3(kFwdThreads), smem, stream, pdl, a, lg_G, S, BT, lg_Q);
 }
 
 // Unrolled instructions per edge and lane of all paths in one launch.
@@ -480,9 +495,12 @@ constexpr int fwd_all_cost() {
 template <class PS>
 using FwdPlan = Plan<PS, kByL3, kFwdVec, false, CGTP_FWD_BUDGET>;
 // the fused double-backward forward carries about three times the code per
-// path (three T products): chunks of a third of the budget
+// path (three T products): its own budget (730 measured best of 366 ... 2000)
+#ifndef CGTP_DD_FWD_BUDGET
+#define CGTP_DD_FWD_BUDGET 730
+#endif
 template <class PS>
-using FwdPlanDD = Plan<PS, kByL3, kFwdVec, false, CGTP_FWD_BUDGET / 3>;
+using FwdPlanDD = Plan<PS, kByL3, kFwdVec, false, CGTP_DD_FWD_BUDGET>;
 
 // Output blocks l3 that no path reaches are zero.
 template <class PS>
