@@ -364,7 +364,7 @@ __device__ __forceinline__ void bwd_edge_dd(const float* __restrict__ T, const f
 // of the chunk's paths and a partial grad_Y over them.
 template <class PS, bool NEED_GY, int CH, int KMULT, int VAR>
 __global__ void CGTP_BWD_BOUNDS
-conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt, int lg_Q) {
+conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt, int lg_Q_rt) {
   constexpr int VEC = kBwdVec;
   constexpr bool EXT = (VAR & kVarExt) != 0, PP = (VAR & kVarPerPath) != 0;
   constexpr bool WSH = (VAR & kVarWShared) != 0, DD = (VAR & kVarDD) != 0;
@@ -415,6 +415,8 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt,
   // Row split: Q = 2^lg_Q groups of lanes share one work item (source row),
   // group `part` taking the row's edges part, part + Q, ...; their grad_x
   // accumulators are summed by shuffles at the end.
+  // (a compile-time multiplicity fills the warp with one item: no split)
+  const int lg_Q = KMULT ? 0 : lg_Q_rt;
   const int Q = 1 << lg_Q, part = grp & (Q - 1), ipw = gpw >> lg_Q;  // items per warp
   const uint64_t wpol = stream_policy();
   const long long n_items = (long long)a.n_nodes * S;

@@ -256,7 +256,7 @@ __device__ __forceinline__ void fwd_edge_dd(const float* __restrict__ T, const f
 // onto that chunk's rows (GR::FIRST false).
 template <class PS, class GR, int KMULT, bool WSH, bool DD>
 __global__ void CGTP_FWD_BOUNDS
-conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT, int lg_Q) {
+conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT, int lg_Q_rt) {
   // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x 4
   // channels, so every row offset below folds into an immediate.
   const int mult = KMULT ? KMULT : a.mult;
@@ -290,6 +290,8 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT, int lg_Q) {
   // Row split: Q = 2^lg_Q groups of lanes share one work item, group `part`
   // taking the row's edges part, part + Q, ...; their accumulators are summed
   // by shuffles at the end (more warps for graphs with few rows).
+  // (a compile-time multiplicity fills the warp with one item: no split)
+  const int lg_Q = KMULT ? 0 : lg_Q_rt;
   const int Q = 1 << lg_Q, part = grp & (Q - 1), ipw = gpw >> lg_Q;  // items per warp
   const uint64_t wpol = stream_policy();
   const long long n_items = (long long)a.n_nodes * S;
