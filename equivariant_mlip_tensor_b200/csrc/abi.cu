@@ -653,26 +653,34 @@ cgtp_status cgtp_uvw_forward(cgtp_plan p, int n_nodes, int n_edges, const int* r
   void* gws = (char*)packed + round256(sizeof(float) * L.packed_floats);
   const size_t gws_bytes = workspace_bytes - round256(sizeof(float) * L.t_floats) -
                            round256(sizeof(float) * L.packed_floats);
-  // stage 1: per-path messages t (channelwise convolution, paths kept apart)
+  // Per l3 block, on the block's lane: stage 1, the per-path messages t of the
+  // block's paths (channelwise convolution, paths kept apart); the block's
+  // packed mixing matrices; stage 2, the block's mixing GEMM (tensor cores).
+  // The blocks' lanes overlap, so one block's GEMM runs beside the next
+  // block's messages.  Output blocks that no path reaches are zero.
   ConvFwdArgs a{n_nodes, row_ptr, col, edge_vec, x, w, t, p->mult};
   cudaError_t e = validate_graph(p, n_nodes, n_edges, row_ptr, col, edge_vec, nullptr, nullptr, nullptr, sms, s,
                                  &a.abort_flag);
   if (e != cudaSuccess) return cuda_fail(e);
-  e = cudaErrorNotSupported;
-#define CGTP_UVW_PATHS_ENTRY(A, B, C) \
-  if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_paths<A, B, C>(a, sms, s);
-  CGTP_VARIANT_CONFIGS(CGTP_UVW_PATHS_ENTRY)
-  if (e != cudaSuccess) return cuda_fail(e);
-  // stage 2: per-l3 mixing GEMMs; output blocks no path reaches are zero
-  e = launch_uvw_pack(p->n_paths, p->mult, mult_out, p->lo, L.order, L.count_l3, mix, packed, s);
   for (int l3 = 0; l3 <= p->lo && e == cudaSuccess; ++l3)
     if (L.count_l3[l3] == 0) {
       const int no = (p->lo + 1) * (p->lo + 1);
       e = cudaMemset2DAsync(out + (size_t)l3 * l3 * mult_out, sizeof(float) * no * mult_out, 0,
                             sizeof(float) * (2 * l3 + 1) * mult_out, n_nodes, s);
     }
-  if (e == cudaSuccess) e = launch_uvw_gemm(n_nodes, p->lo, L.count_l3, p->mult, mult_out, t, packed, out, gws,
-                                            gws_bytes, s);
+  auto stage1 = [&](int l3, cudaStream_t st) -> cudaError_t {
+    if (L.count_l3[l3] == 0) return cudaSuccess;
+    cudaError_t r = cudaErrorNotSupported;
+#define CGTP_UVW_PATHS_ENTRY(A, B, C) \
+    if (p->li == A && p->ls == B && p->lo == C) r = launch_conv_paths<A, B, C>(a, sms, st, l3);
+    CGTP_VARIANT_CONFIGS(CGTP_UVW_PATHS_ENTRY)
+    if (r == cudaSuccess)
+      r = launch_uvw_pack_l3(p->n_paths, p->mult, mult_out, p->lo, L.order, L.count_l3, mix, packed, l3, st);
+    return r;
+  };
+  if (e == cudaSuccess)
+    e = launch_uvw_gemm_after(n_nodes, p->lo, L.count_l3, p->mult, mult_out, t, packed, out, gws, gws_bytes, s,
+                              stage1);
   if (e == cudaErrorNotSupported) return CGTP_ERR_UNSUPPORTED;
   return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
 }

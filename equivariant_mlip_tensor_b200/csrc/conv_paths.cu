@@ -67,22 +67,27 @@ void conv_path_order(int* order, int* count_l3) {
 
 // Per-path messages t: a.out is t, whose block for l3 holds
 // [n_nodes][2 l3 + 1][paths of l3][mult] and follows the blocks of smaller l3.
+// only_l3 >= 0: the chunks of that l3 block alone (the fully connected
+// forward runs each block's chunks on its own lane, ahead of its GEMM).
 template <int LI, int LS, int LO>
-cudaError_t launch_conv_paths(const ConvFwdArgs& a, int num_sms, cudaStream_t stream) {
+cudaError_t launch_conv_paths(const ConvFwdArgs& a, int num_sms, cudaStream_t stream, int only_l3) {
   using PS = PathSet<LI, LS, LO>;
   using PL = PathPlan<PS>;
   cudaError_t err = cudaSuccess;
+  bool first = true;
   static_for_host<0, PL::N>([&](auto Cc) {
     constexpr int CH = decltype(Cc)::value;
     using GR = PathRowsGrp<PS, PL, CH>;
+    if (only_l3 >= 0 && GR::KEY != only_l3) return;
     size_t off = 0;  // floats before the l3 = KEY block
     for (int c = 0; c < PL::P.n; ++c)
       if (PL::P.key[c] < GR::KEY) off += (size_t)PL::P.count[c] * (2 * PL::P.key[c] + 1);
     ConvFwdArgs b = a;
     b.out = a.out + off * (size_t)a.n_nodes * a.mult;
     b.accumulate = 0;
-    // chunks write disjoint rows: all but the first may overlap the one before
-    if (err == cudaSuccess) err = launch_fwd_group<PS, GR, false>(b, num_sms, CH > 0, stream);
+    // chunks write disjoint rows: all but the first launched may overlap the one before
+    if (err == cudaSuccess) err = launch_fwd_group<PS, GR, false>(b, num_sms, !first, stream);
+    first = false;
   });
   return err;
 }
@@ -94,7 +99,7 @@ cudaError_t launch_conv_bwd_paths(const ConvBwdArgs& a, int num_sms, cudaStream_
 
 // One translation unit per shape (the build passes CGTP_CFG_LI/LS/LO).
 template cudaError_t launch_conv_paths<CGTP_CFG_LI, CGTP_CFG_LS, CGTP_CFG_LO>(const ConvFwdArgs&, int,
-                                                                           cudaStream_t);
+                                                                           cudaStream_t, int);
 template void conv_path_order<CGTP_CFG_LI, CGTP_CFG_LS, CGTP_CFG_LO>(int*, int*);
 template cudaError_t launch_conv_bwd_paths<CGTP_CFG_LI, CGTP_CFG_LS, CGTP_CFG_LO>(const ConvBwdArgs&, int,
                                                                                 cudaStream_t);

@@ -4,6 +4,7 @@
 
 #include <cuda_runtime.h>
 
+#include <functional>
 #include <mutex>
 
 #include "common.cuh"
@@ -61,7 +62,7 @@ cudaError_t launch_cp_bwd(const CPArgs& a, cudaStream_t stream);
 template <int LI, int LS, int LO>
 cudaError_t launch_conv_fwd(const ConvFwdArgs& a, int num_sms, cudaStream_t stream);
 template <int LI, int LS, int LO>
-cudaError_t launch_conv_paths(const ConvFwdArgs& a, int num_sms, cudaStream_t stream);
+cudaError_t launch_conv_paths(const ConvFwdArgs& a, int num_sms, cudaStream_t stream, int only_l3 = -1);
 template <int LI, int LS, int LO>
 void conv_path_order(int* order, int* count_l3);
 template <int LI, int LS, int LO>
@@ -115,6 +116,15 @@ size_t uvw_gemm_workspace(int n_nodes, int lmax_out, const int* count_l3, int mu
 cudaError_t launch_uvw_gemm(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out,
                             const float* t, const float* packed, float* out, void* ws, size_t ws_bytes,
                             cudaStream_t stream);
+// The same GEMMs with each l3 block's producer work first on the block's
+// lane: before(l3, lane stream) launches what the block's GEMM reads (its
+// per-path messages and packed mixing matrices), so the blocks overlap.
+cudaError_t launch_uvw_gemm_after(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out,
+                                  const float* t, const float* packed, float* out, void* ws, size_t ws_bytes,
+                                  cudaStream_t stream, const std::function<cudaError_t(int, cudaStream_t)>& before);
+// Packing of one l3 block's mixing matrices (l3 < 0: every block).
+cudaError_t launch_uvw_pack_l3(int n_paths, int mult, int mult_out, int lmax_out, const int* order,
+                               const int* count_l3, const float* mix, float* packed, int l3, cudaStream_t stream);
 cudaError_t launch_uvw_pack_t(int n_paths, int mult, int mult_out, int lmax_out, const int* order,
                               const int* count_l3, const float* mix, float* packed_t, cudaStream_t stream);
 size_t uvw_bwd_gemm_workspace(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out);

@@ -217,15 +217,16 @@ Gemm::Arguments block_args(int n_nodes, int l3, int lmax_out, int K, int mult_ou
 
 }  // namespace
 
-cudaError_t launch_uvw_pack(int n_paths, int mult, int mult_out, int lmax_out, const int* order, const int* count_l3,
-                            const float* mix, float* packed, cudaStream_t stream) {
+cudaError_t launch_uvw_pack_l3(int n_paths, int mult, int mult_out, int lmax_out, const int* order,
+                               const int* count_l3, const float* mix, float* packed, int only_l3,
+                               cudaStream_t stream) {
   PathOrder po{};
   for (int k = 0; k < n_paths && k < kMaxPaths; ++k) po.order[k] = order[k];
   int rank0 = 0;
   size_t off = 0;
   for (int l3 = 0; l3 <= lmax_out; ++l3) {
     const int npk = count_l3[l3], n3 = 2 * l3 + 1;
-    if (npk > 0) {
+    if (npk > 0 && (only_l3 < 0 || l3 == only_l3)) {
       uvw_pack_kernel<<<256, 256, 0, stream>>>(po, mult, mult_out, rank0, npk, n3, mix, packed + off);
       const cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return e;
@@ -234,6 +235,11 @@ cudaError_t launch_uvw_pack(int n_paths, int mult, int mult_out, int lmax_out, c
     rank0 += npk;
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_uvw_pack(int n_paths, int mult, int mult_out, int lmax_out, const int* order, const int* count_l3,
+                            const float* mix, float* packed, cudaStream_t stream) {
+  return launch_uvw_pack_l3(n_paths, mult, mult_out, lmax_out, order, count_l3, mix, packed, -1, stream);
 }
 
 size_t uvw_gemm_workspace(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out) {
@@ -251,8 +257,10 @@ size_t uvw_gemm_workspace(int n_nodes, int lmax_out, const int* count_l3, int mu
 #endif
 }
 
-cudaError_t launch_uvw_gemm(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out, const float* t,
-                            const float* packed, float* out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+cudaError_t launch_uvw_gemm_after(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out,
+                                  const float* t, const float* packed, float* out, void* ws, size_t ws_bytes,
+                                  cudaStream_t stream,
+                                  const std::function<cudaError_t(int, cudaStream_t)>& before) {
 #if defined(CGTP_NO_CUTLASS)
   return cudaErrorNotSupported;
 #else
@@ -265,8 +273,9 @@ cudaError_t launch_uvw_gemm(int n_nodes, int lmax_out, const int* count_l3, int 
   size_t t_off = 0, p_off = 0;
   for (int l3 = 0; l3 <= lmax_out && e == cudaSuccess; ++l3) {
     const int npk = count_l3[l3], n3 = 2 * l3 + 1, K = npk * mult;
-    if (npk > 0) {
-      cudaStream_t st = lane(Ls, stream, l3);
+    cudaStream_t st = lane(Ls, stream, l3);
+    if (before) e = before(l3, st);
+    if (npk > 0 && e == cudaSuccess) {
       void* w = (char*)ws + (size_t)(l3 % kLanes) * slice;
       Gemm g;
       auto args = block_args(n_nodes, l3, lmax_out, K, mult_out, t + t_off, packed + p_off, out);
@@ -282,6 +291,12 @@ cudaError_t launch_uvw_gemm(int n_nodes, int lmax_out, const int* count_l3, int 
   if (e != cudaSuccess) return e;
   return ej != cudaSuccess ? ej : cudaGetLastError();
 #endif
+}
+
+cudaError_t launch_uvw_gemm(int n_nodes, int lmax_out, const int* count_l3, int mult, int mult_out, const float* t,
+                            const float* packed, float* out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  return launch_uvw_gemm_after(n_nodes, lmax_out, count_l3, mult, mult_out, t, packed, out, ws, ws_bytes, stream,
+                               nullptr);
 }
 
 cudaError_t launch_uvw_pack_t(int n_paths, int mult, int mult_out, int lmax_out, const int* order,
