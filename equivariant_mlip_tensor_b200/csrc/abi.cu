@@ -494,20 +494,23 @@ cgtp_status cgtp_conv_double_backward(cgtp_plan p, int n_nodes, int n_edges, con
 
   // Every cotangent given: the fused passes.  d grad_out by one forward that
   // reads W and gg_W once; d x, d W and the edge-vector term by one
-  // source-centric pass that reads them once more and writes d W once.
+  // source-centric pass that reads them once more and writes d W once.  The
+  // two passes write disjoint outputs: the forward runs on a side lane,
+  // forked from `s` and joined back, beside the (compute-heavier) source pass.
   if (gg_x != nullptr && gg_w != nullptr && gr) {
-    if (d_grad_out != nullptr) {
-      ConvFwdArgs a{n_nodes, row_ptr, col, edge_vec, x, w, d_grad_out, p->mult};
-      a.abort_flag = abort_flag;
-      a.x2 = gg_x;
-      a.w2 = gg_w;
-      a.gr_dir = gg_edge_vec;
-      e = cudaErrorNotSupported;
-#define CGTP_DDF_ENTRY(A, B, C) \
-      if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_dd_fwd<A, B, C>(a, sms, s);
-      CGTP_CONFIGS(CGTP_DDF_ENTRY)
+    const bool want_fwd = d_grad_out != nullptr;
+    const bool want_bwd = d_x != nullptr || d_w != nullptr || d_edge_vec != nullptr;
+    std::unique_lock<std::mutex> turn(side_lanes_mutex(kLanesDD), std::defer_lock);
+    SideLanes* L = nullptr;
+    cudaStream_t fs = s;
+    if (want_fwd && want_bwd) {
+      turn.lock();
+      e = side_lanes(kLanesDD, &L);
+      if (e == cudaSuccess) e = lanes_fork(L, 1, s);
+      if (e != cudaSuccess) return cuda_fail(e);
+      fs = L->side[0];
     }
-    if (e == cudaSuccess && (d_x != nullptr || d_w != nullptr || d_edge_vec != nullptr)) {
+    if (want_bwd) {
       ConvBwdArgs a{n_nodes, n_edges, csc_ptr, csc_edge, csc_dst, edge_vec, x, w, grad_out,
                     d_x, d_w, d_edge_vec, gsh, p->mult};
       a.abort_flag = abort_flag;
@@ -518,6 +521,21 @@ cgtp_status cgtp_conv_double_backward(cgtp_plan p, int n_nodes, int n_edges, con
 #define CGTP_DDB_ENTRY(A, B, C) \
       if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_dd_bwd<A, B, C>(a, sms, s);
       CGTP_CONFIGS(CGTP_DDB_ENTRY)
+    }
+    if (e == cudaSuccess && want_fwd) {
+      ConvFwdArgs a{n_nodes, row_ptr, col, edge_vec, x, w, d_grad_out, p->mult};
+      a.abort_flag = abort_flag;
+      a.x2 = gg_x;
+      a.w2 = gg_w;
+      a.gr_dir = gg_edge_vec;
+      e = cudaErrorNotSupported;
+#define CGTP_DDF_ENTRY(A, B, C) \
+      if (p->li == A && p->ls == B && p->lo == C) e = launch_conv_dd_fwd<A, B, C>(a, sms, fs);
+      CGTP_CONFIGS(CGTP_DDF_ENTRY)
+    }
+    if (L != nullptr) {  // join even after an error, so the lane is not left forked
+      const cudaError_t ej = lanes_join(L, 1, s);
+      if (e == cudaSuccess) e = ej;
     }
     return e == cudaSuccess ? CGTP_OK : cuda_fail(e);
   }

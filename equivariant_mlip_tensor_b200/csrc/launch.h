@@ -17,7 +17,7 @@ namespace cgtp {
 // (lanes_join: the caller's stream waits for them).  A host thread holds
 // side_lanes_mutex(pool) from the fork to the join (the events are shared).
 constexpr int kMaxSideLanes = 4;
-enum { kLanesBwd = 0, kLanesUvw = 1, kLanePools = 2 };
+enum { kLanesBwd = 0, kLanesUvw = 1, kLanesDD = 2, kLanePools = 3 };
 struct SideLanes {
   cudaStream_t side[kMaxSideLanes];
   cudaEvent_t fork, join[kMaxSideLanes];
