@@ -41,12 +41,10 @@ enum : int { kVarExt = 1, kVarPerPath = 2, kVarWShared = 8, kVarDD = 16 };
 
 namespace {
 
-// Warps per block, persistent grid or one group of lanes per item, and the
-// shared-memory budget per warp (floats) that sizes the edge batch (as in
-// the forward: one-warp blocks let the block scheduler balance the rows).
-#ifndef CGTP_BWD_WARPS
-#define CGTP_BWD_WARPS 1
-#endif
+// Persistent grid or one block per item, and the shared-memory budget per
+// warp (floats) that sizes the edge batch (as in the forward: blocks of one
+// warp, or of the few warps that split one item, let the block scheduler
+// balance the rows).
 #ifndef CGTP_BWD_PERSISTENT
 #define CGTP_BWD_PERSISTENT 0
 #endif
@@ -59,11 +57,18 @@ namespace {
 #ifndef CGTP_BWD_MINB
 #define CGTP_BWD_MINB 0
 #endif
-constexpr int kBwdThreads = 32 * CGTP_BWD_WARPS;
+// (blocks of the compile-time multiplicity keep one warp, and their launch
+// bound says so: with a bound of 128 threads the molecules backward took
+// 0.518 ms instead of 0.504)
+constexpr int kBwdMaxWarps = 4;
+// Warps that split one item (source rows of graphs with few rows): 1, 2 or 4.
+#ifndef CGTP_BWD_MAX_WARPS
+#define CGTP_BWD_MAX_WARPS 4
+#endif
 #if CGTP_BWD_MINB > 0
-#define CGTP_BWD_BOUNDS __launch_bounds__(kBwdThreads, CGTP_BWD_MINB)
+#define CGTP_BWD_BOUNDS(KM) __launch_bounds__((KM) ? 32 : 32 * kBwdMaxWarps, CGTP_BWD_MINB)
 #else
-#define CGTP_BWD_BOUNDS __launch_bounds__(kBwdThreads)
+#define CGTP_BWD_BOUNDS(KM) __launch_bounds__((KM) ? 32 : 32 * kBwdMaxWarps)
 #endif
 // Channels per lane (float4: measured faster than 2 at every shape with
 // one-warp blocks and budgeted chunks).
@@ -363,8 +368,8 @@ __device__ __forceinline__ void bwd_edge_dd(const float* __restrict__ T, const f
 // (written by the block's first chunk, accumulated by the others), grad_W
 // of the chunk's paths and a partial grad_Y over them.
 template <class PS, bool NEED_GY, int CH, int KMULT, int VAR>
-__global__ void CGTP_BWD_BOUNDS
-conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt, int lg_Q_rt) {
+__global__ void CGTP_BWD_BOUNDS(KMULT)
+conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt, int lg_Q_rt, int lg_W_rt) {
   constexpr int VEC = kBwdVec;
   constexpr bool EXT = (VAR & kVarExt) != 0, PP = (VAR & kVarPerPath) != 0;
   constexpr bool WSH = (VAR & kVarWShared) != 0, DD = (VAR & kVarDD) != 0;
@@ -375,6 +380,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt,
   const int lg_G = KMULT ? 5 : lg_G_rt;
   const int S = KMULT ? KMULT / (32 * VEC) : S_rt;
   const int slice_base = KMULT ? CH * S : slice_base_rt;
+  const int lg_W = KMULT ? 0 : lg_W_rt;  // warps of the block that share its items
   using PL = BwdPlan<PS, NEED_GY, VAR & kVarDD>;
   using GR = ChunkGrp<PS, PL, CH, kByL1>;
   constexpr int OWN0 = GR::OWN0;  // first x / grad_x row of the chunk's l1 blocks
@@ -400,7 +406,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt,
   // by the 8 lanes of one 128-bit access phase fall in distinct banks)
   const int rs = G + 4;
   // (two such buffers in the fused double-backward pass: its A and B sums)
-  float* red = smem + (kBwdThreads / 32) * gpw * group_floats +
+  float* red = smem + (gpw << lg_W) * group_floats +
                (warp * gpw + grp) * bwd_red_floats(NS, G) * (DD ? 2 : 1);
   [[maybe_unused]] const int slices_total = S * PL::N;  // the B partials follow the A partials
 
@@ -412,27 +418,31 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt,
     grid_dependency_wait();
     return;
   }
-  // Row split: Q = 2^lg_Q groups of lanes share one work item (source row),
-  // group `part` taking the row's edges part, part + Q, ...; their grad_x
-  // accumulators are summed by shuffles at the end.
-  // (a compile-time multiplicity fills the warp with one item: no split)
+  // Row split: Q = 2^lg_Q groups of lanes of each of the block's 2^lg_W
+  // warps share one work item (source row), part p = warp Q + (group mod Q)
+  // taking the row's edges p, p + Q 2^lg_W, ...; their grad_x accumulators
+  // are summed by shuffles, then across the warps through shared memory.
+  // The block's warps all take the same items.
+  // (a compile-time multiplicity fills the warp with one item: no split
+  // inside the warp)
+  // (nor across warps: one warp per item)
   const int lg_Q = KMULT ? 0 : lg_Q_rt;
-  const int Q = 1 << lg_Q, part = grp & (Q - 1), ipw = gpw >> lg_Q;  // items per warp
+  const int lg_QT = lg_Q + lg_W, nwarps = 1 << lg_W;
+  const int Q = 1 << lg_Q, QT = 1 << lg_QT, part = (warp << lg_Q) | (grp & (Q - 1));
+  const int ipw = gpw >> lg_Q;  // items per block
   const uint64_t wpol = stream_policy();
   const long long n_items = (long long)a.n_nodes * S;
-  const long long warps_total = (long long)gridDim.x * (kBwdThreads / 32);
-  for (long long base = ((long long)blockIdx.x * (kBwdThreads / 32) + warp) * ipw; base < n_items;
-       base += warps_total * ipw) {
+  for (long long base = (long long)blockIdx.x * ipw; base < n_items; base += (long long)gridDim.x * ipw) {
     const long long item = base + (grp >> lg_Q);
     const bool active = item < n_items;
     const long long node = active ? item / S : 0;
     const int slice = active ? int(item % S) : 0;
     const int c0 = (slice * G + gl) * VEC;
-    int k0 = 0, cnt = 0;  // this group's CSC slots: k0 + part + Q t, t < cnt
+    int k0 = 0, cnt = 0;  // this group's CSC slots: k0 + part + QT t, t < cnt
     if (active) {
       k0 = __ldg(a.csc_ptr + node);
       const int deg = __ldg(a.csc_ptr + node + 1) - k0;
-      cnt = deg > part ? (deg - part + Q - 1) >> lg_Q : 0;
+      cnt = deg > part ? (deg - part + QT - 1) >> lg_QT : 0;
       k0 += part;
     }
     const int maxdeg = __reduce_max_sync(0xffffffffu, cnt);
@@ -494,7 +504,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt,
 
     for (int b0 = 0; b0 < maxdeg; b0 += BT) {
       for (int k = gl; k < BT; k += G) {
-        const int kk = k0 + ((b0 + k) << lg_Q);
+        const int kk = k0 + ((b0 + k) << lg_QT);
         if (active && b0 + k < cnt) {
           const int e = __ldg(a.csc_edge + kk);
           float Y[NS];
@@ -587,6 +597,32 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt,
       for (int r = 0; r < NR; ++r)
 #pragma unroll
         for (int c = 0; c < VEC; ++c) gx[r][c] += __shfl_xor_sync(0xffffffffu, gx[r][c], sh * G);
+    }
+    if (lg_W > 0) {
+      // then the warps' sums, in warp order, by warp 0: each warp's part-0
+      // groups leave theirs at the start of their own shared-memory region
+      // (NR rows of G x VEC floats, within the group's region)
+      cp_async_wait<0>();
+      __syncthreads();
+      const bool head = (grp & (Q - 1)) == 0;
+      if (warp > 0 && head) {
+#pragma unroll
+        for (int r = 0; r < NR; ++r) VecIO<VEC>::st(Tg + r * rowf + gl * VEC, gx[r]);
+      }
+      __syncthreads();
+      if (warp == 0 && head) {
+        for (int w = 1; w < nwarps; ++w) {
+          const float* theirs = smem + (w * gpw + grp) * group_floats + gl * VEC;
+#pragma unroll
+          for (int r = 0; r < NR; ++r) {
+            float v[VEC];
+            VecIO<VEC>::lds(v, theirs + r * rowf);
+#pragma unroll
+            for (int c = 0; c < VEC; ++c) gx[r][c] += v[c];
+          }
+        }
+      }
+      __syncthreads();
     }
     if (active && part == 0 && a.grad_x != nullptr) {
       if (!GR::FIRST || (EXT && a.accumulate)) {
@@ -711,37 +747,45 @@ cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t str
   const int BT = pick_batch(gpw, GR::NT * mul, stage_floats, CGTP_BWD_BATCH_FLOATS, CGTP_BWD_MAX_BATCH);
   // the kernel's indexing reaches gpw groups x warps of group_floats, then
   // (with NEED_GY) as many reduction buffers
-  const size_t groups = (size_t)gpw * (kBwdThreads / 32);
-  const size_t smem = sizeof(float) * (groups * bwd_group_floats(BT, GR::NT * mul, stage_floats) +
-                                       (NEED_GY ? groups * bwd_red_floats(PS::NS, G) * mul : 0));
+  const long long items = (long long)a.n_nodes * S;
+  const bool ext = a.sh != nullptr || a.accumulate;
+  // the compile-time multiplicity for the common case (one warp per item);
+  // the per-path layout keeps the run-time one
+  constexpr bool kAllow128 = (VAR & kVarPerPath) == 0;
+  const bool kmult = !ext && kAllow128 && a.mult == 128;
+  int lg_W = 0;
+  const int lg_Q = row_split(items, gpw, num_sms, kmult ? 1 : CGTP_BWD_MAX_WARPS, &lg_W);
+  const int gfl = bwd_group_floats(BT, GR::NT * mul, stage_floats);
+  const int per_group = gfl + (NEED_GY ? bwd_red_floats(PS::NS, G) * mul : 0);
+  // fewer warps per item when the block's shared memory would not fit, or a
+  // group's region could not hold the warps' sums (NOWN rows of G x VEC floats)
+  while (lg_W > 0 && (sizeof(float) * (size_t)per_group * (gpw << lg_W) > smem_limit() || GR::NOWN * G * kBwdVec > gfl))
+    --lg_W;
+  const int threads = 32 << lg_W;
+  const size_t groups = (size_t)gpw << lg_W;
+  const size_t smem = sizeof(float) * (groups * gfl + (NEED_GY ? groups * bwd_red_floats(PS::NS, G) * mul : 0));
   cudaError_t err = check_smem(smem);
   if (err != cudaSuccess) return err;
-  const long long items = (long long)a.n_nodes * S;
-  const int lg_Q = row_split(items, gpw, num_sms);
-  const long long items_per_block = (long long)(gpw >> lg_Q) * (kBwdThreads / 32);
+  const long long items_per_block = (long long)(gpw >> lg_Q);
   const long long blocks = (items + items_per_block - 1) / items_per_block;
-  const bool ext = a.sh != nullptr || a.accumulate;
   if (ext && (VAR & (kVarPerPath | kVarWShared | kVarDD))) return cudaErrorInvalidValue;  // not built
-  // the compile-time multiplicity for the common case; the per-path layout
-  // keeps the run-time one
-  constexpr bool kAllow128 = (VAR & kVarPerPath) == 0;
   constexpr int kExtVar = (VAR & (kVarPerPath | kVarWShared | kVarDD)) ? VAR : (VAR | kVarExt);
   auto kern = ext ? conv_bwd_kernel<PS, NEED_GY, CH, 0, kExtVar>
-              : (kAllow128 && a.mult == 128) ? conv_bwd_kernel<PS, NEED_GY, CH, kAllow128 ? 128 : 0, VAR>
-                                             : conv_bwd_kernel<PS, NEED_GY, CH, 0, VAR>;
+              : kmult ? conv_bwd_kernel<PS, NEED_GY, CH, kAllow128 ? 128 : 0, VAR>
+                      : conv_bwd_kernel<PS, NEED_GY, CH, 0, VAR>;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   long long cap = 0x7fffffffLL;  // the kernel loops over items beyond the grid
   if (CGTP_BWD_PERSISTENT) {
     int per_sm = 0;
-    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBwdThreads, smem);
+    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
     if (err != cudaSuccess) return err;
     cap = (long long)num_sms * (per_sm < 1 ? 1 : per_sm);
   }
   long long nb = blocks > cap ? cap : blocks;
   if (nb < 1) nb = 1;
-  return launch_kernel(kern, dim3((unsigned)nb), dim3(kBwdThreads), smem, stream, CGTP_BWD_PDL && pdl, a, lg_G,
-                       S, BT, CH * S, lg_Q);
+  return launch_kernel(kern, dim3((unsigned)nb), dim3(threads), smem, stream, CGTP_BWD_PDL && pdl, a, lg_G,
+                       S, BT, CH * S, lg_Q, lg_W);
 }
 
 // grad_x blocks that no path reaches (l1 with no path) are zero.

@@ -317,34 +317,78 @@ struct ChunkGrp : Chunk<PS, PL, CH> {
 // Checks a launch's dynamic shared memory against the device's per-block
 // opt-in limit before the attribute is set (a request beyond it is refused
 // here rather than by the launch).
-inline cudaError_t check_smem(size_t smem) {
-  static int limit = -1;  // the same for every B200 in the process
+// Dynamic shared memory a block may opt in to (bytes; the same for every
+// B200 in the process), or 0 when the device cannot be queried.
+inline size_t smem_limit() {
+  static int limit = -1;
   if (limit < 0) {
     int dev = 0, v = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    if (e != cudaSuccess) return e;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return 0;
     limit = v;
   }
-  return smem <= (size_t)limit ? cudaSuccess : cudaErrorInvalidConfiguration;
+  return (size_t)limit;
+}
+inline cudaError_t check_smem(size_t smem) {
+  const size_t limit = smem_limit();
+  if (limit == 0) return cudaErrorInvalidDevice;
+  return smem <= limit ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
+// Blocks of `threads` threads that one SM holds at once with `smem` bytes of
+// dynamic shared memory and `regs` registers per thread (the limits of the
+// device, read once: shared memory per SM and reserved per block, registers
+// per SM in per-warp units of 256, blocks per SM).
+inline int resident_blocks_per_sm(size_t smem, int regs, int threads) {
+  static int sm_smem = -1, reserved = 0, sm_regs = 0, max_blocks = 0;
+  if (sm_smem < 0) {
+    int dev = 0, a = 0, b = 0, c = 0, d = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&a, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&b, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&c, cudaDevAttrMaxRegistersPerMultiprocessor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d, cudaDevAttrMaxBlocksPerMultiprocessor, dev) != cudaSuccess)
+      return 1;
+    reserved = b, sm_regs = c, max_blocks = d;
+    sm_smem = a;
+  }
+  const int warps = (threads + 31) / 32;
+  const int warp_regs = ((regs * 32 + 255) / 256) * 256;
+  int n = max_blocks;
+  if (warp_regs > 0) n = std::min(n, sm_regs / (warps * warp_regs));
+  n = std::min(n, (int)(sm_smem / (smem + reserved)));
+  return n;
 }
 
 // Edges per batch: T matrices of BT edges per group of lanes, sized so that a
 // group's shared memory stays near 24 KB.
-inline int pick_batch(int gpw, int t_floats, int stage_floats, int budget_floats = 6144, int max_bt = 16) {
-  const int budget = budget_floats / gpw - 2 * stage_floats;
+inline int pick_batch_staged(int gpw, int t_floats, int staging_floats, int budget_floats = 6144, int max_bt = 16) {
+  const int budget = budget_floats / gpw - staging_floats;
   int bt = budget / (t_floats + 3);
   if (bt > max_bt) bt = max_bt;
   return bt < 1 ? 1 : bt;
 }
+// the same with two pipeline stages of stage_floats
+inline int pick_batch(int gpw, int t_floats, int stage_floats, int budget_floats = 6144, int max_bt = 16) {
+  return pick_batch_staged(gpw, t_floats, 2 * stage_floats, budget_floats, max_bt);
+}
 
 // Row split (log2 of the groups of lanes that share one work item): with few
 // items, a warp holds one item instead of 32 / G, its groups taking every
-// Q-th edge of the row, until there are about 8 warps per SM.
-inline int row_split(long long items, int gpw, int num_sms) {
+// Q-th edge of the row, until there are about 8 warps per SM.  With
+// max_warps > 1 and still few warps, *lg_W (log2 of the warps of one block,
+// which then all take the same items) doubles while the grid stays within
+// about 4 waves of 8 warps per SM.
+inline int row_split(long long items, int gpw, int num_sms, int max_warps = 1, int* lg_W = nullptr) {
   int lg_Q = 0;
   const long long target = 8LL * num_sms;
   while ((1 << (lg_Q + 1)) <= gpw && items * (1LL << lg_Q) / gpw < target) ++lg_Q;
+  if (lg_W != nullptr) {
+    *lg_W = 0;
+    const long long warps = items * (1LL << lg_Q) / gpw;
+    while ((2 << *lg_W) <= max_warps && warps * (2LL << *lg_W) <= 4 * target) ++*lg_W;
+  }
   return lg_Q;
 }
 

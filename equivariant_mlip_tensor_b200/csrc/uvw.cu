@@ -116,11 +116,44 @@ using Epilogue = typename cutlass::epilogue::collective::CollectiveBuilder<
     cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, TileShape, ClusterShape,
     cutlass::epilogue::collective::EpilogueTileAuto, float, float, float, Layout, kAlign, float, Layout, kAlign,
     cutlass::epilogue::collective::EpilogueScheduleAuto>::CollectiveOp;
-using Mainloop = typename cutlass::gemm::collective::CollectiveBuilder<
-    cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, float, Layout, kAlign, float, Layout, kAlign, float,
-    TileShape, ClusterShape,
-    cutlass::gemm::collective::StageCountAutoCarveout<static_cast<int>(sizeof(typename Epilogue::SharedStorage))>,
-    cutlass::gemm::KernelTmaWarpSpecialized1SmFastFP32Sm100>::CollectiveOp;
+// Product bands of the fp32-accurate mode: each operand is split into three
+// bf16 terms x = x0 + x1 + x2 (|x1| <= 2^-9 |x|, |x2| <= 2^-18 |x|), and band
+// k holds the products x_i y_j with i + j = k.  Bands 0..2 (six products)
+// leave out terms below 2^-26 |x y|, under fp32 rounding; the library's
+// builder computes all five (nine products).  Three bands: molecules forward
+// 0.517 -> 0.510 ms.
+#ifndef CGTP_UVW_BANDS
+#define CGTP_UVW_BANDS 3
+#endif
+template <int NB, class CM>
+struct WithBands {
+  using type = CM;
+};
+template <int NB, int L2T, int T2M, int SP, int AP, int NB0, int SF, int PI, class Cl, class Cp, class Ar,
+          class... Rest>
+struct WithBands<NB, cutlass::gemm::collective::CollectiveMma<
+                         cutlass::gemm::MainloopSm100TmaUmmaWarpSpecializedFastF32<L2T, T2M, SP, AP, NB0, SF, PI, Cl,
+                                                                                   Cp, Ar>,
+                         Rest...>> {
+  using type = cutlass::gemm::collective::CollectiveMma<
+      cutlass::gemm::MainloopSm100TmaUmmaWarpSpecializedFastF32<L2T, T2M, SP, AP, NB, SF, PI, Cl, Cp, Ar>, Rest...>;
+};
+using Mainloop = typename WithBands<
+    CGTP_UVW_BANDS,
+    typename cutlass::gemm::collective::CollectiveBuilder<
+        cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, float, Layout, kAlign, float, Layout, kAlign, float,
+        TileShape, ClusterShape,
+        cutlass::gemm::collective::StageCountAutoCarveout<static_cast<int>(sizeof(typename Epilogue::SharedStorage))>,
+        cutlass::gemm::KernelTmaWarpSpecialized1SmFastFP32Sm100>::CollectiveOp>::type;
+static_assert(CGTP_UVW_BANDS == 5 || !std::is_same_v<Mainloop,
+                                                      typename cutlass::gemm::collective::CollectiveBuilder<
+                                                          cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, float,
+                                                          Layout, kAlign, float, Layout, kAlign, float, TileShape,
+                                                          ClusterShape,
+                                                          cutlass::gemm::collective::StageCountAutoCarveout<
+                                                              static_cast<int>(sizeof(typename Epilogue::SharedStorage))>,
+                                                          cutlass::gemm::KernelTmaWarpSpecialized1SmFastFP32Sm100>::CollectiveOp>,
+              "the band count did not reach the mainloop");
 using Kernel = cutlass::gemm::kernel::GemmUniversal<Shape<int, int, int, int>, Mainloop, Epilogue>;
 using Gemm = cutlass::gemm::device::GemmUniversalAdapter<Kernel>;
 
@@ -134,11 +167,13 @@ using EpilogueT = typename cutlass::epilogue::collective::CollectiveBuilder<
     cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, TileShapeT, ClusterShape,
     cutlass::epilogue::collective::EpilogueTileAuto, float, float, float, Layout, kAlign, float, Layout, kAlign,
     cutlass::epilogue::collective::EpilogueScheduleAuto>::CollectiveOp;
-using MainloopT = typename cutlass::gemm::collective::CollectiveBuilder<
-    cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, float, LayoutCol, kAlign, float, Layout, kAlign, float,
-    TileShapeT, ClusterShape,
-    cutlass::gemm::collective::StageCountAutoCarveout<static_cast<int>(sizeof(typename EpilogueT::SharedStorage))>,
-    cutlass::gemm::KernelTmaWarpSpecialized1SmFastFP32Sm100>::CollectiveOp;
+using MainloopT = typename WithBands<
+    CGTP_UVW_BANDS,
+    typename cutlass::gemm::collective::CollectiveBuilder<
+        cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, float, LayoutCol, kAlign, float, Layout, kAlign, float,
+        TileShapeT, ClusterShape,
+        cutlass::gemm::collective::StageCountAutoCarveout<static_cast<int>(sizeof(typename EpilogueT::SharedStorage))>,
+        cutlass::gemm::KernelTmaWarpSpecialized1SmFastFP32Sm100>::CollectiveOp>::type;
 using KernelT = cutlass::gemm::kernel::GemmUniversal<Shape<int, int, int, int>, MainloopT, EpilogueT>;
 using GemmT = cutlass::gemm::device::GemmUniversalAdapter<KernelT>;
 
