@@ -66,9 +66,9 @@ constexpr int kBwdMaxWarps = 4;
 #define CGTP_BWD_MAX_WARPS 4
 #endif
 #if CGTP_BWD_MINB > 0
-#define CGTP_BWD_BOUNDS(KM) __launch_bounds__((KM) ? 32 : 32 * kBwdMaxWarps, CGTP_BWD_MINB)
+#define CGTP_BWD_BOUNDS(KM) __launch_bounds__(kmult_whole_warp(KM, kBwdVec) ? 32 : 32 * kBwdMaxWarps, CGTP_BWD_MINB)
 #else
-#define CGTP_BWD_BOUNDS(KM) __launch_bounds__((KM) ? 32 : 32 * kBwdMaxWarps)
+#define CGTP_BWD_BOUNDS(KM) __launch_bounds__(kmult_whole_warp(KM, kBwdVec) ? 32 : 32 * kBwdMaxWarps)
 #endif
 // Channels per lane (float4: measured faster than 2 at every shape with
 // one-warp blocks and budgeted chunks).
@@ -374,13 +374,15 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt,
   constexpr bool EXT = (VAR & kVarExt) != 0, PP = (VAR & kVarPerPath) != 0;
   constexpr bool WSH = (VAR & kVarWShared) != 0, DD = (VAR & kVarDD) != 0;
   static_assert(!DD || (VAR == kVarDD), "the fused double-backward pass is a variant of its own");
-  // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x VEC
-  // channels, so every row offset below folds into an immediate.
+  // KMULT > 0: the multiplicity is a compile-time constant (128: one item of
+  // 32 lanes x VEC channels per warp; 64: two items of 16 lanes, whose rows
+  // may still be split), so every row offset below folds into an immediate.
   const int mult = KMULT ? KMULT : a.mult;
-  const int lg_G = KMULT ? 5 : lg_G_rt;
-  const int S = KMULT ? KMULT / (32 * VEC) : S_rt;
+  constexpr bool WHOLE = kmult_whole_warp(KMULT, VEC);  // one item fills the warp
+  const int lg_G = KMULT ? kmult_lg_G(KMULT, VEC) : lg_G_rt;
+  const int S = KMULT ? kmult_S(KMULT, VEC) : S_rt;
   const int slice_base = KMULT ? CH * S : slice_base_rt;
-  const int lg_W = KMULT ? 0 : lg_W_rt;  // warps of the block that share its items
+  const int lg_W = WHOLE ? 0 : lg_W_rt;  // warps of the block that share its items
   using PL = BwdPlan<PS, NEED_GY, VAR & kVarDD>;
   using GR = ChunkGrp<PS, PL, CH, kByL1>;
   constexpr int OWN0 = GR::OWN0;  // first x / grad_x row of the chunk's l1 blocks
@@ -426,7 +428,7 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt,
   // (a compile-time multiplicity fills the warp with one item: no split
   // inside the warp)
   // (nor across warps: one warp per item)
-  const int lg_Q = KMULT ? 0 : lg_Q_rt;
+  const int lg_Q = WHOLE ? 0 : lg_Q_rt;
   const int lg_QT = lg_Q + lg_W, nwarps = 1 << lg_W;
   const int Q = 1 << lg_Q, QT = 1 << lg_QT, part = (warp << lg_Q) | (grp & (Q - 1));
   const int ipw = gpw >> lg_Q;  // items per block
@@ -751,8 +753,11 @@ cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t str
   const bool ext = a.sh != nullptr || a.accumulate;
   // the compile-time multiplicity for the common case (one warp per item);
   // the per-path layout keeps the run-time one
+  // (and 64 for the plain backward)
   constexpr bool kAllow128 = (VAR & kVarPerPath) == 0;
+  constexpr bool kAllow64 = CGTP_KMULT64 && (VAR & (kVarPerPath | kVarWShared | kVarDD)) == 0;
   const bool kmult = !ext && kAllow128 && a.mult == 128;
+  const bool kmult64 = !ext && kAllow64 && a.mult == 64;
   int lg_W = 0;
   const int lg_Q = row_split(items, gpw, num_sms, kmult ? 1 : CGTP_BWD_MAX_WARPS, &lg_W);
   const int gfl = bwd_group_floats(BT, GR::NT * mul, stage_floats);
@@ -771,8 +776,9 @@ cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t str
   if (ext && (VAR & (kVarPerPath | kVarWShared | kVarDD))) return cudaErrorInvalidValue;  // not built
   constexpr int kExtVar = (VAR & (kVarPerPath | kVarWShared | kVarDD)) ? VAR : (VAR | kVarExt);
   auto kern = ext ? conv_bwd_kernel<PS, NEED_GY, CH, 0, kExtVar>
-              : kmult ? conv_bwd_kernel<PS, NEED_GY, CH, kAllow128 ? 128 : 0, VAR>
-                      : conv_bwd_kernel<PS, NEED_GY, CH, 0, VAR>;
+              : kmult   ? conv_bwd_kernel<PS, NEED_GY, CH, kAllow128 ? 128 : 0, VAR>
+              : kmult64 ? conv_bwd_kernel<PS, NEED_GY, CH, kAllow64 ? 64 : 0, VAR>
+                        : conv_bwd_kernel<PS, NEED_GY, CH, 0, VAR>;
   err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   long long cap = 0x7fffffffLL;  // the kernel loops over items beyond the grid

@@ -392,6 +392,23 @@ inline int row_split(long long items, int gpw, int num_sms, int max_warps = 1, i
   return lg_Q;
 }
 
+// log2 of the channel lanes per group and the channel slices of a
+// compile-time multiplicity km at vec channels per lane (as lane_geometry).
+constexpr int kmult_lg_G(int km, int vec) {
+  int g = 1, lg = 0;
+  while (g < 32 && (km / vec) % (2 * g) == 0) g *= 2, ++lg;
+  return lg;
+}
+constexpr int kmult_S(int km, int vec) { return km / vec / (1 << kmult_lg_G(km, vec)); }
+// Plain forward and backward kernels also specialised for multiplicity 64 (1)
+// or only 128 (0).
+#ifndef CGTP_KMULT64
+#define CGTP_KMULT64 1
+#endif
+// A compile-time multiplicity of at least 32 lanes x vec channels fills the
+// warp with one item: no split of its rows inside or across warps.
+constexpr bool kmult_whole_warp(int km, int vec) { return km >= 32 * vec; }
+
 // Channel lanes per group (G, a power of two <= 32) and channel slices S for
 // mult channels at VEC channels per lane.
 inline void lane_geometry(int mult, int vec, int& G, int& lg_G, int& S) {

@@ -62,9 +62,9 @@ namespace {
 #endif
 constexpr int kFwdMaxWarps = 4;
 #if CGTP_FWD_MINB > 0
-#define CGTP_FWD_BOUNDS(KM) __launch_bounds__((KM) ? 32 : 32 * kFwdMaxWarps, CGTP_FWD_MINB)
+#define CGTP_FWD_BOUNDS(KM) __launch_bounds__(kmult_whole_warp(KM, kFwdVec) ? 32 : 32 * kFwdMaxWarps, CGTP_FWD_MINB)
 #else
-#define CGTP_FWD_BOUNDS(KM) __launch_bounds__((KM) ? 32 : 32 * kFwdMaxWarps)
+#define CGTP_FWD_BOUNDS(KM) __launch_bounds__(kmult_whole_warp(KM, kFwdVec) ? 32 : 32 * kFwdMaxWarps)
 #endif
 #ifndef CGTP_FWD_VEC
 #define CGTP_FWD_VEC 4
@@ -304,12 +304,14 @@ __device__ __forceinline__ void fwd_edge_dd(const float* __restrict__ T, const f
 template <class PS, class GR, int KMULT, bool WSH, bool DD>
 __global__ void CGTP_FWD_BOUNDS(KMULT)
 conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT, int lg_Q_rt, int lg_W_rt) {
-  // KMULT > 0: the multiplicity is a compile-time multiple of 32 lanes x 4
-  // channels, so every row offset below folds into an immediate.
+  // KMULT > 0: the multiplicity is a compile-time constant (128: one item of
+  // 32 lanes x 4 channels per warp; 64: two items of 16 lanes, whose rows
+  // may still be split), so every row offset below folds into an immediate.
   const int mult = KMULT ? KMULT : a.mult;
-  const int lg_G = KMULT ? 5 : lg_G_rt;
-  const int S = KMULT ? KMULT / (32 * kFwdVec) : S_rt;
-  const int lg_W = KMULT ? 0 : lg_W_rt;  // warps of the block that share its items
+  constexpr bool WHOLE = kmult_whole_warp(KMULT, kFwdVec);  // one item fills the warp
+  const int lg_G = KMULT ? kmult_lg_G(KMULT, kFwdVec) : lg_G_rt;
+  const int S = KMULT ? kmult_S(KMULT, kFwdVec) : S_rt;
+  const int lg_W = WHOLE ? 0 : lg_W_rt;  // warps of the block that share its items
   constexpr int NI = PS::NI, NO = PS::NO, NS = PS::NS, NT = GR::NT;
   constexpr int NW = (WSH ? 1 : GR::NP) * (DD ? 2 : 1);  // staged weight rows (W, then gg_W)
   constexpr int NXR = GR::NROW * (DD ? 2 : 1);            // staged feature rows (x, then gg_x)
@@ -349,7 +351,7 @@ conv_fwd_kernel(ConvFwdArgs a, int lg_G_rt, int S_rt, int BT, int lg_Q_rt, int l
   // (a compile-time multiplicity fills the warp with one item: no split
   // inside the warp)
   // (nor across warps: one warp per item)
-  const int lg_Q = KMULT ? 0 : lg_Q_rt;
+  const int lg_Q = WHOLE ? 0 : lg_Q_rt;
   const int lg_QT = lg_Q + lg_W, nwarps = 1 << lg_W;
   const int Q = 1 << lg_Q, QT = 1 << lg_QT, part = (warp << lg_Q) | (grp & (Q - 1));
   const int ipw = gpw >> lg_Q;  // items per block
@@ -581,7 +583,12 @@ cudaError_t launch_fwd_group(const ConvFwdArgs& a, int num_sms, bool pdl, cudaSt
   const int gpw = 32 / G;
   const int mul = DD ? 2 : 1;  // the fused double-backward pass stages and builds everything twice
   const int w_floats = fwd_w_floats((WSH ? 1 : GR::NP) * mul, G), x_floats = fwd_x_floats(GR::NROW * mul, G);
-  auto kern = a.mult == 128 ? conv_fwd_kernel<PS, GR, 128, WSH, DD> : conv_fwd_kernel<PS, GR, 0, WSH, DD>;
+  // compile-time multiplicities: 128 for every launch, 64 for the plain
+  // forward (the others keep the run-time one there)
+  constexpr bool kAllow64 = CGTP_KMULT64 && !WSH && !DD && !GR::PERPATH;
+  auto kern = a.mult == 128               ? conv_fwd_kernel<PS, GR, 128, WSH, DD>
+              : (kAllow64 && a.mult == 64) ? conv_fwd_kernel<PS, GR, kAllow64 ? 64 : 0, WSH, DD>
+                                           : conv_fwd_kernel<PS, GR, 0, WSH, DD>;
   const long long items = (long long)a.n_nodes * S;
   constexpr bool RING = fwd_ring<GR>();
   int BT = pick_batch_staged(gpw, GR::NT * mul, fwd_staging_floats(w_floats, x_floats, RING), CGTP_FWD_BATCH_FLOATS,
@@ -604,7 +611,8 @@ cudaError_t launch_fwd_group(const ConvFwdArgs& a, int num_sms, bool pdl, cudaSt
     // A grid that one wave would hold with smaller edge batches (few rows,
     // e.g. one periodic cell) gets the largest batch that makes it fit: the
     // T matrices are most of a group's shared memory.
-    static int regs = -1;  // per instantiation
+    static int regs_of[3] = {-1, -1, -1};  // per kernel of this instantiation (multiplicity 128, 64, run time)
+    int& regs = regs_of[a.mult == 128 ? 0 : (kAllow64 && a.mult == 64) ? 1 : 2];
     if (regs < 0) {
       cudaFuncAttributes fa;
       if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return cudaGetLastError();
