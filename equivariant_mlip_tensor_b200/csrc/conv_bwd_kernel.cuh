@@ -76,6 +76,12 @@ constexpr int kBwdMaxWarps = 4;
 #define CGTP_BWD_VEC 4
 #endif
 constexpr int kBwdVec = CGTP_BWD_VEC;
+// The per-path-layout variant (fully connected convolution) with the
+// compile-time multiplicity 128 too (1: its backward at molecules 1.97 ->
+// 1.76 ms, bit-identical), or only the run-time one (0).
+#ifndef CGTP_PP_KMULT
+#define CGTP_PP_KMULT 1
+#endif
 // Programmatic dependent launch between the chunks of one backward call
 // (1) or plain stream order (0).
 #ifndef CGTP_BWD_PDL
@@ -751,10 +757,9 @@ cudaError_t launch_bwd_chunk(const ConvBwdArgs& a, int num_sms, cudaStream_t str
   // (with NEED_GY) as many reduction buffers
   const long long items = (long long)a.n_nodes * S;
   const bool ext = a.sh != nullptr || a.accumulate;
-  // the compile-time multiplicity for the common case (one warp per item);
-  // the per-path layout keeps the run-time one
-  // (and 64 for the plain backward)
-  constexpr bool kAllow128 = (VAR & kVarPerPath) == 0;
+  // the compile-time multiplicity for the common case (one warp per item),
+  // and 64 for the plain backward
+  constexpr bool kAllow128 = CGTP_PP_KMULT || (VAR & kVarPerPath) == 0;
   constexpr bool kAllow64 = CGTP_KMULT64 && (VAR & (kVarPerPath | kVarWShared | kVarDD)) == 0;
   const bool kmult = !ext && kAllow128 && a.mult == 128;
   const bool kmult64 = !ext && kAllow64 && a.mult == 64;

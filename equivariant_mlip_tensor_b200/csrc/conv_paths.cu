@@ -25,7 +25,10 @@ namespace {
 // Per-path rows: chunks of same-l3 paths that keep one block of 2 l3 + 1
 // output rows per path, at most kPathRowsMax rows per chunk (the
 // accumulators stay in registers).
-constexpr int kPathRowsMax = 16;
+#ifndef CGTP_PATH_ROWS
+#define CGTP_PATH_ROWS 16
+#endif
+constexpr int kPathRowsMax = CGTP_PATH_ROWS;
 template <class PS>
 using PathPlan = Plan<PS, kByL3, kFwdVec, false, CGTP_FWD_BUDGET, kPathRowsMax>;
 
