@@ -60,7 +60,15 @@ namespace {
 #ifndef CGTP_FWD_MINB
 #define CGTP_FWD_MINB 1
 #endif
-constexpr int kFwdMaxWarps = 4;
+// Warps that split one item (rows of the forward's graphs with few rows): 1,
+// 2 or 4.  More than one measured slower for the forward at the 1 000-atom
+// periodic cell (four-warp blocks of its large per-warp staging leave fewer
+// warps per SM), so the default keeps one.
+#ifndef CGTP_FWD_MAX_WARPS
+#define CGTP_FWD_MAX_WARPS 1
+#endif
+// (the kernels' launch bound follows it: 32 threads by default)
+constexpr int kFwdMaxWarps = CGTP_FWD_MAX_WARPS;
 #if CGTP_FWD_MINB > 0
 #define CGTP_FWD_BOUNDS(KM) __launch_bounds__(kmult_whole_warp(KM, kFwdVec) ? 32 : 32 * kFwdMaxWarps, CGTP_FWD_MINB)
 #else
@@ -101,13 +109,7 @@ template <class GR>
 constexpr bool fwd_ring() {
   return kFwdRing && !GR::PERPATH;
 }
-// Warps that split one item (rows of the forward's graphs with few rows): 1,
-// 2 or 4.  More than one measured slower for the forward at the 1 000-atom
-// periodic cell (four-warp blocks of its large per-warp staging leave fewer
-// warps per SM), so the default keeps one.
-#ifndef CGTP_FWD_MAX_WARPS
-#define CGTP_FWD_MAX_WARPS 1
-#endif
+
 
 // One launch over all paths while their unrolled code per edge and lane stays
 // within CGTP_FWD_SINGLE_MAX instructions; otherwise one launch per chunk of
@@ -594,7 +596,7 @@ cudaError_t launch_fwd_group(const ConvFwdArgs& a, int num_sms, bool pdl, cudaSt
   int BT = pick_batch_staged(gpw, GR::NT * mul, fwd_staging_floats(w_floats, x_floats, RING), CGTP_FWD_BATCH_FLOATS,
                              CGTP_FWD_MAX_BATCH);
   int lg_W = 0;
-  const int lg_Q = row_split(items, gpw, num_sms, a.mult == 128 ? 1 : CGTP_FWD_MAX_WARPS, &lg_W);
+  const int lg_Q = row_split(items, gpw, num_sms, a.mult == 128 ? 1 : kFwdMaxWarps, &lg_W);
   // fewer warps per item when the block's shared memory would not fit, or a
   // group's region could not hold the warps' sums (NOWN rows of G x 4 floats)
   const int gfl = fwd_group_floats(BT, GR::NT * mul, w_floats, x_floats, RING);
