@@ -82,6 +82,17 @@ constexpr int kBwdVec = CGTP_BWD_VEC;
 #ifndef CGTP_PP_KMULT
 #define CGTP_PP_KMULT 1
 #endif
+// The harmonic Jacobian epilogue launched with programmatic dependent launch
+// (1) or in plain stream order (0), and the largest l1 block's chain of
+// chunks on the caller's stream, the others on side lanes (1), or the
+// smallest block's (0).  Together: molecules backward 0.509 -> 0.503 ms
+// (0.355 -> 0.351 ms without the Jacobian), bit-identical.
+#ifndef CGTP_SH_PDL
+#define CGTP_SH_PDL 1
+#endif
+#ifndef CGTP_BWD_LONG_MAIN
+#define CGTP_BWD_LONG_MAIN 1
+#endif
 // Programmatic dependent launch between the chunks of one backward call
 // (1) or plain stream order (0).
 #ifndef CGTP_BWD_PDL
@@ -657,13 +668,18 @@ conv_bwd_kernel(ConvBwdArgs a, int lg_G_rt, int S_rt, int BT, int slice_base_rt,
   grid_dependency_wait();
 }
 
-// grad_edge_vec[e] (= or +=) (dY_e/dr_e)^T sum_s grad_sh[s][e]
+// grad_edge_vec[e] (= or +=) (dY_e/dr_e)^T sum_s grad_sh[s][e].  Launched
+// with programmatic dependent launch after the chunks: the Jacobian needs only
+// the edge vectors, so it is evaluated before waiting for the chunks' partials.
 template <int LS>
 __global__ void sh_backward_kernel(int n_edges, int S, const float* __restrict__ edge_vec,
                                    const float* __restrict__ grad_sh, float* __restrict__ grad_edge_vec, int add) {
   constexpr int NS = (LS + 1) * (LS + 1);
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n_edges;
        e += (long long)gridDim.x * blockDim.x) {
+    Dual3 Y[NS];
+    sh_grad_of_vec<LS>(edge_vec[3 * e], edge_vec[3 * e + 1], edge_vec[3 * e + 2], Y);
+    grid_dependency_wait();  // the partials (and the caller's grad_edge_vec) from here on
     float g[NS];
 #pragma unroll
     for (int b = 0; b < NS; ++b) g[b] = 0.f;
@@ -672,8 +688,6 @@ __global__ void sh_backward_kernel(int n_edges, int S, const float* __restrict__
 #pragma unroll
       for (int b = 0; b < NS; ++b) g[b] += src[b];
     }
-    Dual3 Y[NS];
-    sh_grad_of_vec<LS>(edge_vec[3 * e], edge_vec[3 * e + 1], edge_vec[3 * e + 2], Y);
     float d0 = 0.f, d1 = 0.f, d2 = 0.f;
 #pragma unroll
     for (int b = 0; b < NS; ++b) {
@@ -690,6 +704,7 @@ __global__ void sh_backward_kernel(int n_edges, int S, const float* __restrict__
     grad_edge_vec[3 * e + 1] = d1;
     grad_edge_vec[3 * e + 2] = d2;
   }
+  grid_dependency_wait();  // complete only after the chunks (threads without an edge too)
 }
 
 // grad_edge_vec[e] (= or +=) sum_b G_b (d2Y_b/dr2) q_e with G = sum_s grad_sh[s][e]:
@@ -848,7 +863,10 @@ cudaError_t launch_bwd_chunks(const ConvBwdArgs& a, int num_sms, cudaStream_t st
     if (err == cudaSuccess) err = lanes_fork(L, NKEYS - 1, stream);
     static_for_host<0, NCH>([&](auto Cc) {
       constexpr int CH = decltype(Cc)::value;
-      constexpr int lane = PL::P.key[CH] - PL::P.key[0];  // the key's lane; lane 0 is the caller's stream
+      // the key's lane; lane 0 is the caller's stream (with CGTP_BWD_LONG_MAIN
+      // the last key, the largest l1 block, takes it: the epilogue then follows
+      // the longest chain in stream order)
+      constexpr int lane = CGTP_BWD_LONG_MAIN ? PL::P.key[NCH - 1] - PL::P.key[CH] : PL::P.key[CH] - PL::P.key[0];
       if (err == cudaSuccess)
         err = launch_bwd_chunk<PS, NEED_GY, CH, VAR>(a, num_sms, lane == 0 ? stream : L->side[lane - 1],
                                                      !PL::P.first_of_key[CH]);
@@ -873,8 +891,9 @@ cudaError_t launch_sh_backward(const ConvBwdArgs& a, int slices, int num_sms, cu
     sh_backward_hess_kernel<LS><<<(unsigned)nbk, threads, 0, stream>>>(a.n_edges, slices, a.edge_vec, a.grad_sh,
                                                                       a.gr_dir, a.grad_edge_vec, a.gr_mode == 2);
   } else {
-    sh_backward_kernel<LS><<<(unsigned)nbk, threads, 0, stream>>>(a.n_edges, slices, a.edge_vec, a.grad_sh,
-                                                                 a.grad_edge_vec, a.gr_mode == 1);
+    return launch_kernel(sh_backward_kernel<LS>, dim3((unsigned)nbk), dim3(threads), 0, stream, CGTP_SH_PDL != 0,
+                         (int)a.n_edges, slices, a.edge_vec, (const float*)a.grad_sh, a.grad_edge_vec,
+                         (int)(a.gr_mode == 1));
   }
   return cudaGetLastError();
 }
