@@ -193,6 +193,7 @@ struct ChunkPlan {
   int first[kMaxPaths];         // chunk c is order[first[c] .. first[c] + count[c])
   int count[kMaxPaths];
   bool first_of_key[kMaxPaths];
+  int chain[kMaxPaths];         // chunks that continue a key's rows follow their predecessor: one chain each
   int order[kMaxPaths];         // paths sorted by (key, l2, lexicographic)
 };
 
@@ -210,7 +211,7 @@ constexpr int path_cost(int p, int kind, int vec, bool gy) {
 // accumulators per path.
 template <class PS>
 constexpr ChunkPlan make_chunk_plan(int kind, int vec, bool gy, int budget, int max_rows = 1 << 30,
-                                   bool merge = false) {
+                                   bool merge = false, bool merge_tail = false) {
   ChunkPlan c{};
   int k = 0;
   const int kmax = kind == kByL1 ? PS::LI : PS::LO;
@@ -242,7 +243,34 @@ constexpr ChunkPlan make_chunk_plan(int kind, int vec, bool gy, int budget, int 
           kr += 2 * PS::D.l3[c.order[e2]] + 1;
           ++e2;
         }
-        if (cost + kc > budget || rows + kr > max_rows) break;
+        if (cost + kc > budget || rows + kr > max_rows) {
+          // merge_tail: the paths that would form the next key's last (small)
+          // chunk, when they fit, start that key's rows here instead, and its
+          // other chunks continue them
+          if (merge_tail) {
+            int ls = end, lc = 0, lr = 0;  // greedy chunks of key nk alone: the last one is [ls, e2)
+            for (int q = end; q < e2; ++q) {
+              const int pc = path_cost<PS>(c.order[q], kind, vec, gy);
+              const int pr = 2 * PS::D.l3[c.order[q]] + 1;
+              if (q > ls && (lc + pc > budget || lr + pr > max_rows)) ls = q, lc = 0, lr = 0;
+              lc += pc;
+              lr += pr;
+            }
+            if (ls > end && cost + lc <= budget && rows + lr <= max_rows) {
+              // move order[ls, e2) to order[end, ...): one contiguous chunk
+              for (int q = ls; q < e2; ++q) {
+                const int p = c.order[q];
+                for (int r = q; r > end + (q - ls); --r) c.order[r] = c.order[r - 1];
+                c.order[end + (q - ls)] = p;
+              }
+              end += e2 - ls;
+              cost += lc;
+              rows += lr;
+              key_hi = nk;
+            }
+          }
+          break;
+        }
         cost += kc;
         rows += kr;
         end = e2;
@@ -254,16 +282,19 @@ constexpr ChunkPlan make_chunk_plan(int kind, int vec, bool gy, int budget, int 
     c.first[c.n] = start;
     c.count[c.n] = end - start;
     c.first_of_key[c.n] = c.n == 0 || c.key_hi[c.n - 1] != key;
+    c.chain[c.n] = c.n == 0 ? 0 : c.chain[c.n - 1] + (c.first_of_key[c.n] ? 1 : 0);
     ++c.n;
     start = end;
   }
   return c;
 }
 
-template <class PS, int KIND, int VEC, bool GY, int BUDGET, int MAX_ROWS = (1 << 30), bool MERGE = false>
+template <class PS, int KIND, int VEC, bool GY, int BUDGET, int MAX_ROWS = (1 << 30), bool MERGE = false,
+          bool MERGE_TAIL = false>
 struct Plan {
-  static constexpr ChunkPlan P = make_chunk_plan<PS>(KIND, VEC, GY, BUDGET, MAX_ROWS, MERGE);
+  static constexpr ChunkPlan P = make_chunk_plan<PS>(KIND, VEC, GY, BUDGET, MAX_ROWS, MERGE, MERGE_TAIL);
   static constexpr int N = P.n;
+  static constexpr int CHAINS = P.n ? P.chain[P.n - 1] + 1 : 0;
 };
 
 // The paths of chunk CH of plan PL, with the same interface as Grp.
