@@ -5,9 +5,10 @@
 // reply to reviewer cmnz: the fully connected CG tensor product).  The GEMM
 // runs on the 5th-generation tensor cores through CUTLASS's sm100 collective
 // (TMA-staged operands, tcgen05 MMA into tensor memory) in its fp32-accurate
-// mode: each fp32 operand is split into three bf16 terms and the nine
-// products are accumulated in fp32, which keeps the result within fp32
-// rounding of the exact product.  Cluster shape 1x1x1: no multicast loads.
+// mode: each fp32 operand is split into three bf16 terms and, of the nine
+// products, the six above fp32 rounding are accumulated in fp32, which keeps
+// the result within fp32 rounding of the exact product.  Cluster shape 1x1x1: every CTA loads its own
+// operand tiles from this GPU's memory.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
